@@ -1,0 +1,173 @@
+/*
+ * dsa_decode.h -- C ABI of libdsa.so: the decode/verify step of a DeepSeek
+ * Sparse Attention (DSA) layer with a GQA-4 backbone, on one NVIDIA B200.
+ *
+ * The step (NaiveAI research page, naive.ai/en/research):
+ *   1. Indexer scan.  "Technical Details > Model Architecture": a lightweight
+ *      indexer scores the full history.  "Hybrid SWA-DSA Architecture": the
+ *      indexer has 16 query heads.  The page does not print the scoring rule;
+ *      this library uses the DSA indexer's form
+ *          I[t,s] = scale[s] * sum_{j<16} w[t,j] * ReLU(q_idx[t,j,:] . k_idx[s,:])
+ *      over 64-dim keys (scale = 1 unless a per-token scale is given).
+ *   2. Causal top-k.  "Hybrid SWA-DSA Architecture": DSA selects the top
+ *      2,048 tokens.  Query t sits at position pos[t] and may select
+ *      s in [0, pos[t]].  If pos[t] + 1 <= topk every visible position is
+ *      selected; otherwise the topk largest scores, equal scores going to the
+ *      lower position, which makes the result unique.  "NaiveRT > Why
+ *      single-stream speed matters for RL" requires bitwise-identical results
+ *      run to run; every kernel here is deterministic.
+ *   3. Sparse attention.  "Hybrid SWA-DSA Architecture": GQA with four KV
+ *      groups; "NaiveRT > Optimizing inside the kernel": eight query heads
+ *      per GPU under TP8, i.e. 64 query heads.  For head h (group g = h / 16)
+ *          out[t,h,:] = sum_{s in S_t} softmax_s(q[t,h,:] . K[s,g,:] / sqrt(128)) V[s,g,:]
+ *      over the selected set S_t only.
+ *
+ * Conventions for every entry point:
+ *   - Device pointers unless stated otherwise.  The caller owns every buffer;
+ *     the library keeps no pointer after a call returns.  Outputs must not
+ *     alias inputs.
+ *   - All work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and is asynchronous: results are valid once the stream reaches
+ *     that point.  No entry point synchronises, except dsa_device_status.
+ *   - Arguments are checked on the host before any launch; a failed check
+ *     returns DSA_ERR_INVALID_ARG (or DSA_ERR_UNSUPPORTED for a shape this
+ *     build does not handle) and launches nothing; dsa_last_error() then
+ *     describes it.  Kernels never trap: an anomaly found on the device (an
+ *     out-of-range selected index given to dsa_sparse_attn, a bounded wait that
+ *     ran out) sets a device error word that dsa_device_status reports.
+ *   - Inputs with NaN (an E4M3 code S.1111.111, a NaN bf16) give unspecified
+ *     output values but never an out-of-bounds access.
+ */
+#ifndef DSA_DECODE_H
+#define DSA_DECODE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define DSA_API __attribute__((visibility("default")))
+#else
+#define DSA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A cudaStream_t, declared without the CUDA headers. */
+typedef struct CUstream_st *dsa_stream_t;
+
+typedef enum {
+    DSA_OK = 0,
+    DSA_ERR_INVALID_ARG = 1, /* a null pointer, bad shape, stride, alignment, dtype, pos or topk */
+    DSA_ERR_UNSUPPORTED = 2, /* head shape or size outside what this build implements */
+    DSA_ERR_CUDA = 3,        /* a CUDA runtime call failed (launch, allocation, ...) */
+    DSA_ERR_DEVICE = 4       /* a kernel reported an anomaly (see dsa_device_status) */
+} dsa_status_t;
+
+typedef enum {
+    DSA_BF16 = 0,     /* bfloat16, 2 bytes */
+    DSA_FP8_E4M3 = 1, /* OCP FP8 E4M3, 1 byte */
+    DSA_F32 = 2,      /* IEEE binary32 */
+    DSA_I32 = 3       /* int32 */
+} dsa_dtype_t;
+
+/* A strided tensor view.  Strides are in elements; the innermost dimension must
+ * have stride 1 and every other stride must keep rows 16-byte aligned.  `scale`
+ * is read only for the indexer key cache: a per-token fp32 scale [L] (device),
+ * or NULL for 1. */
+typedef struct {
+    void *data;
+    int32_t dtype;      /* dsa_dtype_t */
+    int32_t ndim;
+    int64_t shape[4];
+    int64_t stride[4];
+    const float *scale;
+} dsa_tensor_t;
+
+/* Shapes (T = query tokens, 1..8; L = cached positions, including the query
+ * tokens' own; topk in 1..2048):
+ *   q            [T][64][128]      bf16, contiguous        backbone queries (post-RoPE)
+ *   q_idx        [T][16][64]       bf16, contiguous        indexer queries
+ *   w_idx        [T][16]           f32, contiguous         indexer head weights
+ *   k_idx_cache  [L][64]           bf16 or fp8-e4m3, row stride >= 64 and a multiple
+ *                                  of 16 bytes; optional per-token scale [L] f32 (> 0)
+ *   kv_cache     [L][2][4][128]    bf16; per token the K rows of the 4 groups, then
+ *                                  the V rows; token stride >= 1024 elements and a
+ *                                  multiple of 8; inner dims contiguous
+ *   pos          HOST int32 [T],   0 <= pos[t] < L
+ *   out          [T][64][128]      bf16, contiguous        attention output
+ *   sel_idx      [T][topk]         int32, row stride >= topk: the selected positions of
+ *                                  query t in ascending order, then -1 padding
+ * All device base addresses must be 16-byte aligned. */
+
+/* Bytes of workspace dsa_decode_ws needs for these sizes (0 if they are invalid). */
+DSA_API size_t dsa_workspace_bytes(int32_t T, int64_t L, int32_t topk);
+
+/* The whole step: indexer scan, causal top-k, sparse attention.  Takes its
+ * workspace stream-ordered (cudaMallocAsync / cudaFreeAsync on `stream`), so it
+ * must not be captured into a CUDA graph on a device without memory-pool
+ * support; use dsa_decode_ws for graphs. */
+DSA_API dsa_status_t dsa_decode(const dsa_tensor_t *q, const dsa_tensor_t *q_idx, const dsa_tensor_t *w_idx,
+                        const dsa_tensor_t *k_idx_cache, const dsa_tensor_t *kv_cache,
+                        const int32_t *pos, int32_t topk, dsa_tensor_t *out, dsa_tensor_t *sel_idx,
+                        dsa_stream_t stream);
+
+/* Same as dsa_decode with a caller-provided device workspace of at least
+ * dsa_workspace_bytes(T, L, topk) bytes, 256-byte aligned.  Makes no allocation
+ * and no synchronisation, so it can be captured in a CUDA graph (pos is read
+ * on the host at call time and baked into the launches). */
+DSA_API dsa_status_t dsa_decode_ws(const dsa_tensor_t *q, const dsa_tensor_t *q_idx, const dsa_tensor_t *w_idx,
+                           const dsa_tensor_t *k_idx_cache, const dsa_tensor_t *kv_cache,
+                           const int32_t *pos, int32_t topk, dsa_tensor_t *out, dsa_tensor_t *sel_idx,
+                           dsa_stream_t stream, void *workspace, size_t workspace_bytes);
+
+/* Stage 1 alone: scores [T][ld] f32 (ld >= L, a multiple of 4).  scores[t][s] is
+ * I[t,s] for s <= pos[t] and -inf for s > pos[t].  The sum is taken in fp32
+ * (tensor-core dot products, then a fixed-order weighted sum over heads). */
+DSA_API dsa_status_t dsa_index_scores(const dsa_tensor_t *q_idx, const dsa_tensor_t *w_idx,
+                              const dsa_tensor_t *k_idx_cache, const int32_t *pos, float *scores,
+                              int64_t ld, dsa_stream_t stream);
+
+/* Stage 2 alone: causal top-k of caller scores [T][ld] (f32, ld >= L, a multiple
+ * of 4; entries s > pos[t] are ignored).  -0 and +0 compare equal.  Writes sel_idx
+ * [T][sel_ld] (sel_ld >= topk).  Workspace: dsa_workspace_bytes(T, L, topk). */
+DSA_API dsa_status_t dsa_topk_from_scores(const float *scores, int32_t T, int64_t L, int64_t ld,
+                                  const int32_t *pos, int32_t topk, int32_t *sel_idx, int64_t sel_ld,
+                                  dsa_stream_t stream, void *workspace, size_t workspace_bytes);
+
+/* Stage 3 alone: attention of q over the rows listed in sel_idx [T][topk]
+ * (entries < 0 are skipped; an entry outside [0, pos[t]] is skipped and flags
+ * DSA_ERR_DEVICE).  `sink` is NULL or a per-head logit [64] f32 (device) that
+ * joins each head's softmax denominator with no value row (an attention sink).
+ * Workspace: dsa_workspace_bytes(T, L, topk). */
+DSA_API dsa_status_t dsa_sparse_attn(const dsa_tensor_t *q, const dsa_tensor_t *kv_cache,
+                             const dsa_tensor_t *sel_idx, const int32_t *pos, const float *sink,
+                             dsa_tensor_t *out, dsa_stream_t stream, void *workspace,
+                             size_t workspace_bytes);
+
+/* Synchronises `stream`, then reads and clears the device error word of the
+ * current device: DSA_OK, DSA_ERR_DEVICE (an anomaly was flagged since the last
+ * call), or DSA_ERR_CUDA (the stream reported an error). */
+DSA_API dsa_status_t dsa_device_status(dsa_stream_t stream);
+
+/* Static description of a status code. */
+DSA_API const char *dsa_status_str(dsa_status_t status);
+
+/* Detail of the last failed call on this host thread ("" if none). */
+DSA_API const char *dsa_last_error(void);
+
+/* Number of kernels this library has launched in this process (all devices). */
+DSA_API uint64_t dsa_launch_count(void);
+
+/* Profiling hook for the calling host thread.  With n == 5, dsa_decode and
+ * dsa_decode_ws record five cudaEvent_t on their stream: events[0] before the
+ * first launch, events[1] after the indexer scan, events[2] after the top-k
+ * selection, events[3] after the split attention kernel and events[4] after the
+ * split combine.  n == 0 disables; any other n is ignored. */
+DSA_API void dsa_set_stage_events(void *const *events, int32_t n);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DSA_DECODE_H */

@@ -1,0 +1,529 @@
+// dsa_api.cu -- the C ABI of libdsa.so (declared in include/dsa_decode.h):
+// argument checks, workspace layout, TMA descriptor set-up and launch sequencing
+// of the three stages.  No compute happens on the host.
+#include <atomic>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include "../../include/dsa_decode.h"
+#include "dsa_internal.h"
+
+namespace dsa {
+
+__device__ uint32_t g_err_word;
+
+namespace {
+
+thread_local std::string t_last_error;
+thread_local void* t_stage_events[5] = {nullptr, nullptr, nullptr, nullptr, nullptr};
+thread_local bool t_stage_events_on = false;
+std::atomic<uint64_t> g_launches{0};
+
+dsa_status_t fail(dsa_status_t st, const char* fmt, ...)
+{
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    t_last_error = buf;
+    return st;
+}
+
+dsa_status_t cuda_fail(cudaError_t e, const char* what)
+{
+    return fail(DSA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+struct DeviceInfo {
+    int sms = 0;
+    uint32_t* err = nullptr;
+};
+
+dsa_status_t device_info(DeviceInfo& info)
+{
+    static DeviceInfo cache[64];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= 64) return fail(DSA_ERR_UNSUPPORTED, "device ordinal %d", dev);
+    if (cache[dev].sms == 0) {
+        DeviceInfo d;
+        e = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+        e = cudaGetSymbolAddress(reinterpret_cast<void**>(&d.err), g_err_word);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress");
+        cache[dev] = d;
+    }
+    info = cache[dev];
+    return DSA_OK;
+}
+
+void stage_event(int i, cudaStream_t s)
+{
+    if (t_stage_events_on && t_stage_events[i]) cudaEventRecord(static_cast<cudaEvent_t>(t_stage_events[i]), s);
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
+
+// ------------------------------------------------------------------ checks
+struct Shape {
+    int T = 0;
+    int64_t L = 0;
+    bool fp8 = false;
+    int64_t k_ld = 0;    // elements per indexer key row
+    int64_t kv_ld = 0;   // elements per cached token row
+};
+
+dsa_status_t check_contig(const dsa_tensor_t* x, const char* name, int dtype, int ndim, const int64_t* dims)
+{
+    if (!x || !x->data) return fail(DSA_ERR_INVALID_ARG, "%s: null", name);
+    if (x->dtype != dtype) return fail(DSA_ERR_INVALID_ARG, "%s: dtype %d, expected %d", name, x->dtype, dtype);
+    if (x->ndim != ndim) return fail(DSA_ERR_INVALID_ARG, "%s: ndim %d, expected %d", name, x->ndim, ndim);
+    int64_t expect = 1;
+    for (int i = ndim - 1; i >= 0; --i) {
+        if (dims[i] >= 0 && x->shape[i] != dims[i])
+            return fail(i == 0 ? DSA_ERR_INVALID_ARG : DSA_ERR_UNSUPPORTED, "%s: shape[%d] = %lld, expected %lld",
+                        name, i, (long long)x->shape[i], (long long)dims[i]);
+        if (x->stride[i] != expect)
+            return fail(DSA_ERR_INVALID_ARG, "%s: must be contiguous (stride[%d] = %lld)", name, i,
+                        (long long)x->stride[i]);
+        expect *= x->shape[i];
+    }
+    if (!aligned16(x->data)) return fail(DSA_ERR_INVALID_ARG, "%s: base not 16-byte aligned", name);
+    return DSA_OK;
+}
+
+dsa_status_t check_T(int64_t T)
+{
+    if (T < 1 || T > kMaxT) return fail(DSA_ERR_UNSUPPORTED, "T = %lld query tokens (1..%d supported)", (long long)T, kMaxT);
+    return DSA_OK;
+}
+
+dsa_status_t check_indexer_inputs(const dsa_tensor_t* q_idx, const dsa_tensor_t* w_idx, const dsa_tensor_t* k,
+                                  const int32_t* pos, Shape& sh)
+{
+    if (!q_idx) return fail(DSA_ERR_INVALID_ARG, "q_idx: null");
+    sh.T = static_cast<int>(q_idx->shape[0]);
+    dsa_status_t st = check_T(q_idx->shape[0]);
+    if (st) return st;
+    const int64_t qd[3] = {sh.T, kHI, kDI};
+    if ((st = check_contig(q_idx, "q_idx", DSA_BF16, 3, qd))) return st;
+    const int64_t wd[2] = {sh.T, kHI};
+    if ((st = check_contig(w_idx, "w_idx", DSA_F32, 2, wd))) return st;
+    if (!k || !k->data) return fail(DSA_ERR_INVALID_ARG, "k_idx_cache: null");
+    if (k->dtype != DSA_BF16 && k->dtype != DSA_FP8_E4M3)
+        return fail(DSA_ERR_INVALID_ARG, "k_idx_cache: dtype must be bf16 or fp8-e4m3");
+    if (k->ndim != 2) return fail(DSA_ERR_INVALID_ARG, "k_idx_cache: ndim must be 2");
+    if (k->shape[1] != kDI) return fail(DSA_ERR_UNSUPPORTED, "k_idx_cache: dim %lld (64 supported)", (long long)k->shape[1]);
+    sh.L = k->shape[0];
+    if (sh.L < 1 || sh.L > INT32_MAX - 4096) return fail(DSA_ERR_INVALID_ARG, "k_idx_cache: L = %lld", (long long)sh.L);
+    sh.fp8 = k->dtype == DSA_FP8_E4M3;
+    const int64_t es = sh.fp8 ? 1 : 2;
+    if (k->stride[1] != 1 || k->stride[0] < kDI || (k->stride[0] * es) % 16)
+        return fail(DSA_ERR_INVALID_ARG, "k_idx_cache: row stride must be >= 64 elements and a multiple of 16 bytes");
+    if (!aligned16(k->data)) return fail(DSA_ERR_INVALID_ARG, "k_idx_cache: base not 16-byte aligned");
+    if (k->scale && !aligned16(k->scale)) return fail(DSA_ERR_INVALID_ARG, "k_idx_cache.scale: not 16-byte aligned");
+    sh.k_ld = k->stride[0];
+    if (!pos) return fail(DSA_ERR_INVALID_ARG, "pos: null");
+    for (int t = 0; t < sh.T; ++t)
+        if (pos[t] < 0 || pos[t] >= sh.L)
+            return fail(DSA_ERR_INVALID_ARG, "pos[%d] = %d outside [0, L = %lld)", t, pos[t], (long long)sh.L);
+    return DSA_OK;
+}
+
+dsa_status_t check_kv(const dsa_tensor_t* kv, Shape& sh)
+{
+    if (!kv || !kv->data) return fail(DSA_ERR_INVALID_ARG, "kv_cache: null");
+    if (kv->dtype != DSA_BF16) return fail(DSA_ERR_INVALID_ARG, "kv_cache: dtype must be bf16");
+    if (kv->ndim != 4) return fail(DSA_ERR_INVALID_ARG, "kv_cache: ndim must be 4");
+    if (kv->shape[1] != 2 || kv->shape[2] != kG || kv->shape[3] != kD)
+        return fail(DSA_ERR_UNSUPPORTED, "kv_cache: shape [L][2][4][128] supported");
+    if (kv->stride[3] != 1 || kv->stride[2] != kD || kv->stride[1] != kG * kD || kv->stride[0] < 2 * kG * kD ||
+        kv->stride[0] % 8)
+        return fail(DSA_ERR_INVALID_ARG, "kv_cache: token rows must be [2][4][128] contiguous, stride a multiple of 8");
+    if (!aligned16(kv->data)) return fail(DSA_ERR_INVALID_ARG, "kv_cache: base not 16-byte aligned");
+    if (sh.L && kv->shape[0] != sh.L)
+        return fail(DSA_ERR_INVALID_ARG, "kv_cache: L = %lld but the key cache has %lld", (long long)kv->shape[0],
+                    (long long)sh.L);
+    sh.L = kv->shape[0];
+    sh.kv_ld = kv->stride[0];
+    return DSA_OK;
+}
+
+dsa_status_t check_topk(int32_t topk)
+{
+    if (topk < 1 || topk > kMaxTopk) return fail(DSA_ERR_INVALID_ARG, "topk = %d outside [1, %d]", topk, kMaxTopk);
+    return DSA_OK;
+}
+
+dsa_status_t check_sel(const dsa_tensor_t* sel, int T, int32_t topk)
+{
+    if (!sel || !sel->data) return fail(DSA_ERR_INVALID_ARG, "sel_idx: null");
+    if (sel->dtype != DSA_I32 || sel->ndim != 2) return fail(DSA_ERR_INVALID_ARG, "sel_idx: int32 [T][topk] expected");
+    if (sel->shape[0] != T || sel->shape[1] != topk)
+        return fail(DSA_ERR_INVALID_ARG, "sel_idx: shape [%lld][%lld], expected [%d][%d]", (long long)sel->shape[0],
+                    (long long)sel->shape[1], T, topk);
+    if (sel->stride[1] != 1 || sel->stride[0] < topk)
+        return fail(DSA_ERR_INVALID_ARG, "sel_idx: rows must be contiguous with stride >= topk");
+    if (!aligned16(sel->data)) return fail(DSA_ERR_INVALID_ARG, "sel_idx: base not 16-byte aligned");
+    return DSA_OK;
+}
+
+// ------------------------------------------------------------------ workspace
+struct Layout {
+    int64_t ld = 0;            // score / candidate row stride (elements)
+    size_t hist = 0, tickets = 0, zero_bytes = 0;
+    size_t counts = 0, scores = 0, cand = 0, part_o = 0, part_ml = 0;
+    size_t total = 0;
+};
+
+Layout layout(int T, int64_t L)
+{
+    Layout l;
+    l.ld = round_up(L, 64);
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t at = off;
+        off += static_cast<size_t>(round_up(static_cast<int64_t>(bytes), 256));
+        return at;
+    };
+    l.hist = take(sizeof(uint32_t) * (size_t)T * kHistBins + sizeof(uint32_t) * kMaxT);
+    l.tickets = l.hist + sizeof(uint32_t) * (size_t)T * kHistBins;
+    l.zero_bytes = off;
+    l.counts = take(sizeof(uint32_t) * (size_t)T * kMaxChunks);
+    l.scores = take(sizeof(float) * (size_t)T * l.ld);
+    l.cand = take(sizeof(uint2) * (size_t)T * l.ld);
+    l.part_o = take(sizeof(float) * (size_t)T * kMaxSplits * kH * kD);
+    l.part_ml = take(sizeof(float2) * (size_t)T * kMaxSplits * kH);
+    l.total = off;
+    return l;
+}
+
+dsa_status_t check_ws(void* ws, size_t bytes, const Layout& l)
+{
+    if (!ws) return fail(DSA_ERR_INVALID_ARG, "workspace: null");
+    if (reinterpret_cast<uintptr_t>(ws) & 255u) return fail(DSA_ERR_INVALID_ARG, "workspace: not 256-byte aligned");
+    if (bytes < l.total)
+        return fail(DSA_ERR_INVALID_ARG, "workspace: %zu bytes, %zu needed", bytes, l.total);
+    return DSA_OK;
+}
+
+template <typename P>
+P* at(void* ws, size_t off) { return reinterpret_cast<P*>(static_cast<char*>(ws) + off); }
+
+// ------------------------------------------------------------------ stage launches
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        cudaDriverEntryPointQueryResult q;
+        void* p = nullptr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+dsa_status_t run_indexer(const dsa_tensor_t* q_idx, const dsa_tensor_t* w_idx, const dsa_tensor_t* k,
+                         const int32_t* pos, const Shape& sh, float* scores, int64_t ld, const DeviceInfo& dev,
+                         cudaStream_t stream)
+{
+    auto enc = encode_fn();
+    if (!enc) return fail(DSA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+    CUtensorMap map;
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(kDI), static_cast<cuuint64_t>(sh.L)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(sh.k_ld * (sh.fp8 ? 1 : 2))};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(kDI), static_cast<cuuint32_t>(kKeyTile)};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(&map, sh.fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, k->data, dims,
+                     strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     sh.fp8 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(DSA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+    IndexerParams p{};
+    p.q_idx = static_cast<const uint16_t*>(q_idx->data);
+    p.w = static_cast<const float*>(w_idx->data);
+    p.scale = k->scale;
+    p.scores = scores;
+    p.ld = ld;
+    p.L = static_cast<int32_t>(sh.L);
+    int n_max = 0;
+    for (int t = 0; t < sh.T; ++t) {
+        p.pos[t] = pos[t];
+        n_max = pos[t] + 1 > n_max ? pos[t] + 1 : n_max;
+    }
+    p.n_max = n_max;
+    p.err = dev.err;
+    const int ntiles = static_cast<int>((n_max + kKeyTile - 1) / kKeyTile);
+    int grid = dev.sms * indexer_max_ctas_per_sm(sh.T, sh.fp8);
+    if (grid > ntiles) grid = ntiles;
+    if (grid < 1) grid = 1;
+    cudaError_t e = launch_indexer(&map, p, sh.T, sh.fp8, grid, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "indexer launch");
+    g_launches += 1;
+    return DSA_OK;
+}
+
+dsa_status_t run_topk(const float* scores, int64_t ld, int T, const int32_t* pos, int32_t topk, int32_t* sel,
+                      int64_t sel_ld, void* ws, const Layout& l, const DeviceInfo& dev, cudaStream_t stream)
+{
+    TopkParams p{};
+    p.scores = scores;
+    p.ld = ld;
+    p.T = T;
+    p.topk = topk;
+    int64_t n_max = 0;
+    for (int t = 0; t < T; ++t) {
+        p.pos[t] = pos[t];
+        n_max = pos[t] + 1 > n_max ? pos[t] + 1 : n_max;
+    }
+    // About two blocks per SM over all queries, chunks a multiple of 2048 scores.
+    const int64_t per_query = (2 * dev.sms + T - 1) / T;
+    int64_t chunk = round_up((n_max + per_query - 1) / per_query, 2048);
+    if (chunk < 4096) chunk = 4096;
+    while ((n_max + chunk - 1) / chunk > kMaxChunks) chunk += 2048;
+    p.chunk = static_cast<int32_t>(chunk);
+    p.nchunks = static_cast<int32_t>((n_max + chunk - 1) / chunk);
+    p.hist = at<uint32_t>(ws, l.hist);
+    p.tickets = at<uint32_t>(ws, l.tickets);
+    p.counts = at<uint32_t>(ws, l.counts);
+    p.cand = at<uint2>(ws, l.cand);
+    p.sel = sel;
+    p.sel_ld = sel_ld;
+    p.err = dev.err;
+    cudaError_t e = cudaMemsetAsync(ws, 0, l.zero_bytes, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "workspace clear");
+    if ((e = launch_topk_hist(p, stream)) != cudaSuccess) return cuda_fail(e, "top-k histogram launch");
+    if ((e = launch_topk_select(p, stream)) != cudaSuccess) return cuda_fail(e, "top-k select launch");
+    g_launches += 2;
+    return DSA_OK;
+}
+
+dsa_status_t run_attention(const dsa_tensor_t* q, const dsa_tensor_t* kv, const int32_t* sel, int64_t sel_ld,
+                           int32_t topk, const int32_t* pos, const float* sink, dsa_tensor_t* out, const Shape& sh,
+                           void* ws, const Layout& l, const DeviceInfo& dev, cudaStream_t stream)
+{
+    AttnParams p{};
+    p.q = static_cast<const uint16_t*>(q->data);
+    p.kv = static_cast<const uint16_t*>(kv->data);
+    p.kv_ld = sh.kv_ld;
+    p.sel = sel;
+    p.sel_ld = sel_ld;
+    p.L = static_cast<int32_t>(sh.L);
+    p.rows = topk;
+    int64_t nsplit = (2 * dev.sms + sh.T - 1) / sh.T;
+    if (nsplit > kMaxSplits) nsplit = kMaxSplits;
+    int64_t rps = round_up((topk + nsplit - 1) / nsplit, 16);
+    p.rows_per_split = static_cast<int32_t>(rps);
+    p.nsplit = static_cast<int32_t>((topk + rps - 1) / rps);
+    for (int t = 0; t < sh.T; ++t) p.pos[t] = pos[t];
+    p.sink = sink;
+    p.part_o = at<float>(ws, l.part_o);
+    p.part_ml = at<float2>(ws, l.part_ml);
+    p.out = static_cast<uint16_t*>(out->data);
+    p.err = dev.err;
+    cudaError_t e = launch_attention(p, sh.T, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "attention launch");
+    stage_event(3, stream);
+    if ((e = launch_combine(p, sh.T, stream)) != cudaSuccess) return cuda_fail(e, "combine launch");
+    g_launches += 2;
+    return DSA_OK;
+}
+
+dsa_status_t check_decode_args(const dsa_tensor_t* q, const dsa_tensor_t* q_idx, const dsa_tensor_t* w_idx,
+                               const dsa_tensor_t* k_idx_cache, const dsa_tensor_t* kv_cache, const int32_t* pos,
+                               int32_t topk, dsa_tensor_t* out, dsa_tensor_t* sel_idx, Shape& sh)
+{
+    dsa_status_t st = check_indexer_inputs(q_idx, w_idx, k_idx_cache, pos, sh);
+    if (st) return st;
+    const int64_t qd[3] = {sh.T, kH, kD};
+    if ((st = check_contig(q, "q", DSA_BF16, 3, qd))) return st;
+    if ((st = check_kv(kv_cache, sh))) return st;
+    if ((st = check_topk(topk))) return st;
+    if ((st = check_contig(out, "out", DSA_BF16, 3, qd))) return st;
+    if ((st = check_sel(sel_idx, sh.T, topk))) return st;
+    return DSA_OK;
+}
+
+}  // namespace
+}  // namespace dsa
+
+using namespace dsa;
+
+extern "C" {
+
+size_t dsa_workspace_bytes(int32_t T, int64_t L, int32_t topk)
+{
+    if (T < 1 || T > kMaxT || L < 1 || L > INT32_MAX - 4096 || topk < 1 || topk > kMaxTopk) return 0;
+    return layout(T, L).total;
+}
+
+dsa_status_t dsa_decode_ws(const dsa_tensor_t* q, const dsa_tensor_t* q_idx, const dsa_tensor_t* w_idx,
+                           const dsa_tensor_t* k_idx_cache, const dsa_tensor_t* kv_cache, const int32_t* pos,
+                           int32_t topk, dsa_tensor_t* out, dsa_tensor_t* sel_idx, dsa_stream_t stream_,
+                           void* workspace, size_t workspace_bytes)
+{
+    t_last_error.clear();
+    Shape sh;
+    dsa_status_t st = check_decode_args(q, q_idx, w_idx, k_idx_cache, kv_cache, pos, topk, out, sel_idx, sh);
+    if (st) return st;
+    const Layout l = layout(sh.T, sh.L);
+    if ((st = check_ws(workspace, workspace_bytes, l))) return st;
+    DeviceInfo dev;
+    if ((st = device_info(dev))) return st;
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    float* scores = at<float>(workspace, l.scores);
+    stage_event(0, stream);
+    if ((st = run_indexer(q_idx, w_idx, k_idx_cache, pos, sh, scores, l.ld, dev, stream))) return st;
+    stage_event(1, stream);
+    int32_t* sel = static_cast<int32_t*>(sel_idx->data);
+    if ((st = run_topk(scores, l.ld, sh.T, pos, topk, sel, sel_idx->stride[0], workspace, l, dev, stream))) return st;
+    stage_event(2, stream);
+    if ((st = run_attention(q, kv_cache, sel, sel_idx->stride[0], topk, pos, nullptr, out, sh, workspace, l, dev,
+                            stream)))
+        return st;
+    stage_event(4, stream);
+    return DSA_OK;
+}
+
+dsa_status_t dsa_decode(const dsa_tensor_t* q, const dsa_tensor_t* q_idx, const dsa_tensor_t* w_idx,
+                        const dsa_tensor_t* k_idx_cache, const dsa_tensor_t* kv_cache, const int32_t* pos,
+                        int32_t topk, dsa_tensor_t* out, dsa_tensor_t* sel_idx, dsa_stream_t stream_)
+{
+    t_last_error.clear();
+    Shape sh;
+    dsa_status_t st = check_decode_args(q, q_idx, w_idx, k_idx_cache, kv_cache, pos, topk, out, sel_idx, sh);
+    if (st) return st;
+    const size_t bytes = layout(sh.T, sh.L).total;
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    void* ws = nullptr;
+    cudaError_t e = cudaMallocAsync(&ws, bytes, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMallocAsync(workspace)");
+    st = dsa_decode_ws(q, q_idx, w_idx, k_idx_cache, kv_cache, pos, topk, out, sel_idx, stream_, ws, bytes);
+    e = cudaFreeAsync(ws, stream);
+    if (st == DSA_OK && e != cudaSuccess) return cuda_fail(e, "cudaFreeAsync(workspace)");
+    return st;
+}
+
+dsa_status_t dsa_index_scores(const dsa_tensor_t* q_idx, const dsa_tensor_t* w_idx, const dsa_tensor_t* k_idx_cache,
+                              const int32_t* pos, float* scores, int64_t ld, dsa_stream_t stream_)
+{
+    t_last_error.clear();
+    Shape sh;
+    dsa_status_t st = check_indexer_inputs(q_idx, w_idx, k_idx_cache, pos, sh);
+    if (st) return st;
+    if (!scores || !aligned16(scores)) return fail(DSA_ERR_INVALID_ARG, "scores: null or not 16-byte aligned");
+    if (ld < sh.L || ld % 4) return fail(DSA_ERR_INVALID_ARG, "scores: ld = %lld must be >= L and a multiple of 4", (long long)ld);
+    DeviceInfo dev;
+    if ((st = device_info(dev))) return st;
+    return run_indexer(q_idx, w_idx, k_idx_cache, pos, sh, scores, ld, dev, reinterpret_cast<cudaStream_t>(stream_));
+}
+
+dsa_status_t dsa_topk_from_scores(const float* scores, int32_t T, int64_t L, int64_t ld, const int32_t* pos,
+                                  int32_t topk, int32_t* sel_idx, int64_t sel_ld, dsa_stream_t stream_,
+                                  void* workspace, size_t workspace_bytes)
+{
+    t_last_error.clear();
+    dsa_status_t st = check_T(T);
+    if (st) return st;
+    if ((st = check_topk(topk))) return st;
+    if (L < 1 || L > INT32_MAX - 4096) return fail(DSA_ERR_INVALID_ARG, "L = %lld", (long long)L);
+    if (!scores || !aligned16(scores)) return fail(DSA_ERR_INVALID_ARG, "scores: null or not 16-byte aligned");
+    if (ld < L || ld % 4) return fail(DSA_ERR_INVALID_ARG, "scores: ld must be >= L and a multiple of 4");
+    if (!sel_idx || !aligned16(sel_idx) || sel_ld < topk)
+        return fail(DSA_ERR_INVALID_ARG, "sel_idx: null, unaligned, or sel_ld < topk");
+    if (!pos) return fail(DSA_ERR_INVALID_ARG, "pos: null");
+    for (int t = 0; t < T; ++t)
+        if (pos[t] < 0 || pos[t] >= L) return fail(DSA_ERR_INVALID_ARG, "pos[%d] = %d outside [0, L)", t, pos[t]);
+    const Layout l = layout(T, L);
+    if ((st = check_ws(workspace, workspace_bytes, l))) return st;
+    DeviceInfo dev;
+    if ((st = device_info(dev))) return st;
+    return run_topk(scores, ld, T, pos, topk, sel_idx, sel_ld, workspace, l, dev, reinterpret_cast<cudaStream_t>(stream_));
+}
+
+dsa_status_t dsa_sparse_attn(const dsa_tensor_t* q, const dsa_tensor_t* kv_cache, const dsa_tensor_t* sel_idx,
+                             const int32_t* pos, const float* sink, dsa_tensor_t* out, dsa_stream_t stream_,
+                             void* workspace, size_t workspace_bytes)
+{
+    t_last_error.clear();
+    if (!q) return fail(DSA_ERR_INVALID_ARG, "q: null");
+    Shape sh;
+    sh.T = static_cast<int>(q->shape[0]);
+    dsa_status_t st = check_T(q->shape[0]);
+    if (st) return st;
+    const int64_t qd[3] = {sh.T, kH, kD};
+    if ((st = check_contig(q, "q", DSA_BF16, 3, qd))) return st;
+    if ((st = check_kv(kv_cache, sh))) return st;
+    if (!sel_idx) return fail(DSA_ERR_INVALID_ARG, "sel_idx: null");
+    const int32_t topk = static_cast<int32_t>(sel_idx->shape[1]);
+    if ((st = check_topk(topk))) return st;
+    if ((st = check_sel(sel_idx, sh.T, topk))) return st;
+    if ((st = check_contig(out, "out", DSA_BF16, 3, qd))) return st;
+    if (!pos) return fail(DSA_ERR_INVALID_ARG, "pos: null");
+    for (int t = 0; t < sh.T; ++t)
+        if (pos[t] < 0 || pos[t] >= sh.L) return fail(DSA_ERR_INVALID_ARG, "pos[%d] = %d outside [0, L)", t, pos[t]);
+    if (sink && !aligned16(sink)) return fail(DSA_ERR_INVALID_ARG, "sink: not 16-byte aligned");
+    const Layout l = layout(sh.T, sh.L);
+    if ((st = check_ws(workspace, workspace_bytes, l))) return st;
+    DeviceInfo dev;
+    if ((st = device_info(dev))) return st;
+    return run_attention(q, kv_cache, static_cast<const int32_t*>(sel_idx->data), sel_idx->stride[0], topk, pos, sink,
+                         out, sh, workspace, l, dev, reinterpret_cast<cudaStream_t>(stream_));
+}
+
+dsa_status_t dsa_device_status(dsa_stream_t stream_)
+{
+    t_last_error.clear();
+    cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream_));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+    uint32_t word = 0;
+    e = cudaMemcpyFromSymbol(&word, g_err_word, sizeof word);
+    if (e != cudaSuccess) return cuda_fail(e, "read device error word");
+    if (word) {
+        const uint32_t zero = 0;
+        e = cudaMemcpyToSymbol(g_err_word, &zero, sizeof zero);
+        if (e != cudaSuccess) return cuda_fail(e, "clear device error word");
+        return fail(DSA_ERR_DEVICE, "device error word 0x%x (1: wait timeout, 2: bad selected index, 4: top-k state)",
+                    word);
+    }
+    return DSA_OK;
+}
+
+const char* dsa_status_str(dsa_status_t s)
+{
+    switch (s) {
+    case DSA_OK: return "ok";
+    case DSA_ERR_INVALID_ARG: return "invalid argument";
+    case DSA_ERR_UNSUPPORTED: return "unsupported shape or size";
+    case DSA_ERR_CUDA: return "CUDA runtime error";
+    case DSA_ERR_DEVICE: return "device-side anomaly";
+    }
+    return "unknown status";
+}
+
+const char* dsa_last_error(void) { return t_last_error.c_str(); }
+
+uint64_t dsa_launch_count(void) { return g_launches.load(); }
+
+void dsa_set_stage_events(void* const* events, int32_t n)
+{
+    if (n == 5 && events) {
+        for (int i = 0; i < 5; ++i) t_stage_events[i] = events[i];
+        t_stage_events_on = true;
+    } else if (n == 0) {
+        t_stage_events_on = false;
+    }
+}
+
+}  // extern "C"
