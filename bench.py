@@ -230,13 +230,16 @@ def main():
         kernels_per_step = dsa.dsa_launch_count() - n0
     stream.synchronize()
     dsa.dsa_device_status(stream)
+    # torch only reports elapsed time for events it has recorded itself once.
+    for e in ev:
+        e.record(stream)
+    stream.synchronize()
     graph = torch.cuda.CUDAGraph()
-    dsa.dsa_set_stage_events(ev)
     with torch.cuda.graph(graph, stream=stream):
         step()
-    dsa.dsa_set_stage_events(None)
 
     def timed_step():
+        """Cold L2, then one graph replay of the whole step, timed by events."""
         flush.zero_()
         s0 = torch.cuda.Event(enable_timing=True)
         s1 = torch.cuda.Event(enable_timing=True)
@@ -246,18 +249,32 @@ def main():
             graph.replay()
             s1.record(stream)
         stream.synchronize()
-        stages = [ev[i].elapsed_time(ev[i + 1]) for i in range(4)]
-        return s0.elapsed_time(s1), stages
+        return s0.elapsed_time(s1)
+
+    def staged_step():
+        """Cold L2, then the step launched eagerly with an event after every kernel.
+        A spin on the stream first lets the host enqueue all launches, so the
+        gaps between events are device time only."""
+        flush.zero_()
+        with torch.cuda.stream(stream):
+            stream.wait_stream(torch.cuda.current_stream())
+            torch.cuda._sleep(200000)
+            dsa.dsa_set_stage_events(ev)
+            step()
+            dsa.dsa_set_stage_events(None)
+        stream.synchronize()
+        return [ev[i].elapsed_time(ev[i + 1]) for i in range(4)]
 
     for _ in range(args.warmup):
         timed_step()
+        staged_step()
     barrier(world)
     clocks = Clocks(local)
     totals, stage_sum = [], [0.0] * 4
     for _ in range(args.steps):
-        t, stages = timed_step()
-        totals.append(t)
-        stage_sum = [a + b for a, b in zip(stage_sum, stages)]
+        totals.append(timed_step())
+    for _ in range(args.steps):
+        stage_sum = [a + b for a, b in zip(stage_sum, staged_step())]
     barrier(world)
     clk = clocks.stop()
     dsa.dsa_device_status(stream)
