@@ -136,6 +136,26 @@ DSA_API dsa_status_t dsa_topk_from_scores(const float *scores, int32_t T, int64_
                                   const int32_t *pos, int32_t topk, int32_t *sel_idx, int64_t sel_ld,
                                   dsa_stream_t stream, void *workspace, size_t workspace_bytes);
 
+/* Stage 2 without any allocation: the same computation and arguments as
+ * dsa_topk_from_scores, minus the workspace.  It is for callers that cannot
+ * allocate device memory when they run this step: code inside a CUDA graph
+ * capture or a real-time decode loop that forbids allocation after start-up,
+ * or a host whose device memory is entirely owned by another allocator.  The
+ * paper has no counterpart; this is an interface choice of this library.
+ * Its scratch is a static device array of about 4.3 MB inside libdsa.so; every
+ * GPU that loads the library holds it until the process exits.
+ *   - Limits: T <= 8 and L <= 65536 scores per query; larger L returns
+ *     DSA_ERR_INVALID_ARG (say "exceeds the no-allocation scratch limit").
+ *   - The first call on a device looks up the array's device address (with
+ *     that device current) and caches it; make that first call outside any
+ *     stream capture.
+ *   - Every call shares the one array and clears the parts that must start at
+ *     zero; calls whose work overlaps on the GPU (other streams, other host
+ *     threads) race on it and must be serialised by the caller. */
+DSA_API dsa_status_t dsa_topk_from_scores_noalloc(const float *scores, int32_t T, int64_t L, int64_t ld,
+                                                  const int32_t *pos, int32_t topk, int32_t *sel_idx,
+                                                  int64_t sel_ld, dsa_stream_t stream);
+
 /* Stage 3 alone: attention of q over the rows listed in sel_idx [T][topk]
  * (entries < 0 are skipped; an entry outside [0, pos[t]] is skipped and flags
  * DSA_ERR_DEVICE).  `sink` is NULL or a per-head logit [64] f32 (device) that

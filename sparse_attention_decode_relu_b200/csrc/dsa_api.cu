@@ -355,6 +355,57 @@ dsa_status_t check_decode_args(const dsa_tensor_t* q, const dsa_tensor_t* q_idx,
     return DSA_OK;
 }
 
+
+// ------------------------------------------------------------------ no-allocation top-k
+// Scratch for dsa_topk_from_scores_noalloc: a file-scope device array, so that
+// entry point never allocates.  Sized for T <= 8 queries and L <= 65536 scores
+// per query: the zeroed histogram/ticket block, the per-chunk counts and the
+// candidate regions of the top-k stage (about 4.3 MB per device, held until
+// the process exits).
+constexpr int64_t kNoAllocMaxL = 65536;
+constexpr size_t ru256(size_t x) { return (x + 255) / 256 * 256; }
+constexpr size_t kNoAllocHist = ru256(sizeof(uint32_t) * kMaxT * kHistBins + sizeof(uint32_t) * kMaxT);
+constexpr size_t kNoAllocCounts = ru256(sizeof(uint32_t) * kMaxT * kMaxChunks);
+constexpr size_t kNoAllocCand = ru256(sizeof(uint2) * kMaxT * static_cast<size_t>(kNoAllocMaxL));
+constexpr size_t kNoAllocBytes = kNoAllocHist + kNoAllocCounts + kNoAllocCand;
+
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocBytes];
+
+// The top-k stage's layout packed into the static scratch (no score or
+// attention regions).
+Layout topk_only_layout(int T, int64_t L)
+{
+    Layout l;
+    l.ld = round_up(L, 64);
+    l.hist = 0;
+    l.tickets = sizeof(uint32_t) * (size_t)T * kHistBins;
+    l.zero_bytes = ru256(l.tickets + sizeof(uint32_t) * kMaxT);
+    l.counts = l.zero_bytes;
+    l.cand = l.counts + ru256(sizeof(uint32_t) * (size_t)T * kMaxChunks);
+    l.total = l.cand + ru256(sizeof(uint2) * (size_t)T * l.ld);
+    return l;
+}
+
+// Device address of the scratch array on the current device.  The host-side
+// name g_noalloc_scratch is only a stand-in, so the address is looked up once
+// per device (with that device current) and cached.
+std::atomic<void*> g_noalloc_ptr[64];
+
+dsa_status_t noalloc_scratch(void** ptr)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= 64) return fail(DSA_ERR_UNSUPPORTED, "device ordinal %d", dev);
+    void* p = g_noalloc_ptr[dev].load();
+    if (!p) {
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(no-allocation scratch)");
+        g_noalloc_ptr[dev].store(p);
+    }
+    *ptr = p;
+    return DSA_OK;
+}
 }  // namespace
 }  // namespace dsa
 
@@ -450,6 +501,34 @@ dsa_status_t dsa_topk_from_scores(const float* scores, int32_t T, int64_t L, int
     DeviceInfo dev;
     if ((st = device_info(dev))) return st;
     return run_topk(scores, ld, T, pos, topk, sel_idx, sel_ld, workspace, l, dev, reinterpret_cast<cudaStream_t>(stream_));
+}
+
+dsa_status_t dsa_topk_from_scores_noalloc(const float* scores, int32_t T, int64_t L, int64_t ld,
+                                          const int32_t* pos, int32_t topk, int32_t* sel_idx, int64_t sel_ld,
+                                          dsa_stream_t stream_)
+{
+    t_last_error.clear();
+    dsa_status_t st = check_T(T);
+    if (st) return st;
+    if ((st = check_topk(topk))) return st;
+    if (L < 1) return fail(DSA_ERR_INVALID_ARG, "L = %lld", (long long)L);
+    if (L > kNoAllocMaxL)
+        return fail(DSA_ERR_INVALID_ARG, "L = %lld exceeds the no-allocation scratch limit of %lld scores per query",
+                    (long long)L, (long long)kNoAllocMaxL);
+    if (!scores || !aligned16(scores)) return fail(DSA_ERR_INVALID_ARG, "scores: null or not 16-byte aligned");
+    if (ld < L || ld % 4) return fail(DSA_ERR_INVALID_ARG, "scores: ld must be >= L and a multiple of 4");
+    if (!sel_idx || !aligned16(sel_idx) || sel_ld < topk)
+        return fail(DSA_ERR_INVALID_ARG, "sel_idx: null, unaligned, or sel_ld < topk");
+    if (!pos) return fail(DSA_ERR_INVALID_ARG, "pos: null");
+    for (int t = 0; t < T; ++t)
+        if (pos[t] < 0 || pos[t] >= L) return fail(DSA_ERR_INVALID_ARG, "pos[%d] = %d outside [0, L)", t, pos[t]);
+    const Layout l = topk_only_layout(T, L);
+    if (l.total > kNoAllocBytes) return fail(DSA_ERR_INVALID_ARG, "no-allocation scratch too small");
+    void* ws = nullptr;
+    if ((st = noalloc_scratch(&ws))) return st;
+    DeviceInfo dev;
+    if ((st = device_info(dev))) return st;
+    return run_topk(scores, ld, T, pos, topk, sel_idx, sel_ld, ws, l, dev, reinterpret_cast<cudaStream_t>(stream_));
 }
 
 dsa_status_t dsa_sparse_attn(const dsa_tensor_t* q, const dsa_tensor_t* kv_cache, const dsa_tensor_t* sel_idx,

@@ -63,6 +63,9 @@ def lib():
             L.dsa_topk_from_scores.restype = st
             L.dsa_topk_from_scores.argtypes = [P, ctypes.c_int32, ctypes.c_int64, ctypes.c_int64, P, ctypes.c_int32,
                                                P, ctypes.c_int64, P, P, ctypes.c_size_t]
+            L.dsa_topk_from_scores_noalloc.restype = st
+            L.dsa_topk_from_scores_noalloc.argtypes = [P, ctypes.c_int32, ctypes.c_int64, ctypes.c_int64, P,
+                                                       ctypes.c_int32, P, ctypes.c_int64, P]
             L.dsa_sparse_attn.restype = st
             L.dsa_sparse_attn.argtypes = [T, T, T, P, P, T, P, P, ctypes.c_size_t]
             L.dsa_device_status.restype = st
@@ -160,6 +163,18 @@ def dsa_topk_from_scores(scores, L, pos, topk, sel_idx, workspace, stream=None):
     _check(lib().dsa_topk_from_scores(scores.data_ptr(), scores.shape[0], int(L), scores.stride(0), _pos(pos),
                                       int(topk), sel_idx.data_ptr(), sel_idx.stride(0), _stream(stream),
                                       workspace.data_ptr(), workspace.numel() * workspace.element_size()))
+
+
+def dsa_topk_from_scores_noalloc(scores, L, pos, topk, sel_idx, stream=None):
+    """dsa_topk_from_scores with the library's static scratch instead of a
+    workspace (T <= 8, L <= 65536; concurrent calls on the GPU race)."""
+    if scores.dtype != torch.float32 or scores.dim() != 2 or scores.stride(1) != 1:
+        raise ValueError("scores must be float32 [T][ld] with unit inner stride")
+    if sel_idx.dtype != torch.int32 or sel_idx.stride(1) != 1:
+        raise ValueError("sel_idx must be int32 [T][>= topk] with unit inner stride")
+    _check(lib().dsa_topk_from_scores_noalloc(scores.data_ptr(), scores.shape[0], int(L), scores.stride(0),
+                                              _pos(pos), int(topk), sel_idx.data_ptr(), sel_idx.stride(0),
+                                              _stream(stream)))
 
 
 def dsa_sparse_attn(q, kv_cache, sel_idx, pos, out, workspace, stream=None, *, sink=None):
