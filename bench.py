@@ -263,14 +263,14 @@ def main():
             step()
             dsa.dsa_set_stage_events(None)
         stream.synchronize()
-        return [ev[i].elapsed_time(ev[i + 1]) for i in range(4)]
+        return [ev[i].elapsed_time(ev[i + 1]) for i in range(4)] + [ev[0].elapsed_time(ev[4])]
 
     for _ in range(args.warmup):
         timed_step()
         staged_step()
     barrier(world)
     clocks = Clocks(local)
-    totals, stage_sum = [], [0.0] * 4
+    totals, stage_sum = [], [0.0] * 5
     for _ in range(args.steps):
         totals.append(timed_step())
     for _ in range(args.steps):
@@ -279,7 +279,8 @@ def main():
     clk = clocks.stop()
     dsa.dsa_device_status(stream)
     ms = reduce_max(statistics.mean(totals), world)
-    stage_ms = [s / args.steps for s in stage_sum]
+    stage_ms = [s / args.steps for s in stage_sum[:4]]
+    eager_ms = stage_sum[4] / args.steps
 
     sel_np = sel.cpu().numpy()
     ab = algorithmic_bytes(w, sel_np)
@@ -321,7 +322,7 @@ def main():
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e_ms, 4)}
 
     # Roofline of the dominant kernel (largest share of the step).
-    names = ["indexer", "topk", "attention", "combine"]
+    names = ["indexer", "topk", "attention", "tail"]
     dom = int(np.argmax(stage_ms))
     peak, which = peaks()
     alg = {"indexer": ab["indexer"], "attention": ab["attention"]}
@@ -346,6 +347,7 @@ def main():
                    "gathered_kv_rows": ab["gathered_rows"]},
         "frac_of_peak_hbm": round(ab["step"] / (ms * 1e-3) / 1e9 / peak, 4),
         "stage_us": {n: round(s * 1e3, 2) for n, s in zip(names, stage_ms)},
+        "eager_us_per_step": round(eager_ms * 1e3, 2),
         "roofline": roof,
         "e2e": e2e,
         "gpu_launches": int(kernels_per_step * args.steps),

@@ -142,9 +142,9 @@ DSA_API dsa_status_t dsa_topk_from_scores(const float *scores, int32_t T, int64_
  * capture or a real-time decode loop that forbids allocation after start-up,
  * or a host whose device memory is entirely owned by another allocator.  The
  * paper has no counterpart; this is an interface choice of this library.
- * Its scratch is a static device array of about 4.3 MB inside libdsa.so; every
+ * Its scratch is a static device array of about 16.4 MB inside libdsa.so; every
  * GPU that loads the library holds it until the process exits.
- *   - Limits: T <= 8 and L <= 65536 scores per query; larger L returns
+ *   - Limits: T <= 8 and L <= 262144 scores per query; larger L returns
  *     DSA_ERR_INVALID_ARG (say "exceeds the no-allocation scratch limit").
  *   - The first call on a device looks up the array's device address (with
  *     that device current) and caches it; make that first call outside any
@@ -183,8 +183,8 @@ DSA_API uint64_t dsa_launch_count(void);
 /* Profiling hook for the calling host thread.  With n == 5, dsa_decode and
  * dsa_decode_ws record five cudaEvent_t on their stream: events[0] before the
  * first launch, events[1] after the indexer scan, events[2] after the top-k
- * selection, events[3] after the split attention kernel and events[4] after the
- * split combine.  n == 0 disables; any other n is ignored. */
+ * selection, events[3] after the attention and events[4] at the end of the
+ * call.  n == 0 disables; any other n is ignored. */
 DSA_API void dsa_set_stage_events(void *const *events, int32_t n);
 
 #ifdef __cplusplus

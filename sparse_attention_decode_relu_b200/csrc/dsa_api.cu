@@ -182,7 +182,7 @@ dsa_status_t check_sel(const dsa_tensor_t* sel, int T, int32_t topk)
 struct Layout {
     int64_t ld = 0;            // score / candidate row stride (elements)
     size_t hist = 0, tickets = 0, zero_bytes = 0;
-    size_t counts = 0, scores = 0, cand = 0, part_o = 0, part_ml = 0;
+    size_t counts = 0, scores = 0, cand = 0, mm = 0;
     size_t total = 0;
 };
 
@@ -200,10 +200,9 @@ Layout layout(int T, int64_t L)
     l.tickets = l.hist + sizeof(uint32_t) * (size_t)T * kHistBins;
     l.zero_bytes = off;
     l.counts = take(sizeof(uint32_t) * (size_t)T * kMaxChunks);
+    l.mm = take(sizeof(uint2) * (size_t)kMaxSlots * kMaxT);
     l.scores = take(sizeof(float) * (size_t)T * l.ld);
     l.cand = take(sizeof(uint2) * (size_t)T * l.ld);
-    l.part_o = take(sizeof(float) * (size_t)T * kMaxSplits * kH * kD);
-    l.part_ml = take(sizeof(float2) * (size_t)T * kMaxSplits * kH);
     l.total = off;
     return l;
 }
@@ -236,7 +235,8 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
 
 dsa_status_t run_indexer(const dsa_tensor_t* q_idx, const dsa_tensor_t* w_idx, const dsa_tensor_t* k,
                          const int32_t* pos, const Shape& sh, float* scores, int64_t ld, const DeviceInfo& dev,
-                         cudaStream_t stream)
+                         cudaStream_t stream, uint32_t* zero = nullptr, size_t zero_bytes = 0,
+                         uint32_t* mm = nullptr, int* mm_slots = nullptr)
 {
     auto enc = encode_fn();
     if (!enc) return fail(DSA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
@@ -250,6 +250,18 @@ dsa_status_t run_indexer(const dsa_tensor_t* q_idx, const dsa_tensor_t* w_idx, c
                      sh.fp8 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B,
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(DSA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+    CUtensorMap smap;
+    std::memset(&smap, 0, sizeof smap);
+    if (k->scale) {   // per-token scales, 128 per tile; reads past L are filled with zeros
+        const cuuint64_t sdims[1] = {static_cast<cuuint64_t>(sh.L)};
+        const cuuint64_t sstr[1] = {static_cast<cuuint64_t>(sh.L * 4)};
+        const cuuint32_t sbox[1] = {static_cast<cuuint32_t>(kKeyTile)};
+        const cuuint32_t sestr[1] = {1};
+        r = enc(&smap, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 1, const_cast<float*>(k->scale), sdims, sstr, sbox, sestr,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) return fail(DSA_ERR_CUDA, "cuTensorMapEncodeTiled (scale) failed (%d)", static_cast<int>(r));
+    }
     IndexerParams p{};
     p.q_idx = static_cast<const uint16_t*>(q_idx->data);
     p.w = static_cast<const float*>(w_idx->data);
@@ -263,19 +275,25 @@ dsa_status_t run_indexer(const dsa_tensor_t* q_idx, const dsa_tensor_t* w_idx, c
         n_max = pos[t] + 1 > n_max ? pos[t] + 1 : n_max;
     }
     p.n_max = n_max;
+    p.zero = zero;
+    p.zero_words = static_cast<int32_t>(zero_bytes / 4);
+    p.mm = mm;
     p.err = dev.err;
     const int ntiles = static_cast<int>((n_max + kKeyTile - 1) / kKeyTile);
     int grid = dev.sms * indexer_max_ctas_per_sm(sh.T, sh.fp8);
     if (grid > ntiles) grid = ntiles;
+    if (grid > kMaxSlots) grid = kMaxSlots;
     if (grid < 1) grid = 1;
-    cudaError_t e = launch_indexer(&map, p, sh.T, sh.fp8, grid, stream);
+    if (mm_slots) *mm_slots = grid;
+    cudaError_t e = launch_indexer(&map, &smap, p, sh.T, sh.fp8, grid, stream);
     if (e != cudaSuccess) return cuda_fail(e, "indexer launch");
     g_launches += 1;
     return DSA_OK;
 }
 
 dsa_status_t run_topk(const float* scores, int64_t ld, int T, const int32_t* pos, int32_t topk, int32_t* sel,
-                      int64_t sel_ld, void* ws, const Layout& l, const DeviceInfo& dev, cudaStream_t stream)
+                      int64_t sel_ld, void* ws, const Layout& l, const DeviceInfo& dev, cudaStream_t stream,
+                      bool zeroed = false, int mm_slots = 0)
 {
     TopkParams p{};
     p.scores = scores;
@@ -298,11 +316,26 @@ dsa_status_t run_topk(const float* scores, int64_t ld, int T, const int32_t* pos
     p.tickets = at<uint32_t>(ws, l.tickets);
     p.counts = at<uint32_t>(ws, l.counts);
     p.cand = at<uint2>(ws, l.cand);
+    p.mm = at<uint32_t>(ws, l.mm);
+    p.mm_slots = mm_slots;
     p.sel = sel;
     p.sel_ld = sel_ld;
     p.err = dev.err;
-    cudaError_t e = cudaMemsetAsync(ws, 0, l.zero_bytes, stream);
-    if (e != cudaSuccess) return cuda_fail(e, "workspace clear");
+    cudaError_t e;
+    if (n_max <= topk_cluster_capacity()) {   // one block cluster per query, keys in shared memory
+        if ((e = launch_topk_cluster(p, stream)) != cudaSuccess) return cuda_fail(e, "top-k launch");
+        g_launches += 1;
+        return DSA_OK;
+    }
+    if (!zeroed) {
+        e = cudaMemsetAsync(ws, 0, l.zero_bytes, stream);
+        if (e != cudaSuccess) return cuda_fail(e, "workspace clear");
+    }
+    if (mm_slots == 0) {   // no producer left key ranges: one pass to find them
+        p.mm_slots = p.nchunks;
+        if ((e = launch_topk_minmax(p, stream)) != cudaSuccess) return cuda_fail(e, "top-k range launch");
+        g_launches += 1;
+    }
     if ((e = launch_topk_hist(p, stream)) != cudaSuccess) return cuda_fail(e, "top-k histogram launch");
     if ((e = launch_topk_select(p, stream)) != cudaSuccess) return cuda_fail(e, "top-k select launch");
     g_launches += 2;
@@ -321,22 +354,17 @@ dsa_status_t run_attention(const dsa_tensor_t* q, const dsa_tensor_t* kv, const 
     p.sel_ld = sel_ld;
     p.L = static_cast<int32_t>(sh.L);
     p.rows = topk;
-    int64_t nsplit = (2 * dev.sms + sh.T - 1) / sh.T;
-    if (nsplit > kMaxSplits) nsplit = kMaxSplits;
-    int64_t rps = round_up((topk + nsplit - 1) / nsplit, 16);
+    const int C = attention_cluster_size(sh.T);
+    const int64_t rps = round_up((topk + C - 1) / C, 16);
     p.rows_per_split = static_cast<int32_t>(rps);
-    p.nsplit = static_cast<int32_t>((topk + rps - 1) / rps);
+    p.nsplit = C;
     for (int t = 0; t < sh.T; ++t) p.pos[t] = pos[t];
     p.sink = sink;
-    p.part_o = at<float>(ws, l.part_o);
-    p.part_ml = at<float2>(ws, l.part_ml);
     p.out = static_cast<uint16_t*>(out->data);
     p.err = dev.err;
     cudaError_t e = launch_attention(p, sh.T, stream);
     if (e != cudaSuccess) return cuda_fail(e, "attention launch");
-    stage_event(3, stream);
-    if ((e = launch_combine(p, sh.T, stream)) != cudaSuccess) return cuda_fail(e, "combine launch");
-    g_launches += 2;
+    g_launches += 1;
     return DSA_OK;
 }
 
@@ -358,16 +386,18 @@ dsa_status_t check_decode_args(const dsa_tensor_t* q, const dsa_tensor_t* q_idx,
 
 // ------------------------------------------------------------------ no-allocation top-k
 // Scratch for dsa_topk_from_scores_noalloc: a file-scope device array, so that
-// entry point never allocates.  Sized for T <= 8 queries and L <= 65536 scores
-// per query: the zeroed histogram/ticket block, the per-chunk counts and the
-// candidate regions of the top-k stage (about 4.3 MB per device, held until
-// the process exits).
-constexpr int64_t kNoAllocMaxL = 65536;
+// entry point never allocates.  Sized for T <= 8 queries and L <= 262144 scores
+// per query: the zeroed histogram/ticket block, the per-chunk counts, the
+// candidate regions and the per-block key ranges of the top-k stage (about
+// 16.4 MB per device, held until the process exits).  Queries short enough for
+// the cluster path use none of it.
+constexpr int64_t kNoAllocMaxL = 262144;
 constexpr size_t ru256(size_t x) { return (x + 255) / 256 * 256; }
 constexpr size_t kNoAllocHist = ru256(sizeof(uint32_t) * kMaxT * kHistBins + sizeof(uint32_t) * kMaxT);
 constexpr size_t kNoAllocCounts = ru256(sizeof(uint32_t) * kMaxT * kMaxChunks);
 constexpr size_t kNoAllocCand = ru256(sizeof(uint2) * kMaxT * static_cast<size_t>(kNoAllocMaxL));
-constexpr size_t kNoAllocBytes = kNoAllocHist + kNoAllocCounts + kNoAllocCand;
+constexpr size_t kNoAllocRanges = ru256(sizeof(uint2) * kMaxSlots * kMaxT);
+constexpr size_t kNoAllocBytes = kNoAllocHist + kNoAllocCounts + kNoAllocCand + kNoAllocRanges;
 
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocBytes];
 
@@ -382,7 +412,8 @@ Layout topk_only_layout(int T, int64_t L)
     l.zero_bytes = ru256(l.tickets + sizeof(uint32_t) * kMaxT);
     l.counts = l.zero_bytes;
     l.cand = l.counts + ru256(sizeof(uint32_t) * (size_t)T * kMaxChunks);
-    l.total = l.cand + ru256(sizeof(uint2) * (size_t)T * l.ld);
+    l.mm = l.cand + ru256(sizeof(uint2) * (size_t)T * l.ld);
+    l.total = l.mm + ru256(sizeof(uint2) * kMaxSlots * kMaxT);
     return l;
 }
 
@@ -435,14 +466,21 @@ dsa_status_t dsa_decode_ws(const dsa_tensor_t* q, const dsa_tensor_t* q_idx, con
     cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
     float* scores = at<float>(workspace, l.scores);
     stage_event(0, stream);
-    if ((st = run_indexer(q_idx, w_idx, k_idx_cache, pos, sh, scores, l.ld, dev, stream))) return st;
+    // The indexer clears the top-k counters the large-context path accumulates into.
+    int mm_slots = 0;
+    if ((st = run_indexer(q_idx, w_idx, k_idx_cache, pos, sh, scores, l.ld, dev, stream,
+                          at<uint32_t>(workspace, l.hist), l.zero_bytes, at<uint32_t>(workspace, l.mm), &mm_slots)))
+        return st;
     stage_event(1, stream);
     int32_t* sel = static_cast<int32_t*>(sel_idx->data);
-    if ((st = run_topk(scores, l.ld, sh.T, pos, topk, sel, sel_idx->stride[0], workspace, l, dev, stream))) return st;
+    if ((st = run_topk(scores, l.ld, sh.T, pos, topk, sel, sel_idx->stride[0], workspace, l, dev, stream, true,
+                       mm_slots)))
+        return st;
     stage_event(2, stream);
     if ((st = run_attention(q, kv_cache, sel, sel_idx->stride[0], topk, pos, nullptr, out, sh, workspace, l, dev,
                             stream)))
         return st;
+    stage_event(3, stream);
     stage_event(4, stream);
     return DSA_OK;
 }

@@ -12,11 +12,12 @@
 // keys arrive by TMA (cp.async.bulk.tensor) into a 4-stage shared-memory ring
 // completed on mbarriers; bf16 keys land 128B-swizzled so the warp MMA operand
 // loads are bank-conflict free, FP8-E4M3 keys are widened exactly to bf16 in
-// shared memory first.  Each warp owns 16 keys of a tile: keys are the M side of
-// m16n8k16 tensor-core products, the T x 16 indexer query heads are the N side
-// and stay in registers for the whole scan.  The epilogue applies ReLU and the
-// head weights, reduces the 16 heads in a fixed order (two quad shuffles), and
-// writes fp32 scores.  Positions beyond a query's pos[t] get -inf.
+// shared memory first.  The indexer queries and head weights arrive once by
+// bulk copy.  Each warp owns one query (or a share of one when T < 8) and keeps
+// its 16 heads x 64 dims in registers as the N side of m16n8k16 tensor-core
+// products whose M side is 16 keys at a time.  The epilogue applies ReLU and
+// the head weights, reduces the 16 heads in a fixed order (two quad shuffles),
+// and writes fp32 scores.  Positions beyond a query's pos[t] get -inf.
 #include "common.cuh"
 #include "dsa_internal.h"
 
@@ -24,69 +25,110 @@ namespace dsa {
 namespace {
 
 constexpr int kStages = 4;
-constexpr int kThreads = 256;   // 8 warps x 16 keys = one 128-key tile
+constexpr int kThreads = 256;   // 8 warps; a 128-key tile is 8 blocks of 16 keys
 
 template <bool FP8>
 struct IndexerSmem {
     static constexpr int raw_bytes = kKeyTile * kDI * (FP8 ? 1 : 2);
     static constexpr int cvt_bytes = FP8 ? kKeyTile * kDI * 2 : 0;
-    static constexpr int bytes = 1024 /*align slack*/ + kStages * raw_bytes + cvt_bytes + kStages * 8 + kMaxT * kHI * 4;
+    static constexpr int q_bytes = kMaxT * kHI * kDI * 2;
+    static constexpr int scale_bytes = kKeyTile * 4;
+    static constexpr int bytes = 1024 /*align slack*/ + kStages * raw_bytes + cvt_bytes + q_bytes + kMaxT * kHI * 4 +
+                                 kStages * scale_bytes + (kStages + 1) * 8;
+};
+
+// Warps per query: 8 / T rounded to a power of two, so every query gets the
+// same share of the tile.  A warp keeps its query's 16 x 64 indexer heads in
+// registers and walks its share of the tile's 16-key blocks.
+template <int T>
+struct WarpMap {
+    static constexpr int TP = T <= 1 ? 1 : T <= 2 ? 2 : T <= 4 ? 4 : 8;
+    static constexpr int kWpq = 8 / TP;        // warps per query
+    static constexpr int kBlocks = 8 / kWpq;   // 16-key blocks per warp per tile
 };
 
 template <int T, bool FP8>
-__global__ void __launch_bounds__(kThreads, 1)
-    indexer_kernel(const __grid_constant__ CUtensorMap kmap, const IndexerParams p)
+__global__ void __launch_bounds__(kThreads, 2)
+    indexer_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap smap,
+                   const IndexerParams p)
 {
     using S = IndexerSmem<FP8>;
+    using M = WarpMap<T>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* ring = smem;                                            // kStages x raw tile
-    uint8_t* cvt = smem + kStages * S::raw_bytes;                    // FP8: widened bf16 tile (swizzled)
-    uint64_t* full = reinterpret_cast<uint64_t*>(cvt + S::cvt_bytes);
-    float* w_s = reinterpret_cast<float*>(full + kStages);
+    uint8_t* cvt = ring + kStages * S::raw_bytes;                    // FP8: widened bf16 tile (swizzled)
+    uint16_t* q_s = reinterpret_cast<uint16_t*>(cvt + S::cvt_bytes); // [T][16][64] bf16
+    float* w_s = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(q_s) + S::q_bytes);
+    float* sc_s = w_s + kMaxT * kHI;                                 // kStages x 128 per-token scales
+    uint64_t* full = reinterpret_cast<uint64_t*>(sc_s + kStages * kKeyTile);
+    uint64_t* setup = full + kStages;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int g = lane >> 2, c = lane & 3;
     const int ntiles = (p.n_max + kKeyTile - 1) / kKeyTile;
-
-    if (tid == 0) {
-        prefetch_tmap(&kmap);
-        for (int s = 0; s < kStages; ++s) mbar_init(&full[s], 1);
-        fence_mbar_init();
-    }
-    if (tid < T * kHI) w_s[tid] = p.w[tid];
-    __syncthreads();
-
-    // Indexer queries as B fragments: B[k = dim][n = head], n-tile nt covers heads 8nt..8nt+7.
-    uint32_t qb[T][2][4][2];
-#pragma unroll
-    for (int t = 0; t < T; ++t)
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-                const uint16_t* src = p.q_idx + (size_t)(t * kHI + nt * 8 + g) * kDI + kk * 16 + 2 * c;
-                qb[t][nt][kk][0] = *reinterpret_cast<const uint32_t*>(src);
-                qb[t][nt][kk][1] = *reinterpret_cast<const uint32_t*>(src + 8);
-            }
+    const bool scaled = p.scale != nullptr;
+    const uint32_t tile_tx = S::raw_bytes + (scaled ? S::scale_bytes : 0);
+    // One tile: 128 key rows, plus their per-token scales when there are any.
+    auto load_tile = [&](int stage, int tile) {
+        mbar_arrive_expect_tx(&full[stage], tile_tx);
+        tma_load_2d(ring + stage * S::raw_bytes, &kmap, 0, tile * kKeyTile, &full[stage]);
+        if (scaled) tma_load_1d(sc_s + stage * kKeyTile, &smap, tile * kKeyTile, &full[stage]);
+    };
 
     int issued = 0;   // tiles issued by thread 0
     if (tid == 0) {
+        prefetch_tmap(&kmap);
+        if (scaled) prefetch_tmap(&smap);
+        for (int s = 0; s < kStages + 1; ++s) mbar_init(&full[s], 1);
+        fence_mbar_init();
+        mbar_arrive_expect_tx(setup, T * kHI * kDI * 2 + T * kHI * 4);
+        bulk_g2s(q_s, p.q_idx, T * kHI * kDI * 2, setup);
+        bulk_g2s(w_s, p.w, T * kHI * 4, setup);
         for (int s = 0; s < kStages; ++s) {
             const int tile = blockIdx.x + s * gridDim.x;
             if (tile >= ntiles) break;
-            mbar_arrive_expect_tx(&full[s], S::raw_bytes);
-            tma_load_2d(ring + s * S::raw_bytes, &kmap, 0, tile * kKeyTile, &full[s]);
+            load_tile(s, tile);
             ++issued;
         }
     }
+    if (p.zero != nullptr)   // clear the next stage's counters (nothing reads them before this grid ends)
+        for (int i = blockIdx.x * kThreads + tid; i < p.zero_words; i += gridDim.x * kThreads) p.zero[i] = 0u;
+    __syncthreads();
+    bool ok = mbar_wait(setup, 0, p.err);
+
+    const int t = warp / M::kWpq;           // this warp's query
+    const bool active = t < T;
+    const int kb0 = warp % M::kWpq;
+    int pos_t = -1;
+#pragma unroll
+    for (int i = 0; i < T; ++i)
+        if (i == t) pos_t = p.pos[i];
+    // B fragments: B[k = dim][n = head]; n-tile nt = heads 8nt..8nt+7.  ldmatrix
+    // rows are heads (128 B apart), matrices are consecutive 8-dim slices.
+    uint32_t qb[2][4][2];
+    float w0 = 0.f, w1 = 0.f, w8 = 0.f, w9 = 0.f;
+    uint32_t klo = 0xFFFFFFFFu, khi = 0u;   // key range of the visible scores this lane wrote
+    if (active && ok) {
+        const uint32_t qbase = smem_u32(q_s + t * kHI * kDI);
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int kp = 0; kp < 2; ++kp) {
+                const uint32_t a = qbase + (nt * 8 + (lane & 7)) * (kDI * 2) + (kp * 32 + (lane >> 3) * 8) * 2;
+                ldsm_x4(a, qb[nt][2 * kp][0], qb[nt][2 * kp][1], qb[nt][2 * kp + 1][0], qb[nt][2 * kp + 1][1]);
+            }
+        w0 = w_s[t * kHI + 2 * c];
+        w1 = w_s[t * kHI + 2 * c + 1];
+        w8 = w_s[t * kHI + 8 + 2 * c];
+        w9 = w_s[t * kHI + 9 + 2 * c];
+    }
 
     int it = 0;
-    bool aborted = false;
-    for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
+    bool aborted = __syncthreads_or(!ok);
+    for (int tile = blockIdx.x; !aborted && tile < ntiles; tile += gridDim.x, ++it) {
         const int stage = it % kStages;
-        const uint32_t parity = (it / kStages) & 1;
-        const bool ok = mbar_wait(&full[stage], parity, p.err);
+        ok = mbar_wait(&full[stage], (it / kStages) & 1, p.err);
         if (__syncthreads_or(!ok)) {
             aborted = true;
             break;
@@ -114,47 +156,51 @@ __global__ void __launch_bounds__(kThreads, 1)
             ktile = cvt;
         }
 
-        // Keys of this warp as A fragments (16 keys x 64 dims), 128B-swizzled rows.
-        uint32_t a[4][4];
-        {
-            const int row = warp * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
-            const uint32_t base = smem_u32(ktile) + row * 128;
+        if (active) {
+#pragma unroll 2
+            for (int j = 0; j < M::kBlocks; ++j) {
+                const int kb = kb0 + M::kWpq * j;
+                // Keys kb*16 .. kb*16+15 as A fragments (16 keys x 64 dims), 128B-swizzled rows.
+                uint32_t a[4][4];
+                const int row = kb * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+                const uint32_t base = smem_u32(ktile) + row * 128;
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-                const int chunk = 2 * kk + (lane >> 4);
-                ldsm_x4(base + ((chunk ^ (row & 7)) << 4), a[kk][0], a[kk][1], a[kk][2], a[kk][3]);
-            }
-        }
-        const int s_base = tile * kKeyTile + warp * 16;
-        const int s_mine = s_base + g + 8 * (c & 1);   // the key this lane writes (lanes c = 0, 1)
-        float scale = 1.0f;
-        if (p.scale != nullptr && c < 2 && s_mine < p.L) scale = p.scale[s_mine];
-
+                for (int kk = 0; kk < 4; ++kk) {
+                    const int chunk = 2 * kk + (lane >> 4);
+                    ldsm_x4(base + ((chunk ^ (row & 7)) << 4), a[kk][0], a[kk][1], a[kk][2], a[kk][3]);
+                }
+                float acc0[4] = {0.f, 0.f, 0.f, 0.f}, acc1[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int t = 0; t < T; ++t) {
-            float acc0[4] = {0.f, 0.f, 0.f, 0.f}, acc1[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-                mma_bf16_16816(acc0, a[kk], qb[t][0][kk][0], qb[t][0][kk][1]);
-                mma_bf16_16816(acc1, a[kk], qb[t][1][kk][0], qb[t][1][kk][1]);
-            }
-            const float w0 = w_s[t * kHI + 2 * c], w1 = w_s[t * kHI + 2 * c + 1];
-            const float w8 = w_s[t * kHI + 8 + 2 * c], w9 = w_s[t * kHI + 9 + 2 * c];
-            float pa = fmaxf(acc0[0], 0.f) * w0;
-            pa = fmaf(fmaxf(acc0[1], 0.f), w1, pa);
-            pa = fmaf(fmaxf(acc1[0], 0.f), w8, pa);
-            pa = fmaf(fmaxf(acc1[1], 0.f), w9, pa);
-            float pb = fmaxf(acc0[2], 0.f) * w0;
-            pb = fmaf(fmaxf(acc0[3], 0.f), w1, pb);
-            pb = fmaf(fmaxf(acc1[2], 0.f), w8, pb);
-            pb = fmaf(fmaxf(acc1[3], 0.f), w9, pb);
-            pa += __shfl_xor_sync(0xffffffffu, pa, 1);
-            pb += __shfl_xor_sync(0xffffffffu, pb, 1);
-            pa += __shfl_xor_sync(0xffffffffu, pa, 2);
-            pb += __shfl_xor_sync(0xffffffffu, pb, 2);
-            if (c < 2 && s_mine < p.L) {
-                const float v = (c == 0 ? pa : pb) * scale;
-                p.scores[(int64_t)t * p.ld + s_mine] = (s_mine <= p.pos[t]) ? v : -INFINITY;
+                for (int kk = 0; kk < 4; ++kk) {
+                    mma_bf16_16816(acc0, a[kk], qb[0][kk][0], qb[0][kk][1]);
+                    mma_bf16_16816(acc1, a[kk], qb[1][kk][0], qb[1][kk][1]);
+                }
+                // ReLU, head weights, then the 16 heads summed in a fixed order.
+                float pa = fmaxf(acc0[0], 0.f) * w0;
+                pa = fmaf(fmaxf(acc0[1], 0.f), w1, pa);
+                pa = fmaf(fmaxf(acc1[0], 0.f), w8, pa);
+                pa = fmaf(fmaxf(acc1[1], 0.f), w9, pa);
+                float pb = fmaxf(acc0[2], 0.f) * w0;
+                pb = fmaf(fmaxf(acc0[3], 0.f), w1, pb);
+                pb = fmaf(fmaxf(acc1[2], 0.f), w8, pb);
+                pb = fmaf(fmaxf(acc1[3], 0.f), w9, pb);
+                pa += __shfl_xor_sync(0xffffffffu, pa, 1);
+                pb += __shfl_xor_sync(0xffffffffu, pb, 1);
+                pa += __shfl_xor_sync(0xffffffffu, pa, 2);
+                pb += __shfl_xor_sync(0xffffffffu, pb, 2);
+                const int s = tile * kKeyTile + kb * 16 + g + 8 * (c & 1);   // lanes c = 0, 1 write
+                if (c < 2 && s < p.L) {
+                    const float scale = scaled ? sc_s[stage * kKeyTile + kb * 16 + g + 8 * (c & 1)] : 1.0f;
+                    const float v = (c == 0 ? pa : pb) * scale;
+                    if (s <= pos_t) {
+                        p.scores[(int64_t)t * p.ld + s] = v;
+                        const uint32_t k = score_key(v);
+                        klo = min(klo, k);
+                        khi = max(khi, k);
+                    } else {
+                        p.scores[(int64_t)t * p.ld + s] = -INFINITY;
+                    }
+                }
             }
         }
 
@@ -162,31 +208,56 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (tid == 0) {
             const int next = tile + kStages * gridDim.x;
             if (next < ntiles) {
-                mbar_arrive_expect_tx(&full[stage], S::raw_bytes);
-                tma_load_2d(ring + stage * S::raw_bytes, &kmap, 0, next * kKeyTile, &full[stage]);
+                load_tile(stage, next);
                 ++issued;
             }
         }
     }
 
+    griddep_launch_dependents();
     if (aborted) {
         // Let copies still in flight land before the block's shared memory goes away.
         if (tid == 0) {
+            mbar_wait(setup, 0, p.err);
             for (int k = it; k < issued; ++k) mbar_wait(&full[k % kStages], (k / kStages) & 1, p.err);
         }
         __syncthreads();
         return;
     }
 
+    // Per-block key range of each query's visible scores, for the top-k stage.
+    if (p.mm != nullptr) {
+        __shared__ uint32_t wr[2][8];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            klo = min(klo, __shfl_xor_sync(0xffffffffu, klo, o));
+            khi = max(khi, __shfl_xor_sync(0xffffffffu, khi, o));
+        }
+        if (lane == 0) {
+            wr[0][warp] = klo;
+            wr[1][warp] = khi;
+        }
+        __syncthreads();
+        if (tid < T) {
+            uint32_t lo = 0xFFFFFFFFu, hi = 0u;
+            for (int w = tid * M::kWpq; w < (tid + 1) * M::kWpq; ++w) {
+                lo = min(lo, wr[0][w]);
+                hi = max(hi, wr[1][w]);
+            }
+            reinterpret_cast<uint2*>(p.mm)[(int64_t)blockIdx.x * kMaxT + tid] = make_uint2(lo, hi);
+        }
+    }
+
     // Positions no query can see (s >= n_max): -inf, as the stage's contract states.
     const int64_t tail0 = (int64_t)ntiles * kKeyTile;
     for (int64_t s = tail0 + (int64_t)blockIdx.x * kThreads + tid; s < p.L; s += (int64_t)gridDim.x * kThreads)
 #pragma unroll
-        for (int t = 0; t < T; ++t) p.scores[(int64_t)t * p.ld + s] = -INFINITY;
+        for (int tt = 0; tt < T; ++tt) p.scores[(int64_t)tt * p.ld + s] = -INFINITY;
 }
 
 template <int T, bool FP8>
-cudaError_t launch_t(const CUtensorMap* kmap, const IndexerParams& p, int grid, cudaStream_t s)
+cudaError_t launch_t(const CUtensorMap* kmap, const CUtensorMap* smap, const IndexerParams& p, int grid,
+                     cudaStream_t s)
 {
     constexpr int smem = IndexerSmem<FP8>::bytes;
     static bool configured[64] = {};
@@ -197,7 +268,7 @@ cudaError_t launch_t(const CUtensorMap* kmap, const IndexerParams& p, int grid, 
         if (e != cudaSuccess) return e;
         configured[dev] = true;
     }
-    indexer_kernel<T, FP8><<<grid, kThreads, smem, s>>>(*kmap, p);
+    indexer_kernel<T, FP8><<<grid, kThreads, smem, s>>>(*kmap, *smap, p);
     return cudaGetLastError();
 }
 
@@ -231,10 +302,10 @@ int occupancy_t()
     default: return fp8 ? FN<8, true>(__VA_ARGS__) : FN<8, false>(__VA_ARGS__);    \
     }
 
-cudaError_t launch_indexer(const CUtensorMap* kmap, const IndexerParams& p, int T, bool fp8, int grid,
-                           cudaStream_t s)
+cudaError_t launch_indexer(const CUtensorMap* kmap, const CUtensorMap* smap, const IndexerParams& p, int T, bool fp8,
+                           int grid, cudaStream_t s)
 {
-    DSA_INDEXER_DISPATCH(launch_t, kmap, p, grid, s)
+    DSA_INDEXER_DISPATCH(launch_t, kmap, smap, p, grid, s)
 }
 
 int indexer_max_ctas_per_sm(int T, bool fp8)

@@ -31,7 +31,11 @@ def _scores(rng, T, L, kind):
 @pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")
 def test_noalloc_topk_matches_workspace_entry_two_calls_in_a_row():
     rng = np.random.default_rng(2024)
-    cases = [(8, 65536, 2048, "ties", [65535 - i for i in range(8)]),
+    # The first two calls take the multi-block path that works in the scratch array
+    # (the second finds the first one's leftovers there); 40000 scores per query
+    # take the cluster path that needs none.
+    cases = [(8, 262144, 2048, "ties", [262143 - i for i in range(8)]),
+             (3, 200000, 777, "normal", [199999, 1000, 150000]),
              (3, 40000, 777, "normal", [39999, 1000, 20000])]
     for T, L, k, kind, pos in cases:
         scores = _scores(rng, T, L, kind)
@@ -46,9 +50,9 @@ def test_noalloc_topk_matches_workspace_entry_two_calls_in_a_row():
 
 @pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")
 def test_noalloc_rejects_sizes_beyond_its_scratch():
-    scores = torch.zeros((1, 65540), dtype=torch.float32, device="cuda")
+    scores = torch.zeros((1, 262148), dtype=torch.float32, device="cuda")
     sel = torch.empty((1, 16), dtype=torch.int32, device="cuda")
     with pytest.raises(dsa.DsaError) as e:
-        dsa.dsa_topk_from_scores_noalloc(scores, 65537, [10], 16, sel)
+        dsa.dsa_topk_from_scores_noalloc(scores, 262145, [10], 16, sel)
     assert e.value.status == dsa.ERR_INVALID_ARG
     assert "no-allocation scratch limit" in str(e.value)
