@@ -5,8 +5,9 @@ sparse GQA attention) on B200.
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl ours|reference]
 
 A step is one full pass of the path over one batch of synthetic inputs that are
-resident in HBM.  Each timed step starts with a cold L2 (a write of twice the L2
-size runs before it, outside the timed region) and is replayed from a CUDA graph
+resident in HBM.  Each timed step starts with a cold L2 (outside the timed
+region a buffer of twice the L2 size is written, then another one is read, so no
+dirty lines of the flush are left to write back) and is replayed from a CUDA graph
 of dsa_decode_ws; its time is taken with CUDA events on the launching stream.
 `value` is algorithmic HBM bytes per step (indexer keys, unique selected K/V
 rows, queries, outputs, indices) over the step time, summed over ranks.  With
@@ -64,42 +65,50 @@ def algorithmic_bytes(w, sel):
 
 
 class Clocks:
-    """nvidia-smi sampler running during the timed region."""
+    """NVML sampler (a background thread, ~1 ms period) running during the timed
+    region: SM clock and the clock-event (throttle) reasons."""
 
-    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
-              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
-              "clocks_event_reasons.sw_power_cap")
+    REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+               "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80}
 
     def __init__(self, index):
-        self.p = None
+        import threading
+
+        self.samples, self.reasons, self.max_mhz, self.err = [], set(), None, None
+        self.stop_flag = False
         try:
-            self.p = subprocess.Popen(["nvidia-smi", "-i", str(index), "--query-gpu=" + self.FIELDS,
-                                       "--format=csv,noheader,nounits", "-lms", "100"],
-                                      stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-        except Exception:
-            self.p = None
+            import pynvml
+
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # no NVML: report it
+            self.nv, self.err = None, str(e)
+        self.thread = threading.Thread(target=self._run, daemon=True)
+        self.thread.start()
+
+    def _run(self):
+        if self.nv is None:
+            return
+        while not self.stop_flag:
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for n, bit in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(n)
+            except Exception as e:
+                self.err = str(e)
+                return
+            time.sleep(0.001)
 
     def stop(self):
-        if self.p is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.p.terminate()
-        out, _ = self.p.communicate(timeout=10)
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in out.strip().splitlines():
-            f = [x.strip() for x in line.split(",")]
-            if len(f) < 7:
-                continue
-            try:
-                sm.append(float(f[0]))
-                mx = float(f[1])
-            except ValueError:
-                continue
-            for n, v in zip(names, f[3:7]):
-                if v.lower().startswith("active"):
-                    reasons.add(n)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        self.stop_flag = True
+        self.thread.join(timeout=5)
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None, "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples), "source": "nvml",
+                **({"error": self.err} if self.err else {})}
 
 
 def dist_setup(n):
@@ -215,32 +224,39 @@ def main():
     sel = torch.empty((T, topk), dtype=torch.int32, device=dev)
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     flush = torch.empty(2 * l2, dtype=torch.uint8, device=dev)
+    sweep = torch.ones(2 * l2 // 4, dtype=torch.float32, device=dev)
+
+    def flush_l2():
+        # Write a buffer twice the L2 size (evicts everything, writing back our
+        # outputs), then read another one (the L2 ends up full of clean lines, so
+        # the timed step does not pay for write-backs of the flush itself).
+        flush.zero_()
+        sweep.amax()
     stream = torch.cuda.Stream(device=dev)
-    ev = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+    grid = dsa.dsa_step_grid(w.key_dtype == "fp8")
+    trace = torch.zeros(grid * 32, dtype=torch.int64, device=dev)
 
     def step():
         dsa.dsa_decode_ws(d["q"], d["q_idx"], d["w_idx"], d["k_idx"], d["kv"], d["pos"], topk, out, sel, ws,
                           k_scale=d["k_scale"])
 
-    # One eager call counts the kernels of a step; then capture the step (with its
-    # stage events) into a graph.
+    # One eager call counts the kernels of a step; then capture the step in a graph.
     with torch.cuda.stream(stream):
         n0 = dsa.dsa_launch_count()
         step()
         kernels_per_step = dsa.dsa_launch_count() - n0
     stream.synchronize()
     dsa.dsa_device_status(stream)
-    # torch only reports elapsed time for events it has recorded itself once.
-    for e in ev:
-        e.record(stream)
-    stream.synchronize()
+    # The graph carries the in-kernel phase stamps (a few stores per block).
     graph = torch.cuda.CUDAGraph()
+    dsa.dsa_set_step_trace(trace)
     with torch.cuda.graph(graph, stream=stream):
         step()
+    dsa.dsa_set_step_trace(None)
 
     def timed_step():
         """Cold L2, then one graph replay of the whole step, timed by events."""
-        flush.zero_()
+        flush_l2()
         s0 = torch.cuda.Event(enable_timing=True)
         s1 = torch.cuda.Event(enable_timing=True)
         with torch.cuda.stream(stream):
@@ -251,36 +267,40 @@ def main():
         stream.synchronize()
         return s0.elapsed_time(s1)
 
-    def staged_step():
-        """Cold L2, then the step launched eagerly with an event after every kernel.
-        A spin on the stream first lets the host enqueue all launches, so the
-        gaps between events are device time only."""
-        flush.zero_()
-        with torch.cuda.stream(stream):
-            stream.wait_stream(torch.cuda.current_stream())
-            torch.cuda._sleep(200000)
-            dsa.dsa_set_stage_events(ev)
-            step()
-            dsa.dsa_set_stage_events(None)
-        stream.synchronize()
-        return [ev[i].elapsed_time(ev[i + 1]) for i in range(4)] + [ev[0].elapsed_time(ev[4])]
+    def phases():
+        """Phase spans of the last replay, from the in-kernel stamps."""
+        t = trace.view(grid, 32).cpu().numpy().astype(np.int64)
+        # phase k runs from its start stamp (earliest block) to its end stamp (latest block)
+        spans = {}
+        for name, a, b in (("indexer", 0, 1), ("topk_hist", 2, 3), ("topk_extract", 4, 5), ("topk_emit", 6, 7),
+                           ("attention", 8, 9), ("merge", 10, 11)):
+            spans[name] = (t[:, b].max() - t[:, a].min()) / 1e3
+        spans["kernel"] = (t[:, 30].max() - t[:, 0].min()) / 1e3
+        spans["sm_mhz_in_kernel"] = float((t[0, 29] - t[0, 28]) / max(1, t[0, 30] - t[0, 0]) * 1e3)
+        spans["start_skew"] = (t[:, 0].max() - t[:, 0].min()) / 1e3
+        fast = t[:, 12] > 0   # blocks that ran the top-k emission's single-block path
+        if fast.any():
+            for name, a, b in (("emit_cut", 6, 12), ("emit_list", 12, 13), ("emit_tau", 13, 14),
+                               ("emit_ties", 14, 15), ("emit_out", 15, 7)):
+                spans[name] = (t[fast, b] - t[fast, a]).max() / 1e3
+        return spans
 
     for _ in range(args.warmup):
         timed_step()
-        staged_step()
     barrier(world)
     clocks = Clocks(local)
-    totals, stage_sum = [], [0.0] * 5
+    totals = []
+    phase_sum = {}
     for _ in range(args.steps):
+        trace.zero_()
         totals.append(timed_step())
-    for _ in range(args.steps):
-        stage_sum = [a + b for a, b in zip(stage_sum, staged_step())]
+        for k, v in phases().items():
+            phase_sum[k] = phase_sum.get(k, 0.0) + v
     barrier(world)
     clk = clocks.stop()
     dsa.dsa_device_status(stream)
     ms = reduce_max(statistics.mean(totals), world)
-    stage_ms = [s / args.steps for s in stage_sum[:4]]
-    eager_ms = stage_sum[4] / args.steps
+    phase_us = {k: round(v / args.steps, 2) for k, v in phase_sum.items()}
 
     sel_np = sel.cpu().numpy()
     ab = algorithmic_bytes(w, sel_np)
@@ -309,7 +329,7 @@ def main():
     stream.synchronize()
     e_times = []
     for _ in range(args.steps):
-        flush.zero_()
+        flush_l2()
         torch.cuda.current_stream().synchronize()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
@@ -321,33 +341,25 @@ def main():
     e2e = {"value": round(world * ab["step"] / (e_ms * 1e-3) / 1e9, 3), "unit": "GB/s",
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e_ms, 4)}
 
-    # Roofline of the dominant kernel (largest share of the step).
-    names = ["indexer", "topk", "attention", "tail"]
-    dom = int(np.argmax(stage_ms))
+    # Roofline of the step kernel (the only kernel: every phase of the step runs in
+    # one cooperative launch), timed by the events around each graph replay.
     peak, which = peaks()
-    alg = {"indexer": ab["indexer"], "attention": ab["attention"]}
-    roof = None
-    if names[dom] in alg:
-        achieved = alg[names[dom]] / (stage_ms[dom] * 1e-3) / 1e9
-        roof = {"kernel": names[dom], "bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                "frac": round(achieved / peak, 4), "peak_source": which, "traffic": None,
-                "algorithmic_bytes": alg[names[dom]]}
-    else:
-        roof = {"kernel": names[dom], "bound": "hbm", "achieved": None, "peak": peak, "unit": "GB/s", "frac": None,
-                "peak_source": which, "traffic": None}
+    achieved = ab["step"] / (ms * 1e-3) / 1e9
+    roof = {"kernel": "step_kernel", "bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+            "frac": round(achieved / peak, 4), "peak_source": which, "traffic": None,
+            "algorithmic_bytes": ab["step"]}
 
     line = {
         "metric": METRIC, "value": round(value, 3), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms, 5), "us_per_step": round(ms * 1e3, 2),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": w.name, "L": L, "T": T, "topk": topk, "key_dtype": w.key_dtype, "recipe": w.recipe,
-                   "seed": w.seed, "parallelism": f"replicas{world}", "l2": "flushed before every step",
+                   "seed": w.seed, "parallelism": f"replicas{world}", "l2": "flushed before every step (write 2x L2, then read another 2x L2: cold and clean)",
                    "timing": "CUDA-graph replay of dsa_decode_ws, CUDA events per step",
                    "algorithmic_bytes_per_step": ab["step"], "unique_kv_rows": ab["unique_rows"],
                    "gathered_kv_rows": ab["gathered_rows"]},
         "frac_of_peak_hbm": round(ab["step"] / (ms * 1e-3) / 1e9 / peak, 4),
-        "stage_us": {n: round(s * 1e3, 2) for n, s in zip(names, stage_ms)},
-        "eager_us_per_step": round(eager_ms * 1e3, 2),
+        "phase_us": phase_us,
         "roofline": roof,
         "e2e": e2e,
         "gpu_launches": int(kernels_per_step * args.steps),

@@ -187,6 +187,19 @@ DSA_API uint64_t dsa_launch_count(void);
  * call.  n == 0 disables; any other n is ignored. */
 DSA_API void dsa_set_stage_events(void *const *events, int32_t n);
 
+/* Profiling hook for the calling host thread: when device_buffer is not NULL,
+ * every launch records, per block b and slot k < 32, the GPU global timer (ns)
+ * into ((uint64_t*)device_buffer)[b * 32 + k] at the phase boundaries of the
+ * step: 0 start, 1 indexer scan done, 2/3 histogram start/end, 4/5 candidate
+ * extraction, 6/7 ordered emission, 8/9 split attention, 10/11 merge, 12-15
+ * inside the emission, 30 end; slots 28/29 hold the SM clock counter at start
+ * and end.  The buffer must hold dsa_step_grid(...) * 32 entries.  NULL
+ * disables. */
+DSA_API void dsa_set_step_trace(void *device_buffer);
+
+/* Blocks of the step kernel on the current device (one per SM); 0 on error. */
+DSA_API int32_t dsa_step_grid(int32_t fp8_keys);
+
 #ifdef __cplusplus
 }
 #endif

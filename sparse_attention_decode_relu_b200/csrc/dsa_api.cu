@@ -23,6 +23,7 @@ namespace {
 thread_local std::string t_last_error;
 thread_local void* t_stage_events[5] = {nullptr, nullptr, nullptr, nullptr, nullptr};
 thread_local bool t_stage_events_on = false;
+thread_local unsigned long long* t_trace = nullptr;
 std::atomic<uint64_t> g_launches{0};
 
 dsa_status_t fail(dsa_status_t st, const char* fmt, ...)
@@ -179,30 +180,43 @@ dsa_status_t check_sel(const dsa_tensor_t* sel, int T, int32_t topk)
 }
 
 // ------------------------------------------------------------------ workspace
+// Device workspace of one step: barrier words, the top-k counters the indexer
+// clears, per-block key ranges, per-chunk counts, fp32 scores, candidate lists,
+// and the attention splits' partial states.
 struct Layout {
     int64_t ld = 0;            // score / candidate row stride (elements)
-    size_t hist = 0, tickets = 0, zero_bytes = 0;
-    size_t counts = 0, scores = 0, cand = 0, mm = 0;
+    size_t ctrl = 0, hist = 0, list_n = 0, zero_bytes = 0;
+    size_t mm = 0, above = 0, cuts = 0, scores = 0, list = 0, po = 0, pml = 0;
     size_t total = 0;
 };
 
-Layout layout(int T, int64_t L)
+constexpr size_t ru256(size_t x) { return (x + 255) / 256 * 256; }
+
+// with_scores / with_attn: whether the layout carries the score and the
+// attention regions (the allocation-free top-k needs neither).
+Layout layout(int T, int64_t L, bool with_scores = true, bool with_attn = true)
 {
     Layout l;
     l.ld = round_up(L, 64);
     size_t off = 0;
     auto take = [&](size_t bytes) {
         const size_t at = off;
-        off += static_cast<size_t>(round_up(static_cast<int64_t>(bytes), 256));
+        off += ru256(bytes);
         return at;
     };
+    l.ctrl = take(kBarCtrlBytes + 128);
     l.hist = take(sizeof(uint32_t) * (size_t)T * kHistBins + sizeof(uint32_t) * kMaxT);
-    l.tickets = l.hist + sizeof(uint32_t) * (size_t)T * kHistBins;
-    l.zero_bytes = off;
-    l.counts = take(sizeof(uint32_t) * (size_t)T * kMaxChunks);
-    l.mm = take(sizeof(uint2) * (size_t)kMaxSlots * kMaxT);
-    l.scores = take(sizeof(float) * (size_t)T * l.ld);
-    l.cand = take(sizeof(uint2) * (size_t)T * l.ld);
+    l.list_n = l.hist + sizeof(uint32_t) * (size_t)T * kHistBins;
+    l.zero_bytes = sizeof(uint32_t) * ((size_t)T * kHistBins + kMaxT);
+    l.mm = take(sizeof(uint2) * (size_t)kMaxGrid * kMaxT);
+    l.above = take(sizeof(uint32_t) * (size_t)kMaxT * kMaxChunksStep);
+    l.cuts = take(sizeof(uint32_t) * 4 * kMaxT);
+    l.list = take(sizeof(uint2) * (size_t)T * l.ld);
+    if (with_scores) l.scores = take(sizeof(float) * (size_t)T * l.ld);
+    if (with_attn) {
+        l.po = take(sizeof(float) * (size_t)kMaxAttnItems * kH * kD);
+        l.pml = take(sizeof(float2) * (size_t)kMaxAttnItems * kH);
+    }
     l.total = off;
     return l;
 }
@@ -219,7 +233,7 @@ dsa_status_t check_ws(void* ws, size_t bytes, const Layout& l)
 template <typename P>
 P* at(void* ws, size_t off) { return reinterpret_cast<P*>(static_cast<char*>(ws) + off); }
 
-// ------------------------------------------------------------------ stage launches
+// ------------------------------------------------------------------ the step kernel
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
 {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -233,14 +247,12 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
     return fn;
 }
 
-dsa_status_t run_indexer(const dsa_tensor_t* q_idx, const dsa_tensor_t* w_idx, const dsa_tensor_t* k,
-                         const int32_t* pos, const Shape& sh, float* scores, int64_t ld, const DeviceInfo& dev,
-                         cudaStream_t stream, uint32_t* zero = nullptr, size_t zero_bytes = 0,
-                         uint32_t* mm = nullptr, int* mm_slots = nullptr)
+// TMA descriptors of the indexer key cache (128-key tiles; bf16 rows land
+// 128B-swizzled) and of its per-token scales (128 per tile).
+dsa_status_t encode_key_maps(const dsa_tensor_t* k, const Shape& sh, CUtensorMap& map, CUtensorMap& smap)
 {
     auto enc = encode_fn();
     if (!enc) return fail(DSA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
-    CUtensorMap map;
     const cuuint64_t dims[2] = {static_cast<cuuint64_t>(kDI), static_cast<cuuint64_t>(sh.L)};
     const cuuint64_t strides[1] = {static_cast<cuuint64_t>(sh.k_ld * (sh.fp8 ? 1 : 2))};
     const cuuint32_t box[2] = {static_cast<cuuint32_t>(kDI), static_cast<cuuint32_t>(kKeyTile)};
@@ -250,9 +262,8 @@ dsa_status_t run_indexer(const dsa_tensor_t* q_idx, const dsa_tensor_t* w_idx, c
                      sh.fp8 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B,
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(DSA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
-    CUtensorMap smap;
     std::memset(&smap, 0, sizeof smap);
-    if (k->scale) {   // per-token scales, 128 per tile; reads past L are filled with zeros
+    if (k->scale) {
         const cuuint64_t sdims[1] = {static_cast<cuuint64_t>(sh.L)};
         const cuuint64_t sstr[1] = {static_cast<cuuint64_t>(sh.L * 4)};
         const cuuint32_t sbox[1] = {static_cast<cuuint32_t>(kKeyTile)};
@@ -262,110 +273,82 @@ dsa_status_t run_indexer(const dsa_tensor_t* q_idx, const dsa_tensor_t* w_idx, c
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
         if (r != CUDA_SUCCESS) return fail(DSA_ERR_CUDA, "cuTensorMapEncodeTiled (scale) failed (%d)", static_cast<int>(r));
     }
-    IndexerParams p{};
-    p.q_idx = static_cast<const uint16_t*>(q_idx->data);
-    p.w = static_cast<const float*>(w_idx->data);
-    p.scale = k->scale;
-    p.scores = scores;
-    p.ld = ld;
-    p.L = static_cast<int32_t>(sh.L);
+    return DSA_OK;
+}
+
+int grid_blocks(const DeviceInfo& dev, bool fp8)
+{
+    static int cache[64][2] = {};
+    int d = 0;
+    cudaGetDevice(&d);
+    if (d >= 0 && d < 64 && cache[d][fp8]) return cache[d][fp8];
+    int g = step_max_blocks(fp8);
+    if (g > kMaxGrid) g = kMaxGrid;
+    if (g < 1) g = dev.sms > 0 ? dev.sms : 1;
+    if (d >= 0 && d < 64) cache[d][fp8] = g;
+    return g;
+}
+
+// Fill the top-k part of the parameters (work split, workspace pointers).
+void topk_params(StepParams& p, void* ws, const Layout& l)
+{
+    p.hist = at<uint32_t>(ws, l.hist);
+    p.list_n = at<uint32_t>(ws, l.list_n);
+    p.list = at<uint2>(ws, l.list);
+    p.above = at<uint32_t>(ws, l.above);
+    p.cuts = at<uint32_t>(ws, l.cuts);
+    p.mm = at<uint2>(ws, l.mm);
+    p.mm_slots = p.grid;
+    p.zero = at<uint32_t>(ws, l.hist);
+    p.zero_words = static_cast<int32_t>(l.zero_bytes / 4);
+    int nchunk = p.grid / p.T;
+    if (nchunk < 1) nchunk = 1;
+    if (nchunk > kMaxChunksStep) nchunk = kMaxChunksStep;
+    int64_t chunk = round_up((p.n_max + nchunk - 1) / nchunk, 4);
+    if (chunk < 4) chunk = 4;
+    p.chunk = static_cast<int32_t>(chunk);
+    p.nchunk = static_cast<int32_t>((p.n_max + chunk - 1) / chunk);
+    if (p.nchunk < 1) p.nchunk = 1;
+}
+
+void attn_params(StepParams& p, void* ws, const Layout& l, int32_t topk)
+{
+    int64_t nsplit = p.grid / p.T;
+    if (nsplit * p.T > kMaxAttnItems) nsplit = kMaxAttnItems / p.T;
+    if (nsplit < 1) nsplit = 1;
+    int64_t rps = round_up((topk + nsplit - 1) / nsplit, 16);
+    if (rps > kMaxRowsPerSplit) rps = kMaxRowsPerSplit;
+    p.rows = topk;
+    p.rows_per_split = static_cast<int32_t>(rps);
+    p.nsplit = static_cast<int32_t>((topk + rps - 1) / rps);
+    p.po = at<float>(ws, l.po);
+    p.pml = at<float2>(ws, l.pml);
+}
+
+dsa_status_t launch(const CUtensorMap& map, const CUtensorMap& smap, StepParams& p, bool fp8, void* ws,
+                    const Layout& l, cudaStream_t stream)
+{
+    cudaError_t e;
+    if (p.phases & (kPhaseTopk | kPhaseAttend)) {   // grid barriers are used: start the counter at zero
+        p.bar_ctrl = at<uint32_t>(ws, l.ctrl);
+        if ((e = cudaMemsetAsync(p.bar_ctrl, 0, sizeof(uint32_t), stream)) != cudaSuccess)
+            return cuda_fail(e, "barrier reset");
+    }
+    p.trace = t_trace;
+    if ((e = launch_step(&map, &smap, p, fp8, stream)) != cudaSuccess) return cuda_fail(e, "step launch");
+    g_launches += 1;
+    return DSA_OK;
+}
+
+void set_pos(StepParams& p, const int32_t* pos, int T)
+{
+    p.T = T;
     int n_max = 0;
-    for (int t = 0; t < sh.T; ++t) {
-        p.pos[t] = pos[t];
-        n_max = pos[t] + 1 > n_max ? pos[t] + 1 : n_max;
+    for (int t = 0; t < kMaxT; ++t) {
+        p.pos[t] = t < T ? pos[t] : 0;
+        if (t < T && pos[t] + 1 > n_max) n_max = pos[t] + 1;
     }
     p.n_max = n_max;
-    p.zero = zero;
-    p.zero_words = static_cast<int32_t>(zero_bytes / 4);
-    p.mm = mm;
-    p.err = dev.err;
-    const int ntiles = static_cast<int>((n_max + kKeyTile - 1) / kKeyTile);
-    int grid = dev.sms * indexer_max_ctas_per_sm(sh.T, sh.fp8);
-    if (grid > ntiles) grid = ntiles;
-    if (grid > kMaxSlots) grid = kMaxSlots;
-    if (grid < 1) grid = 1;
-    if (mm_slots) *mm_slots = grid;
-    cudaError_t e = launch_indexer(&map, &smap, p, sh.T, sh.fp8, grid, stream);
-    if (e != cudaSuccess) return cuda_fail(e, "indexer launch");
-    g_launches += 1;
-    return DSA_OK;
-}
-
-dsa_status_t run_topk(const float* scores, int64_t ld, int T, const int32_t* pos, int32_t topk, int32_t* sel,
-                      int64_t sel_ld, void* ws, const Layout& l, const DeviceInfo& dev, cudaStream_t stream,
-                      bool zeroed = false, int mm_slots = 0)
-{
-    TopkParams p{};
-    p.scores = scores;
-    p.ld = ld;
-    p.T = T;
-    p.topk = topk;
-    int64_t n_max = 0;
-    for (int t = 0; t < T; ++t) {
-        p.pos[t] = pos[t];
-        n_max = pos[t] + 1 > n_max ? pos[t] + 1 : n_max;
-    }
-    // About two blocks per SM over all queries, chunks a multiple of 2048 scores.
-    const int64_t per_query = (2 * dev.sms + T - 1) / T;
-    int64_t chunk = round_up((n_max + per_query - 1) / per_query, 2048);
-    if (chunk < 4096) chunk = 4096;
-    while ((n_max + chunk - 1) / chunk > kMaxChunks) chunk += 2048;
-    p.chunk = static_cast<int32_t>(chunk);
-    p.nchunks = static_cast<int32_t>((n_max + chunk - 1) / chunk);
-    p.hist = at<uint32_t>(ws, l.hist);
-    p.tickets = at<uint32_t>(ws, l.tickets);
-    p.counts = at<uint32_t>(ws, l.counts);
-    p.cand = at<uint2>(ws, l.cand);
-    p.mm = at<uint32_t>(ws, l.mm);
-    p.mm_slots = mm_slots;
-    p.sel = sel;
-    p.sel_ld = sel_ld;
-    p.err = dev.err;
-    cudaError_t e;
-    if (n_max <= topk_cluster_capacity()) {   // one block cluster per query, keys in shared memory
-        if ((e = launch_topk_cluster(p, stream)) != cudaSuccess) return cuda_fail(e, "top-k launch");
-        g_launches += 1;
-        return DSA_OK;
-    }
-    if (!zeroed) {
-        e = cudaMemsetAsync(ws, 0, l.zero_bytes, stream);
-        if (e != cudaSuccess) return cuda_fail(e, "workspace clear");
-    }
-    if (mm_slots == 0) {   // no producer left key ranges: one pass to find them
-        p.mm_slots = p.nchunks;
-        if ((e = launch_topk_minmax(p, stream)) != cudaSuccess) return cuda_fail(e, "top-k range launch");
-        g_launches += 1;
-    }
-    if ((e = launch_topk_hist(p, stream)) != cudaSuccess) return cuda_fail(e, "top-k histogram launch");
-    if ((e = launch_topk_select(p, stream)) != cudaSuccess) return cuda_fail(e, "top-k select launch");
-    g_launches += 2;
-    return DSA_OK;
-}
-
-dsa_status_t run_attention(const dsa_tensor_t* q, const dsa_tensor_t* kv, const int32_t* sel, int64_t sel_ld,
-                           int32_t topk, const int32_t* pos, const float* sink, dsa_tensor_t* out, const Shape& sh,
-                           void* ws, const Layout& l, const DeviceInfo& dev, cudaStream_t stream)
-{
-    AttnParams p{};
-    p.q = static_cast<const uint16_t*>(q->data);
-    p.kv = static_cast<const uint16_t*>(kv->data);
-    p.kv_ld = sh.kv_ld;
-    p.sel = sel;
-    p.sel_ld = sel_ld;
-    p.L = static_cast<int32_t>(sh.L);
-    p.rows = topk;
-    const int C = attention_cluster_size(sh.T);
-    const int64_t rps = round_up((topk + C - 1) / C, 16);
-    p.rows_per_split = static_cast<int32_t>(rps);
-    p.nsplit = C;
-    for (int t = 0; t < sh.T; ++t) p.pos[t] = pos[t];
-    p.sink = sink;
-    p.out = static_cast<uint16_t*>(out->data);
-    p.err = dev.err;
-    cudaError_t e = launch_attention(p, sh.T, stream);
-    if (e != cudaSuccess) return cuda_fail(e, "attention launch");
-    g_launches += 1;
-    return DSA_OK;
 }
 
 dsa_status_t check_decode_args(const dsa_tensor_t* q, const dsa_tensor_t* q_idx, const dsa_tensor_t* w_idx,
@@ -383,39 +366,19 @@ dsa_status_t check_decode_args(const dsa_tensor_t* q, const dsa_tensor_t* q_idx,
     return DSA_OK;
 }
 
-
 // ------------------------------------------------------------------ no-allocation top-k
 // Scratch for dsa_topk_from_scores_noalloc: a file-scope device array, so that
 // entry point never allocates.  Sized for T <= 8 queries and L <= 262144 scores
-// per query: the zeroed histogram/ticket block, the per-chunk counts, the
-// candidate regions and the per-block key ranges of the top-k stage (about
-// 16.4 MB per device, held until the process exits).  Queries short enough for
-// the cluster path use none of it.
+// per query: barrier words, the top-k counters, per-block key ranges, per-chunk
+// counts and the candidate lists (about 16.4 MB per device, held until the
+// process exits).
 constexpr int64_t kNoAllocMaxL = 262144;
-constexpr size_t ru256(size_t x) { return (x + 255) / 256 * 256; }
-constexpr size_t kNoAllocHist = ru256(sizeof(uint32_t) * kMaxT * kHistBins + sizeof(uint32_t) * kMaxT);
-constexpr size_t kNoAllocCounts = ru256(sizeof(uint32_t) * kMaxT * kMaxChunks);
-constexpr size_t kNoAllocCand = ru256(sizeof(uint2) * kMaxT * static_cast<size_t>(kNoAllocMaxL));
-constexpr size_t kNoAllocRanges = ru256(sizeof(uint2) * kMaxSlots * kMaxT);
-constexpr size_t kNoAllocBytes = kNoAllocHist + kNoAllocCounts + kNoAllocCand + kNoAllocRanges;
+constexpr size_t kNoAllocBytes = ru256(kBarCtrlBytes + 128) + ru256(sizeof(uint32_t) * ((size_t)kMaxT * kHistBins + kMaxT)) +
+                                 ru256(sizeof(uint2) * (size_t)kMaxGrid * kMaxT) +
+                                 ru256(sizeof(uint32_t) * (size_t)kMaxT * kMaxChunksStep) + ru256(sizeof(uint32_t) * 4 * kMaxT) +
+                                 ru256(sizeof(uint2) * (size_t)kMaxT * ((kNoAllocMaxL + 63) / 64 * 64));
 
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocBytes];
-
-// The top-k stage's layout packed into the static scratch (no score or
-// attention regions).
-Layout topk_only_layout(int T, int64_t L)
-{
-    Layout l;
-    l.ld = round_up(L, 64);
-    l.hist = 0;
-    l.tickets = sizeof(uint32_t) * (size_t)T * kHistBins;
-    l.zero_bytes = ru256(l.tickets + sizeof(uint32_t) * kMaxT);
-    l.counts = l.zero_bytes;
-    l.cand = l.counts + ru256(sizeof(uint32_t) * (size_t)T * kMaxChunks);
-    l.mm = l.cand + ru256(sizeof(uint2) * (size_t)T * l.ld);
-    l.total = l.mm + ru256(sizeof(uint2) * kMaxSlots * kMaxT);
-    return l;
-}
 
 // Device address of the scratch array on the current device.  The host-side
 // name g_noalloc_scratch is only a stand-in, so the address is looked up once
@@ -437,6 +400,31 @@ dsa_status_t noalloc_scratch(void** ptr)
     *ptr = p;
     return DSA_OK;
 }
+
+dsa_status_t run_topk_stage(const float* scores, int32_t T, int64_t L, int64_t ld, const int32_t* pos, int32_t topk,
+                            int32_t* sel_idx, int64_t sel_ld, void* ws, const Layout& l, cudaStream_t stream)
+{
+    DeviceInfo dev;
+    dsa_status_t st = device_info(dev);
+    if (st) return st;
+    StepParams p{};
+    p.phases = kPhaseRanges | kPhaseTopk;
+    p.grid = grid_blocks(dev, false);
+    set_pos(p, pos, T);
+    p.L = static_cast<int32_t>(L);
+    p.topk = topk;
+    p.scores = const_cast<float*>(scores);
+    p.ld = ld;
+    p.sel = sel_idx;
+    p.sel_ld = sel_ld;
+    p.err = dev.err;
+    topk_params(p, ws, l);
+    p.list = at<uint2>(ws, l.list);
+    CUtensorMap none;
+    std::memset(&none, 0, sizeof none);
+    return launch(none, none, p, false, ws, l, stream);
+}
+
 }  // namespace
 }  // namespace dsa
 
@@ -464,25 +452,32 @@ dsa_status_t dsa_decode_ws(const dsa_tensor_t* q, const dsa_tensor_t* q_idx, con
     DeviceInfo dev;
     if ((st = device_info(dev))) return st;
     cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
-    float* scores = at<float>(workspace, l.scores);
+    CUtensorMap map, smap;
+    if ((st = encode_key_maps(k_idx_cache, sh, map, smap))) return st;
+    StepParams p{};
+    p.phases = kPhaseIndex | kPhaseTopk | kPhaseAttend;
+    p.grid = grid_blocks(dev, sh.fp8);
+    set_pos(p, pos, sh.T);
+    p.L = static_cast<int32_t>(sh.L);
+    p.topk = topk;
+    p.q_idx = static_cast<const uint16_t*>(q_idx->data);
+    p.w = static_cast<const float*>(w_idx->data);
+    p.scale = k_idx_cache->scale;
+    p.scores = at<float>(workspace, l.scores);
+    p.ld = l.ld;
+    p.sel = static_cast<int32_t*>(sel_idx->data);
+    p.sel_ld = sel_idx->stride[0];
+    p.q = static_cast<const uint16_t*>(q->data);
+    p.kv = static_cast<const uint16_t*>(kv_cache->data);
+    p.kv_ld = sh.kv_ld;
+    p.out = static_cast<uint16_t*>(out->data);
+    p.err = dev.err;
+    topk_params(p, workspace, l);
+    attn_params(p, workspace, l, topk);
     stage_event(0, stream);
-    // The indexer clears the top-k counters the large-context path accumulates into.
-    int mm_slots = 0;
-    if ((st = run_indexer(q_idx, w_idx, k_idx_cache, pos, sh, scores, l.ld, dev, stream,
-                          at<uint32_t>(workspace, l.hist), l.zero_bytes, at<uint32_t>(workspace, l.mm), &mm_slots)))
-        return st;
-    stage_event(1, stream);
-    int32_t* sel = static_cast<int32_t*>(sel_idx->data);
-    if ((st = run_topk(scores, l.ld, sh.T, pos, topk, sel, sel_idx->stride[0], workspace, l, dev, stream, true,
-                       mm_slots)))
-        return st;
-    stage_event(2, stream);
-    if ((st = run_attention(q, kv_cache, sel, sel_idx->stride[0], topk, pos, nullptr, out, sh, workspace, l, dev,
-                            stream)))
-        return st;
-    stage_event(3, stream);
-    stage_event(4, stream);
-    return DSA_OK;
+    st = launch(map, smap, p, sh.fp8, workspace, l, stream);
+    for (int i = 1; i < 5; ++i) stage_event(i, stream);
+    return st;
 }
 
 dsa_status_t dsa_decode(const dsa_tensor_t* q, const dsa_tensor_t* q_idx, const dsa_tensor_t* w_idx,
@@ -515,7 +510,21 @@ dsa_status_t dsa_index_scores(const dsa_tensor_t* q_idx, const dsa_tensor_t* w_i
     if (ld < sh.L || ld % 4) return fail(DSA_ERR_INVALID_ARG, "scores: ld = %lld must be >= L and a multiple of 4", (long long)ld);
     DeviceInfo dev;
     if ((st = device_info(dev))) return st;
-    return run_indexer(q_idx, w_idx, k_idx_cache, pos, sh, scores, ld, dev, reinterpret_cast<cudaStream_t>(stream_));
+    CUtensorMap map, smap;
+    if ((st = encode_key_maps(k_idx_cache, sh, map, smap))) return st;
+    StepParams p{};
+    p.phases = kPhaseIndex;
+    p.grid = grid_blocks(dev, sh.fp8);
+    set_pos(p, pos, sh.T);
+    p.L = static_cast<int32_t>(sh.L);
+    p.q_idx = static_cast<const uint16_t*>(q_idx->data);
+    p.w = static_cast<const float*>(w_idx->data);
+    p.scale = k_idx_cache->scale;
+    p.scores = scores;
+    p.ld = ld;
+    p.err = dev.err;
+    const Layout l{};
+    return launch(map, smap, p, sh.fp8, nullptr, l, reinterpret_cast<cudaStream_t>(stream_));
 }
 
 dsa_status_t dsa_topk_from_scores(const float* scores, int32_t T, int64_t L, int64_t ld, const int32_t* pos,
@@ -536,9 +545,8 @@ dsa_status_t dsa_topk_from_scores(const float* scores, int32_t T, int64_t L, int
         if (pos[t] < 0 || pos[t] >= L) return fail(DSA_ERR_INVALID_ARG, "pos[%d] = %d outside [0, L)", t, pos[t]);
     const Layout l = layout(T, L);
     if ((st = check_ws(workspace, workspace_bytes, l))) return st;
-    DeviceInfo dev;
-    if ((st = device_info(dev))) return st;
-    return run_topk(scores, ld, T, pos, topk, sel_idx, sel_ld, workspace, l, dev, reinterpret_cast<cudaStream_t>(stream_));
+    return run_topk_stage(scores, T, L, ld, pos, topk, sel_idx, sel_ld, workspace, l,
+                          reinterpret_cast<cudaStream_t>(stream_));
 }
 
 dsa_status_t dsa_topk_from_scores_noalloc(const float* scores, int32_t T, int64_t L, int64_t ld,
@@ -560,13 +568,11 @@ dsa_status_t dsa_topk_from_scores_noalloc(const float* scores, int32_t T, int64_
     if (!pos) return fail(DSA_ERR_INVALID_ARG, "pos: null");
     for (int t = 0; t < T; ++t)
         if (pos[t] < 0 || pos[t] >= L) return fail(DSA_ERR_INVALID_ARG, "pos[%d] = %d outside [0, L)", t, pos[t]);
-    const Layout l = topk_only_layout(T, L);
+    const Layout l = layout(T, L, false, false);
     if (l.total > kNoAllocBytes) return fail(DSA_ERR_INVALID_ARG, "no-allocation scratch too small");
     void* ws = nullptr;
     if ((st = noalloc_scratch(&ws))) return st;
-    DeviceInfo dev;
-    if ((st = device_info(dev))) return st;
-    return run_topk(scores, ld, T, pos, topk, sel_idx, sel_ld, ws, l, dev, reinterpret_cast<cudaStream_t>(stream_));
+    return run_topk_stage(scores, T, L, ld, pos, topk, sel_idx, sel_ld, ws, l, reinterpret_cast<cudaStream_t>(stream_));
 }
 
 dsa_status_t dsa_sparse_attn(const dsa_tensor_t* q, const dsa_tensor_t* kv_cache, const dsa_tensor_t* sel_idx,
@@ -595,8 +601,24 @@ dsa_status_t dsa_sparse_attn(const dsa_tensor_t* q, const dsa_tensor_t* kv_cache
     if ((st = check_ws(workspace, workspace_bytes, l))) return st;
     DeviceInfo dev;
     if ((st = device_info(dev))) return st;
-    return run_attention(q, kv_cache, static_cast<const int32_t*>(sel_idx->data), sel_idx->stride[0], topk, pos, sink,
-                         out, sh, workspace, l, dev, reinterpret_cast<cudaStream_t>(stream_));
+    StepParams p{};
+    p.phases = kPhaseAttend;
+    p.grid = grid_blocks(dev, false);
+    set_pos(p, pos, sh.T);
+    p.L = static_cast<int32_t>(sh.L);
+    p.topk = topk;
+    p.sel = static_cast<int32_t*>(sel_idx->data);
+    p.sel_ld = sel_idx->stride[0];
+    p.q = static_cast<const uint16_t*>(q->data);
+    p.kv = static_cast<const uint16_t*>(kv_cache->data);
+    p.kv_ld = sh.kv_ld;
+    p.sink = sink;
+    p.out = static_cast<uint16_t*>(out->data);
+    p.err = dev.err;
+    attn_params(p, workspace, l, topk);
+    CUtensorMap none;
+    std::memset(&none, 0, sizeof none);
+    return launch(none, none, p, false, workspace, l, reinterpret_cast<cudaStream_t>(stream_));
 }
 
 dsa_status_t dsa_device_status(dsa_stream_t stream_)
@@ -632,6 +654,15 @@ const char* dsa_status_str(dsa_status_t s)
 const char* dsa_last_error(void) { return t_last_error.c_str(); }
 
 uint64_t dsa_launch_count(void) { return g_launches.load(); }
+
+void dsa_set_step_trace(void* device_buffer) { t_trace = static_cast<unsigned long long*>(device_buffer); }
+
+int32_t dsa_step_grid(int32_t fp8_keys)
+{
+    DeviceInfo dev;
+    if (device_info(dev)) return 0;
+    return grid_blocks(dev, fp8_keys != 0);
+}
 
 void dsa_set_stage_events(void* const* events, int32_t n)
 {

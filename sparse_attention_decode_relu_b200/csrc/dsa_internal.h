@@ -15,73 +15,66 @@ constexpr int kMaxT = 8;
 constexpr int kMaxTopk = 2048;
 constexpr int kKeyTile = 128;              // keys per indexer tile
 constexpr int kHistBins = 4096;            // first-level radix bins (top 12 key bits)
-constexpr int kMaxChunks = 512;            // top-k chunks per query
-constexpr int kMaxSplits = 32;             // attention splits per query
-constexpr int kMaxSlots = 1024;            // per-block key-range slots
 
-struct IndexerParams {
+constexpr int kMaxRowsPerSplit = 256;       // selected rows one attention work item gathers
+constexpr int kMaxChunksStep = 1024;        // top-k chunks per query (<= grid)
+constexpr int kMaxGrid = 1024;              // blocks of the step kernel
+constexpr int kMaxAttnItems = 512;          // (query, split) attention work items
+constexpr int kTraceSlots = 32;             // phase-boundary stamps per block
+constexpr int kBarCtrlBytes = 128;          // grid barrier arrival counter
+
+// Phases of the step kernel.
+enum : int {
+    kPhaseIndex = 1,    // indexer scan (scores + per-block key ranges)
+    kPhaseRanges = 2,   // per-block key ranges of caller-provided scores
+    kPhaseTopk = 4,     // histogram, candidates, ordered emission
+    kPhaseAttend = 8,   // split attention + merge
+};
+
+struct StepParams {
+    int32_t phases;
+    int32_t grid;            // blocks (one per SM, all co-resident)
+    int32_t T, L, n_max, topk;
+    int32_t pos[kMaxT];
+    // indexer
     const uint16_t* q_idx;   // [T][16][64] bf16
     const float* w;          // [T][16]
     const float* scale;      // [L] or nullptr
     float* scores;           // [T][ld]
     int64_t ld;
-    int32_t L;
-    int32_t n_max;           // max_t pos[t] + 1: keys at or beyond it are never visible
-    int32_t pos[kMaxT];
-    uint32_t* zero;          // words the next stage needs zeroed (or nullptr)
-    int32_t zero_words;
-    uint32_t* mm;            // [gridDim.x][kMaxT] (min, max) key of the block's visible scores, or nullptr
-    uint32_t* err;
-};
-
-struct TopkParams {
-    const float* scores;     // [T][ld]
-    int64_t ld;
-    int32_t T;
-    int32_t topk;
-    int32_t chunk;           // elements per chunk (multiple of 2048)
-    int32_t nchunks;
-    int32_t pos[kMaxT];
-    uint32_t* hist;          // [T][kHistBins], zero on entry of the histogram kernel
-    uint32_t* tickets;       // [T], zero on entry of the select kernel
-    uint32_t* counts;        // [T][kMaxChunks]
-    uint2* cand;             // [T][ld]: (key, position) per chunk region
-    uint32_t* mm;            // [mm_slots][kMaxT] per-block (min, max) keys
+    // top-k
+    uint2* mm;               // [grid][kMaxT] per-block (min, max) key of visible scores
     int32_t mm_slots;
+    uint32_t* hist;          // [T][kHistBins]
+    uint32_t* list_n;        // [kMaxT] candidates per query
+    uint2* list;             // [T][ld] (key, position) candidates
+    uint32_t* above;         // [T][kMaxChunksStep]
+    uint32_t* cuts;          // [kMaxT][4]: threshold bin (cut, ctop) and #keys above it, per query
+    uint32_t* zero;          // words phase 1 clears (hist, list_n)
+    int32_t zero_words;
+    int32_t chunk, nchunk;   // top-k work items: nchunk chunks of `chunk` positions per query
     int32_t* sel;            // [T][sel_ld]
     int64_t sel_ld;
-    uint32_t* err;
-};
-
-struct AttnParams {
+    // attention
     const uint16_t* q;       // [T][64][128] bf16
     const uint16_t* kv;      // [L][kv_ld] bf16
-    int64_t kv_ld;           // elements per token row (>= 1024)
-    const int32_t* sel;      // [T][sel_ld]
-    int64_t sel_ld;
-    int32_t L;
+    int64_t kv_ld;
     int32_t rows;            // selected rows per query to read (= topk)
-    int32_t rows_per_split;  // multiple of 16
-    int32_t nsplit;          // blocks per query = cluster size
-    int32_t pos[kMaxT];
+    int32_t rows_per_split;  // multiple of 16, <= kMaxRowsPerSplit
+    int32_t nsplit;
     const float* sink;       // [64] or nullptr
+    float* po;               // [T][nsplit][64][128] partial outputs
+    float2* pml;             // [T][nsplit][64] (max in log2 units, sum)
     uint16_t* out;           // [T][64][128] bf16
+    // control
+    unsigned long long* trace;   // [grid][kTraceSlots] globaltimer stamps at phase boundaries, or nullptr
+    uint32_t* bar_ctrl;      // grid barrier arrival counter (zero at launch)
     uint32_t* err;
 };
 
-// Launchers return cudaGetLastError() after the launch.  Kernels after the
-// first of a step are launched with programmatic stream serialisation: they
-// start their prologue early and wait for the preceding grid before reading
-// its output.
-cudaError_t launch_indexer(const CUtensorMap* kmap, const CUtensorMap* smap, const IndexerParams& p, int T, bool fp8,
-                           int grid, cudaStream_t s);
-int indexer_max_ctas_per_sm(int T, bool fp8);
-cudaError_t launch_topk_cluster(const TopkParams& p, cudaStream_t s);
-int64_t topk_cluster_capacity();   // largest n the cluster path holds
-cudaError_t launch_topk_minmax(const TopkParams& p, cudaStream_t s);
-cudaError_t launch_topk_hist(const TopkParams& p, cudaStream_t s);
-cudaError_t launch_topk_select(const TopkParams& p, cudaStream_t s);
-cudaError_t launch_attention(const AttnParams& p, int T, cudaStream_t s);
-int attention_cluster_size(int T);   // blocks per query (16, 8 or 4)
+int step_smem_bytes();
+int step_max_blocks(bool fp8);
+cudaError_t launch_step(const CUtensorMap* kmap, const CUtensorMap* smap, const StepParams& p, bool fp8,
+                        cudaStream_t s);
 
 }  // namespace dsa

@@ -1,0 +1,1277 @@
+// step.cu -- the DSA decode/verify step as one cooperative persistent kernel.
+//
+// NaiveAI research page (naive.ai/en/research), "NaiveRT > A DSA layer: from 29
+// kernels to one": a DSA layer runs as a single cooperative kernel across 148
+// CTAs in one grid.  Here one block per SM runs every phase of the step, with a
+// bounded grid barrier between phases, so no kernel boundary (launch latency,
+// ramp, drain) separates the stages:
+//
+//   1 index   : ReLU indexer scan over the key cache (TMA tiles, tensor cores),
+//               fp32 scores plus each block's per-query key range
+//   2 hist    : first radix pass of the top-k, per (query, chunk) work item:
+//               4096 bins over the query's key range, summed in global memory
+//   3 extract : the bin holding the topk-th key; every key in that bin goes to
+//               the query's candidate list, keys above it are counted per chunk
+//   4 emit    : tau and the tie count from the candidate list (small), then
+//               each chunk writes its selected positions in order
+//   5 attend  : gathered sparse attention per (query, row split): whole K/V rows
+//               by bulk async copy, tensor-core QK and PV, online softmax;
+//               partial (max, sum, output) states to global memory
+//   6 merge   : per (query, head group), the splits merged in a fixed order
+//
+// Stage entry points run a sub-range of the phases.  Every reduction is either
+// integer or in a fixed order, so results are bitwise reproducible.
+#include "common.cuh"
+#include "dsa_internal.h"
+
+namespace dsa {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+constexpr float kLog2e = 1.4426950408889634f;
+
+// ---- shared memory map (dynamic, 1024-aligned base) --------------------------
+constexpr int kIdxStages = 4;
+constexpr int kAttStages = 6;
+constexpr int kTileRows = 16;
+constexpr int kRowBytes = 2048;
+constexpr int kPitch = 2064;              // bank-conflict-free ldmatrix rows
+constexpr int kDataBytes = kAttStages * kTileRows * kPitch + kAttStages * kTileRows * 4 + kMaxRowsPerSplit * 4;
+constexpr int kBarOffset = (kDataBytes + 127) / 128 * 128;
+constexpr int kStepSmem = 1024 + kBarOffset + 256;
+static_assert(kIdxStages * 16384 + 16384 + kMaxT * kHI * kDI * 2 + kMaxT * kHI * 4 + kIdxStages * kKeyTile * 4 <=
+                  kDataBytes, "indexer buffers fit the data region");
+
+__device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p)
+{
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void st_release(uint32_t* p, uint32_t v)
+{
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Grid-wide barrier among the co-resident blocks of a cooperative launch.  The
+// arrival counter only grows during a launch (it is zero at launch): barrier k
+// ends when it reaches k * gridDim.x.  Each block adds 1 with release semantics
+// and polls with acquire loads, giving up (error bit, false) after
+// kWaitLimitCycles.
+struct GridBarrier {
+    uint32_t* count;
+    uint32_t* err;
+    uint32_t next;     // count value that ends the next barrier
+
+    __device__ bool sync(int* ok_s)
+    {
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            const uint32_t target = next;
+            bool ok = true;
+            asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(count) : "memory");
+            const long long t0 = clock64();
+            while (ld_acquire(count) < target) {
+                if (clock64() - t0 > kWaitLimitCycles) {
+                    atomicOr(err, ERR_WAIT_TIMEOUT);
+                    ok = false;
+                    break;
+                }
+            }
+            *ok_s = ok ? 1 : 0;
+        }
+        __syncthreads();
+        next += gridDim.x;
+        return *ok_s != 0;
+    }
+};
+
+// Phase-boundary timestamp (when the caller asked for a trace).
+__device__ __forceinline__ void stamp(const StepParams& p, int slot)
+{
+    if (p.trace != nullptr && threadIdx.x == 0) {
+        unsigned long long t;
+        asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+        p.trace[(int64_t)blockIdx.x * kTraceSlots + slot] = t;
+    }
+}
+
+// ---- block-wide helpers ----------------------------------------------------------
+__device__ __forceinline__ uint32_t warp_incl_scan(uint32_t v)
+{
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += y;
+    }
+    return v;
+}
+
+// Exclusive prefix sum over the block (thread order); `total` gets the sum.
+__device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t& total, uint32_t* scratch)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const uint32_t x = warp_incl_scan(v);
+    if (lane == 31) scratch[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+        const uint32_t w = lane < kWarps ? scratch[lane] : 0u;
+        const uint32_t wi = warp_incl_scan(w);
+        if (lane < kWarps) scratch[lane] = wi;
+    }
+    __syncthreads();
+    const uint32_t before = warp ? scratch[warp - 1] : 0u;
+    total = scratch[kWarps - 1];
+    __syncthreads();
+    return before + x - v;
+}
+
+__device__ __forceinline__ uint32_t block_sum(uint32_t v, uint32_t* scratch)
+{
+    uint32_t total;
+    block_excl_scan(v, total, scratch);
+    return total;
+}
+
+__device__ __forceinline__ void block_minmax(uint32_t& lo, uint32_t& hi, uint32_t* scratch)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+        hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+    }
+    if (lane == 0) {
+        scratch[warp] = lo;
+        scratch[32 + warp] = hi;
+    }
+    __syncthreads();
+    lo = scratch[0];
+    hi = scratch[32];
+    for (int w = 1; w < kWarps; ++w) {
+        lo = min(lo, scratch[w]);
+        hi = max(hi, scratch[32 + w]);
+    }
+    __syncthreads();
+}
+
+// Right shift that maps the key range [lo, hi] onto at most 4096 bins.
+__device__ __forceinline__ int range_shift(uint32_t lo, uint32_t hi)
+{
+    const int bits = 32 - __clz(hi - lo);
+    return bits > 12 ? bits - 12 : 0;
+}
+
+// Highest key of the bin that starts at `start` (bins of width 2^shift), clamped to hi.
+__device__ __forceinline__ uint32_t bin_top(uint32_t start, int shift, uint32_t hi)
+{
+    const uint32_t width = (1u << shift) - 1u;   // shift <= 20
+    return (start > 0xFFFFFFFFu - width) ? hi : min(hi, start + width);
+}
+
+// Bin b of an NB-bin histogram (h global or shared) holding the need-th largest
+// entry: #(bins > b) < need <= #(bins >= b).  res = {b, #(bins > b), found}.
+template <int NB>
+__device__ void find_from_top(const uint32_t* h, uint32_t need, uint32_t* res, uint32_t* scratch, bool global_h)
+{
+    constexpr int PER = NB / kThreads;
+    const int top = NB - PER * threadIdx.x;   // thread 0 owns the highest bins
+    uint32_t cnt[PER];
+    uint32_t sum = 0;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+        cnt[i] = global_h ? __ldcg(h + top - 1 - i) : h[top - 1 - i];
+        sum += cnt[i];
+    }
+    if (threadIdx.x == 0) res[2] = 0;
+    uint32_t total;
+    uint32_t run = block_excl_scan(sum, total, scratch);
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+        if (run < need && run + cnt[i] >= need) {
+            res[0] = static_cast<uint32_t>(top - 1 - i);
+            res[1] = run;
+            res[2] = 1;
+        }
+        run += cnt[i];
+    }
+    __syncthreads();
+}
+
+// Work item i of `items` assigned to this block in round r (i = block + r*grid).
+__device__ __forceinline__ int item_of(int r) { return blockIdx.x + r * gridDim.x; }
+
+// ==================================================================================
+// Phase 1: indexer scan.  Tiles of 128 keys by TMA into a 4-stage ring; each warp
+// owns one query (or a share of one when T < 8) and keeps its 16 indexer heads x
+// 64 dims in registers as the N side of m16n8k16 tensor-core products whose M side
+// is 16 keys at a time.  ReLU, head weights, a fixed-order sum over heads.
+// ==================================================================================
+template <bool FP8>
+__device__ void phase_index(const CUtensorMap& kmap, const CUtensorMap& smap, const StepParams& p, uint8_t* smem,
+                            uint64_t* bars, uint32_t* scratch)
+{
+    constexpr int raw_bytes = kKeyTile * kDI * (FP8 ? 1 : 2);
+    uint8_t* ring = smem;
+    uint8_t* cvt = ring + kIdxStages * raw_bytes;
+    uint16_t* q_s = reinterpret_cast<uint16_t*>(cvt + (FP8 ? kKeyTile * kDI * 2 : 0));
+    float* w_s = reinterpret_cast<float*>(q_s + kMaxT * kHI * kDI);
+    float* sc_s = w_s + kMaxT * kHI;
+    uint64_t* full = bars;                  // [kIdxStages]
+    uint64_t* setup = bars + kIdxStages;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int g = lane >> 2, c = lane & 3;
+    const int T = p.T;
+    const int ntiles = (p.n_max + kKeyTile - 1) / kKeyTile;
+    const bool scaled = p.scale != nullptr;
+    const uint32_t tile_tx = raw_bytes + (scaled ? kKeyTile * 4 : 0);
+    auto load_tile = [&](int stage, int tile) {
+        mbar_arrive_expect_tx(&full[stage], tile_tx);
+        tma_load_2d(ring + stage * raw_bytes, &kmap, 0, tile * kKeyTile, &full[stage]);
+        if (scaled) tma_load_1d(sc_s + stage * kKeyTile, &smap, tile * kKeyTile, &full[stage]);
+    };
+
+    int issued = 0;
+    if (tid == 0) {
+        prefetch_tmap(&kmap);
+        if (scaled) prefetch_tmap(&smap);
+        for (int s = 0; s < kIdxStages + 1; ++s) mbar_init(&bars[s], 1);
+        fence_mbar_init();
+        mbar_arrive_expect_tx(setup, T * kHI * kDI * 2 + T * kHI * 4);
+        bulk_g2s(q_s, p.q_idx, T * kHI * kDI * 2, setup);
+        bulk_g2s(w_s, p.w, T * kHI * 4, setup);
+        for (int s = 0; s < kIdxStages; ++s) {
+            const int tile = blockIdx.x + s * gridDim.x;
+            if (tile >= ntiles) break;
+            load_tile(s, tile);
+            ++issued;
+        }
+    }
+    // Counters the top-k phases accumulate into start at zero.
+    for (int i = blockIdx.x * kThreads + tid; i < p.zero_words; i += gridDim.x * kThreads) p.zero[i] = 0u;
+    __syncthreads();
+    bool ok = mbar_wait(setup, 0, p.err);
+
+    // Warps per query: 8 / T rounded down to a power of two.
+    const int tp = T <= 1 ? 1 : T <= 2 ? 2 : T <= 4 ? 4 : 8;
+    const int wpq = kWarps / tp, nblk = kWarps / wpq;
+    const int t = warp / wpq;
+    const bool active = t < T;
+    const int kb0 = warp % wpq;
+    int pos_t = -1;
+#pragma unroll
+    for (int i = 0; i < kMaxT; ++i)
+        if (i == t) pos_t = p.pos[i];
+    uint32_t qb[2][4][2];
+    float w0 = 0.f, w1 = 0.f, w8 = 0.f, w9 = 0.f;
+    uint32_t klo = 0xFFFFFFFFu, khi = 0u;
+    if (active && ok) {
+        const uint32_t qbase = smem_u32(q_s + t * kHI * kDI);
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int kp = 0; kp < 2; ++kp) {
+                const uint32_t a = qbase + (nt * 8 + (lane & 7)) * (kDI * 2) + (kp * 32 + (lane >> 3) * 8) * 2;
+                ldsm_x4(a, qb[nt][2 * kp][0], qb[nt][2 * kp][1], qb[nt][2 * kp + 1][0], qb[nt][2 * kp + 1][1]);
+            }
+        w0 = w_s[t * kHI + 2 * c];
+        w1 = w_s[t * kHI + 2 * c + 1];
+        w8 = w_s[t * kHI + 8 + 2 * c];
+        w9 = w_s[t * kHI + 9 + 2 * c];
+    }
+
+    int it = 0;
+    bool aborted = __syncthreads_or(!ok);
+    for (int tile = blockIdx.x; !aborted && tile < ntiles; tile += gridDim.x, ++it) {
+        const int stage = it % kIdxStages;
+        ok = mbar_wait(&full[stage], (it / kIdxStages) & 1, p.err);
+        if (__syncthreads_or(!ok)) {
+            aborted = true;
+            break;
+        }
+        const uint8_t* ktile = ring + stage * raw_bytes;
+        if constexpr (FP8) {
+            // Widen 128 x 64 E4M3 codes to bf16 (exact) in the 128B-swizzled layout.
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                const int chunk = tid + r * kThreads;
+                const int row = chunk >> 2, piece = chunk & 3;
+                const uint4 v = *reinterpret_cast<const uint4*>(ktile + row * 64 + piece * 16);
+                const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+                uint32_t o[8];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    o[2 * i] = e4m3x2_to_bf16x2(static_cast<uint16_t>(w4[i] & 0xFFFFu));
+                    o[2 * i + 1] = e4m3x2_to_bf16x2(static_cast<uint16_t>(w4[i] >> 16));
+                }
+                const int c0 = (2 * piece) ^ (row & 7), c1 = (2 * piece + 1) ^ (row & 7);
+                *reinterpret_cast<uint4*>(cvt + row * 128 + c0 * 16) = make_uint4(o[0], o[1], o[2], o[3]);
+                *reinterpret_cast<uint4*>(cvt + row * 128 + c1 * 16) = make_uint4(o[4], o[5], o[6], o[7]);
+            }
+            __syncthreads();
+            ktile = cvt;
+        }
+        if (active) {
+#pragma unroll 2
+            for (int j = 0; j < nblk; ++j) {
+                const int kb = kb0 + wpq * j;
+                uint32_t a[4][4];
+                const int row = kb * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+                const uint32_t base = smem_u32(ktile) + row * 128;
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                    const int chunk = 2 * kk + (lane >> 4);
+                    ldsm_x4(base + ((chunk ^ (row & 7)) << 4), a[kk][0], a[kk][1], a[kk][2], a[kk][3]);
+                }
+                float acc0[4] = {0.f, 0.f, 0.f, 0.f}, acc1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                    mma_bf16_16816(acc0, a[kk], qb[0][kk][0], qb[0][kk][1]);
+                    mma_bf16_16816(acc1, a[kk], qb[1][kk][0], qb[1][kk][1]);
+                }
+                float pa = fmaxf(acc0[0], 0.f) * w0;
+                pa = fmaf(fmaxf(acc0[1], 0.f), w1, pa);
+                pa = fmaf(fmaxf(acc1[0], 0.f), w8, pa);
+                pa = fmaf(fmaxf(acc1[1], 0.f), w9, pa);
+                float pb = fmaxf(acc0[2], 0.f) * w0;
+                pb = fmaf(fmaxf(acc0[3], 0.f), w1, pb);
+                pb = fmaf(fmaxf(acc1[2], 0.f), w8, pb);
+                pb = fmaf(fmaxf(acc1[3], 0.f), w9, pb);
+                pa += __shfl_xor_sync(0xffffffffu, pa, 1);
+                pb += __shfl_xor_sync(0xffffffffu, pb, 1);
+                pa += __shfl_xor_sync(0xffffffffu, pa, 2);
+                pb += __shfl_xor_sync(0xffffffffu, pb, 2);
+                const int s = tile * kKeyTile + kb * 16 + g + 8 * (c & 1);   // lanes c = 0, 1 write
+                if (c < 2 && s < p.L) {
+                    const float scale = scaled ? sc_s[stage * kKeyTile + kb * 16 + g + 8 * (c & 1)] : 1.0f;
+                    const float v = (c == 0 ? pa : pb) * scale;
+                    if (s <= pos_t) {
+                        p.scores[(int64_t)t * p.ld + s] = v;
+                        const uint32_t k = score_key(v);
+                        klo = min(klo, k);
+                        khi = max(khi, k);
+                    } else {
+                        p.scores[(int64_t)t * p.ld + s] = -INFINITY;
+                    }
+                }
+            }
+        }
+        __syncthreads();   // every warp is done with this stage (and with cvt)
+        if (tid == 0) {
+            const int next = tile + kIdxStages * gridDim.x;
+            if (next < ntiles) {
+                load_tile(stage, next);
+                ++issued;
+            }
+        }
+    }
+    if (aborted) {   // let copies still in flight land before the smem is reused
+        if (tid == 0) {
+            mbar_wait(setup, 0, p.err);
+            for (int k = it; k < issued; ++k) mbar_wait(&full[k % kIdxStages], (k / kIdxStages) & 1, p.err);
+        }
+        __syncthreads();
+    }
+
+    // This block's key range of each query's visible scores (slot [block][t]).
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        klo = min(klo, __shfl_xor_sync(0xffffffffu, klo, o));
+        khi = max(khi, __shfl_xor_sync(0xffffffffu, khi, o));
+    }
+    if (lane == 0) {
+        scratch[warp] = klo;
+        scratch[32 + warp] = khi;
+    }
+    __syncthreads();
+    if (tid < kMaxT && p.mm != nullptr) {
+        uint32_t lo = 0xFFFFFFFFu, hi = 0u;
+        if (tid < T)
+            for (int w = tid * wpq; w < (tid + 1) * wpq; ++w) {
+                lo = min(lo, scratch[w]);
+                hi = max(hi, scratch[32 + w]);
+            }
+        p.mm[(int64_t)blockIdx.x * kMaxT + tid] = make_uint2(lo, hi);
+    }
+    // Positions no query can see (s >= n_max): -inf, as the stage contract states.
+    const int64_t tail0 = (int64_t)ntiles * kKeyTile;
+    for (int64_t s = tail0 + (int64_t)blockIdx.x * kThreads + tid; s < p.L; s += (int64_t)gridDim.x * kThreads)
+        for (int tt = 0; tt < T; ++tt) p.scores[(int64_t)tt * p.ld + s] = -INFINITY;
+    __syncthreads();
+}
+
+// Phase 1 for caller-provided scores: each block's key range per query.
+__device__ void phase_ranges(const StepParams& p, uint32_t* scratch)
+{
+    for (int i = blockIdx.x * kThreads + threadIdx.x; i < p.zero_words; i += gridDim.x * kThreads) p.zero[i] = 0u;
+    for (int t = 0; t < p.T; ++t) {
+        const int n = p.pos[t] + 1;
+        uint32_t lo = 0xFFFFFFFFu, hi = 0u;
+        const float* row = p.scores + (int64_t)t * p.ld;
+        for (int s = blockIdx.x * kThreads + threadIdx.x; s < n; s += gridDim.x * kThreads) {
+            const uint32_t k = score_key(__ldcg(row + s));
+            lo = min(lo, k);
+            hi = max(hi, k);
+        }
+        block_minmax(lo, hi, scratch);
+        if (threadIdx.x == 0) p.mm[(int64_t)blockIdx.x * kMaxT + t] = make_uint2(lo, hi);
+    }
+    for (int t = p.T + threadIdx.x; t < kMaxT; t += kThreads)
+        p.mm[(int64_t)blockIdx.x * kMaxT + t] = make_uint2(0xFFFFFFFFu, 0u);
+}
+
+// ==================================================================================
+// Phases 2-4: causal top-k by radix select over the query's own key range.
+// Work items are (query t, chunk c): positions [c*S, min((c+1)*S, n_t)).  A chunk
+// that fits is bulk-copied into shared memory once (phase 2) and stays there for
+// phase 3; longer chunks are streamed with several vector loads in flight.
+// ==================================================================================
+constexpr int kChunkSmem = 40960;        // scores of one chunk kept in shared memory
+
+struct Item {
+    int t, c, s0, s1, n;
+};
+
+__device__ __forceinline__ Item topk_item(const StepParams& p, int i)
+{
+    Item it;
+    it.t = i / p.nchunk;
+    it.c = i % p.nchunk;
+    int pos_t = 0;
+#pragma unroll
+    for (int k = 0; k < kMaxT; ++k)
+        if (k == it.t) pos_t = p.pos[k];
+    it.n = pos_t + 1;
+    it.s0 = min(it.n, it.c * p.chunk);
+    it.s1 = min(it.n, it.s0 + p.chunk);
+    return it;
+}
+
+// Key range [lo, hi] of query t from the per-block ranges of phase 1.
+__device__ void query_range(const StepParams& p, int t, uint32_t& lo, uint32_t& hi, uint32_t* scratch)
+{
+    lo = 0xFFFFFFFFu;
+    hi = 0u;
+    for (int b = threadIdx.x; b < p.mm_slots; b += kThreads) {
+        const uint2 v = __ldcg(p.mm + (int64_t)b * kMaxT + t);
+        lo = min(lo, v.x);
+        hi = max(hi, v.y);
+    }
+    block_minmax(lo, hi, scratch);
+}
+
+// The chunk's keys: from shared memory (after phase 2 put them there) or global.
+struct ChunkKeys {
+    const uint32_t* smem;   // keys of positions [s0, s1) or nullptr
+    const float* row;       // scores of the query
+    int s0;
+    __device__ __forceinline__ uint32_t operator()(int s) const
+    {
+        return smem ? smem[s - s0] : score_key(__ldcg(row + s));
+    }
+};
+
+__device__ void phase_hist(const StepParams& p, uint8_t* smem, uint64_t* bar, uint32_t* scratch)
+{
+    uint32_t* keys = reinterpret_cast<uint32_t*>(smem);                       // [kChunkSmem]
+    uint32_t* h = keys + kChunkSmem;                                          // [kHistBins]
+    int uses = 0;   // phases of `bar` completed so far
+    for (int r = 0;; ++r) {
+        const int i = item_of(r);
+        if (i >= p.T * p.nchunk) break;
+        const Item it = topk_item(p, i);
+        if (it.n <= p.topk || it.s0 >= it.s1) continue;
+        uint32_t lo, hi;
+        query_range(p, it.t, lo, hi, scratch);
+        const int shift = range_shift(lo, hi);
+        const float* row = p.scores + (int64_t)it.t * p.ld;
+        const int cnt = it.s1 - it.s0;
+        const int c4 = (cnt + 3) & ~3;   // rows have a stride that is a multiple of 4 scores
+        const bool in_smem = r == 0 && c4 <= kChunkSmem;   // a block's first item stays in smem
+        if (in_smem) {
+            if (threadIdx.x == 0) {
+                mbar_arrive_expect_tx(bar, static_cast<uint32_t>(c4) * 4u);
+                bulk_g2s(keys, row + it.s0, static_cast<uint32_t>(c4) * 4u, bar);
+            }
+        }
+        for (int b = threadIdx.x; b < kHistBins; b += kThreads) h[b] = 0u;
+        if (in_smem) {
+            const bool ok = mbar_wait(bar, uses & 1, p.err);
+            ++uses;
+            if (!__syncthreads_and(ok)) return;
+            for (int j = threadIdx.x; j < cnt; j += kThreads) {
+                const uint32_t k = score_key(__uint_as_float(keys[j]));
+                keys[j] = k;
+                atomicAdd(&h[(k - lo) >> shift], 1u);
+            }
+        } else {
+            __syncthreads();
+            for (int s = it.s0 + threadIdx.x * 4; s < it.s1; s += kThreads * 16) {
+                float4 v[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int su = s + u * kThreads * 4;
+                    v[u] = su + 4 <= it.s1 ? __ldcg(reinterpret_cast<const float4*>(row + su))
+                                           : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int su = s + u * kThreads * 4;
+                    if (su + 4 <= it.s1) {
+                        atomicAdd(&h[(score_key(v[u].x) - lo) >> shift], 1u);
+                        atomicAdd(&h[(score_key(v[u].y) - lo) >> shift], 1u);
+                        atomicAdd(&h[(score_key(v[u].z) - lo) >> shift], 1u);
+                        atomicAdd(&h[(score_key(v[u].w) - lo) >> shift], 1u);
+                    } else {
+                        for (int j = su; j < it.s1 && j < su + 4; ++j)
+                            atomicAdd(&h[(score_key(__ldcg(row + j)) - lo) >> shift], 1u);
+                    }
+                }
+            }
+        }
+        __syncthreads();
+        uint32_t* gh = p.hist + (int64_t)it.t * kHistBins;
+        for (int b = threadIdx.x; b < kHistBins; b += kThreads)
+            if (h[b]) atomicAdd(gh + b, h[b]);
+        __syncthreads();
+    }
+}
+
+// Per query: threshold bin [cut, ctop] and #(keys > ctop), from the histogram.
+struct Cut {
+    uint32_t cut, ctop, above;
+};
+
+__device__ Cut query_cut(const StepParams& p, int t, uint32_t* res, uint32_t* scratch)
+{
+    uint32_t lo, hi;
+    query_range(p, t, lo, hi, scratch);
+    const int shift = range_shift(lo, hi);
+    find_from_top<kHistBins>(p.hist + (int64_t)t * kHistBins, static_cast<uint32_t>(p.topk), res, scratch, true);
+    Cut cu;
+    if (!res[2]) {   // histogram and scores disagree: cannot happen for consistent input
+        if (threadIdx.x == 0) atomicOr(p.err, ERR_TOPK_STATE);
+        cu.cut = lo;
+        cu.ctop = hi;
+        cu.above = 0;
+    } else {
+        cu.cut = lo + (res[0] << shift);
+        cu.ctop = bin_top(cu.cut, shift, hi);
+        cu.above = res[1];
+    }
+    __syncthreads();
+    return cu;
+}
+
+// Phase 3: every key >= cut (the threshold bin and above) goes to the query's
+// candidate list with its position; keys above the bin are also counted per
+// chunk.  One atomic per block reserves the block's slots of the list.
+__device__ void phase_extract(const StepParams& p, uint8_t* smem, uint32_t* res, uint32_t* scratch)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const uint32_t* keys = reinterpret_cast<const uint32_t*>(smem);
+    for (int r = 0;; ++r) {
+        const int i = item_of(r);
+        if (i >= p.T * p.nchunk) break;
+        const Item it = topk_item(p, i);
+        if (it.n <= p.topk) continue;
+        const Cut cu = query_cut(p, it.t, res, scratch);
+        if (it.c == 0 && threadIdx.x == 0)
+            reinterpret_cast<uint4*>(p.cuts)[it.t] = make_uint4(cu.cut, cu.ctop, cu.above, 0u);
+        const int cnt = it.s1 - it.s0;
+        const ChunkKeys key{r == 0 && ((cnt + 3) & ~3) <= kChunkSmem ? keys : nullptr, p.scores + (int64_t)it.t * p.ld,
+                            it.s0};
+        // Pass 1: candidates per warp (warp w owns lanes w*32.. of every 256-position step).
+        uint32_t above = 0, wcnt = 0;
+        for (int base = it.s0; base < it.s1; base += kThreads * 4) {
+            uint32_t k[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int s = base + u * kThreads + threadIdx.x;
+                k[u] = s < it.s1 ? key(s) : 0u;
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int s = base + u * kThreads + threadIdx.x;
+                above += s < it.s1 && k[u] > cu.ctop;
+                wcnt += __popc(__ballot_sync(0xffffffffu, s < it.s1 && k[u] >= cu.cut));
+            }
+        }
+        if (lane == 0) scratch[warp] = wcnt;
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            uint32_t tot = 0;
+            for (int w = 0; w < kWarps; ++w) {
+                const uint32_t x = scratch[w];
+                scratch[w] = tot;
+                tot += x;
+            }
+            scratch[kWarps] = tot ? atomicAdd(p.list_n + it.t, tot) : 0u;
+        }
+        __syncthreads();
+        uint32_t at = scratch[kWarps] + scratch[warp];
+        __syncthreads();
+        // Pass 2: the same positions in the same order, written at the reserved slots.
+        uint2* list = p.list + (int64_t)it.t * p.ld;
+        for (int base = it.s0; base < it.s1; base += kThreads * 4) {
+            uint32_t k[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int s = base + u * kThreads + threadIdx.x;
+                k[u] = s < it.s1 ? key(s) : 0u;
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int s = base + u * kThreads + threadIdx.x;
+                const bool c = s < it.s1 && k[u] >= cu.cut;
+                const uint32_t bal = __ballot_sync(0xffffffffu, c);
+                if (c) list[at + __popc(bal & ((1u << lane) - 1u))] = make_uint2(k[u], static_cast<uint32_t>(s));
+                at += __popc(bal);
+            }
+        }
+        above = block_sum(above, scratch);
+        if (threadIdx.x == 0) p.above[(int64_t)it.t * kMaxChunksStep + it.c] = above;
+    }
+}
+
+// Radix select over n values read through get(j) (only those in [lo, hi] count),
+// `need` of them still to find from the top.  On return lo == hi is the need-th
+// largest value and need = how many entries equal to it are to be taken.
+template <typename Get>
+__device__ void radix_select(Get get, uint32_t n, uint32_t& lo, uint32_t& hi, uint32_t& need, uint32_t* h,
+                             uint32_t* res, uint32_t* scratch, uint32_t* err)
+{
+#pragma unroll 1
+    for (int pass = 0; pass < 4 && lo != hi; ++pass) {
+        const int shift = range_shift(lo, hi);
+        for (int b = threadIdx.x; b < kHistBins; b += kThreads) h[b] = 0u;
+        __syncthreads();
+        for (uint32_t j = threadIdx.x; j < n; j += kThreads) {
+            const uint32_t k = get(j);
+            if (k >= lo && k <= hi) atomicAdd(&h[(k - lo) >> shift], 1u);
+        }
+        __syncthreads();
+        find_from_top<kHistBins>(h, need, res, scratch, false);
+        if (!res[2]) {
+            if (threadIdx.x == 0) atomicOr(err, ERR_TOPK_STATE);
+            res[0] = 0;
+            res[1] = 0;
+        }
+        const uint32_t nlo = lo + (res[0] << shift);
+        hi = bin_top(nlo, shift, hi);
+        lo = nlo;
+        need -= res[1];
+        __syncthreads();
+    }
+}
+
+// The need-th largest of the n values v[0..n) in shared memory (n <= kSmallSel):
+// each thread ranks its values against all of them.  Returns the value; `need`
+// becomes how many entries equal to it are to be taken.
+constexpr int kSmallSel = 64;
+
+__device__ uint32_t rank_select(const uint32_t* v, uint32_t n, uint32_t& need, uint32_t* res, uint32_t* err)
+{
+    if (threadIdx.x == 0) res[2] = 0;
+    __syncthreads();
+    for (uint32_t j = threadIdx.x; j < n; j += kThreads) {
+        const uint32_t x = v[j];
+        uint32_t gt = 0, eq = 0, eq_before = 0;
+        for (uint32_t q = 0; q < n; ++q) {
+            const uint32_t y = v[q];
+            gt += y > x;
+            eq += y == x;
+            eq_before += (y == x) && q < j;
+        }
+        // the first copy (lowest index) of the value that holds the need-th place reports it
+        if (eq_before == 0 && gt < need && gt + eq >= need) {
+            res[0] = x;
+            res[1] = gt;
+            res[2] = 1;
+        }
+    }
+    __syncthreads();
+    if (!res[2]) {
+        if (threadIdx.x == 0) atomicOr(err, ERR_TOPK_STATE);
+        __syncthreads();
+        return 0u;
+    }
+    const uint32_t x = res[0];
+    need -= res[1];
+    __syncthreads();
+    return x;
+}
+
+// Phase 4.  The common case: the query's candidate list (every key >= cut,
+// with its position) fits in shared memory and the context fits the bitmap.
+// Block (t, chunk 0) then finds tau and the tie cut among the candidates, marks
+// the selected positions in a bitmap and writes them in position order.
+// Otherwise every chunk block sweeps its positions in order.
+constexpr int kListSmem = 4096;          // candidates a block keeps in shared memory
+constexpr int kBitmapBits = 1 << 20;     // positions the ordered emission marks in shared memory
+static_assert(kListSmem * 8 + kHistBins * 4 + kBitmapBits / 8 + kSmallSel * 8 <= kDataBytes, "emit buffers fit");
+static_assert(kChunkSmem * 4 + kHistBins * 4 <= kDataBytes, "chunk buffers fit");
+
+__device__ void phase_emit(const StepParams& p, uint8_t* smem, uint64_t* bar, uint32_t* res, uint32_t* scratch)
+{
+    uint2* lst = reinterpret_cast<uint2*>(smem);                                  // [kListSmem]
+    uint32_t* h = reinterpret_cast<uint32_t*>(smem + kListSmem * 8);              // [kHistBins]
+    uint32_t* bitmap = h + kHistBins;                                             // [kBitmapBits / 32]
+    uint32_t* small = bitmap + kBitmapBits / 32;                                  // [2 * kSmallSel]
+    __shared__ uint32_t nsmall;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int uses = 0;
+    for (int r = 0;; ++r) {
+        const int i = item_of(r);
+        if (i >= p.T * p.nchunk) break;
+        const Item it = topk_item(p, i);
+        int32_t* sel = p.sel + (int64_t)it.t * p.sel_ld;
+        if (it.n <= p.topk) {   // everything visible is selected
+            for (int s = it.s0 + threadIdx.x; s < it.s1; s += kThreads) sel[s] = s;
+            if (it.c == 0)
+                for (int j = it.n + threadIdx.x; j < p.topk; j += kThreads) sel[j] = -1;
+            continue;
+        }
+        const uint32_t m = __ldcg(p.list_n + it.t);
+        const bool fast = m <= static_cast<uint32_t>(kListSmem) && it.n <= kBitmapBits;
+        if (fast && it.c != 0) continue;
+        const uint4 cq = __ldcg(reinterpret_cast<const uint4*>(p.cuts) + it.t);
+        const Cut cu{cq.x, cq.y, cq.z};
+        const uint2* glist = p.list + (int64_t)it.t * p.ld;
+        stamp(p, 12);
+        if (fast) {
+            // The list in one bulk copy (8-byte entries; an odd count reads one spare entry).
+            const uint32_t bytes = ((m * 8u) + 15u) & ~15u;
+            if (threadIdx.x == 0) {
+                mbar_arrive_expect_tx(bar, bytes);
+                bulk_g2s(lst, glist, bytes, bar);
+            }
+            if (!__syncthreads_and(mbar_wait(bar, uses & 1, p.err))) return;
+            ++uses;
+        }
+        auto cand = [&](uint32_t j) -> uint2 { return fast ? lst[j] : __ldcg(glist + j); };
+        stamp(p, 13);
+
+        // tau: keys above ctop are all taken; select among the keys in the bin.
+        uint32_t need = static_cast<uint32_t>(p.topk) - cu.above;
+        uint32_t tau;
+        if (threadIdx.x == 0) nsmall = 0;
+        __syncthreads();
+        if (fast) {   // gather the bin's keys (order does not matter for the rank of a value)
+            for (uint32_t j = threadIdx.x; j < m; j += kThreads) {
+                const uint32_t k = lst[j].x;
+                if (k <= cu.ctop) {
+                    const uint32_t at = atomicAdd(&nsmall, 1u);
+                    if (at < kSmallSel) small[at] = k;
+                }
+            }
+        }
+        __syncthreads();
+        if (fast && nsmall <= kSmallSel) {
+            tau = rank_select(small, nsmall, need, res, p.err);
+        } else {
+            uint32_t lo = cu.cut, hi = cu.ctop;
+            radix_select([&](uint32_t j) { return cand(j).x; }, m, lo, hi, need, h, res, scratch, p.err);
+            tau = lo;
+        }
+        const uint32_t rties = need;   // take every key > tau and the first rties keys == tau
+        stamp(p, 14);
+
+        if (fast) {
+            // Ties at tau: the rties lowest positions.  e = #(key == tau).
+            if (threadIdx.x == 0) nsmall = 0;
+            __syncthreads();
+            uint32_t e = 0;
+            for (uint32_t j = threadIdx.x; j < m; j += kThreads) {
+                const uint2 v = lst[j];
+                if (v.x == tau) {
+                    ++e;
+                    const uint32_t at = atomicAdd(&nsmall, 1u);
+                    if (at < kSmallSel) small[kSmallSel + at] = ~v.y;   // ~position: largest = lowest position
+                }
+            }
+            e = block_sum(e, scratch);
+            uint32_t pcut = 0xFFFFFFFFu;   // ties with position <= pcut are taken
+            if (rties < e) {
+                uint32_t need_p = rties;
+                if (e <= static_cast<uint32_t>(kSmallSel)) {
+                    pcut = ~rank_select(small + kSmallSel, e, need_p, res, p.err);
+                } else {
+                    uint32_t plo = 0xFFFFFFFFu, phi = 0u;
+                    for (uint32_t j = threadIdx.x; j < m; j += kThreads)
+                        if (lst[j].x == tau) {
+                            plo = min(plo, ~lst[j].y);
+                            phi = max(phi, ~lst[j].y);
+                        }
+                    block_minmax(plo, phi, scratch);
+                    radix_select([&](uint32_t j) { const uint2 v = lst[j]; return v.x == tau ? ~v.y : 0u; }, m, plo,
+                                 phi, need_p, h, res, scratch, p.err);
+                    pcut = ~plo;
+                }
+            }
+            stamp(p, 15);
+            const int nwords = (it.n + 31) >> 5;
+            for (int w = threadIdx.x; w < nwords; w += kThreads) bitmap[w] = 0u;
+            __syncthreads();
+            for (uint32_t j = threadIdx.x; j < m; j += kThreads) {
+                const uint2 v = lst[j];
+                if (v.x > tau || (v.x == tau && v.y <= pcut)) atomicOr(&bitmap[v.y >> 5], 1u << (v.y & 31));
+            }
+            __syncthreads();
+            // Warp w owns words [w*per, (w+1)*per); lanes read consecutive words.
+            const int per = ((nwords + kWarps - 1) / kWarps + 31) / 32 * 32;
+            const int w0 = min(nwords, warp * per), w1 = min(nwords, w0 + per);
+            uint32_t cnt = 0;
+            for (int w = w0 + lane; w < w1; w += 32) cnt += __popc(bitmap[w]);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+            if (lane == 0) scratch[32 + warp] = cnt;
+            __syncthreads();
+            uint32_t o = 0, total = 0;
+            for (int w = 0; w < kWarps; ++w) {
+                const uint32_t x = scratch[32 + w];
+                if (w < warp) o += x;
+                total += x;
+            }
+            for (int base = w0; base < w1; base += 32) {
+                const int w = base + lane;
+                uint32_t b = w < w1 ? bitmap[w] : 0u;
+                const uint32_t c = __popc(b);
+                const uint32_t incl = warp_incl_scan(c);
+                uint32_t oo = o + incl - c;
+                while (b) {
+                    const int bit = __ffs(b) - 1;
+                    b &= b - 1;
+                    if (oo < static_cast<uint32_t>(p.topk)) sel[oo] = (w << 5) + bit;
+                    ++oo;
+                }
+                o += __shfl_sync(0xffffffffu, incl, 31);
+            }
+            if (threadIdx.x == 0 && total != static_cast<uint32_t>(p.topk)) atomicOr(p.err, ERR_TOPK_STATE);
+            __syncthreads();
+            continue;
+        }
+
+        // Fallback: this chunk's output offset and tie rank from the candidates of
+        // earlier chunks, then an ordered sweep of the chunk.
+        uint32_t before_gt = 0, before_eq = 0;
+        for (uint32_t j = threadIdx.x; j < m; j += kThreads) {
+            const uint2 v = cand(j);
+            if (static_cast<int>(v.y) < it.s0) {
+                before_gt += v.x > tau;
+                before_eq += v.x == tau;
+            }
+        }
+        before_gt = block_sum(before_gt, scratch);
+        before_eq = block_sum(before_eq, scratch);
+        uint32_t out = before_gt + min(before_eq, rties);
+        uint32_t tie_rank = before_eq;
+        const float* row = p.scores + (int64_t)it.t * p.ld;
+        for (int base = it.s0; base < it.s1; base += kThreads * 4) {
+            const int s = base + threadIdx.x * 4;
+            uint32_t gtm = 0, eqm = 0;
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                if (s + j < it.s1) {
+                    const uint32_t k = score_key(__ldcg(row + s + j));
+                    if (k > tau) gtm |= 1u << j;
+                    if (k == tau) eqm |= 1u << j;
+                }
+            if (!__syncthreads_or((gtm | eqm) != 0u)) continue;
+            uint32_t tie_total;
+            uint32_t rank = tie_rank + block_excl_scan(__popc(eqm), tie_total, scratch);
+            uint32_t take = gtm;
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                if (eqm & (1u << j)) {
+                    if (rank < rties) take |= 1u << j;
+                    ++rank;
+                }
+            uint32_t taken_total;
+            uint32_t o = out + block_excl_scan(__popc(take), taken_total, scratch);
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                if ((take & (1u << j)) && o < static_cast<uint32_t>(p.topk)) sel[o++] = s + j;
+            out += taken_total;
+            tie_rank += tie_total;
+        }
+    }
+}
+
+// ==================================================================================
+// Phase 5: sparse attention per (query t, row split).  Warp 4 gathers whole
+// 2 KiB token rows (K then V of the 4 groups) by bulk async copy into a 6-stage
+// ring of 16-row tiles; warp g < 4 owns KV group g, i.e. query heads
+// 16g .. 16g+15 -- the 16 rows of an m16n8k16 tile, so nothing is padded.
+// Online softmax in the exp2 domain; the partial (max, sum, output) of every
+// head goes to global memory for phase 6.
+// ==================================================================================
+__device__ void phase_attend(const StepParams& p, uint8_t* smem, uint64_t* bars)
+{
+    uint8_t* ring = smem;
+    int32_t* rowidx = reinterpret_cast<int32_t*>(smem + kAttStages * kTileRows * kPitch);   // [stage][16]
+    int32_t* sel_s = rowidx + kAttStages * kTileRows;
+    uint64_t* full = bars + 8;
+    uint64_t* empty = full + kAttStages;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int gq = lane >> 2, c = lane & 3;
+    constexpr int kConsumers = 4;
+    const float sm_scale = kLog2e * rsqrtf(static_cast<float>(kD));
+
+    int phase_base = 0;   // tiles consumed by this block so far (mbarrier phase bookkeeping)
+    if (tid == 0) {
+        for (int s = 0; s < kAttStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], kConsumers);
+        }
+        fence_mbar_init();
+    }
+    __syncthreads();
+
+    for (int r = 0;; ++r) {
+        const int i = item_of(r);
+        if (i >= p.T * p.nsplit) break;
+        const int t = i / p.nsplit, split = i % p.nsplit;
+        int pos_t = 0;
+#pragma unroll
+        for (int k = 0; k < kMaxT; ++k)
+            if (k == t) pos_t = p.pos[k];
+        const int rows_t = min(p.rows, pos_t + 1);
+        const int r0 = split * p.rows_per_split;
+        const int r1 = min(r0 + p.rows_per_split, rows_t);
+        const int ntile = r1 > r0 ? (r1 - r0 + kTileRows - 1) / kTileRows : 0;
+
+        bool failed = false;
+        float oacc[16][4];
+        float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+#pragma unroll
+        for (int k = 0; k < 16; ++k) oacc[k][0] = oacc[k][1] = oacc[k][2] = oacc[k][3] = 0.f;
+
+        if (warp == kConsumers) {
+            // producer: validate the selected rows, gather them whole
+            const int32_t* selrow = p.sel + (int64_t)t * p.sel_ld + r0;
+            for (int j = lane; j < r1 - r0; j += 32) sel_s[j] = __ldcg(selrow + j);
+            __syncwarp();
+            for (int k = 0; k < ntile; ++k) {
+                const int kk = phase_base + k;
+                const int stage = kk % kAttStages;
+                if (kk >= kAttStages && !mbar_wait(&empty[stage], ((kk / kAttStages) - 1) & 1, p.err)) {
+                    failed = true;
+                    break;
+                }
+                uint8_t* dst = ring + stage * kTileRows * kPitch;
+                int s = -1;
+                bool valid = false;
+                if (lane < kTileRows) {
+                    const int j = k * kTileRows + lane;
+                    if (r0 + j < r1) {
+                        s = sel_s[j];
+                        valid = s >= 0 && s <= pos_t && s < p.L;
+                        if (s >= 0 && !valid) atomicOr(p.err, ERR_BAD_INDEX);
+                    }
+                    rowidx[stage * kTileRows + lane] = valid ? s : -1;
+                }
+                const uint32_t vmask = __ballot_sync(0xffffffffu, valid);
+                // Rows with nothing to load get a zero V half, so P = 0 never meets stale data.
+                uint32_t none = ~vmask & 0xFFFFu;
+                while (none) {
+                    const int z = __ffs(none) - 1;
+                    none &= none - 1;
+                    uint4* v = reinterpret_cast<uint4*>(dst + z * kPitch + kRowBytes / 2);
+                    v[lane] = make_uint4(0u, 0u, 0u, 0u);
+                    v[lane + 32] = make_uint4(0u, 0u, 0u, 0u);
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_expect_tx(&full[stage], __popc(vmask) * kRowBytes);
+                __syncwarp();
+                if (valid) bulk_g2s(dst + lane * kPitch, p.kv + (int64_t)s * p.kv_ld, kRowBytes, &full[stage]);
+            }
+        } else if (warp < kConsumers) {
+            const int grp = warp;
+            uint32_t qa[8][4];
+            const uint16_t* qbp = p.q + ((int64_t)t * kH + grp * 16) * kD;
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                qa[kk][0] = __ldg(reinterpret_cast<const uint32_t*>(qbp + gq * kD + kk * 16 + 2 * c));
+                qa[kk][1] = __ldg(reinterpret_cast<const uint32_t*>(qbp + (gq + 8) * kD + kk * 16 + 2 * c));
+                qa[kk][2] = __ldg(reinterpret_cast<const uint32_t*>(qbp + gq * kD + kk * 16 + 8 + 2 * c));
+                qa[kk][3] = __ldg(reinterpret_cast<const uint32_t*>(qbp + (gq + 8) * kD + kk * 16 + 8 + 2 * c));
+            }
+            for (int k = 0; k < ntile; ++k) {
+                const int kk0 = phase_base + k;
+                const int stage = kk0 % kAttStages;
+                if (!mbar_wait(&full[stage], (kk0 / kAttStages) & 1, p.err)) {
+                    failed = true;
+                    break;
+                }
+                const uint32_t base = smem_u32(ring + stage * kTileRows * kPitch);
+                const int32_t* ridx = rowidx + stage * kTileRows;
+                float sacc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+                float sodd[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+                for (int kk2 = 0; kk2 < 4; ++kk2) {
+#pragma unroll
+                    for (int nt = 0; nt < 2; ++nt) {
+                        const int key = nt * 8 + (lane & 7);
+                        const int dim = kk2 * 32 + (lane >> 3) * 8;
+                        uint32_t b0, b1, b2, b3;
+                        ldsm_x4(base + key * kPitch + grp * 256 + dim * 2, b0, b1, b2, b3);
+                        mma_bf16_16816(sacc[nt], qa[2 * kk2], b0, b1);
+                        mma_bf16_16816(sodd[nt], qa[2 * kk2 + 1], b2, b3);
+                    }
+                }
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int key = nt * 8 + 2 * c + (e & 1);
+                        const float z = sacc[nt][e] + sodd[nt][e];
+                        sacc[nt][e] = ridx[key] >= 0 ? z * sm_scale : -INFINITY;
+                    }
+                float mx0 = fmaxf(fmaxf(sacc[0][0], sacc[0][1]), fmaxf(sacc[1][0], sacc[1][1]));
+                float mx1 = fmaxf(fmaxf(sacc[0][2], sacc[0][3]), fmaxf(sacc[1][2], sacc[1][3]));
+                mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+                mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+                mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+                mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+                const float n0 = fmaxf(m0, mx0), n1 = fmaxf(m1, mx1);
+                const float z0 = n0 == -INFINITY ? 0.f : n0, z1 = n1 == -INFINITY ? 0.f : n1;
+                const float alpha0 = exp2f(m0 - z0), alpha1 = exp2f(m1 - z1);
+                m0 = n0;
+                m1 = n1;
+                float pr[2][4];
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt) {
+                    pr[nt][0] = exp2f(sacc[nt][0] - z0);
+                    pr[nt][1] = exp2f(sacc[nt][1] - z0);
+                    pr[nt][2] = exp2f(sacc[nt][2] - z1);
+                    pr[nt][3] = exp2f(sacc[nt][3] - z1);
+                }
+                l0 = l0 * alpha0 + (pr[0][0] + pr[0][1]) + (pr[1][0] + pr[1][1]);
+                l1 = l1 * alpha1 + (pr[0][2] + pr[0][3]) + (pr[1][2] + pr[1][3]);
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    oacc[e][0] *= alpha0;
+                    oacc[e][1] *= alpha0;
+                    oacc[e][2] *= alpha1;
+                    oacc[e][3] *= alpha1;
+                }
+                uint32_t pa[4];
+                pa[0] = pack_bf16(pr[0][0], pr[0][1]);
+                pa[1] = pack_bf16(pr[0][2], pr[0][3]);
+                pa[2] = pack_bf16(pr[1][0], pr[1][1]);
+                pa[3] = pack_bf16(pr[1][2], pr[1][3]);
+#pragma unroll
+                for (int nd2 = 0; nd2 < 8; ++nd2) {
+                    const int key = (lane & 7) + 8 * ((lane >> 3) & 1);
+                    const int dim = nd2 * 16 + 8 * (lane >> 4);
+                    uint32_t v0, v1, v2, v3;
+                    ldsm_x4_t(base + key * kPitch + kRowBytes / 2 + grp * 256 + dim * 2, v0, v1, v2, v3);
+                    mma_bf16_16816(oacc[2 * nd2], pa, v0, v1);
+                    mma_bf16_16816(oacc[2 * nd2 + 1], pa, v2, v3);
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty[stage]);
+            }
+        }
+        if (__syncthreads_or(failed)) {
+            // A bounded wait ran out: let the copies in flight land; the partial is empty.
+            if (tid == kConsumers * 32)
+                for (int k = max(0, ntile - kAttStages); k < ntile; ++k)
+                    mbar_wait(&full[(phase_base + k) % kAttStages], ((phase_base + k) / kAttStages) & 1, p.err);
+            __syncthreads();
+            m0 = m1 = -INFINITY;
+            l0 = l1 = 0.f;
+#pragma unroll
+            for (int k = 0; k < 16; ++k) oacc[k][0] = oacc[k][1] = oacc[k][2] = oacc[k][3] = 0.f;
+        }
+        if (warp < kConsumers) {
+            l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
+            l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+            l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
+            l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+            const int h0 = warp * 16 + gq, h1 = h0 + 8;
+            const int64_t part = (int64_t)t * p.nsplit + split;
+            if (c == 0) {
+                p.pml[part * kH + h0] = make_float2(m0, l0);
+                p.pml[part * kH + h1] = make_float2(m1, l1);
+            }
+            float* o0 = p.po + (part * kH + h0) * kD;
+            float* o1 = p.po + (part * kH + h1) * kD;
+#pragma unroll
+            for (int nd = 0; nd < 16; ++nd) {
+                *reinterpret_cast<float2*>(o0 + nd * 8 + 2 * c) = make_float2(oacc[nd][0], oacc[nd][1]);
+                *reinterpret_cast<float2*>(o1 + nd * 8 + 2 * c) = make_float2(oacc[nd][2], oacc[nd][3]);
+            }
+        }
+        phase_base += ntile;
+        __syncthreads();
+    }
+}
+
+// Phase 6: merge the splits of each (query, head) in split order.  Thread
+// (g, d) sums splits g, g+4, ... for dims 2d, 2d+1; the four partial sums are
+// then added in a fixed order.
+__device__ void phase_merge(const StepParams& p, uint8_t* smem, uint32_t* scratch)
+{
+    float* part = reinterpret_cast<float*>(smem);   // [4][128] partial sums + [4] denominators
+    const int items = p.T * kH;
+    const int grp = threadIdx.x >> 6, d2 = threadIdx.x & 63;
+    for (int r = 0;; ++r) {
+        const int i = item_of(r);
+        if (i >= items) break;
+        const int t = i / kH, h = i % kH;
+        const float2* ml = p.pml + (int64_t)t * p.nsplit * kH + h;
+        // running max over all splits (each thread reads a quarter, then combine)
+        float M = -INFINITY;
+        for (int s = grp; s < p.nsplit; s += 4) M = fmaxf(M, __ldcg(ml + (int64_t)s * kH).x);
+        if (d2 == 0) scratch[grp] = __float_as_uint(M);
+        __syncthreads();
+        M = fmaxf(fmaxf(__uint_as_float(scratch[0]), __uint_as_float(scratch[1])),
+                  fmaxf(__uint_as_float(scratch[2]), __uint_as_float(scratch[3])));
+        float sink = -INFINITY;
+        if (p.sink != nullptr) {
+            sink = p.sink[h] * kLog2e;
+            M = fmaxf(M, sink);
+        }
+        float den = 0.f, ax = 0.f, ay = 0.f;
+#pragma unroll 4
+        for (int s = grp; s < p.nsplit; s += 4) {
+            const float2 v = __ldcg(ml + (int64_t)s * kH);
+            if (v.x == -INFINITY) continue;
+            const float w = exp2f(v.x - M);
+            den += w * v.y;
+            const float2 o = __ldcg(reinterpret_cast<const float2*>(
+                p.po + (((int64_t)t * p.nsplit + s) * kH + h) * kD + 2 * d2));
+            ax += w * o.x;
+            ay += w * o.y;
+        }
+        part[grp * kD + 2 * d2] = ax;
+        part[grp * kD + 2 * d2 + 1] = ay;
+        if (d2 == 0) part[4 * kD + grp] = den;
+        __syncthreads();
+        if (grp == 0) {
+            float dd = (p.sink != nullptr && M != -INFINITY) ? exp2f(sink - M) : 0.f;
+            float x = 0.f, y = 0.f;
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+                dd += part[4 * kD + g];
+                x += part[g * kD + 2 * d2];
+                y += part[g * kD + 2 * d2 + 1];
+            }
+            const float inv = dd > 0.f ? 1.0f / dd : 0.f;
+            *reinterpret_cast<uint32_t*>(p.out + ((int64_t)t * kH + h) * kD + 2 * d2) = pack_bf16(x * inv, y * inv);
+        }
+        __syncthreads();
+    }
+}
+
+// ==================================================================================
+template <bool FP8>
+__global__ void __launch_bounds__(kThreads, 1)
+    step_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap smap, const StepParams p)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kBarOffset);
+    __shared__ uint32_t scratch[64];
+    __shared__ uint32_t res[3];
+    __shared__ int ok_s;
+
+    GridBarrier gb{p.bar_ctrl, p.err, gridDim.x};
+
+    if (threadIdx.x == 0) {
+        mbar_init(bars + 24, 1);
+        mbar_init(bars + 25, 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    // Stamps (when tracing): 0 start, 1 indexer done, 2-3 histogram, 4-5 extract,
+    // 6-7 emit, 8-9 attention, 10-11 merge (even: phase starts after its barrier).
+    bool ok = true;
+    stamp(p, 0);
+    if (p.trace != nullptr && threadIdx.x == 0) p.trace[(int64_t)blockIdx.x * kTraceSlots + 28] = clock64();
+    if (p.phases & kPhaseIndex) {
+        phase_index<FP8>(kmap, smap, p, smem, bars, scratch);
+    } else if (p.phases & kPhaseRanges) {
+        phase_ranges(p, scratch);
+    }
+    stamp(p, 1);
+    if (p.phases & kPhaseTopk) {
+        ok = gb.sync(&ok_s);
+        stamp(p, 2);
+        if (ok) phase_hist(p, smem, bars + 24, scratch);
+        stamp(p, 3);
+        ok = gb.sync(&ok_s) && ok;
+        stamp(p, 4);
+        if (ok) phase_extract(p, smem, res, scratch);
+        stamp(p, 5);
+        ok = gb.sync(&ok_s) && ok;
+        stamp(p, 6);
+        if (ok) phase_emit(p, smem, bars + 25, res, scratch);
+        stamp(p, 7);
+    }
+    if (p.phases & kPhaseAttend) {
+        if (p.phases & (kPhaseIndex | kPhaseTopk)) ok = gb.sync(&ok_s) && ok;
+        stamp(p, 8);
+        if (ok) phase_attend(p, smem, bars);
+        stamp(p, 9);
+        ok = gb.sync(&ok_s) && ok;
+        stamp(p, 10);
+        if (ok) phase_merge(p, smem, scratch);
+        stamp(p, 11);
+    }
+    if (p.trace != nullptr && threadIdx.x == 0) {
+        p.trace[(int64_t)blockIdx.x * kTraceSlots + 29] = clock64();
+        stamp(p, 30);
+    }
+}
+
+bool g_configured[64][2] = {};
+
+}  // namespace
+
+int step_smem_bytes() { return kStepSmem; }
+
+cudaError_t launch_step(const CUtensorMap* kmap, const CUtensorMap* smap, const StepParams& p, bool fp8,
+                        cudaStream_t s)
+{
+    int dev = 0;
+    cudaGetDevice(&dev);
+    auto kern = fp8 ? step_kernel<true> : step_kernel<false>;
+    if (dev >= 0 && dev < 64 && !g_configured[dev][fp8]) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kStepSmem);
+        if (e != cudaSuccess) return e;
+        g_configured[dev][fp8] = true;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(p.grid, 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = kStepSmem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, *kmap, *smap, p);
+}
+
+int step_max_blocks(bool fp8)
+{
+    int dev = 0, sms = 0, n = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    auto kern = fp8 ? step_kernel<true> : step_kernel<false>;
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kStepSmem);
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, kThreads, kStepSmem) != cudaSuccess || n < 1) n = 1;
+    cudaGetLastError();
+    return sms * (n > 1 ? 1 : n);   // one block per SM
+}
+
+}  // namespace dsa

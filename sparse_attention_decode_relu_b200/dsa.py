@@ -74,6 +74,10 @@ def lib():
             L.dsa_status_str.argtypes = [st]
             L.dsa_last_error.restype = ctypes.c_char_p
             L.dsa_launch_count.restype = ctypes.c_uint64
+            L.dsa_set_step_trace.restype = None
+            L.dsa_set_step_trace.argtypes = [P]
+            L.dsa_step_grid.restype = ctypes.c_int32
+            L.dsa_step_grid.argtypes = [ctypes.c_int32]
             L.dsa_set_stage_events.restype = None
             L.dsa_set_stage_events.argtypes = [ctypes.POINTER(ctypes.c_void_p), ctypes.c_int32]
             _lib = L
@@ -193,6 +197,16 @@ def dsa_device_status(stream=None):
 
 def dsa_launch_count() -> int:
     return int(lib().dsa_launch_count())
+
+
+def dsa_set_step_trace(buf: Optional[torch.Tensor]):
+    """Record per-block phase-boundary timestamps into buf (int64 CUDA tensor of
+    dsa_step_grid(...) * 32 entries) on the following calls; None disables."""
+    lib().dsa_set_step_trace(None if buf is None else buf.data_ptr())
+
+
+def dsa_step_grid(fp8_keys: bool = False) -> int:
+    return int(lib().dsa_step_grid(1 if fp8_keys else 0))
 
 
 def dsa_set_stage_events(events: Optional[Sequence[torch.cuda.Event]]):
