@@ -28,6 +28,7 @@ import sys
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
+SPIN_CYCLES = 200_000   # ~0.1 ms of GPU-side spin before each timed region
 sys.path.insert(0, ROOT)
 
 import numpy as np  # noqa: E402
@@ -255,12 +256,15 @@ def main():
     dsa.dsa_set_step_trace(None)
 
     def timed_step():
-        """Cold L2, then one graph replay of the whole step, timed by events."""
+        """Cold L2, then one graph replay of the whole step, timed by events.  A
+        short GPU-side spin ahead of the first event keeps the host's graph
+        submission out of the timed region (the GPU never waits for the host)."""
         flush_l2()
         s0 = torch.cuda.Event(enable_timing=True)
         s1 = torch.cuda.Event(enable_timing=True)
+        stream.wait_stream(torch.cuda.current_stream())   # the flush (and trace reset) come first
         with torch.cuda.stream(stream):
-            stream.wait_stream(torch.cuda.current_stream())
+            torch.cuda._sleep(SPIN_CYCLES)
             s0.record(stream)
             graph.replay()
             s1.record(stream)

@@ -101,11 +101,20 @@ typedef struct {
  *                                  query t in ascending order, then -1 padding
  * All device base addresses must be 16-byte aligned. */
 
-/* Bytes of workspace dsa_decode_ws needs for these sizes (0 if they are invalid). */
+/* Bytes of workspace dsa_decode_ws needs for these sizes (0 if they are invalid).
+ * Workspace contract (dsa_decode_ws, dsa_topk_from_scores, dsa_sparse_attn): the
+ * caller owns the memory; its first DSA_WS_CTRL_BYTES bytes are grid-barrier
+ * control words that must be zero before the workspace's first use (one
+ * cudaMemsetAsync when it is created); every call leaves them zero again, so
+ * later calls need no reset.  A launch that finds them non-zero flags
+ * DSA_ERR_DEVICE (bit 8 of the error word).  One workspace serves one call at a
+ * time: calls that may overlap on the GPU need separate workspaces. */
+#define DSA_WS_CTRL_BYTES 256
 DSA_API size_t dsa_workspace_bytes(int32_t T, int64_t L, int32_t topk);
 
 /* The whole step: indexer scan, causal top-k, sparse attention.  Takes its
- * workspace stream-ordered (cudaMallocAsync / cudaFreeAsync on `stream`), so it
+ * workspace stream-ordered (cudaMallocAsync, a zeroing of its control words,
+ * cudaFreeAsync, all on `stream`), so it
  * must not be captured into a CUDA graph on a device without memory-pool
  * support; use dsa_decode_ws for graphs. */
 DSA_API dsa_status_t dsa_decode(const dsa_tensor_t *q, const dsa_tensor_t *q_idx, const dsa_tensor_t *w_idx,

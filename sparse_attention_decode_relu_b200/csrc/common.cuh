@@ -16,6 +16,7 @@ enum : uint32_t {
     ERR_WAIT_TIMEOUT = 1u << 0,   // a bounded mbarrier wait ran out
     ERR_BAD_INDEX = 1u << 1,      // a selected index outside [0, pos[t]]
     ERR_TOPK_STATE = 1u << 2,     // top-k bookkeeping inconsistent (bad input scores)
+    ERR_WORKSPACE_STATE = 1u << 3,  // workspace control words were not zero at launch
 };
 
 // Every spin on an mbarrier gives up after this many SM clocks (~1 s).

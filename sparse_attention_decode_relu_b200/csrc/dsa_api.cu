@@ -204,7 +204,7 @@ Layout layout(int T, int64_t L, bool with_scores = true, bool with_attn = true)
         off += ru256(bytes);
         return at;
     };
-    l.ctrl = take(kBarCtrlBytes + 128);
+    l.ctrl = take(kWsCtrlBytes);
     l.hist = take(sizeof(uint32_t) * (size_t)T * kHistBins + sizeof(uint32_t) * kMaxT);
     l.list_n = l.hist + sizeof(uint32_t) * (size_t)T * kHistBins;
     l.zero_bytes = sizeof(uint32_t) * ((size_t)T * kHistBins + kMaxT);
@@ -329,11 +329,9 @@ dsa_status_t launch(const CUtensorMap& map, const CUtensorMap& smap, StepParams&
                     const Layout& l, cudaStream_t stream)
 {
     cudaError_t e;
-    if (p.phases & (kPhaseTopk | kPhaseAttend)) {   // grid barriers are used: start the counter at zero
-        p.bar_ctrl = at<uint32_t>(ws, l.ctrl);
-        if ((e = cudaMemsetAsync(p.bar_ctrl, 0, sizeof(uint32_t), stream)) != cudaSuccess)
-            return cuda_fail(e, "barrier reset");
-    }
+    // Grid barriers are used: their control words are zero from the workspace's
+    // creation on, and every launch leaves them zero.
+    if (p.phases & (kPhaseTopk | kPhaseAttend)) p.bar_ctrl = at<uint32_t>(ws, l.ctrl);
     p.trace = t_trace;
     if ((e = launch_step(&map, &smap, p, fp8, stream)) != cudaSuccess) return cuda_fail(e, "step launch");
     g_launches += 1;
@@ -373,7 +371,7 @@ dsa_status_t check_decode_args(const dsa_tensor_t* q, const dsa_tensor_t* q_idx,
 // counts and the candidate lists (about 16.4 MB per device, held until the
 // process exits).
 constexpr int64_t kNoAllocMaxL = 262144;
-constexpr size_t kNoAllocBytes = ru256(kBarCtrlBytes + 128) + ru256(sizeof(uint32_t) * ((size_t)kMaxT * kHistBins + kMaxT)) +
+constexpr size_t kNoAllocBytes = ru256(kWsCtrlBytes) + ru256(sizeof(uint32_t) * ((size_t)kMaxT * kHistBins + kMaxT)) +
                                  ru256(sizeof(uint2) * (size_t)kMaxGrid * kMaxT) +
                                  ru256(sizeof(uint32_t) * (size_t)kMaxT * kMaxChunksStep) + ru256(sizeof(uint32_t) * 4 * kMaxT) +
                                  ru256(sizeof(uint2) * (size_t)kMaxT * ((kNoAllocMaxL + 63) / 64 * 64));
@@ -493,6 +491,11 @@ dsa_status_t dsa_decode(const dsa_tensor_t* q, const dsa_tensor_t* q_idx, const 
     void* ws = nullptr;
     cudaError_t e = cudaMallocAsync(&ws, bytes, stream);
     if (e != cudaSuccess) return cuda_fail(e, "cudaMallocAsync(workspace)");
+    e = cudaMemsetAsync(ws, 0, kWsCtrlBytes, stream);
+    if (e != cudaSuccess) {
+        cudaFreeAsync(ws, stream);
+        return cuda_fail(e, "workspace control reset");
+    }
     st = dsa_decode_ws(q, q_idx, w_idx, k_idx_cache, kv_cache, pos, topk, out, sel_idx, stream_, ws, bytes);
     e = cudaFreeAsync(ws, stream);
     if (st == DSA_OK && e != cudaSuccess) return cuda_fail(e, "cudaFreeAsync(workspace)");
@@ -633,7 +636,8 @@ dsa_status_t dsa_device_status(dsa_stream_t stream_)
         const uint32_t zero = 0;
         e = cudaMemcpyToSymbol(g_err_word, &zero, sizeof zero);
         if (e != cudaSuccess) return cuda_fail(e, "clear device error word");
-        return fail(DSA_ERR_DEVICE, "device error word 0x%x (1: wait timeout, 2: bad selected index, 4: top-k state)",
+        return fail(DSA_ERR_DEVICE, "device error word 0x%x (1: wait timeout, 2: bad selected index, 4: top-k state, "
+                    "8: workspace control words not zero at launch)",
                     word);
     }
     return DSA_OK;

@@ -21,7 +21,8 @@ constexpr int kMaxChunksStep = 1024;        // top-k chunks per query (<= grid)
 constexpr int kMaxGrid = 1024;              // blocks of the step kernel
 constexpr int kMaxAttnItems = 512;          // (query, split) attention work items
 constexpr int kTraceSlots = 32;             // phase-boundary stamps per block
-constexpr int kBarCtrlBytes = 128;          // grid barrier arrival counter
+constexpr int kBarCtrlBytes = 128;          // grid barrier arrival counter (its own line)
+constexpr int kWsCtrlBytes = kBarCtrlBytes + 128;  // + the exit counter: workspace bytes [0, 256)
 
 // Phases of the step kernel.
 enum : int {

@@ -59,25 +59,52 @@ __device__ __forceinline__ void st_release(uint32_t* p, uint32_t v)
 // arrival counter only grows during a launch (it is zero at launch): barrier k
 // ends when it reaches k * gridDim.x.  Each block adds 1 with release semantics
 // and polls with acquire loads, giving up (error bit, false) after
-// kWaitLimitCycles.
+// kWaitLimitCycles.  The launch leaves the counter at zero again (see
+// GridBarrier::enter / barrier_exit), so consecutive launches need no reset node.
+// Control words: the arrival count at word 0, the exit count on the next
+// 128-byte line.
+constexpr int kExitWord = 32;
+
 struct GridBarrier {
     uint32_t* count;
     uint32_t* err;
     uint32_t next;     // count value that ends the next barrier
+    uint32_t c0 = 0, x0 = 0;   // (thread 0) both words as this block first saw them
+    bool bad = false;          // (thread 0) they were not zero at launch
+
+    // Thread 0 reads the control words at kernel entry; they are checked at the
+    // first barrier, so the loads overlap the first phase.
+    __device__ void enter()
+    {
+        if (threadIdx.x == 0) {
+            c0 = *reinterpret_cast<volatile uint32_t*>(count);
+            x0 = *reinterpret_cast<volatile uint32_t*>(count + kExitWord);
+        }
+    }
 
     __device__ bool sync(int* ok_s)
     {
         __syncthreads();
         if (threadIdx.x == 0) {
-            const uint32_t target = next;
-            bool ok = true;
-            asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(count) : "memory");
-            const long long t0 = clock64();
-            while (ld_acquire(count) < target) {
-                if (clock64() - t0 > kWaitLimitCycles) {
-                    atomicOr(err, ERR_WAIT_TIMEOUT);
-                    ok = false;
-                    break;
+            // Before its first arrival a block can see at most gridDim.x - 1
+            // arrivals and no exit (nobody passes the first barrier without it);
+            // anything else means the words were not zero at launch.  Such a
+            // block flags it and takes no part in the barriers.
+            if (next == gridDim.x && (x0 != 0u || c0 >= gridDim.x)) {
+                bad = true;
+                atomicOr(err, ERR_WORKSPACE_STATE);
+            }
+            bool ok = !bad;
+            if (ok) {
+                const uint32_t target = next;
+                asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(count) : "memory");
+                const long long t0 = clock64();
+                while (ld_acquire(count) < target) {
+                    if (clock64() - t0 > kWaitLimitCycles) {
+                        atomicOr(err, ERR_WAIT_TIMEOUT);
+                        ok = false;
+                        break;
+                    }
                 }
             }
             *ok_s = ok ? 1 : 0;
@@ -87,6 +114,21 @@ struct GridBarrier {
         return *ok_s != 0;
     }
 };
+
+__device__ __forceinline__ void barrier_exit(const StepParams& p)
+{
+    if (threadIdx.x == 0) {
+        uint32_t old;
+        asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;"
+                     : "=r"(old)
+                     : "l"(p.bar_ctrl + kExitWord)
+                     : "memory");
+        if (old == gridDim.x - 1u) {
+            p.bar_ctrl[0] = 0u;
+            p.bar_ctrl[kExitWord] = 0u;
+        }
+    }
+}
 
 // Phase-boundary timestamp (when the caller asked for a trace).
 __device__ __forceinline__ void stamp(const StepParams& p, int slot)
@@ -1194,6 +1236,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Stamps (when tracing): 0 start, 1 indexer done, 2-3 histogram, 4-5 extract,
     // 6-7 emit, 8-9 attention, 10-11 merge (even: phase starts after its barrier).
     bool ok = true;
+    if (p.bar_ctrl != nullptr) gb.enter();
     stamp(p, 0);
     if (p.trace != nullptr && threadIdx.x == 0) p.trace[(int64_t)blockIdx.x * kTraceSlots + 28] = clock64();
     if (p.phases & kPhaseIndex) {
@@ -1226,6 +1269,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ok) phase_merge(p, smem, scratch);
         stamp(p, 11);
     }
+    if (p.bar_ctrl != nullptr) barrier_exit(p);
     if (p.trace != nullptr && threadIdx.x == 0) {
         p.trace[(int64_t)blockIdx.x * kTraceSlots + 29] = clock64();
         stamp(p, 30);

@@ -20,6 +20,7 @@ from . import build as _build
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_DEVICE = 0, 1, 2, 3, 4
 BF16, FP8_E4M3, F32, I32 = 0, 1, 2, 3
+WS_CTRL_BYTES = 256   # DSA_WS_CTRL_BYTES: leading workspace bytes that must be zero before first use
 
 _lock = threading.Lock()
 _lib = None
@@ -222,7 +223,9 @@ def workspace(T: int, L: int, topk: int, device=None) -> torch.Tensor:
     n = dsa_workspace_bytes(T, L, topk)
     if n == 0:
         raise DsaError(ERR_INVALID_ARG, "invalid sizes for a workspace")
-    return torch.empty(n, dtype=torch.uint8, device=device or "cuda")
+    ws = torch.empty(n, dtype=torch.uint8, device=device or "cuda")
+    ws[:WS_CTRL_BYTES].zero_()   # grid-barrier control words start at zero; calls keep them so
+    return ws
 
 
 def decode(q, q_idx, w_idx, k_idx_cache, kv_cache, pos, topk=2048, *, k_scale=None, ws=None, stream=None):

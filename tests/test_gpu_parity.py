@@ -277,3 +277,23 @@ def test_verify_1m_integer_twin_selection():
     dsa.dsa_topk_from_scores(s, w.L, w.pos, w.topk, sel, dsa.workspace(w.T, w.L, w.topk))
     dsa.dsa_device_status()
     assert np.array_equal(sel.cpu().numpy(), oracle.topk(os_, w.pos, w.topk))
+
+
+def test_workspace_control_words_left_zero_and_checked():
+    """Each launch leaves the workspace's grid-barrier control words at zero, so a
+    workspace needs zeroing only once; a launch that finds them non-zero reports
+    it (device error word) and skips the work that depends on the barrier."""
+    w = synth.config("tiny_decode")
+    d = dsa.to_device(w)
+    ws = dsa.workspace(w.T, w.L, w.topk)
+    ref_o, ref_s = gpu_decode(w, d, ws=ws)
+    assert int(ws[: dsa.WS_CTRL_BYTES].count_nonzero()) == 0
+    ws[:4].view(torch.int32).fill_(1 << 16)       # an arrival count no launch can start from
+    out, sel = dsa.decode(d["q"], d["q_idx"], d["w_idx"], d["k_idx"], d["kv"], d["pos"], w.topk,
+                          k_scale=d["k_scale"], ws=ws)
+    with pytest.raises(dsa.DsaError) as e:
+        dsa.dsa_device_status()
+    assert e.value.status == dsa.ERR_DEVICE and "0x8" in str(e.value)
+    ws[: dsa.WS_CTRL_BYTES].zero_()
+    o2, s2 = gpu_decode(w, d, ws=ws)
+    assert np.array_equal(s2, ref_s) and np.array_equal(o2, ref_o)
