@@ -40,6 +40,32 @@ METRIC = "µs per DSA decode/verify step and achieved HBM GB/s (% of B200 peak) 
 KEY_BYTES = {"bf16": 128, "fp8": 68}
 
 
+def kernel_sources_sha256():
+    """sha256 over the sorted file names and contents of the CUDA sources."""
+    import hashlib
+    d = os.path.join(ROOT, "sparse_attention_decode_relu_b200", "csrc")
+    h = hashlib.sha256()
+    for f in sorted(os.listdir(d)):
+        h.update(f.encode())
+        with open(os.path.join(d, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def profiled_traffic(workload):
+    """DRAM bytes per step-kernel launch from the committed ncu capture of this
+    workload, or None when there is none or the kernel sources changed since."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            rec = json.load(f)["step_kernel"]
+    except (OSError, KeyError, ValueError):
+        return None
+    if rec.get("source_sha256") != kernel_sources_sha256():
+        return None
+    wl = rec.get("per_workload", {}).get(workload)
+    return None if wl is None else wl["dram_bytes_read"] + wl["dram_bytes_write"]
+
+
 def peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -350,7 +376,7 @@ def main():
     peak, which = peaks()
     achieved = ab["step"] / (ms * 1e-3) / 1e9
     roof = {"kernel": "step_kernel", "bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-            "frac": round(achieved / peak, 4), "peak_source": which, "traffic": None,
+            "frac": round(achieved / peak, 4), "peak_source": which, "traffic": profiled_traffic(w.name),
             "algorithmic_bytes": ab["step"]}
 
     line = {
