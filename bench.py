@@ -308,10 +308,10 @@ def main():
         spans["kernel"] = (t[:, 30].max() - t[:, 0].min()) / 1e3
         spans["sm_mhz_in_kernel"] = float((t[0, 29] - t[0, 28]) / max(1, t[0, 30] - t[0, 0]) * 1e3)
         spans["start_skew"] = (t[:, 0].max() - t[:, 0].min()) / 1e3
-        fast = t[:, 12] > 0   # blocks that ran the top-k emission's single-block path
+        fast = t[:, 15] > 0   # blocks that took the list-driven emission
         if fast.any():
-            for name, a, b in (("emit_cut", 6, 12), ("emit_list", 12, 13), ("emit_tau", 13, 14),
-                               ("emit_ties", 14, 15), ("emit_out", 15, 7)):
+            for name, a, b in (("emit_load", 6, 12), ("emit_subbin", 12, 13), ("emit_listpass", 13, 14),
+                               ("emit_select", 14, 15), ("emit_out", 15, 7)):
                 spans[name] = (t[fast, b] - t[fast, a]).max() / 1e3
         return spans
 

@@ -39,7 +39,8 @@ constexpr int kRowBytes = 2048;
 constexpr int kPitch = 2064;              // bank-conflict-free ldmatrix rows
 constexpr int kDataBytes = kAttStages * kTileRows * kPitch + kAttStages * kTileRows * 4 + kMaxRowsPerSplit * 4;
 constexpr int kBarOffset = (kDataBytes + 127) / 128 * 128;
-constexpr int kStepSmem = 1024 + kBarOffset + 256;
+constexpr int kBarSlots = 64;             // mbarriers (8 bytes each) after the data region
+constexpr int kStepSmem = 1024 + kBarOffset + kBarSlots * 8;
 static_assert(kIdxStages * 16384 + 16384 + kMaxT * kHI * kDI * 2 + kMaxT * kHI * 4 + kIdxStages * kKeyTile * 4 <=
                   kDataBytes, "indexer buffers fit the data region");
 
@@ -48,11 +49,6 @@ __device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p)
     uint32_t v;
     asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
-}
-
-__device__ __forceinline__ void st_release(uint32_t* p, uint32_t v)
-{
-    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
 // Grid-wide barrier among the co-resident blocks of a cooperative launch.  The
@@ -200,6 +196,24 @@ __device__ __forceinline__ void block_minmax(uint32_t& lo, uint32_t& hi, uint32_
     __syncthreads();
 }
 
+// Append the values x of the lanes with `take` set to v[*count ..] (one shared
+// atomic per warp; entries past cap are counted but not stored).  Every lane of
+// the warp must call it.
+template <typename V>
+__device__ __forceinline__ void warp_append(bool take, V x, V* v, uint32_t* count, uint32_t cap)
+{
+    const int lane = threadIdx.x & 31;
+    const uint32_t bal = __ballot_sync(0xffffffffu, take);
+    if (!bal) return;
+    uint32_t base = 0;
+    if (lane == 0) base = atomicAdd(count, static_cast<uint32_t>(__popc(bal)));
+    base = __shfl_sync(0xffffffffu, base, 0);
+    if (take) {
+        const uint32_t at = base + __popc(bal & ((1u << lane) - 1u));
+        if (at < cap) v[at] = x;
+    }
+}
+
 // Right shift that maps the key range [lo, hi] onto at most 4096 bins.
 __device__ __forceinline__ int range_shift(uint32_t lo, uint32_t hi)
 {
@@ -210,7 +224,7 @@ __device__ __forceinline__ int range_shift(uint32_t lo, uint32_t hi)
 // Highest key of the bin that starts at `start` (bins of width 2^shift), clamped to hi.
 __device__ __forceinline__ uint32_t bin_top(uint32_t start, int shift, uint32_t hi)
 {
-    const uint32_t width = (1u << shift) - 1u;   // shift <= 20
+    const uint32_t width = (1u << shift) - 1u;   // shift <= 24
     return (start > 0xFFFFFFFFu - width) ? hi : min(hi, start + width);
 }
 
@@ -468,11 +482,65 @@ __device__ void phase_ranges(const StepParams& p, uint32_t* scratch)
 
 // ==================================================================================
 // Phases 2-4: causal top-k by radix select over the query's own key range.
-// Work items are (query t, chunk c): positions [c*S, min((c+1)*S, n_t)).  A chunk
-// that fits is bulk-copied into shared memory once (phase 2) and stays there for
-// phase 3; longer chunks are streamed with several vector loads in flight.
+// Work items are (query t, chunk c): positions [c*S, min((c+1)*S, n_t)); a block
+// has at most one.  A chunk that fits is bulk-copied into shared memory once
+// (phase 2) and stays there for phase 3; a longer one streams through a ring
+// of bulk-copied tiles in both phases.
 // ==================================================================================
-constexpr int kChunkSmem = 40960;        // scores of one chunk kept in shared memory
+constexpr int kChunkSmem = 32768;        // scores of one chunk kept in shared memory (128 KiB)
+constexpr int kStreamStages = 8;         // ring of score tiles for longer chunks
+constexpr int kStreamTile = 4096;        // scores per tile (16 KiB)
+constexpr int kStreamBar = 32;           // first of the ring's mbarriers
+constexpr int kStageCap = 8192;          // candidates phase 3 stages in shared memory before a flush
+static_assert(kStreamStages * kStreamTile <= kChunkSmem, "the ring fits the chunk region");
+static_assert(kChunkSmem * 4 + kStageCap * 8 <= kDataBytes, "chunk + candidate staging fit");
+static_assert(kChunkSmem * 4 + kHistBins * 4 <= kDataBytes, "chunk + histogram fit");
+static_assert(kStreamBar + kStreamStages <= kBarSlots, "ring mbarriers fit");
+
+// Streams row[s0, s1) through the ring: for tile j, f(tile, a, c) runs on all
+// threads with tile[0, c) = the scores of positions a .. a + c - 1.  `seq`
+// counts the tiles this block has streamed so far (it keeps each stage's
+// mbarrier parity in step across calls).  False if a wait ran out (error bit
+// set; the copies still in flight are waited for before returning).
+template <typename F>
+__device__ bool stream_scores(const float* row, int s0, int s1, float* ring, uint64_t* full, uint32_t& seq,
+                              uint32_t* err, F f)
+{
+    const int ntiles = s1 > s0 ? (s1 - s0 + kStreamTile - 1) / kStreamTile : 0;
+    auto issue = [&](int j) {
+        const int a = s0 + j * kStreamTile;
+        const int c = min(kStreamTile, s1 - a);
+        const uint32_t bytes = static_cast<uint32_t>((c + 3) & ~3) * 4u;   // rows have a stride of 4k scores
+        const uint32_t st = (seq + j) % kStreamStages;
+        mbar_arrive_expect_tx(&full[st], bytes);
+        bulk_g2s(ring + st * kStreamTile, row + a, bytes, &full[st]);
+    };
+    fence_proxy_async_smem();   // earlier generic writes to the ring region come first
+    __syncthreads();
+    if (threadIdx.x == 0)
+        for (int j = 0; j < min(ntiles, kStreamStages); ++j) issue(j);
+    int j = 0;
+    bool ok = true;
+    for (; j < ntiles; ++j) {
+        const uint32_t g = seq + j, st = g % kStreamStages;
+        if (!__syncthreads_and(mbar_wait(&full[st], (g / kStreamStages) & 1u, err))) {
+            ok = false;
+            break;
+        }
+        const int a = s0 + j * kStreamTile;
+        f(ring + st * kStreamTile, a, min(kStreamTile, s1 - a));
+        __syncthreads();
+        if (threadIdx.x == 0 && j + kStreamStages < ntiles) issue(j + kStreamStages);
+    }
+    if (!ok && threadIdx.x == 0)   // drain what is still in flight (bounded waits)
+        for (int k = j; k < min(ntiles, j + kStreamStages); ++k) {
+            const uint32_t g = seq + k;
+            mbar_wait(&full[g % kStreamStages], (g / kStreamStages) & 1u, err);
+        }
+    seq += ntiles;
+    __syncthreads();
+    return ok;
+}
 
 struct Item {
     int t, c, s0, s1, n;
@@ -506,22 +574,11 @@ __device__ void query_range(const StepParams& p, int t, uint32_t& lo, uint32_t& 
     block_minmax(lo, hi, scratch);
 }
 
-// The chunk's keys: from shared memory (after phase 2 put them there) or global.
-struct ChunkKeys {
-    const uint32_t* smem;   // keys of positions [s0, s1) or nullptr
-    const float* row;       // scores of the query
-    int s0;
-    __device__ __forceinline__ uint32_t operator()(int s) const
-    {
-        return smem ? smem[s - s0] : score_key(__ldcg(row + s));
-    }
-};
-
-__device__ void phase_hist(const StepParams& p, uint8_t* smem, uint64_t* bar, uint32_t* scratch)
+__device__ void phase_hist(const StepParams& p, uint8_t* smem, uint64_t* bar, uint64_t* ring_full, uint32_t& seq,
+                           uint32_t* scratch)
 {
-    uint32_t* keys = reinterpret_cast<uint32_t*>(smem);                       // [kChunkSmem]
+    uint32_t* keys = reinterpret_cast<uint32_t*>(smem);                       // [kChunkSmem] (or the ring)
     uint32_t* h = keys + kChunkSmem;                                          // [kHistBins]
-    int uses = 0;   // phases of `bar` completed so far
     for (int r = 0;; ++r) {
         const int i = item_of(r);
         if (i >= p.T * p.nchunk) break;
@@ -535,6 +592,8 @@ __device__ void phase_hist(const StepParams& p, uint8_t* smem, uint64_t* bar, ui
         const int c4 = (cnt + 3) & ~3;   // rows have a stride that is a multiple of 4 scores
         const bool in_smem = r == 0 && c4 <= kChunkSmem;   // a block's first item stays in smem
         if (in_smem) {
+            fence_proxy_async_smem();
+            __syncthreads();
             if (threadIdx.x == 0) {
                 mbar_arrive_expect_tx(bar, static_cast<uint32_t>(c4) * 4u);
                 bulk_g2s(keys, row + it.s0, static_cast<uint32_t>(c4) * 4u, bar);
@@ -542,8 +601,7 @@ __device__ void phase_hist(const StepParams& p, uint8_t* smem, uint64_t* bar, ui
         }
         for (int b = threadIdx.x; b < kHistBins; b += kThreads) h[b] = 0u;
         if (in_smem) {
-            const bool ok = mbar_wait(bar, uses & 1, p.err);
-            ++uses;
+            const bool ok = mbar_wait(bar, 0, p.err);   // this barrier completes once per launch
             if (!__syncthreads_and(ok)) return;
             for (int j = threadIdx.x; j < cnt; j += kThreads) {
                 const uint32_t k = score_key(__uint_as_float(keys[j]));
@@ -551,29 +609,12 @@ __device__ void phase_hist(const StepParams& p, uint8_t* smem, uint64_t* bar, ui
                 atomicAdd(&h[(k - lo) >> shift], 1u);
             }
         } else {
-            __syncthreads();
-            for (int s = it.s0 + threadIdx.x * 4; s < it.s1; s += kThreads * 16) {
-                float4 v[4];
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int su = s + u * kThreads * 4;
-                    v[u] = su + 4 <= it.s1 ? __ldcg(reinterpret_cast<const float4*>(row + su))
-                                           : make_float4(0.f, 0.f, 0.f, 0.f);
-                }
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int su = s + u * kThreads * 4;
-                    if (su + 4 <= it.s1) {
-                        atomicAdd(&h[(score_key(v[u].x) - lo) >> shift], 1u);
-                        atomicAdd(&h[(score_key(v[u].y) - lo) >> shift], 1u);
-                        atomicAdd(&h[(score_key(v[u].z) - lo) >> shift], 1u);
-                        atomicAdd(&h[(score_key(v[u].w) - lo) >> shift], 1u);
-                    } else {
-                        for (int j = su; j < it.s1 && j < su + 4; ++j)
-                            atomicAdd(&h[(score_key(__ldcg(row + j)) - lo) >> shift], 1u);
-                    }
-                }
-            }
+            const bool ok = stream_scores(row, it.s0, it.s1, reinterpret_cast<float*>(keys), ring_full, seq, p.err,
+                                          [&](const float* tile, int, int c) {
+                                              for (int j = threadIdx.x; j < c; j += kThreads)
+                                                  atomicAdd(&h[(score_key(tile[j]) - lo) >> shift], 1u);
+                                          });
+            if (!ok) return;
         }
         __syncthreads();
         uint32_t* gh = p.hist + (int64_t)it.t * kHistBins;
@@ -611,11 +652,16 @@ __device__ Cut query_cut(const StepParams& p, int t, uint32_t* res, uint32_t* sc
 
 // Phase 3: every key >= cut (the threshold bin and above) goes to the query's
 // candidate list with its position; keys above the bin are also counted per
-// chunk.  One atomic per block reserves the block's slots of the list.
-__device__ void phase_extract(const StepParams& p, uint8_t* smem, uint32_t* res, uint32_t* scratch)
+// chunk.  Candidates are staged in shared memory (one shared atomic per warp
+// step) and flushed to the list with one global atomic per flush; the list's
+// order is not used by phase 4.
+__device__ void phase_extract(const StepParams& p, uint8_t* smem, uint64_t* ring_full, uint32_t& seq, uint32_t* res,
+                              uint32_t* scratch)
 {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const uint32_t* keys = reinterpret_cast<const uint32_t*>(smem);
+    const uint32_t* keys = reinterpret_cast<const uint32_t*>(smem);             // resident chunk (phase 2)
+    uint2* stage = reinterpret_cast<uint2*>(smem + kChunkSmem * 4);              // [kStageCap]
+    __shared__ uint32_t nstage;
+    __shared__ uint32_t flush_at;
     for (int r = 0;; ++r) {
         const int i = item_of(r);
         if (i >= p.T * p.nchunk) break;
@@ -624,57 +670,59 @@ __device__ void phase_extract(const StepParams& p, uint8_t* smem, uint32_t* res,
         const Cut cu = query_cut(p, it.t, res, scratch);
         if (it.c == 0 && threadIdx.x == 0)
             reinterpret_cast<uint4*>(p.cuts)[it.t] = make_uint4(cu.cut, cu.ctop, cu.above, 0u);
-        const int cnt = it.s1 - it.s0;
-        const ChunkKeys key{r == 0 && ((cnt + 3) & ~3) <= kChunkSmem ? keys : nullptr, p.scores + (int64_t)it.t * p.ld,
-                            it.s0};
-        // Pass 1: candidates per warp (warp w owns lanes w*32.. of every 256-position step).
-        uint32_t above = 0, wcnt = 0;
-        for (int base = it.s0; base < it.s1; base += kThreads * 4) {
-            uint32_t k[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int s = base + u * kThreads + threadIdx.x;
-                k[u] = s < it.s1 ? key(s) : 0u;
-            }
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int s = base + u * kThreads + threadIdx.x;
-                above += s < it.s1 && k[u] > cu.ctop;
-                wcnt += __popc(__ballot_sync(0xffffffffu, s < it.s1 && k[u] >= cu.cut));
-            }
-        }
-        if (lane == 0) scratch[warp] = wcnt;
+        if (threadIdx.x == 0) nstage = 0;
         __syncthreads();
-        if (threadIdx.x == 0) {
-            uint32_t tot = 0;
-            for (int w = 0; w < kWarps; ++w) {
-                const uint32_t x = scratch[w];
-                scratch[w] = tot;
-                tot += x;
-            }
-            scratch[kWarps] = tot ? atomicAdd(p.list_n + it.t, tot) : 0u;
-        }
-        __syncthreads();
-        uint32_t at = scratch[kWarps] + scratch[warp];
-        __syncthreads();
-        // Pass 2: the same positions in the same order, written at the reserved slots.
         uint2* list = p.list + (int64_t)it.t * p.ld;
-        for (int base = it.s0; base < it.s1; base += kThreads * 4) {
-            uint32_t k[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int s = base + u * kThreads + threadIdx.x;
-                k[u] = s < it.s1 ? key(s) : 0u;
+        // Move the staged candidates to the list (all threads; nstage is uniform here).
+        auto flush = [&]() {
+            const uint32_t n = min(nstage, static_cast<uint32_t>(kStageCap));
+            if (n == 0) return;
+            if (threadIdx.x == 0) flush_at = atomicAdd(p.list_n + it.t, n);
+            __syncthreads();
+            const uint32_t at = flush_at;
+            for (uint32_t j = threadIdx.x; j < n; j += kThreads) list[at + j] = stage[j];
+            __syncthreads();
+            if (threadIdx.x == 0) nstage = 0;
+            __syncthreads();
+        };
+        uint32_t above = 0;
+        uint32_t* hist2 = p.hist2 + (int64_t)it.t * kHistBins;
+        const int shift2 = range_shift(cu.cut, cu.ctop);
+        // Keys of positions a .. a + c - 1 (at most kStreamTile of them): stage the
+        // candidates; the keys inside the threshold bin also go to the second-level
+        // histogram (4096 sub-bins over [cut, ctop]).
+        auto take = [&](auto key_at, int a, int c) {
+            if (nstage + static_cast<uint32_t>(c) > static_cast<uint32_t>(kStageCap)) flush();
+            for (int j0 = 0; j0 < c; j0 += kThreads) {
+                const int j = j0 + threadIdx.x;
+                const uint32_t k = j < c ? key_at(j) : 0u;
+                above += j < c && k > cu.ctop;
+                const bool inb = j < c && k >= cu.cut && k <= cu.ctop;
+                if (__any_sync(0xffffffffu, inb)) {   // one atomic per distinct sub-bin of the warp
+                    const uint32_t sb = inb ? (k - cu.cut) >> shift2 : 0xFFFFFFFFu;
+                    const uint32_t peers = __match_any_sync(0xffffffffu, sb);
+                    if (inb && __ffs(peers) - 1 == (threadIdx.x & 31)) atomicAdd(hist2 + sb, __popc(peers));
+                }
+                warp_append(j < c && k >= cu.cut, make_uint2(k, static_cast<uint32_t>(a + j)), stage, &nstage,
+                             kStageCap);
             }
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int s = base + u * kThreads + threadIdx.x;
-                const bool c = s < it.s1 && k[u] >= cu.cut;
-                const uint32_t bal = __ballot_sync(0xffffffffu, c);
-                if (c) list[at + __popc(bal & ((1u << lane) - 1u))] = make_uint2(k[u], static_cast<uint32_t>(s));
-                at += __popc(bal);
+        };
+        const int cnt = it.s1 - it.s0;
+        bool ok = true;
+        if (r == 0 && ((cnt + 3) & ~3) <= kChunkSmem) {
+            for (int a = 0; a < cnt; a += kStreamTile) {
+                take([&](int j) { return keys[a + j]; }, it.s0 + a, min(kStreamTile, cnt - a));
+                __syncthreads();
             }
+        } else {
+            const float* row = p.scores + (int64_t)it.t * p.ld;
+            ok = stream_scores(row, it.s0, it.s1, reinterpret_cast<float*>(smem), ring_full, seq, p.err,
+                               [&](const float* tile, int a, int c) {
+                                   take([&](int j) { return score_key(tile[j]); }, a, c);
+                               });
         }
+        if (!ok) return;
+        flush();
         above = block_sum(above, scratch);
         if (threadIdx.x == 0) p.above[(int64_t)it.t * kMaxChunksStep + it.c] = above;
     }
@@ -711,10 +759,51 @@ __device__ void radix_select(Get get, uint32_t n, uint32_t& lo, uint32_t& hi, ui
     }
 }
 
-// The need-th largest of the n values v[0..n) in shared memory (n <= kSmallSel):
-// each thread ranks its values against all of them.  Returns the value; `need`
-// becomes how many entries equal to it are to be taken.
-constexpr int kSmallSel = 64;
+// The need-th largest of the n values v[0..n) gathered in shared memory: radix
+// select with 256 bins over their own range [min, max] (no pass at all when the
+// values are equal).  Returns the value; `need` becomes how many entries equal
+// to it are to be taken.
+constexpr int kSmallBins = 256;
+
+__device__ uint32_t small_select(const uint32_t* v, uint32_t n, uint32_t& need, uint32_t* h, uint32_t* res,
+                                 uint32_t* scratch, uint32_t* err)
+{
+    uint32_t lo = 0xFFFFFFFFu, hi = 0u;
+    for (uint32_t j = threadIdx.x; j < n; j += kThreads) {
+        lo = min(lo, v[j]);
+        hi = max(hi, v[j]);
+    }
+    block_minmax(lo, hi, scratch);
+#pragma unroll 1
+    for (int pass = 0; pass < 4 && lo != hi; ++pass) {
+        const int bits = 32 - __clz(hi - lo);
+        const int shift = bits > 8 ? bits - 8 : 0;
+        h[threadIdx.x] = 0u;   // kSmallBins == kThreads
+        __syncthreads();
+        for (uint32_t j = threadIdx.x; j < n; j += kThreads) {
+            const uint32_t x = v[j];
+            if (x >= lo && x <= hi) atomicAdd(&h[(x - lo) >> shift], 1u);
+        }
+        __syncthreads();
+        find_from_top<kSmallBins>(h, need, res, scratch, false);
+        if (!res[2]) {
+            if (threadIdx.x == 0) atomicOr(err, ERR_TOPK_STATE);
+            res[0] = 0;
+            res[1] = 0;
+        }
+        const uint32_t nlo = lo + (res[0] << shift);
+        hi = bin_top(nlo, shift, hi);
+        lo = nlo;
+        need -= res[1];
+        __syncthreads();
+    }
+    return lo;
+}
+
+// The need-th largest of the n values v[0..n) in shared memory (n small): each
+// thread ranks its values against all of them, one step.  Returns the value;
+// `need` becomes how many entries equal to it are to be taken.
+constexpr int kRankSel = 64;
 
 __device__ uint32_t rank_select(const uint32_t* v, uint32_t n, uint32_t& need, uint32_t* res, uint32_t* err)
 {
@@ -737,172 +826,196 @@ __device__ uint32_t rank_select(const uint32_t* v, uint32_t n, uint32_t& need, u
         }
     }
     __syncthreads();
-    if (!res[2]) {
-        if (threadIdx.x == 0) atomicOr(err, ERR_TOPK_STATE);
-        __syncthreads();
-        return 0u;
+    uint32_t x = 0u;
+    if (res[2]) {
+        x = res[0];
+        need -= res[1];
+    } else if (threadIdx.x == 0) {
+        atomicOr(err, ERR_TOPK_STATE);
     }
-    const uint32_t x = res[0];
-    need -= res[1];
     __syncthreads();
     return x;
 }
 
-// Phase 4.  The common case: the query's candidate list (every key >= cut,
-// with its position) fits in shared memory and the context fits the bitmap.
-// Block (t, chunk 0) then finds tau and the tie cut among the candidates, marks
-// the selected positions in a bitmap and writes them in position order.
-// Otherwise every chunk block sweeps its positions in order.
-constexpr int kListSmem = 4096;          // candidates a block keeps in shared memory
-constexpr int kBitmapBits = 1 << 20;     // positions the ordered emission marks in shared memory
-static_assert(kListSmem * 8 + kHistBins * 4 + kBitmapBits / 8 + kSmallSel * 8 <= kDataBytes, "emit buffers fit");
-static_assert(kChunkSmem * 4 + kHistBins * 4 <= kDataBytes, "chunk buffers fit");
-
-__device__ void phase_emit(const StepParams& p, uint8_t* smem, uint64_t* bar, uint32_t* res, uint32_t* scratch)
+__device__ __forceinline__ uint32_t exact_select(uint32_t* v, uint32_t n, uint32_t& need, uint32_t* h, uint32_t* res,
+                                                 uint32_t* scratch, uint32_t* err)
 {
-    uint2* lst = reinterpret_cast<uint2*>(smem);                                  // [kListSmem]
-    uint32_t* h = reinterpret_cast<uint32_t*>(smem + kListSmem * 8);              // [kHistBins]
-    uint32_t* bitmap = h + kHistBins;                                             // [kBitmapBits / 32]
-    uint32_t* small = bitmap + kBitmapBits / 32;                                  // [2 * kSmallSel]
-    __shared__ uint32_t nsmall;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    int uses = 0;
+    return n <= static_cast<uint32_t>(kRankSel) ? rank_select(v, n, need, res, err)
+                                                : small_select(v, n, need, h, res, scratch, err);
+}
+
+// Phase 4: ordered emission, one item per (query t, chunk c) as in phases 2-3.
+// Every chunk block of a query derives the threshold tau and the tie cut itself:
+// the second-level histogram names the sub-bin [lo2, hi2] of the threshold bin
+// that holds tau; one pass over the candidate list marks the entries above the
+// sub-bin (all selected) and gathers the sub-bin's entries into shared memory,
+// where tau and the tie cut by position are found exactly.  The block marks the
+// selected positions of its own chunk in a bitmap, counts those before its
+// chunk, and writes its slice of the ascending output with coalesced stores.
+// Very long lists, sub-bins with more than kSubCap entries (heavy ties) and
+// very wide chunks take slower paths over the list and the scores.
+constexpr int kSubCap = 2048;            // sub-bin entries gathered in shared memory
+constexpr int kEmitListMax = 1 << 16;    // longer candidate lists: ordered sweep of the scores
+constexpr int kChunkWords = 16384;       // bitmap words of one chunk (2^19 positions)
+static_assert(kSubCap * 12 + kHistBins * 4 + kChunkWords * 4 + kMaxTopk * 4 <= kDataBytes, "emit buffers fit");
+static_assert(kSmallBins == kThreads, "one small-select bin per thread");
+
+__device__ void phase_emit(const StepParams& p, uint8_t* smem, uint32_t* res, uint32_t* scratch)
+{
+    uint2* sub = reinterpret_cast<uint2*>(smem);                                  // [kSubCap] (key, position)
+    uint32_t* vals = reinterpret_cast<uint32_t*>(sub + kSubCap);                 // [kSubCap]
+    uint32_t* h = vals + kSubCap;                                                 // [kHistBins]
+    uint32_t* bitmap = h + kHistBins;                                             // [kChunkWords]
+    int32_t* outs = reinterpret_cast<int32_t*>(bitmap + kChunkWords);            // [kMaxTopk]
+    __shared__ uint32_t nsub, nval;
+    const int tid = threadIdx.x;
     for (int r = 0;; ++r) {
         const int i = item_of(r);
         if (i >= p.T * p.nchunk) break;
         const Item it = topk_item(p, i);
         int32_t* sel = p.sel + (int64_t)it.t * p.sel_ld;
         if (it.n <= p.topk) {   // everything visible is selected
-            for (int s = it.s0 + threadIdx.x; s < it.s1; s += kThreads) sel[s] = s;
+            for (int s = it.s0 + tid; s < it.s1; s += kThreads) sel[s] = s;
             if (it.c == 0)
-                for (int j = it.n + threadIdx.x; j < p.topk; j += kThreads) sel[j] = -1;
+                for (int j = it.n + tid; j < p.topk; j += kThreads) sel[j] = -1;
             continue;
         }
+        if (it.s0 >= it.s1) continue;   // an empty chunk emits nothing
         const uint32_t m = __ldcg(p.list_n + it.t);
-        const bool fast = m <= static_cast<uint32_t>(kListSmem) && it.n <= kBitmapBits;
-        if (fast && it.c != 0) continue;
         const uint4 cq = __ldcg(reinterpret_cast<const uint4*>(p.cuts) + it.t);
         const Cut cu{cq.x, cq.y, cq.z};
         const uint2* glist = p.list + (int64_t)it.t * p.ld;
         stamp(p, 12);
-        if (fast) {
-            // The list in one bulk copy (8-byte entries; an odd count reads one spare entry).
-            const uint32_t bytes = ((m * 8u) + 15u) & ~15u;
-            if (threadIdx.x == 0) {
-                mbar_arrive_expect_tx(bar, bytes);
-                bulk_g2s(lst, glist, bytes, bar);
-            }
-            if (!__syncthreads_and(mbar_wait(bar, uses & 1, p.err))) return;
-            ++uses;
+
+        // The sub-bin of the threshold bin that holds tau.
+        uint32_t need = static_cast<uint32_t>(p.topk) - cu.above;
+        const int shift2 = range_shift(cu.cut, cu.ctop);
+        find_from_top<kHistBins>(p.hist2 + (int64_t)it.t * kHistBins, need, res, scratch, true);
+        uint32_t lo2 = cu.cut, hi2 = cu.ctop;
+        if (res[2]) {
+            lo2 = cu.cut + (res[0] << shift2);
+            hi2 = bin_top(lo2, shift2, cu.ctop);
+            need -= res[1];
+        } else if (tid == 0) {
+            atomicOr(p.err, ERR_TOPK_STATE);
         }
-        auto cand = [&](uint32_t j) -> uint2 { return fast ? lst[j] : __ldcg(glist + j); };
+        __syncthreads();
         stamp(p, 13);
 
-        // tau: keys above ctop are all taken; select among the keys in the bin.
-        uint32_t need = static_cast<uint32_t>(p.topk) - cu.above;
-        uint32_t tau;
-        if (threadIdx.x == 0) nsmall = 0;
-        __syncthreads();
-        if (fast) {   // gather the bin's keys (order does not matter for the rank of a value)
-            for (uint32_t j = threadIdx.x; j < m; j += kThreads) {
-                const uint32_t k = lst[j].x;
-                if (k <= cu.ctop) {
-                    const uint32_t at = atomicAdd(&nsmall, 1u);
-                    if (at < kSmallSel) small[at] = k;
+        const int span = it.s1 - it.s0;
+        const int R = ((span + 31) / 32 + kThreads - 1) / kThreads;   // bitmap words per thread
+        if (m <= static_cast<uint32_t>(kEmitListMax) && R * kThreads <= kChunkWords) {
+            // Bitmap of this chunk's selected positions, transposed: thread i owns
+            // the R consecutive words [i*R, (i+1)*R), its k-th word at k*256 + i.
+            auto mark = [&](uint32_t pos) -> uint32_t {   // 1 when pos precedes the chunk
+                const int q = static_cast<int>(pos);
+                if (q < it.s0) return 1u;
+                if (q < it.s1) {
+                    const uint32_t rel = static_cast<uint32_t>(q - it.s0), w = rel >> 5, owner = w / R;
+                    atomicOr(&bitmap[(w - owner * R) * kThreads + owner], 1u << (rel & 31));
                 }
-            }
-        }
-        __syncthreads();
-        if (fast && nsmall <= kSmallSel) {
-            tau = rank_select(small, nsmall, need, res, p.err);
-        } else {
-            uint32_t lo = cu.cut, hi = cu.ctop;
-            radix_select([&](uint32_t j) { return cand(j).x; }, m, lo, hi, need, h, res, scratch, p.err);
-            tau = lo;
-        }
-        const uint32_t rties = need;   // take every key > tau and the first rties keys == tau
-        stamp(p, 14);
-
-        if (fast) {
-            // Ties at tau: the rties lowest positions.  e = #(key == tau).
-            if (threadIdx.x == 0) nsmall = 0;
+                return 0u;
+            };
+            for (int w = tid; w < R * kThreads; w += kThreads) bitmap[w] = 0u;
+            if (tid == 0) nsub = 0;
             __syncthreads();
-            uint32_t e = 0;
-            for (uint32_t j = threadIdx.x; j < m; j += kThreads) {
-                const uint2 v = lst[j];
-                if (v.x == tau) {
-                    ++e;
-                    const uint32_t at = atomicAdd(&nsmall, 1u);
-                    if (at < kSmallSel) small[kSmallSel + at] = ~v.y;   // ~position: largest = lowest position
-                }
+            uint32_t before = 0;
+            for (uint32_t j0 = 0; j0 < m; j0 += kThreads) {
+                const uint32_t j = j0 + tid;
+                const uint2 v = j < m ? __ldcg(glist + j) : make_uint2(0u, 0u);
+                if (j < m && v.x > hi2) before += mark(v.y);
+                warp_append(j < m && v.x >= lo2 && v.x <= hi2, v, sub, &nsub, kSubCap);
             }
-            e = block_sum(e, scratch);
-            uint32_t pcut = 0xFFFFFFFFu;   // ties with position <= pcut are taken
-            if (rties < e) {
-                uint32_t need_p = rties;
-                if (e <= static_cast<uint32_t>(kSmallSel)) {
-                    pcut = ~rank_select(small + kSmallSel, e, need_p, res, p.err);
-                } else {
-                    uint32_t plo = 0xFFFFFFFFu, phi = 0u;
-                    for (uint32_t j = threadIdx.x; j < m; j += kThreads)
-                        if (lst[j].x == tau) {
-                            plo = min(plo, ~lst[j].y);
-                            phi = max(phi, ~lst[j].y);
-                        }
-                    block_minmax(plo, phi, scratch);
-                    radix_select([&](uint32_t j) { const uint2 v = lst[j]; return v.x == tau ? ~v.y : 0u; }, m, plo,
-                                 phi, need_p, h, res, scratch, p.err);
+            __syncthreads();
+            stamp(p, 14);
+            const uint32_t n2 = nsub;
+            uint32_t tau, pcut = 0xFFFFFFFFu;   // selected: key > tau, or key == tau and position <= pcut
+            if (n2 <= static_cast<uint32_t>(kSubCap)) {
+                for (uint32_t j = tid; j < n2; j += kThreads) vals[j] = sub[j].x;
+                if (tid == 0) nval = 0;
+                __syncthreads();
+                tau = exact_select(vals, n2, need, h, res, scratch, p.err);
+                const uint32_t rties = need;
+                for (uint32_t j0 = 0; j0 < n2; j0 += kThreads) {   // ~position of the ties: largest = lowest
+                    const uint32_t j = j0 + tid;
+                    const uint2 v = j < n2 ? sub[j] : make_uint2(0u, 0u);
+                    warp_append(j < n2 && v.x == tau, ~v.y, vals, &nval, kSubCap);
+                }
+                __syncthreads();
+                const uint32_t e = nval;
+                if (rties < e) pcut = ~exact_select(vals, e, need, h, res, scratch, p.err);
+                for (uint32_t j = tid; j < n2; j += kThreads) {
+                    const uint2 v = sub[j];
+                    if (v.x > tau || (v.x == tau && v.y <= pcut)) before += mark(v.y);
+                }
+            } else {
+                // Heavy ties: tau and the tie cut by radix select over the list itself.
+                uint32_t lo = lo2, hi = hi2;
+                radix_select([&](uint32_t j) { return __ldcg(glist + j).x; }, m, lo, hi, need, h, res, scratch,
+                             p.err);
+                tau = lo;
+                uint32_t e = 0, plo = 0xFFFFFFFFu, phi = 0u;
+                for (uint32_t j = tid; j < m; j += kThreads) {
+                    const uint2 v = __ldcg(glist + j);
+                    if (v.x == tau) {
+                        ++e;
+                        plo = min(plo, ~v.y);
+                        phi = max(phi, ~v.y);
+                    }
+                }
+                e = block_sum(e, scratch);
+                block_minmax(plo, phi, scratch);
+                if (need < e) {
+                    radix_select(
+                        [&](uint32_t j) {
+                            const uint2 v = __ldcg(glist + j);
+                            return v.x == tau ? ~v.y : 0u;
+                        },
+                        m, plo, phi, need, h, res, scratch, p.err);
                     pcut = ~plo;
                 }
+                for (uint32_t j = tid; j < m; j += kThreads) {
+                    const uint2 v = __ldcg(glist + j);
+                    if (v.x >= lo2 && v.x <= hi2 && (v.x > tau || (v.x == tau && v.y <= pcut))) before += mark(v.y);
+                }
             }
+            before = block_sum(before, scratch);   // also orders the marking before the count
             stamp(p, 15);
-            const int nwords = (it.n + 31) >> 5;
-            for (int w = threadIdx.x; w < nwords; w += kThreads) bitmap[w] = 0u;
-            __syncthreads();
-            for (uint32_t j = threadIdx.x; j < m; j += kThreads) {
-                const uint2 v = lst[j];
-                if (v.x > tau || (v.x == tau && v.y <= pcut)) atomicOr(&bitmap[v.y >> 5], 1u << (v.y & 31));
-            }
-            __syncthreads();
-            // Warp w owns words [w*per, (w+1)*per); lanes read consecutive words.
-            const int per = ((nwords + kWarps - 1) / kWarps + 31) / 32 * 32;
-            const int w0 = min(nwords, warp * per), w1 = min(nwords, w0 + per);
             uint32_t cnt = 0;
-            for (int w = w0 + lane; w < w1; w += 32) cnt += __popc(bitmap[w]);
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
-            if (lane == 0) scratch[32 + warp] = cnt;
-            __syncthreads();
-            uint32_t o = 0, total = 0;
-            for (int w = 0; w < kWarps; ++w) {
-                const uint32_t x = scratch[32 + w];
-                if (w < warp) o += x;
-                total += x;
-            }
-            for (int base = w0; base < w1; base += 32) {
-                const int w = base + lane;
-                uint32_t b = w < w1 ? bitmap[w] : 0u;
-                const uint32_t c = __popc(b);
-                const uint32_t incl = warp_incl_scan(c);
-                uint32_t oo = o + incl - c;
+            for (int k = 0; k < R; ++k) cnt += __popc(bitmap[k * kThreads + tid]);
+            uint32_t total;
+            uint32_t o = block_excl_scan(cnt, total, scratch);
+            for (int k = 0; k < R && cnt; ++k) {
+                uint32_t b = bitmap[k * kThreads + tid];
+                const int base = it.s0 + ((tid * R + k) << 5);
                 while (b) {
                     const int bit = __ffs(b) - 1;
                     b &= b - 1;
-                    if (oo < static_cast<uint32_t>(p.topk)) sel[oo] = (w << 5) + bit;
-                    ++oo;
+                    if (o < static_cast<uint32_t>(kMaxTopk)) outs[o] = base + bit;
+                    ++o;
+                    --cnt;
                 }
-                o += __shfl_sync(0xffffffffu, incl, 31);
             }
-            if (threadIdx.x == 0 && total != static_cast<uint32_t>(p.topk)) atomicOr(p.err, ERR_TOPK_STATE);
+            __syncthreads();
+            const uint32_t lim = before < static_cast<uint32_t>(p.topk) ? static_cast<uint32_t>(p.topk) - before : 0u;
+            for (uint32_t j = tid; j < total && j < lim && j < static_cast<uint32_t>(kMaxTopk); j += kThreads)
+                sel[before + j] = outs[j];
+            if (tid == 0 && (before + total > static_cast<uint32_t>(p.topk) ||
+                             (it.s1 == it.n && before + total != static_cast<uint32_t>(p.topk))))
+                atomicOr(p.err, ERR_TOPK_STATE);
             __syncthreads();
             continue;
         }
 
-        // Fallback: this chunk's output offset and tie rank from the candidates of
-        // earlier chunks, then an ordered sweep of the chunk.
+        // Long lists or wide chunks: tau by radix select over the list, then this
+        // chunk's output offset and tie rank from the candidates of earlier
+        // chunks, then an ordered sweep of the chunk's scores.
+        uint32_t lo = lo2, hi = hi2;
+        radix_select([&](uint32_t j) { return __ldcg(glist + j).x; }, m, lo, hi, need, h, res, scratch, p.err);
+        const uint32_t tau = lo, rties = need;
         uint32_t before_gt = 0, before_eq = 0;
-        for (uint32_t j = threadIdx.x; j < m; j += kThreads) {
-            const uint2 v = cand(j);
+        for (uint32_t j = tid; j < m; j += kThreads) {
+            const uint2 v = __ldcg(glist + j);
             if (static_cast<int>(v.y) < it.s0) {
                 before_gt += v.x > tau;
                 before_eq += v.x == tau;
@@ -914,7 +1027,7 @@ __device__ void phase_emit(const StepParams& p, uint8_t* smem, uint64_t* bar, ui
         uint32_t tie_rank = before_eq;
         const float* row = p.scores + (int64_t)it.t * p.ld;
         for (int base = it.s0; base < it.s1; base += kThreads * 4) {
-            const int s = base + threadIdx.x * 4;
+            const int s = base + tid * 4;
             uint32_t gtm = 0, eqm = 0;
 #pragma unroll
             for (int j = 0; j < 4; ++j)
@@ -1229,13 +1342,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (threadIdx.x == 0) {
         mbar_init(bars + 24, 1);
-        mbar_init(bars + 25, 1);
+        for (int s = 0; s < kStreamStages; ++s) mbar_init(bars + kStreamBar + s, 1);
         fence_mbar_init();
     }
     __syncthreads();
     // Stamps (when tracing): 0 start, 1 indexer done, 2-3 histogram, 4-5 extract,
     // 6-7 emit, 8-9 attention, 10-11 merge (even: phase starts after its barrier).
     bool ok = true;
+    uint32_t seq = 0;   // score tiles this block has streamed (phases 2-3)
     if (p.bar_ctrl != nullptr) gb.enter();
     stamp(p, 0);
     if (p.trace != nullptr && threadIdx.x == 0) p.trace[(int64_t)blockIdx.x * kTraceSlots + 28] = clock64();
@@ -1248,15 +1362,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (p.phases & kPhaseTopk) {
         ok = gb.sync(&ok_s);
         stamp(p, 2);
-        if (ok) phase_hist(p, smem, bars + 24, scratch);
+        if (ok) phase_hist(p, smem, bars + 24, bars + kStreamBar, seq, scratch);
         stamp(p, 3);
         ok = gb.sync(&ok_s) && ok;
         stamp(p, 4);
-        if (ok) phase_extract(p, smem, res, scratch);
+        if (ok) phase_extract(p, smem, bars + kStreamBar, seq, res, scratch);
         stamp(p, 5);
         ok = gb.sync(&ok_s) && ok;
         stamp(p, 6);
-        if (ok) phase_emit(p, smem, bars + 25, res, scratch);
+        if (ok) phase_emit(p, smem, res, scratch);
         stamp(p, 7);
     }
     if (p.phases & kPhaseAttend) {
