@@ -308,11 +308,10 @@ def main():
         spans["kernel"] = (t[:, 30].max() - t[:, 0].min()) / 1e3
         spans["sm_mhz_in_kernel"] = float((t[0, 29] - t[0, 28]) / max(1, t[0, 30] - t[0, 0]) * 1e3)
         spans["start_skew"] = (t[:, 0].max() - t[:, 0].min()) / 1e3
-        fast = t[:, 15] > 0   # blocks that took the list-driven emission
-        if fast.any():
-            for name, a, b in (("emit_load", 6, 12), ("emit_subbin", 12, 13), ("emit_listpass", 13, 14),
-                               ("emit_select", 14, 15), ("emit_out", 15, 7)):
-                spans[name] = (t[fast, b] - t[fast, a]).max() / 1e3
+        emitting = t[:, 13] > 0   # blocks that selected and compacted a chunk
+        if emitting.any():
+            for name, a, b in (("emit_load", 6, 12), ("emit_select", 12, 13), ("emit_out", 13, 7)):
+                spans[name] = (t[emitting, b] - t[emitting, a]).max() / 1e3
         return spans
 
     for _ in range(args.warmup):

@@ -151,7 +151,7 @@ DSA_API dsa_status_t dsa_topk_from_scores(const float *scores, int32_t T, int64_
  * capture or a real-time decode loop that forbids allocation after start-up,
  * or a host whose device memory is entirely owned by another allocator.  The
  * paper has no counterpart; this is an interface choice of this library.
- * Its scratch is a static device array of about 17.1 MB inside libdsa.so; every
+ * Its scratch is a static device array of about 17.0 MB inside libdsa.so; every
  * GPU that loads the library holds it until the process exits.
  *   - Limits: T <= 8 and L <= 262144 scores per query; larger L returns
  *     DSA_ERR_INVALID_ARG (say "exceeds the no-allocation scratch limit").

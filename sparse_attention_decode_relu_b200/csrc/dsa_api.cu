@@ -185,7 +185,7 @@ dsa_status_t check_sel(const dsa_tensor_t* sel, int T, int32_t topk)
 // and the attention splits' partial states.
 struct Layout {
     int64_t ld = 0;            // score / candidate row stride (elements)
-    size_t ctrl = 0, hist = 0, hist2 = 0, list_n = 0, zero_bytes = 0;
+    size_t ctrl = 0, hist = 0, list_n = 0, zero_bytes = 0;
     size_t mm = 0, above = 0, cuts = 0, scores = 0, list = 0, po = 0, pml = 0;
     size_t total = 0;
 };
@@ -205,10 +205,9 @@ Layout layout(int T, int64_t L, bool with_scores = true, bool with_attn = true)
         return at;
     };
     l.ctrl = take(kWsCtrlBytes);
-    l.hist = take(sizeof(uint32_t) * (2 * (size_t)T * kHistBins + kMaxT));
-    l.hist2 = l.hist + sizeof(uint32_t) * (size_t)T * kHistBins;
-    l.list_n = l.hist2 + sizeof(uint32_t) * (size_t)T * kHistBins;
-    l.zero_bytes = sizeof(uint32_t) * (2 * (size_t)T * kHistBins + kMaxT);
+    l.hist = take(sizeof(uint32_t) * ((size_t)T * kHistBins + kMaxT));
+    l.list_n = l.hist + sizeof(uint32_t) * (size_t)T * kHistBins;
+    l.zero_bytes = sizeof(uint32_t) * ((size_t)T * kHistBins + kMaxT);
     l.mm = take(sizeof(uint2) * (size_t)kMaxGrid * kMaxT);
     l.above = take(sizeof(uint32_t) * (size_t)kMaxT * kMaxChunksStep);
     l.cuts = take(sizeof(uint32_t) * 4 * kMaxT);
@@ -294,7 +293,6 @@ int grid_blocks(const DeviceInfo& dev, bool fp8)
 void topk_params(StepParams& p, void* ws, const Layout& l)
 {
     p.hist = at<uint32_t>(ws, l.hist);
-    p.hist2 = at<uint32_t>(ws, l.hist2);
     p.list_n = at<uint32_t>(ws, l.list_n);
     p.list = at<uint2>(ws, l.list);
     p.above = at<uint32_t>(ws, l.above);
@@ -370,10 +368,10 @@ dsa_status_t check_decode_args(const dsa_tensor_t* q, const dsa_tensor_t* q_idx,
 // Scratch for dsa_topk_from_scores_noalloc: a file-scope device array, so that
 // entry point never allocates.  Sized for T <= 8 queries and L <= 262144 scores
 // per query: barrier words, the top-k counters, per-block key ranges, per-chunk
-// counts and the candidate lists (about 17.1 MB per device, held until the
+// counts and the candidate lists (about 17.0 MB per device, held until the
 // process exits).
 constexpr int64_t kNoAllocMaxL = 262144;
-constexpr size_t kNoAllocBytes = ru256(kWsCtrlBytes) + ru256(sizeof(uint32_t) * (2 * (size_t)kMaxT * kHistBins + kMaxT)) +
+constexpr size_t kNoAllocBytes = ru256(kWsCtrlBytes) + ru256(sizeof(uint32_t) * ((size_t)kMaxT * kHistBins + kMaxT)) +
                                  ru256(sizeof(uint2) * (size_t)kMaxGrid * kMaxT) +
                                  ru256(sizeof(uint32_t) * (size_t)kMaxT * kMaxChunksStep) + ru256(sizeof(uint32_t) * 4 * kMaxT) +
                                  ru256(sizeof(uint2) * (size_t)kMaxT * ((kNoAllocMaxL + 63) / 64 * 64));

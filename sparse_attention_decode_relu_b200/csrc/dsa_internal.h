@@ -47,12 +47,11 @@ struct StepParams {
     uint2* mm;               // [grid][kMaxT] per-block (min, max) key of visible scores
     int32_t mm_slots;
     uint32_t* hist;          // [T][kHistBins]
-    uint32_t* hist2;         // [T][kHistBins] second level: the keys inside each query's threshold bin
     uint32_t* list_n;        // [kMaxT] candidates per query
     uint2* list;             // [T][ld] (key, position) candidates
-    uint32_t* above;         // [T][kMaxChunksStep]
+    uint32_t* above;         // [T][kMaxChunksStep] keys above the threshold bin, per chunk
     uint32_t* cuts;          // [kMaxT][4]: threshold bin (cut, ctop) and #keys above it, per query
-    uint32_t* zero;          // words phase 1 clears (hist, hist2, list_n)
+    uint32_t* zero;          // words phase 1 clears (hist, list_n)
     int32_t zero_words;
     int32_t chunk, nchunk;   // top-k work items: nchunk chunks of `chunk` positions per query
     int32_t* sel;            // [T][sel_ld]

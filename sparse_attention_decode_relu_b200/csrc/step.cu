@@ -228,10 +228,10 @@ __device__ __forceinline__ uint32_t bin_top(uint32_t start, int shift, uint32_t 
     return (start > 0xFFFFFFFFu - width) ? hi : min(hi, start + width);
 }
 
-// Bin b of an NB-bin histogram (h global or shared) holding the need-th largest
+// Bin b of an NB-bin histogram in shared memory holding the need-th largest
 // entry: #(bins > b) < need <= #(bins >= b).  res = {b, #(bins > b), found}.
 template <int NB>
-__device__ void find_from_top(const uint32_t* h, uint32_t need, uint32_t* res, uint32_t* scratch, bool global_h)
+__device__ void find_from_top(const uint32_t* h, uint32_t need, uint32_t* res, uint32_t* scratch)
 {
     constexpr int PER = NB / kThreads;
     const int top = NB - PER * threadIdx.x;   // thread 0 owns the highest bins
@@ -239,7 +239,7 @@ __device__ void find_from_top(const uint32_t* h, uint32_t need, uint32_t* res, u
     uint32_t sum = 0;
 #pragma unroll
     for (int i = 0; i < PER; ++i) {
-        cnt[i] = global_h ? __ldcg(h + top - 1 - i) : h[top - 1 - i];
+        cnt[i] = h[top - 1 - i];
         sum += cnt[i];
     }
     if (threadIdx.x == 0) res[2] = 0;
@@ -484,14 +484,18 @@ __device__ void phase_ranges(const StepParams& p, uint32_t* scratch)
 // Phases 2-4: causal top-k by radix select over the query's own key range.
 // Work items are (query t, chunk c): positions [c*S, min((c+1)*S, n_t)); a block
 // has at most one.  A chunk that fits is bulk-copied into shared memory once
-// (phase 2) and stays there for phase 3; a longer one streams through a ring
-// of bulk-copied tiles in both phases.
+// (phase 2) and stays there, as order-preserving keys, until phase 4; a longer
+// one streams through a ring of bulk-copied tiles in each phase.  Phase 3 lists
+// only the keys inside the threshold bin (few) and counts the keys above it per
+// chunk; from those, every chunk block finds the exact threshold and its own
+// offset in the output, then compacts its positions in order.
 // ==================================================================================
 constexpr int kChunkSmem = 32768;        // scores of one chunk kept in shared memory (128 KiB)
 constexpr int kStreamStages = 8;         // ring of score tiles for longer chunks
 constexpr int kStreamTile = 4096;        // scores per tile (16 KiB)
 constexpr int kStreamBar = 32;           // first of the ring's mbarriers
 constexpr int kStageCap = 8192;          // candidates phase 3 stages in shared memory before a flush
+constexpr int kWork = kChunkSmem * 4;    // shared-memory offset of the region after the chunk
 static_assert(kStreamStages * kStreamTile <= kChunkSmem, "the ring fits the chunk region");
 static_assert(kChunkSmem * 4 + kStageCap * 8 <= kDataBytes, "chunk + candidate staging fit");
 static_assert(kChunkSmem * 4 + kHistBins * 4 <= kDataBytes, "chunk + histogram fit");
@@ -574,11 +578,16 @@ __device__ void query_range(const StepParams& p, int t, uint32_t& lo, uint32_t& 
     block_minmax(lo, hi, scratch);
 }
 
+// Per query: threshold bin [cut, ctop] and #(keys > ctop).
+struct Cut {
+    uint32_t cut, ctop, above;
+};
+
 __device__ void phase_hist(const StepParams& p, uint8_t* smem, uint64_t* bar, uint64_t* ring_full, uint32_t& seq,
                            uint32_t* scratch)
 {
     uint32_t* keys = reinterpret_cast<uint32_t*>(smem);                       // [kChunkSmem] (or the ring)
-    uint32_t* h = keys + kChunkSmem;                                          // [kHistBins]
+    uint32_t* h = reinterpret_cast<uint32_t*>(smem + kWork);                  // [kHistBins]
     for (int r = 0;; ++r) {
         const int i = item_of(r);
         if (i >= p.T * p.nchunk) break;
@@ -624,50 +633,47 @@ __device__ void phase_hist(const StepParams& p, uint8_t* smem, uint64_t* bar, ui
     }
 }
 
-// Per query: threshold bin [cut, ctop] and #(keys > ctop), from the histogram.
-struct Cut {
-    uint32_t cut, ctop, above;
-};
-
-__device__ Cut query_cut(const StepParams& p, int t, uint32_t* res, uint32_t* scratch)
+// The threshold bin of query t from its histogram (read with coalesced loads
+// into h, shared memory).
+__device__ Cut query_cut(const StepParams& p, int t, uint32_t* h, uint32_t* res, uint32_t* scratch)
 {
     uint32_t lo, hi;
     query_range(p, t, lo, hi, scratch);
     const int shift = range_shift(lo, hi);
-    find_from_top<kHistBins>(p.hist + (int64_t)t * kHistBins, static_cast<uint32_t>(p.topk), res, scratch, true);
-    Cut cu;
-    if (!res[2]) {   // histogram and scores disagree: cannot happen for consistent input
-        if (threadIdx.x == 0) atomicOr(p.err, ERR_TOPK_STATE);
-        cu.cut = lo;
-        cu.ctop = hi;
-        cu.above = 0;
-    } else {
+    const uint32_t* gh = p.hist + (int64_t)t * kHistBins;
+    for (int b = threadIdx.x; b < kHistBins; b += kThreads) h[b] = __ldcg(gh + b);
+    __syncthreads();
+    find_from_top<kHistBins>(h, static_cast<uint32_t>(p.topk), res, scratch);
+    Cut cu{lo, hi, 0u};
+    if (res[2]) {
         cu.cut = lo + (res[0] << shift);
         cu.ctop = bin_top(cu.cut, shift, hi);
         cu.above = res[1];
+    } else if (threadIdx.x == 0) {   // histogram and scores disagree: cannot happen for consistent input
+        atomicOr(p.err, ERR_TOPK_STATE);
     }
     __syncthreads();
     return cu;
 }
 
 // Phase 3: every key >= cut (the threshold bin and above) goes to the query's
-// candidate list with its position; keys above the bin are also counted per
-// chunk.  Candidates are staged in shared memory (one shared atomic per warp
-// step) and flushed to the list with one global atomic per flush; the list's
-// order is not used by phase 4.
+// candidate list with its position; the keys above the bin are also counted per
+// chunk.
+// Candidates are staged in shared memory (one shared atomic per warp step) and
+// flushed to the list with one global atomic per flush; nothing downstream
+// depends on the list's order.
 __device__ void phase_extract(const StepParams& p, uint8_t* smem, uint64_t* ring_full, uint32_t& seq, uint32_t* res,
                               uint32_t* scratch)
 {
     const uint32_t* keys = reinterpret_cast<const uint32_t*>(smem);             // resident chunk (phase 2)
-    uint2* stage = reinterpret_cast<uint2*>(smem + kChunkSmem * 4);              // [kStageCap]
-    __shared__ uint32_t nstage;
-    __shared__ uint32_t flush_at;
+    uint2* stage = reinterpret_cast<uint2*>(smem + kWork);                       // [kStageCap]
+    __shared__ uint32_t nstage, flush_at;
     for (int r = 0;; ++r) {
         const int i = item_of(r);
         if (i >= p.T * p.nchunk) break;
         const Item it = topk_item(p, i);
         if (it.n <= p.topk) continue;
-        const Cut cu = query_cut(p, it.t, res, scratch);
+        const Cut cu = query_cut(p, it.t, reinterpret_cast<uint32_t*>(smem + kWork), res, scratch);
         if (it.c == 0 && threadIdx.x == 0)
             reinterpret_cast<uint4*>(p.cuts)[it.t] = make_uint4(cu.cut, cu.ctop, cu.above, 0u);
         if (threadIdx.x == 0) nstage = 0;
@@ -686,43 +692,35 @@ __device__ void phase_extract(const StepParams& p, uint8_t* smem, uint64_t* ring
             __syncthreads();
         };
         uint32_t above = 0;
-        uint32_t* hist2 = p.hist2 + (int64_t)it.t * kHistBins;
-        const int shift2 = range_shift(cu.cut, cu.ctop);
-        // Keys of positions a .. a + c - 1 (at most kStreamTile of them): stage the
-        // candidates; the keys inside the threshold bin also go to the second-level
-        // histogram (4096 sub-bins over [cut, ctop]).
+        const int cnt = it.s1 - it.s0;
+        const bool resident = r == 0 && ((cnt + 3) & ~3) <= kChunkSmem;
+        // Keys of positions a .. a + c - 1 (at most kStreamTile of them).
         auto take = [&](auto key_at, int a, int c) {
             if (nstage + static_cast<uint32_t>(c) > static_cast<uint32_t>(kStageCap)) flush();
             for (int j0 = 0; j0 < c; j0 += kThreads) {
                 const int j = j0 + threadIdx.x;
                 const uint32_t k = j < c ? key_at(j) : 0u;
                 above += j < c && k > cu.ctop;
-                const bool inb = j < c && k >= cu.cut && k <= cu.ctop;
-                if (__any_sync(0xffffffffu, inb)) {   // one atomic per distinct sub-bin of the warp
-                    const uint32_t sb = inb ? (k - cu.cut) >> shift2 : 0xFFFFFFFFu;
-                    const uint32_t peers = __match_any_sync(0xffffffffu, sb);
-                    if (inb && __ffs(peers) - 1 == (threadIdx.x & 31)) atomicAdd(hist2 + sb, __popc(peers));
-                }
                 warp_append(j < c && k >= cu.cut, make_uint2(k, static_cast<uint32_t>(a + j)), stage, &nstage,
-                             kStageCap);
+                            kStageCap);
             }
         };
-        const int cnt = it.s1 - it.s0;
-        bool ok = true;
-        if (r == 0 && ((cnt + 3) & ~3) <= kChunkSmem) {
-            for (int a = 0; a < cnt; a += kStreamTile) {
-                take([&](int j) { return keys[a + j]; }, it.s0 + a, min(kStreamTile, cnt - a));
-                __syncthreads();
+        if (cnt > 0) {
+            if (resident) {
+                for (int a = 0; a < cnt; a += kStreamTile) {
+                    take([&](int j) { return keys[a + j]; }, it.s0 + a, min(kStreamTile, cnt - a));
+                    __syncthreads();
+                }
+            } else {
+                const float* row = p.scores + (int64_t)it.t * p.ld;
+                const bool ok = stream_scores(row, it.s0, it.s1, reinterpret_cast<float*>(smem), ring_full, seq,
+                                              p.err, [&](const float* tile, int a, int c) {
+                                                  take([&](int j) { return score_key(tile[j]); }, a, c);
+                                              });
+                if (!ok) return;
             }
-        } else {
-            const float* row = p.scores + (int64_t)it.t * p.ld;
-            ok = stream_scores(row, it.s0, it.s1, reinterpret_cast<float*>(smem), ring_full, seq, p.err,
-                               [&](const float* tile, int a, int c) {
-                                   take([&](int j) { return score_key(tile[j]); }, a, c);
-                               });
+            flush();
         }
-        if (!ok) return;
-        flush();
         above = block_sum(above, scratch);
         if (threadIdx.x == 0) p.above[(int64_t)it.t * kMaxChunksStep + it.c] = above;
     }
@@ -745,7 +743,7 @@ __device__ void radix_select(Get get, uint32_t n, uint32_t& lo, uint32_t& hi, ui
             if (k >= lo && k <= hi) atomicAdd(&h[(k - lo) >> shift], 1u);
         }
         __syncthreads();
-        find_from_top<kHistBins>(h, need, res, scratch, false);
+        find_from_top<kHistBins>(h, need, res, scratch);
         if (!res[2]) {
             if (threadIdx.x == 0) atomicOr(err, ERR_TOPK_STATE);
             res[0] = 0;
@@ -785,7 +783,7 @@ __device__ uint32_t small_select(const uint32_t* v, uint32_t n, uint32_t& need, 
             if (x >= lo && x <= hi) atomicAdd(&h[(x - lo) >> shift], 1u);
         }
         __syncthreads();
-        find_from_top<kSmallBins>(h, need, res, scratch, false);
+        find_from_top<kSmallBins>(h, need, res, scratch);
         if (!res[2]) {
             if (threadIdx.x == 0) atomicOr(err, ERR_TOPK_STATE);
             res[0] = 0;
@@ -844,31 +842,31 @@ __device__ __forceinline__ uint32_t exact_select(uint32_t* v, uint32_t n, uint32
                                                 : small_select(v, n, need, h, res, scratch, err);
 }
 
-// Phase 4: ordered emission, one item per (query t, chunk c) as in phases 2-3.
-// Every chunk block of a query derives the threshold tau and the tie cut itself:
-// the second-level histogram names the sub-bin [lo2, hi2] of the threshold bin
-// that holds tau; one pass over the candidate list marks the entries above the
-// sub-bin (all selected) and gathers the sub-bin's entries into shared memory,
-// where tau and the tie cut by position are found exactly.  The block marks the
-// selected positions of its own chunk in a bitmap, counts those before its
-// chunk, and writes its slice of the ascending output with coalesced stores.
-// Very long lists, sub-bins with more than kSubCap entries (heavy ties) and
-// very wide chunks take slower paths over the list and the scores.
-constexpr int kSubCap = 2048;            // sub-bin entries gathered in shared memory
-constexpr int kEmitListMax = 1 << 16;    // longer candidate lists: ordered sweep of the scores
-constexpr int kChunkWords = 16384;       // bitmap words of one chunk (2^19 positions)
-static_assert(kSubCap * 12 + kHistBins * 4 + kChunkWords * 4 + kMaxTopk * 4 <= kDataBytes, "emit buffers fit");
-static_assert(kSmallBins == kThreads, "one small-select bin per thread");
+// Phase 4: ordered emission, one item per (query t, chunk c).  The block reads
+// the query's threshold-bin candidates (few) and the per-chunk counts of keys
+// above the bin, finds the exact threshold tau (the topk-th largest key) and the
+// tie cut pcut (keys equal to tau are taken at positions <= pcut), and so its
+// first output slot; then it marks the selected positions of its chunk (all in
+// the list) in a bitmap and writes them in ascending order.  More than kInCap
+// candidates (heavy ties) take radix selects over the list in global memory and
+// an ordered compaction of the chunk's keys: each warp owns 512 consecutive
+// positions of a tile, counts them with ballots and writes them after the warps
+// before it.
+constexpr int kInCap = 3584;             // candidates gathered in shared memory
+constexpr int kChunkWords = 16384;       // bitmap words of a streamed chunk (2^19 positions)
+static_assert(kChunkWords * 4 <= kWork, "the bitmap fits below the list");
+static_assert(kWork + kHistBins * 4 + kInCap * 12 <= kDataBytes, "emission buffers fit");
 
-__device__ void phase_emit(const StepParams& p, uint8_t* smem, uint32_t* res, uint32_t* scratch)
+__device__ void phase_emit(const StepParams& p, uint8_t* smem, uint64_t* ring_full, uint32_t& seq, uint32_t* res,
+                           uint32_t* scratch)
 {
-    uint2* sub = reinterpret_cast<uint2*>(smem);                                  // [kSubCap] (key, position)
-    uint32_t* vals = reinterpret_cast<uint32_t*>(sub + kSubCap);                 // [kSubCap]
-    uint32_t* h = vals + kSubCap;                                                 // [kHistBins]
-    uint32_t* bitmap = h + kHistBins;                                             // [kChunkWords]
-    int32_t* outs = reinterpret_cast<int32_t*>(bitmap + kChunkWords);            // [kMaxTopk]
-    __shared__ uint32_t nsub, nval;
-    const int tid = threadIdx.x;
+    const uint32_t* keys = reinterpret_cast<const uint32_t*>(smem);   // resident chunk (phase 2)
+    uint32_t* h = reinterpret_cast<uint32_t*>(smem + kWork);          // [kHistBins] select bins
+    uint2* in = reinterpret_cast<uint2*>(h + kHistBins);              // [kInCap] (key, position)
+    uint32_t* vals = reinterpret_cast<uint32_t*>(in + kInCap);        // [kInCap]
+    __shared__ uint32_t nval;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    constexpr int kSeg = kStreamTile / kWarps;                         // positions per warp and tile
     for (int r = 0;; ++r) {
         const int i = item_of(r);
         if (i >= p.T * p.nchunk) break;
@@ -880,180 +878,160 @@ __device__ void phase_emit(const StepParams& p, uint8_t* smem, uint32_t* res, ui
                 for (int j = it.n + tid; j < p.topk; j += kThreads) sel[j] = -1;
             continue;
         }
-        if (it.s0 >= it.s1) continue;   // an empty chunk emits nothing
+        const int cnt = it.s1 - it.s0;
+        if (cnt <= 0) continue;
         const uint32_t m = __ldcg(p.list_n + it.t);
         const uint4 cq = __ldcg(reinterpret_cast<const uint4*>(p.cuts) + it.t);
         const Cut cu{cq.x, cq.y, cq.z};
         const uint2* glist = p.list + (int64_t)it.t * p.ld;
+        const uint32_t* above = p.above + (int64_t)it.t * kMaxChunksStep;
+        // keys above the bin in the chunks before this one
+        uint32_t before = 0;
+        for (int c = tid; c < it.c; c += kThreads) before += __ldcg(above + c);
+        const bool fits = m <= static_cast<uint32_t>(kInCap);
+        if (fits)
+            for (uint32_t j = tid; j < m; j += kThreads) in[j] = __ldcg(glist + j);
+        if (tid == 0) nval = 0;
+        __syncthreads();
+        uint32_t nin = 0;   // keys inside the threshold bin, gathered in vals
+        if (fits) {
+            for (uint32_t j0 = 0; j0 < m; j0 += kThreads) {
+                const uint32_t j = j0 + tid;
+                const uint32_t k = j < m ? in[j].x : 0xFFFFFFFFu;
+                warp_append(j < m && k <= cu.ctop, k, vals, &nval, kInCap);
+            }
+            __syncthreads();
+            nin = nval;
+            __syncthreads();
+            if (tid == 0) nval = 0;
+        }
         stamp(p, 12);
 
-        // The sub-bin of the threshold bin that holds tau.
         uint32_t need = static_cast<uint32_t>(p.topk) - cu.above;
-        const int shift2 = range_shift(cu.cut, cu.ctop);
-        find_from_top<kHistBins>(p.hist2 + (int64_t)it.t * kHistBins, need, res, scratch, true);
-        uint32_t lo2 = cu.cut, hi2 = cu.ctop;
-        if (res[2]) {
-            lo2 = cu.cut + (res[0] << shift2);
-            hi2 = bin_top(lo2, shift2, cu.ctop);
-            need -= res[1];
-        } else if (tid == 0) {
-            atomicOr(p.err, ERR_TOPK_STATE);
+        uint32_t tau, pcut = 0xFFFFFFFFu;   // selected: key > tau, or key == tau and position <= pcut
+        if (fits) {
+            tau = exact_select(vals, nin, need, h, res, scratch, p.err);   // ends with a barrier
+            const uint32_t rties = need;
+            for (uint32_t j0 = 0; j0 < m; j0 += kThreads) {   // ~position of the ties: largest = lowest
+                const uint32_t j = j0 + tid;
+                const uint2 v = j < m ? in[j] : make_uint2(0u, 0u);
+                warp_append(j < m && v.x == tau, ~v.y, vals, &nval, kInCap);
+            }
+            __syncthreads();
+            const uint32_t e = nval;
+            if (rties < e) pcut = ~exact_select(vals, e, need, h, res, scratch, p.err);
+            for (uint32_t j = tid; j < m; j += kThreads) {
+                const uint2 v = in[j];
+                before += static_cast<int>(v.y) < it.s0 && v.x <= cu.ctop && (v.x > tau || (v.x == tau && v.y <= pcut));
+            }
+        } else {
+            uint32_t lo = cu.cut, hi = cu.ctop;
+            radix_select([&](uint32_t j) { return __ldcg(glist + j).x; }, m, lo, hi, need, h, res, scratch, p.err);
+            tau = lo;   // (keys above ctop in the list fall outside [lo, hi] and are not counted)
+            uint32_t e = 0, plo = 0xFFFFFFFFu, phi = 0u;
+            for (uint32_t j = tid; j < m; j += kThreads) {
+                const uint2 v = __ldcg(glist + j);
+                if (v.x == tau) {
+                    ++e;
+                    plo = min(plo, ~v.y);
+                    phi = max(phi, ~v.y);
+                }
+            }
+            e = block_sum(e, scratch);
+            block_minmax(plo, phi, scratch);
+            if (need < e) {
+                radix_select(
+                    [&](uint32_t j) {
+                        const uint2 v = __ldcg(glist + j);
+                        return v.x == tau ? ~v.y : 0u;
+                    },
+                    m, plo, phi, need, h, res, scratch, p.err);
+                pcut = ~plo;
+            }
+            for (uint32_t j = tid; j < m; j += kThreads) {
+                const uint2 v = __ldcg(glist + j);
+                before += static_cast<int>(v.y) < it.s0 && v.x <= cu.ctop && (v.x > tau || (v.x == tau && v.y <= pcut));
+            }
         }
-        __syncthreads();
+        uint32_t out = block_sum(before, scratch);   // this chunk's first output slot
         stamp(p, 13);
-
-        const int span = it.s1 - it.s0;
-        const int R = ((span + 31) / 32 + kThreads - 1) / kThreads;   // bitmap words per thread
-        if (m <= static_cast<uint32_t>(kEmitListMax) && R * kThreads <= kChunkWords) {
-            // Bitmap of this chunk's selected positions, transposed: thread i owns
-            // the R consecutive words [i*R, (i+1)*R), its k-th word at k*256 + i.
-            auto mark = [&](uint32_t pos) -> uint32_t {   // 1 when pos precedes the chunk
-                const int q = static_cast<int>(pos);
-                if (q < it.s0) return 1u;
-                if (q < it.s1) {
+        const uint32_t topk = static_cast<uint32_t>(p.topk);
+        auto emit_tile = [&](auto key_at, int a, int c) {
+            auto chosen = [&](int j) {
+                if (j >= c) return false;
+                const uint32_t k = key_at(j);
+                return k > tau || (k == tau && static_cast<uint32_t>(a + j) <= pcut);
+            };
+            uint32_t wc = 0;
+#pragma unroll 4
+            for (int u = 0; u < kSeg / 32; ++u)
+                wc += __popc(__ballot_sync(0xffffffffu, chosen(warp * kSeg + u * 32 + lane)));
+            if (lane == 0) scratch[warp] = wc;
+            __syncthreads();
+            uint32_t wo = out, tot = 0;
+#pragma unroll
+            for (int w = 0; w < kWarps; ++w) {
+                const uint32_t x = scratch[w];
+                wo += w < warp ? x : 0u;
+                tot += x;
+            }
+            __syncthreads();
+            const uint32_t wend = wo + wc;
+            for (int u = 0; u < kSeg / 32 && wo < wend; ++u) {
+                const int j = warp * kSeg + u * 32 + lane;
+                const bool s = chosen(j);
+                const uint32_t bal = __ballot_sync(0xffffffffu, s);
+                const uint32_t o = wo + __popc(bal & ((1u << lane) - 1u));
+                if (s && o < topk) sel[o] = a + j;
+                wo += __popc(bal);
+            }
+            out += tot;
+        };
+        const int R = ((cnt + 31) / 32 + kThreads - 1) / kThreads;   // bitmap words per thread
+        if (fits && R * kThreads <= kChunkWords) {
+            // Bitmap of the chunk's selected positions, transposed: thread i owns the
+            // R consecutive words [i*R, (i+1)*R), its k-th word at k*256 + i.
+            uint32_t* bitmap = reinterpret_cast<uint32_t*>(smem);
+            for (int w = tid; w < R * kThreads; w += kThreads) bitmap[w] = 0u;
+            __syncthreads();
+            for (uint32_t j = tid; j < m; j += kThreads) {
+                const uint2 v = in[j];
+                const int q = static_cast<int>(v.y);
+                if (q >= it.s0 && q < it.s1 && (v.x > tau || (v.x == tau && v.y <= pcut))) {
                     const uint32_t rel = static_cast<uint32_t>(q - it.s0), w = rel >> 5, owner = w / R;
                     atomicOr(&bitmap[(w - owner * R) * kThreads + owner], 1u << (rel & 31));
                 }
-                return 0u;
-            };
-            for (int w = tid; w < R * kThreads; w += kThreads) bitmap[w] = 0u;
-            if (tid == 0) nsub = 0;
-            __syncthreads();
-            uint32_t before = 0;
-            for (uint32_t j0 = 0; j0 < m; j0 += kThreads) {
-                const uint32_t j = j0 + tid;
-                const uint2 v = j < m ? __ldcg(glist + j) : make_uint2(0u, 0u);
-                if (j < m && v.x > hi2) before += mark(v.y);
-                warp_append(j < m && v.x >= lo2 && v.x <= hi2, v, sub, &nsub, kSubCap);
             }
             __syncthreads();
-            stamp(p, 14);
-            const uint32_t n2 = nsub;
-            uint32_t tau, pcut = 0xFFFFFFFFu;   // selected: key > tau, or key == tau and position <= pcut
-            if (n2 <= static_cast<uint32_t>(kSubCap)) {
-                for (uint32_t j = tid; j < n2; j += kThreads) vals[j] = sub[j].x;
-                if (tid == 0) nval = 0;
-                __syncthreads();
-                tau = exact_select(vals, n2, need, h, res, scratch, p.err);
-                const uint32_t rties = need;
-                for (uint32_t j0 = 0; j0 < n2; j0 += kThreads) {   // ~position of the ties: largest = lowest
-                    const uint32_t j = j0 + tid;
-                    const uint2 v = j < n2 ? sub[j] : make_uint2(0u, 0u);
-                    warp_append(j < n2 && v.x == tau, ~v.y, vals, &nval, kSubCap);
-                }
-                __syncthreads();
-                const uint32_t e = nval;
-                if (rties < e) pcut = ~exact_select(vals, e, need, h, res, scratch, p.err);
-                for (uint32_t j = tid; j < n2; j += kThreads) {
-                    const uint2 v = sub[j];
-                    if (v.x > tau || (v.x == tau && v.y <= pcut)) before += mark(v.y);
-                }
-            } else {
-                // Heavy ties: tau and the tie cut by radix select over the list itself.
-                uint32_t lo = lo2, hi = hi2;
-                radix_select([&](uint32_t j) { return __ldcg(glist + j).x; }, m, lo, hi, need, h, res, scratch,
-                             p.err);
-                tau = lo;
-                uint32_t e = 0, plo = 0xFFFFFFFFu, phi = 0u;
-                for (uint32_t j = tid; j < m; j += kThreads) {
-                    const uint2 v = __ldcg(glist + j);
-                    if (v.x == tau) {
-                        ++e;
-                        plo = min(plo, ~v.y);
-                        phi = max(phi, ~v.y);
-                    }
-                }
-                e = block_sum(e, scratch);
-                block_minmax(plo, phi, scratch);
-                if (need < e) {
-                    radix_select(
-                        [&](uint32_t j) {
-                            const uint2 v = __ldcg(glist + j);
-                            return v.x == tau ? ~v.y : 0u;
-                        },
-                        m, plo, phi, need, h, res, scratch, p.err);
-                    pcut = ~plo;
-                }
-                for (uint32_t j = tid; j < m; j += kThreads) {
-                    const uint2 v = __ldcg(glist + j);
-                    if (v.x >= lo2 && v.x <= hi2 && (v.x > tau || (v.x == tau && v.y <= pcut))) before += mark(v.y);
-                }
-            }
-            before = block_sum(before, scratch);   // also orders the marking before the count
-            stamp(p, 15);
-            uint32_t cnt = 0;
-            for (int k = 0; k < R; ++k) cnt += __popc(bitmap[k * kThreads + tid]);
+            uint32_t c1 = 0;
+            for (int k = 0; k < R; ++k) c1 += __popc(bitmap[k * kThreads + tid]);
             uint32_t total;
-            uint32_t o = block_excl_scan(cnt, total, scratch);
-            for (int k = 0; k < R && cnt; ++k) {
+            uint32_t o = out + block_excl_scan(c1, total, scratch);
+            for (int k = 0; k < R && c1; ++k) {
                 uint32_t b = bitmap[k * kThreads + tid];
                 const int base = it.s0 + ((tid * R + k) << 5);
                 while (b) {
                     const int bit = __ffs(b) - 1;
                     b &= b - 1;
-                    if (o < static_cast<uint32_t>(kMaxTopk)) outs[o] = base + bit;
+                    if (o < topk) sel[o] = base + bit;
                     ++o;
-                    --cnt;
+                    --c1;
                 }
             }
-            __syncthreads();
-            const uint32_t lim = before < static_cast<uint32_t>(p.topk) ? static_cast<uint32_t>(p.topk) - before : 0u;
-            for (uint32_t j = tid; j < total && j < lim && j < static_cast<uint32_t>(kMaxTopk); j += kThreads)
-                sel[before + j] = outs[j];
-            if (tid == 0 && (before + total > static_cast<uint32_t>(p.topk) ||
-                             (it.s1 == it.n && before + total != static_cast<uint32_t>(p.topk))))
-                atomicOr(p.err, ERR_TOPK_STATE);
-            __syncthreads();
-            continue;
+            out += total;
+        } else if (r == 0 && ((cnt + 3) & ~3) <= kChunkSmem) {
+            for (int a = 0; a < cnt; a += kStreamTile)
+                emit_tile([&](int j) { return keys[a + j]; }, it.s0 + a, min(kStreamTile, cnt - a));
+        } else {
+            const float* row = p.scores + (int64_t)it.t * p.ld;
+            const bool ok = stream_scores(row, it.s0, it.s1, reinterpret_cast<float*>(smem), ring_full, seq, p.err,
+                                          [&](const float* tile, int a, int c) {
+                                              emit_tile([&](int j) { return score_key(tile[j]); }, a, c);
+                                          });
+            if (!ok) return;
         }
-
-        // Long lists or wide chunks: tau by radix select over the list, then this
-        // chunk's output offset and tie rank from the candidates of earlier
-        // chunks, then an ordered sweep of the chunk's scores.
-        uint32_t lo = lo2, hi = hi2;
-        radix_select([&](uint32_t j) { return __ldcg(glist + j).x; }, m, lo, hi, need, h, res, scratch, p.err);
-        const uint32_t tau = lo, rties = need;
-        uint32_t before_gt = 0, before_eq = 0;
-        for (uint32_t j = tid; j < m; j += kThreads) {
-            const uint2 v = __ldcg(glist + j);
-            if (static_cast<int>(v.y) < it.s0) {
-                before_gt += v.x > tau;
-                before_eq += v.x == tau;
-            }
-        }
-        before_gt = block_sum(before_gt, scratch);
-        before_eq = block_sum(before_eq, scratch);
-        uint32_t out = before_gt + min(before_eq, rties);
-        uint32_t tie_rank = before_eq;
-        const float* row = p.scores + (int64_t)it.t * p.ld;
-        for (int base = it.s0; base < it.s1; base += kThreads * 4) {
-            const int s = base + tid * 4;
-            uint32_t gtm = 0, eqm = 0;
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-                if (s + j < it.s1) {
-                    const uint32_t k = score_key(__ldcg(row + s + j));
-                    if (k > tau) gtm |= 1u << j;
-                    if (k == tau) eqm |= 1u << j;
-                }
-            if (!__syncthreads_or((gtm | eqm) != 0u)) continue;
-            uint32_t tie_total;
-            uint32_t rank = tie_rank + block_excl_scan(__popc(eqm), tie_total, scratch);
-            uint32_t take = gtm;
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-                if (eqm & (1u << j)) {
-                    if (rank < rties) take |= 1u << j;
-                    ++rank;
-                }
-            uint32_t taken_total;
-            uint32_t o = out + block_excl_scan(__popc(take), taken_total, scratch);
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-                if ((take & (1u << j)) && o < static_cast<uint32_t>(p.topk)) sel[o++] = s + j;
-            out += taken_total;
-            tie_rank += tie_total;
-        }
+        if (tid == 0 && (out > topk || (it.s1 == it.n && out != topk))) atomicOr(p.err, ERR_TOPK_STATE);
+        __syncthreads();
     }
 }
 
@@ -1370,7 +1348,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         stamp(p, 5);
         ok = gb.sync(&ok_s) && ok;
         stamp(p, 6);
-        if (ok) phase_emit(p, smem, res, scratch);
+        if (ok) phase_emit(p, smem, bars + kStreamBar, seq, res, scratch);
         stamp(p, 7);
     }
     if (p.phases & kPhaseAttend) {
