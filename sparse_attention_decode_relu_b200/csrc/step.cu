@@ -32,7 +32,7 @@ constexpr int kWarps = kThreads / 32;
 constexpr float kLog2e = 1.4426950408889634f;
 
 // ---- shared memory map (dynamic, 1024-aligned base) --------------------------
-constexpr int kIdxStages = 4;
+constexpr int kIdxStages = 6;
 constexpr int kAttStages = 6;
 constexpr int kTileRows = 16;
 constexpr int kRowBytes = 2048;
@@ -41,8 +41,7 @@ constexpr int kDataBytes = kAttStages * kTileRows * kPitch + kAttStages * kTileR
 constexpr int kBarOffset = (kDataBytes + 127) / 128 * 128;
 constexpr int kBarSlots = 64;             // mbarriers (8 bytes each) after the data region
 constexpr int kStepSmem = 1024 + kBarOffset + kBarSlots * 8;
-static_assert(kIdxStages * 16384 + 16384 + kMaxT * kHI * kDI * 2 + kMaxT * kHI * 4 + kIdxStages * kKeyTile * 4 <=
-                  kDataBytes, "indexer buffers fit the data region");
+
 
 __device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p)
 {
@@ -261,195 +260,269 @@ __device__ void find_from_top(const uint32_t* h, uint32_t need, uint32_t* res, u
 __device__ __forceinline__ int item_of(int r) { return blockIdx.x + r * gridDim.x; }
 
 // ==================================================================================
-// Phase 1: indexer scan.  Tiles of 128 keys by TMA into a 4-stage ring; each warp
-// owns one query (or a share of one when T < 8) and keeps its 16 indexer heads x
-// 64 dims in registers as the N side of m16n8k16 tensor-core products whose M side
-// is 16 keys at a time.  ReLU, head weights, a fixed-order sum over heads.
+// Phase 1: indexer scan on the fifth-generation tensor cores.  A tile of 128 keys
+// is the M side of tcgen05.mma (kind::f16: bf16 operands, fp32 accumulators in
+// tensor memory), the T x 16 indexer query heads the N side, the 64 dims K (four
+// K = 16 steps).  TMA brings key tiles into a ring; E4M3 tiles are widened to
+// bf16 (exactly) into a 128B-swizzled buffer.  One thread issues the MMAs; the
+// accumulators of consecutive tiles alternate between two TMEM buffers so that
+// the epilogue of one tile overlaps the MMA of the next.  Epilogue: each thread
+// owns one key row (a TMEM lane) and, per query, applies ReLU, the head weights,
+// a fixed-order sum over the 16 heads and the per-token scale.
 // ==================================================================================
+constexpr uint32_t kTmemCols = 256;        // two accumulator buffers of 128 columns
+constexpr int kMmaBar = 40;                // the two MMA-completion mbarriers
+constexpr int kTileBytesBf16 = kKeyTile * kDI * 2;   // 16 KiB, one 128 x 64 bf16 operand tile
+static_assert(kIdxStages * kTileBytesBf16 + 2 * kTileBytesBf16 + kTileBytesBf16 + kMaxT * kHI * 4 +
+                  (kIdxStages + 2) * kKeyTile * 4 <= kDataBytes, "indexer buffers fit the data region");
+static_assert(kMmaBar + 2 <= kBarSlots && kIdxStages + 1 <= 8, "indexer mbarriers fit");
+
 template <bool FP8>
 __device__ void phase_index(const CUtensorMap& kmap, const CUtensorMap& smap, const StepParams& p, uint8_t* smem,
-                            uint64_t* bars, uint32_t* scratch)
+                            uint64_t* bars, uint32_t* scratch, uint32_t* tmem_slot)
 {
     constexpr int raw_bytes = kKeyTile * kDI * (FP8 ? 1 : 2);
-    uint8_t* ring = smem;
-    uint8_t* cvt = ring + kIdxStages * raw_bytes;
-    uint16_t* q_s = reinterpret_cast<uint16_t*>(cvt + (FP8 ? kKeyTile * kDI * 2 : 0));
-    float* w_s = reinterpret_cast<float*>(q_s + kMaxT * kHI * kDI);
-    float* sc_s = w_s + kMaxT * kHI;
+    uint8_t* ring = smem;                                                  // [kIdxStages][raw_bytes]
+    uint8_t* cvt = ring + kIdxStages * raw_bytes;                          // FP8: [2][16 KiB] bf16 tiles
+    uint8_t* qsw = cvt + (FP8 ? 2 * kTileBytesBf16 : 0);                   // [128 rows][128 B] queries
+    float* w_s = reinterpret_cast<float*>(qsw + kTileBytesBf16);           // [8][16]
+    float* sc_s = w_s + kMaxT * kHI;                                       // [kIdxStages][128] scales
+    float* scl = sc_s + kIdxStages * kKeyTile;                             // [2][128] scales of the TMEM tiles
     uint64_t* full = bars;                  // [kIdxStages]
     uint64_t* setup = bars + kIdxStages;
+    uint64_t* mmab = bars + kMmaBar;        // [2]
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int g = lane >> 2, c = lane & 3;
     const int T = p.T;
     const int ntiles = (p.n_max + kKeyTile - 1) / kKeyTile;
     const bool scaled = p.scale != nullptr;
     const uint32_t tile_tx = raw_bytes + (scaled ? kKeyTile * 4 : 0);
+    auto tile_of = [&](int it) { return blockIdx.x + it * static_cast<int>(gridDim.x); };
     auto load_tile = [&](int stage, int tile) {
         mbar_arrive_expect_tx(&full[stage], tile_tx);
         tma_load_2d(ring + stage * raw_bytes, &kmap, 0, tile * kKeyTile, &full[stage]);
         if (scaled) tma_load_1d(sc_s + stage * kKeyTile, &smap, tile * kKeyTile, &full[stage]);
     };
 
-    int issued = 0;
+    int issued = 0;   // key tiles requested by thread 0
     if (tid == 0) {
         prefetch_tmap(&kmap);
         if (scaled) prefetch_tmap(&smap);
-        for (int s = 0; s < kIdxStages + 1; ++s) mbar_init(&bars[s], 1);
+        for (int s = 0; s <= kIdxStages; ++s) mbar_init(&bars[s], 1);
+        mbar_init(&mmab[0], 1);
+        mbar_init(&mmab[1], 1);
         fence_mbar_init();
-        mbar_arrive_expect_tx(setup, T * kHI * kDI * 2 + T * kHI * 4);
-        bulk_g2s(q_s, p.q_idx, T * kHI * kDI * 2, setup);
+        mbar_arrive_expect_tx(setup, T * kHI * 4);
         bulk_g2s(w_s, p.w, T * kHI * 4, setup);
-        for (int s = 0; s < kIdxStages; ++s) {
-            const int tile = blockIdx.x + s * gridDim.x;
-            if (tile >= ntiles) break;
-            load_tile(s, tile);
+        for (int s = 0; s < kIdxStages && tile_of(s) < ntiles; ++s) {
+            load_tile(s, tile_of(s));
             ++issued;
         }
     }
+    if (warp == 0) tmem_alloc(tmem_slot, kTmemCols);
+    // The indexer queries as the B operand: row r = t*16 + j, 16-byte chunk c at
+    // r*128 + (c ^ (r & 7))*16 (the 128B swizzle); rows >= T*16 are never read.
+    for (int i = tid; i < T * kHI * 8; i += kThreads) {
+        const int r = i >> 3, c = i & 7;
+        const uint4 v = __ldg(reinterpret_cast<const uint4*>(p.q_idx) + i);
+        *reinterpret_cast<uint4*>(qsw + r * 128 + ((c ^ (r & 7)) << 4)) = v;
+    }
     // Counters the top-k phases accumulate into start at zero.
     for (int i = blockIdx.x * kThreads + tid; i < p.zero_words; i += gridDim.x * kThreads) p.zero[i] = 0u;
+    fence_proxy_async_smem();   // the queries are read by the tensor cores (async proxy)
+    tc_fence_before();
     __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
     bool ok = mbar_wait(setup, 0, p.err);
 
-    // Warps per query: 8 / T rounded down to a power of two.
-    const int tp = T <= 1 ? 1 : T <= 2 ? 2 : T <= 4 ? 4 : 8;
-    const int wpq = kWarps / tp, nblk = kWarps / wpq;
-    const int t = warp / wpq;
-    const bool active = t < T;
-    const int kb0 = warp % wpq;
-    int pos_t = -1;
+    // Warp w reads TMEM lanes 32*(w%4) .. +31 (its key rows) and the columns of
+    // queries [qa, qb): warps 0-3 the first ceil(T/2) queries, warps 4-7 the rest.
+    const int quad = warp & 3, half = warp >> 2;
+    const int tsplit = (T + 1) >> 1;
+    const int qa = half ? tsplit : 0, qb = half ? T : tsplit;
+    const int row = quad * 32 + lane;
+    int pos_q[4];
+    uint32_t klo[4], khi[4];
 #pragma unroll
-    for (int i = 0; i < kMaxT; ++i)
-        if (i == t) pos_t = p.pos[i];
-    uint32_t qb[2][4][2];
-    float w0 = 0.f, w1 = 0.f, w8 = 0.f, w9 = 0.f;
-    uint32_t klo = 0xFFFFFFFFu, khi = 0u;
-    if (active && ok) {
-        const uint32_t qbase = smem_u32(q_s + t * kHI * kDI);
+    for (int u = 0; u < 4; ++u) {
+        pos_q[u] = -1;
 #pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-            for (int kp = 0; kp < 2; ++kp) {
-                const uint32_t a = qbase + (nt * 8 + (lane & 7)) * (kDI * 2) + (kp * 32 + (lane >> 3) * 8) * 2;
-                ldsm_x4(a, qb[nt][2 * kp][0], qb[nt][2 * kp][1], qb[nt][2 * kp + 1][0], qb[nt][2 * kp + 1][1]);
-            }
-        w0 = w_s[t * kHI + 2 * c];
-        w1 = w_s[t * kHI + 2 * c + 1];
-        w8 = w_s[t * kHI + 8 + 2 * c];
-        w9 = w_s[t * kHI + 9 + 2 * c];
+        for (int i = 0; i < kMaxT; ++i)
+            if (i == qa + u) pos_q[u] = p.pos[i];
+        klo[u] = 0xFFFFFFFFu;
+        khi[u] = 0u;
     }
+    const uint32_t idesc = umma_idesc_bf16(kKeyTile, T * kHI);
+    const uint64_t bdesc = umma_desc_sw128(smem_u32(qsw));
 
-    int it = 0;
-    bool aborted = __syncthreads_or(!ok);
-    for (int tile = blockIdx.x; !aborted && tile < ntiles; tile += gridDim.x, ++it) {
-        const int stage = it % kIdxStages;
-        ok = mbar_wait(&full[stage], (it / kIdxStages) & 1, p.err);
-        if (__syncthreads_or(!ok)) {
-            aborted = true;
-            break;
-        }
-        const uint8_t* ktile = ring + stage * raw_bytes;
-        if constexpr (FP8) {
-            // Widen 128 x 64 E4M3 codes to bf16 (exact) in the 128B-swizzled layout.
+    int mma_issued = 0, mma_done = 0;
+    // Epilogue of local tile e: wait for its MMA, then scores from TMEM buffer e & 1.
+    auto epilogue = [&](int e) -> bool {
+        const int b = e & 1;
+        const bool okm = __syncthreads_and(mbar_wait(&mmab[b], (e >> 1) & 1, p.err));
+        mma_done = e + 1;
+        tc_fence_after();
+        if (okm && qa < qb) {
+            const int s = tile_of(e) * kKeyTile + row;
+            const float scale = scl[b * kKeyTile + row];
+            const uint32_t tbase = tmem + static_cast<uint32_t>((quad * 32) << 16) + b * 128;
+            // Two queries per TMEM load; the 16-head sum as four interleaved partial
+            // sums over heads {j, j+4, j+8, j+12}, combined in a fixed order.
 #pragma unroll
-            for (int r = 0; r < 2; ++r) {
-                const int chunk = tid + r * kThreads;
-                const int row = chunk >> 2, piece = chunk & 3;
-                const uint4 v = *reinterpret_cast<const uint4*>(ktile + row * 64 + piece * 16);
-                const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-                uint32_t o[8];
+            for (int u0 = 0; u0 < 4; u0 += 2) {
+                const int t0 = qa + u0;
+                if (t0 < qb) {
+                    uint32_t r[32];
+                    tmem_ld32_nowait(tbase + t0 * kHI, r);
+                    tmem_ld_wait();
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    o[2 * i] = e4m3x2_to_bf16x2(static_cast<uint16_t>(w4[i] & 0xFFFFu));
-                    o[2 * i + 1] = e4m3x2_to_bf16x2(static_cast<uint16_t>(w4[i] >> 16));
-                }
-                const int c0 = (2 * piece) ^ (row & 7), c1 = (2 * piece + 1) ^ (row & 7);
-                *reinterpret_cast<uint4*>(cvt + row * 128 + c0 * 16) = make_uint4(o[0], o[1], o[2], o[3]);
-                *reinterpret_cast<uint4*>(cvt + row * 128 + c1 * 16) = make_uint4(o[4], o[5], o[6], o[7]);
-            }
-            __syncthreads();
-            ktile = cvt;
-        }
-        if (active) {
-#pragma unroll 2
-            for (int j = 0; j < nblk; ++j) {
-                const int kb = kb0 + wpq * j;
-                uint32_t a[4][4];
-                const int row = kb * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
-                const uint32_t base = smem_u32(ktile) + row * 128;
+                    for (int h = 0; h < 2; ++h) {
+                        const int u = u0 + h, t = t0 + h;
+                        if (t < qb) {
+                            const float4* w4 = reinterpret_cast<const float4*>(w_s + t * kHI);
+                            float part[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                    const int chunk = 2 * kk + (lane >> 4);
-                    ldsm_x4(base + ((chunk ^ (row & 7)) << 4), a[kk][0], a[kk][1], a[kk][2], a[kk][3]);
-                }
-                float acc0[4] = {0.f, 0.f, 0.f, 0.f}, acc1[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                    mma_bf16_16816(acc0, a[kk], qb[0][kk][0], qb[0][kk][1]);
-                    mma_bf16_16816(acc1, a[kk], qb[1][kk][0], qb[1][kk][1]);
-                }
-                float pa = fmaxf(acc0[0], 0.f) * w0;
-                pa = fmaf(fmaxf(acc0[1], 0.f), w1, pa);
-                pa = fmaf(fmaxf(acc1[0], 0.f), w8, pa);
-                pa = fmaf(fmaxf(acc1[1], 0.f), w9, pa);
-                float pb = fmaxf(acc0[2], 0.f) * w0;
-                pb = fmaf(fmaxf(acc0[3], 0.f), w1, pb);
-                pb = fmaf(fmaxf(acc1[2], 0.f), w8, pb);
-                pb = fmaf(fmaxf(acc1[3], 0.f), w9, pb);
-                pa += __shfl_xor_sync(0xffffffffu, pa, 1);
-                pb += __shfl_xor_sync(0xffffffffu, pb, 1);
-                pa += __shfl_xor_sync(0xffffffffu, pa, 2);
-                pb += __shfl_xor_sync(0xffffffffu, pb, 2);
-                const int s = tile * kKeyTile + kb * 16 + g + 8 * (c & 1);   // lanes c = 0, 1 write
-                if (c < 2 && s < p.L) {
-                    const float scale = scaled ? sc_s[stage * kKeyTile + kb * 16 + g + 8 * (c & 1)] : 1.0f;
-                    const float v = (c == 0 ? pa : pb) * scale;
-                    if (s <= pos_t) {
-                        p.scores[(int64_t)t * p.ld + s] = v;
-                        const uint32_t k = score_key(v);
-                        klo = min(klo, k);
-                        khi = max(khi, k);
-                    } else {
-                        p.scores[(int64_t)t * p.ld + s] = -INFINITY;
+                            for (int g4 = 0; g4 < 4; ++g4) {
+                                const float4 w = w4[g4];
+                                const float* v = reinterpret_cast<const float*>(r + h * 16 + g4 * 4);
+                                part[0] = fmaf(fmaxf(v[0], 0.f), w.x, part[0]);
+                                part[1] = fmaf(fmaxf(v[1], 0.f), w.y, part[1]);
+                                part[2] = fmaf(fmaxf(v[2], 0.f), w.z, part[2]);
+                                part[3] = fmaf(fmaxf(v[3], 0.f), w.w, part[3]);
+                            }
+                            const float acc = ((part[0] + part[1]) + (part[2] + part[3])) * scale;
+                            if (s < p.L) {
+                                if (s <= pos_q[u]) {
+                                    p.scores[(int64_t)t * p.ld + s] = acc;
+                                    const uint32_t k = score_key(acc);
+                                    klo[u] = min(klo[u], k);
+                                    khi[u] = max(khi[u], k);
+                                } else {
+                                    p.scores[(int64_t)t * p.ld + s] = -INFINITY;
+                                }
+                            }
+                        }
                     }
                 }
             }
         }
-        __syncthreads();   // every warp is done with this stage (and with cvt)
-        if (tid == 0) {
-            const int next = tile + kIdxStages * gridDim.x;
-            if (next < ntiles) {
-                load_tile(stage, next);
-                ++issued;
+        tc_fence_before();
+        return okm;
+    };
+
+    bool aborted = __syncthreads_or(!ok);
+    int it = 0;
+    for (; !aborted; ++it) {
+        const int tile = tile_of(it);
+        const bool have = tile < ntiles;
+        if (have) {
+            const int stage = it % kIdxStages;
+            ok = mbar_wait(&full[stage], (it / kIdxStages) & 1, p.err);
+            if (__syncthreads_or(!ok)) {
+                aborted = true;
+                break;
+            }
+            const int b = it & 1;
+            uint32_t a_addr;
+            if constexpr (FP8) {
+                // Widen 128 x 64 E4M3 codes to bf16 (exact) in the 128B-swizzled layout.
+                const uint8_t* raw = ring + stage * raw_bytes;
+                uint8_t* dst = cvt + b * kTileBytesBf16;
+#pragma unroll
+                for (int r = 0; r < 2; ++r) {
+                    const int chunk = tid + r * kThreads;
+                    const int kr = chunk >> 2, piece = chunk & 3;
+                    const uint4 v = *reinterpret_cast<const uint4*>(raw + kr * 64 + piece * 16);
+                    const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+                    uint32_t o[8];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        o[2 * i] = e4m3x2_to_bf16x2(static_cast<uint16_t>(w4[i] & 0xFFFFu));
+                        o[2 * i + 1] = e4m3x2_to_bf16x2(static_cast<uint16_t>(w4[i] >> 16));
+                    }
+                    const int c0 = (2 * piece) ^ (kr & 7), c1 = (2 * piece + 1) ^ (kr & 7);
+                    *reinterpret_cast<uint4*>(dst + kr * 128 + c0 * 16) = make_uint4(o[0], o[1], o[2], o[3]);
+                    *reinterpret_cast<uint4*>(dst + kr * 128 + c1 * 16) = make_uint4(o[4], o[5], o[6], o[7]);
+                }
+                fence_proxy_async_smem();
+                a_addr = smem_u32(dst);
+            } else {
+                a_addr = smem_u32(ring + stage * raw_bytes);
+            }
+            if (tid < kKeyTile) scl[b * kKeyTile + tid] = scaled ? sc_s[stage * kKeyTile + tid] : 1.0f;
+            tc_fence_before();
+            __syncthreads();   // operands ready; the epilogue of local tile it - 2 is done with buffer b
+            if (tid == 0) {
+                tc_fence_after();
+                const uint64_t adesc = umma_desc_sw128(a_addr);
+#pragma unroll
+                for (int k = 0; k < kDI / 16; ++k)
+                    tc_mma_bf16(tmem + b * 128, adesc + 2 * k, bdesc + 2 * k, idesc, k > 0 ? 1u : 0u);
+                tc_commit(&mmab[b]);
+                if constexpr (FP8) {   // the raw tile is consumed: refill its stage now
+                    const int next = tile_of(it + kIdxStages);
+                    if (next < ntiles) {
+                        load_tile(stage, next);
+                        ++issued;
+                    }
+                }
+            }
+            ++mma_issued;
+        }
+        if (it > 0) {
+            if (!epilogue(it - 1)) {
+                aborted = true;
+                break;
+            }
+            if constexpr (!FP8) {   // the MMA of local tile it - 1 is complete: refill its stage
+                const int next = tile_of(it - 1 + kIdxStages);
+                if (tid == 0 && next < ntiles) {
+                    load_tile((it - 1) % kIdxStages, next);
+                    ++issued;
+                }
             }
         }
+        if (!have) break;
     }
-    if (aborted) {   // let copies still in flight land before the smem is reused
+    if (aborted) {   // let copies and MMAs still in flight land before the smem and TMEM are reused
         if (tid == 0) {
             mbar_wait(setup, 0, p.err);
             for (int k = it; k < issued; ++k) mbar_wait(&full[k % kIdxStages], (k / kIdxStages) & 1, p.err);
+            for (int e = mma_done; e < mma_issued; ++e) mbar_wait(&mmab[e & 1], (e >> 1) & 1, p.err);
         }
-        __syncthreads();
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
     }
 
     // This block's key range of each query's visible scores (slot [block][t]).
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        klo = min(klo, __shfl_xor_sync(0xffffffffu, klo, o));
-        khi = max(khi, __shfl_xor_sync(0xffffffffu, khi, o));
+    for (int u = 0; u < 4; ++u) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            klo[u] = min(klo[u], __shfl_xor_sync(0xffffffffu, klo[u], o));
+            khi[u] = max(khi[u], __shfl_xor_sync(0xffffffffu, khi[u], o));
+        }
     }
-    if (lane == 0) {
-        scratch[warp] = klo;
-        scratch[32 + warp] = khi;
-    }
+    // scratch[0..31]: lo of (query t, quad) at t*4 + quad; scratch[32..63]: hi.
+    if (lane == 0)
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+            if (qa + u < qb) {
+                scratch[(qa + u) * 4 + quad] = klo[u];
+                scratch[32 + (qa + u) * 4 + quad] = khi[u];
+            }
     __syncthreads();
     if (tid < kMaxT && p.mm != nullptr) {
         uint32_t lo = 0xFFFFFFFFu, hi = 0u;
         if (tid < T)
-            for (int w = tid * wpq; w < (tid + 1) * wpq; ++w) {
-                lo = min(lo, scratch[w]);
-                hi = max(hi, scratch[32 + w]);
+            for (int q = 0; q < 4; ++q) {
+                lo = min(lo, scratch[tid * 4 + q]);
+                hi = max(hi, scratch[32 + tid * 4 + q]);
             }
         p.mm[(int64_t)blockIdx.x * kMaxT + tid] = make_uint2(lo, hi);
     }
@@ -1315,6 +1388,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __shared__ uint32_t scratch[64];
     __shared__ uint32_t res[3];
     __shared__ int ok_s;
+    __shared__ uint32_t tmem_slot;
 
     GridBarrier gb{p.bar_ctrl, p.err, gridDim.x};
 
@@ -1332,7 +1406,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     stamp(p, 0);
     if (p.trace != nullptr && threadIdx.x == 0) p.trace[(int64_t)blockIdx.x * kTraceSlots + 28] = clock64();
     if (p.phases & kPhaseIndex) {
-        phase_index<FP8>(kmap, smap, p, smem, bars, scratch);
+        phase_index<FP8>(kmap, smap, p, smem, bars, scratch, &tmem_slot);
     } else if (p.phases & kPhaseRanges) {
         phase_ranges(p, scratch);
     }
