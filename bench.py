@@ -174,17 +174,35 @@ def barrier(world):
     torch.cuda.synchronize()
 
 
-def cpu_baseline(w, budget_s=15.0):
+def swa_bytes(w, window):
+    """Sliding-window decode: each unique K/V row of the windows once, plus the
+    queries and outputs."""
+    import oracle
+
+    sel = oracle.window_select(w.pos, window)
+    uniq = np.unique(sel[sel >= 0]).size
+    return {"step": uniq * 2048 + w.T * 2 * 64 * 128 * 2, "unique_rows": uniq, "gathered_rows": int((sel >= 0).sum())}
+
+
+def oracle_step(w, op, window):
+    """One step of the oracle (test infrastructure) for this workload and op."""
+    import oracle
+
+    if op == "swa":
+        return oracle.swa_decode(w.q, w.kv, w.pos, window), oracle.window_select(w.pos, window)
+    return oracle.decode(w.q, w.q_idx, w.w_idx, w.k_idx, w.k_scale, w.kv, w.pos, w.topk)
+
+
+def cpu_baseline(w, budget_s=15.0, op="step", window=128):
     """The oracle as it stands, on this host's cores, over whole steps of the same
     workload until about budget_s seconds have passed."""
     import oracle
 
-    kv = w.kv
     times = []
     t_end = time.perf_counter() + budget_s
     while True:
         t0 = time.perf_counter()
-        _, sel = oracle.decode(w.q, w.q_idx, w.w_idx, w.k_idx, w.k_scale, kv, w.pos, w.topk)
+        _, sel = oracle_step(w, op, window)
         times.append(time.perf_counter() - t0)
         if time.perf_counter() > t_end or len(times) >= 50:
             break
@@ -196,23 +214,22 @@ def run_reference(args, w, rank, world):
         return
     import oracle
 
-    kv = w.kv
     for _ in range(args.warmup):
-        oracle.decode(w.q, w.q_idx, w.w_idx, w.k_idx, w.k_scale, kv, w.pos, w.topk)
+        oracle_step(w, args.op, args.window)
     times = []
     sel = None
     for _ in range(args.steps):
         t0 = time.perf_counter()
-        _, sel = oracle.decode(w.q, w.q_idx, w.w_idx, w.k_idx, w.k_scale, kv, w.pos, w.topk)
+        _, sel = oracle_step(w, args.op, args.window)
         times.append(time.perf_counter() - t0)
-    ab = algorithmic_bytes(w, sel)
+    ab = swa_bytes(w, args.window) if args.op == "swa" else algorithmic_bytes(w, sel)
     t = statistics.mean(times)
     value = ab["step"] / t / 1e9
     line = {
         "impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "GB/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(t * 1e3, 3), "us_per_step": round(t * 1e6, 1),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name, "L": w.L, "T": w.T, "topk": w.topk, "key_dtype": w.key_dtype,
+        "config": {"workload": w.name, "op": args.op, "L": w.L, "T": w.T, "topk": w.topk, "key_dtype": w.key_dtype,
                    "recipe": w.recipe, "seed": w.seed},
         "cpu_baseline": {"value": round(value, 3), "unit": "GB/s", "cores": oracle.threads(), "kind": "oracle",
                          "sample": f"whole steps of {w.name} (fp64 C oracle, OpenMP), {args.steps} timed"},
@@ -230,6 +247,10 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--op", choices=["step", "swa"], default="step",
+                    help="step: the DSA decode/verify step; swa: sliding-window decode on the same q / K/V")
+    ap.add_argument("--window", type=int, default=128, help="window of --op swa")
+    ap.add_argument("--no-bypass", action="store_true", help="score and select even when every query sees <= topk")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
@@ -242,6 +263,7 @@ def main():
 
     from sparse_attention_decode_relu_b200 import dsa
 
+    dsa.dsa_set_short_context_bypass(not args.no_bypass)
     rank, world, local = dist_setup(args.gpus)
     dev = torch.device("cuda", torch.cuda.current_device())
     d = dsa.to_device(w, device=dev)
@@ -264,8 +286,11 @@ def main():
     trace = torch.zeros(grid * 32, dtype=torch.int64, device=dev)
 
     def step():
-        dsa.dsa_decode_ws(d["q"], d["q_idx"], d["w_idx"], d["k_idx"], d["kv"], d["pos"], topk, out, sel, ws,
-                          k_scale=d["k_scale"])
+        if args.op == "swa":
+            dsa.dsa_swa_decode(d["q"], d["kv"], w.pos, args.window, out, ws)
+        else:
+            dsa.dsa_decode_ws(d["q"], d["q_idx"], d["w_idx"], d["k_idx"], d["kv"], d["pos"], topk, out, sel, ws,
+                              k_scale=d["k_scale"])
 
     # One eager call counts the kernels of a step; then capture the step in a graph.
     with torch.cuda.stream(stream):
@@ -331,27 +356,30 @@ def main():
     ms = reduce_max(statistics.mean(totals), world)
     phase_us = {k: round(v / args.steps, 2) for k, v in phase_sum.items()}
 
-    sel_np = sel.cpu().numpy()
-    ab = algorithmic_bytes(w, sel_np)
+    ab = swa_bytes(w, args.window) if args.op == "swa" else algorithmic_bytes(w, sel.cpu().numpy())
     value = world * ab["step"] / (ms * 1e-3) / 1e9
 
     # End to end through the public API: per step the query-side inputs come from
     # pinned host memory and the outputs go back to it; the caches stay resident.
-    h_in = {k: d[k].cpu().pin_memory() for k in ("q", "q_idx", "w_idx")}
+    h_in = {k: d[k].cpu().pin_memory() for k in (("q",) if args.op == "swa" else ("q", "q_idx", "w_idx"))}
     dev_in = {k: torch.empty_like(d[k]) for k in h_in}
     h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
     h_sel = torch.empty(sel.shape, dtype=sel.dtype).pin_memory()
     h2d = sum(v.numel() * v.element_size() for v in h_in.values())
-    d2h = h_out.numel() * h_out.element_size() + h_sel.numel() * h_sel.element_size()
+    d2h = h_out.numel() * h_out.element_size() + (0 if args.op == "swa" else h_sel.numel() * h_sel.element_size())
 
     def e2e_step():
         with torch.cuda.stream(stream):
             for k in h_in:
                 dev_in[k].copy_(h_in[k], non_blocking=True)
-            dsa.dsa_decode_ws(dev_in["q"], dev_in["q_idx"], dev_in["w_idx"], d["k_idx"], d["kv"], d["pos"], topk,
-                              out, sel, ws, k_scale=d["k_scale"])
+            if args.op == "swa":
+                dsa.dsa_swa_decode(dev_in["q"], d["kv"], w.pos, args.window, out, ws)
+            else:
+                dsa.dsa_decode_ws(dev_in["q"], dev_in["q_idx"], dev_in["w_idx"], d["k_idx"], d["kv"], d["pos"], topk,
+                                  out, sel, ws, k_scale=d["k_scale"])
             h_out.copy_(out, non_blocking=True)
-            h_sel.copy_(sel, non_blocking=True)
+            if args.op != "swa":
+                h_sel.copy_(sel, non_blocking=True)
 
     for _ in range(args.warmup):
         e2e_step()
@@ -375,16 +403,19 @@ def main():
     peak, which = peaks()
     achieved = ab["step"] / (ms * 1e-3) / 1e9
     roof = {"kernel": "step_kernel", "bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-            "frac": round(achieved / peak, 4), "peak_source": which, "traffic": profiled_traffic(w.name),
+            "frac": round(achieved / peak, 4), "peak_source": which, "traffic": profiled_traffic(w.name) if args.op == "step" else None,
             "algorithmic_bytes": ab["step"]}
 
     line = {
         "metric": METRIC, "value": round(value, 3), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms, 5), "us_per_step": round(ms * 1e3, 2),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": w.name, "L": L, "T": T, "topk": topk, "key_dtype": w.key_dtype, "recipe": w.recipe,
+        "config": {"workload": w.name, "op": args.op, **({"window": args.window} if args.op == "swa" else {}),
+                   "short_context_bypass": not args.no_bypass,
+                   "L": L, "T": T, "topk": topk, "key_dtype": w.key_dtype, "recipe": w.recipe,
                    "seed": w.seed, "parallelism": f"replicas{world}", "l2": "flushed before every step (write 2x L2, then read another 2x L2: cold and clean)",
-                   "timing": "CUDA-graph replay of dsa_decode_ws, CUDA events per step",
+                   "timing": "CUDA-graph replay of " + ("dsa_swa_decode" if args.op == "swa" else "dsa_decode_ws") +
+                             ", CUDA events per step",
                    "algorithmic_bytes_per_step": ab["step"], "unique_kv_rows": ab["unique_rows"],
                    "gathered_kv_rows": ab["gathered_rows"]},
         "frac_of_peak_hbm": round(ab["step"] / (ms * 1e-3) / 1e9 / peak, 4),
@@ -395,7 +426,7 @@ def main():
         "clocks": clk,
     }
     if rank == 0 and not args.no_cpu_baseline:
-        t_cpu, n_cpu, _, cores = cpu_baseline(w, args.cpu_budget)
+        t_cpu, n_cpu, _, cores = cpu_baseline(w, args.cpu_budget, args.op, args.window)
         line["cpu_baseline"] = {"value": round(ab["step"] / t_cpu / 1e9, 4), "unit": "GB/s", "cores": cores,
                                 "kind": "oracle", "us_per_step": round(t_cpu * 1e6, 1),
                                 "sample": f"{n_cpu} whole steps of {w.name}, median"}

@@ -131,6 +131,35 @@ DSA_API dsa_status_t dsa_decode_ws(const dsa_tensor_t *q, const dsa_tensor_t *q_
                            const int32_t *pos, int32_t topk, dsa_tensor_t *out, dsa_tensor_t *sel_idx,
                            dsa_stream_t stream, void *workspace, size_t workspace_bytes);
 
+/* dsa_decode_ws with an attention sink: `sink` is a per-head logit [64] f32
+ * (device, 16-byte aligned, not NULL) that joins each head's softmax denominator
+ * with no value row.  NaiveAI research page, "Hybrid SWA-DSA Architecture":
+ * both attention types of the model carry a sink bias. */
+DSA_API dsa_status_t dsa_decode_sink_ws(const dsa_tensor_t *q, const dsa_tensor_t *q_idx,
+                                        const dsa_tensor_t *w_idx, const dsa_tensor_t *k_idx_cache,
+                                        const dsa_tensor_t *kv_cache, const int32_t *pos, int32_t topk,
+                                        const float *sink, dsa_tensor_t *out, dsa_tensor_t *sel_idx,
+                                        dsa_stream_t stream, void *workspace, size_t workspace_bytes);
+
+/* Short-context bypass (on by default): when every query of a step sees at most
+ * topk positions (pos[t] + 1 <= topk), the top-k selects everything, so the step
+ * skips the indexer and the selection and takes the visible positions directly.
+ * Results are identical either way; 0 turns the bypass off (process-wide).
+ * NaiveAI research page, "A faster microbenchmark is not a faster model", weighs
+ * the same trade at 200 and 2,200 tokens. */
+DSA_API void dsa_set_short_context_bypass(int32_t enable);
+
+/* Sliding-window decode: attention of q [T][64][128] bf16 over the last
+ * min(pos[t] + 1, window) positions of kv_cache (the same [L][2][4][128] bf16
+ * layout and GQA grouping as the sparse step), 1 <= window <= 2048, optional
+ * sink as in dsa_decode_sink_ws (NULL for none); out [T][64][128] bf16.
+ * Workspace: dsa_workspace_bytes(T, L, window), control words as described
+ * there.  NaiveAI research page, "Hybrid SWA-DSA Architecture": the SWA layers
+ * attend over a 128-token window. */
+DSA_API dsa_status_t dsa_swa_decode(const dsa_tensor_t *q, const dsa_tensor_t *kv_cache, const int32_t *pos,
+                                    int32_t window, const float *sink, dsa_tensor_t *out, dsa_stream_t stream,
+                                    void *workspace, size_t workspace_bytes);
+
 /* Stage 1 alone: scores [T][ld] f32 (ld >= L, a multiple of 4).  scores[t][s] is
  * I[t,s] for s <= pos[t] and -inf for s > pos[t].  The sum is taken in fp32
  * (tensor-core dot products, then a fixed-order weighted sum over heads). */

@@ -137,6 +137,23 @@ def sparse_attn(q, kv, sel, sink=None) -> np.ndarray:
     return out
 
 
+def window_select(pos, window) -> np.ndarray:
+    """Sliding-window selection (NaiveAI research page, "Hybrid SWA-DSA
+    Architecture": SWA layers attend over a 128-token window): query t takes the
+    last min(pos[t] + 1, window) positions, ascending, padded with -1 to window."""
+    pos = np.asarray(pos, np.int64)
+    sel = np.full((pos.shape[0], window), -1, np.int32)
+    for t, p in enumerate(pos):
+        n = min(int(p) + 1, window)
+        sel[t, :n] = np.arange(int(p) + 1 - n, int(p) + 1)
+    return sel
+
+
+def swa_decode(q, kv, pos, window, sink=None) -> np.ndarray:
+    """fp64 sliding-window attention: attention over window_select(pos, window)."""
+    return sparse_attn(q, kv, window_select(pos, window), sink=sink)
+
+
 def decode(q, q_idx, w_idx, k_idx, k_scale, kv, pos, k, want_scores=False):
     """The whole step.  Returns (out fp64 [T][64][128], sel int32 [T][k][, scores])."""
     q = _c(q, np.uint16)

@@ -436,15 +436,20 @@ size_t dsa_workspace_bytes(int32_t T, int64_t L, int32_t topk)
     return layout(T, L).total;
 }
 
-dsa_status_t dsa_decode_ws(const dsa_tensor_t* q, const dsa_tensor_t* q_idx, const dsa_tensor_t* w_idx,
-                           const dsa_tensor_t* k_idx_cache, const dsa_tensor_t* kv_cache, const int32_t* pos,
-                           int32_t topk, dsa_tensor_t* out, dsa_tensor_t* sel_idx, dsa_stream_t stream_,
-                           void* workspace, size_t workspace_bytes)
+// Short-context bypass: when every query sees at most topk positions the top-k
+// selects everything, so the step skips scoring and selects by position.
+static std::atomic<int> g_bypass{1};
+
+static dsa_status_t decode_ws(const dsa_tensor_t* q, const dsa_tensor_t* q_idx, const dsa_tensor_t* w_idx,
+                       const dsa_tensor_t* k_idx_cache, const dsa_tensor_t* kv_cache, const int32_t* pos, int32_t topk,
+                       const float* sink, dsa_tensor_t* out, dsa_tensor_t* sel_idx, dsa_stream_t stream_,
+                       void* workspace, size_t workspace_bytes)
 {
     t_last_error.clear();
     Shape sh;
     dsa_status_t st = check_decode_args(q, q_idx, w_idx, k_idx_cache, kv_cache, pos, topk, out, sel_idx, sh);
     if (st) return st;
+    if (sink && !aligned16(sink)) return fail(DSA_ERR_INVALID_ARG, "sink: not 16-byte aligned");
     const Layout l = layout(sh.T, sh.L);
     if ((st = check_ws(workspace, workspace_bytes, l))) return st;
     DeviceInfo dev;
@@ -456,6 +461,10 @@ dsa_status_t dsa_decode_ws(const dsa_tensor_t* q, const dsa_tensor_t* q_idx, con
     p.phases = kPhaseIndex | kPhaseTopk | kPhaseAttend;
     p.grid = grid_blocks(dev, sh.fp8);
     set_pos(p, pos, sh.T);
+    if (g_bypass.load() && p.n_max <= topk) {
+        p.phases = kPhaseSelectPos | kPhaseAttend;
+        p.window = topk;
+    }
     p.L = static_cast<int32_t>(sh.L);
     p.topk = topk;
     p.q_idx = static_cast<const uint16_t*>(q_idx->data);
@@ -468,6 +477,7 @@ dsa_status_t dsa_decode_ws(const dsa_tensor_t* q, const dsa_tensor_t* q_idx, con
     p.q = static_cast<const uint16_t*>(q->data);
     p.kv = static_cast<const uint16_t*>(kv_cache->data);
     p.kv_ld = sh.kv_ld;
+    p.sink = sink;
     p.out = static_cast<uint16_t*>(out->data);
     p.err = dev.err;
     topk_params(p, workspace, l);
@@ -476,6 +486,71 @@ dsa_status_t dsa_decode_ws(const dsa_tensor_t* q, const dsa_tensor_t* q_idx, con
     st = launch(map, smap, p, sh.fp8, workspace, l, stream);
     for (int i = 1; i < 5; ++i) stage_event(i, stream);
     return st;
+}
+
+dsa_status_t dsa_decode_ws(const dsa_tensor_t* q, const dsa_tensor_t* q_idx, const dsa_tensor_t* w_idx,
+                           const dsa_tensor_t* k_idx_cache, const dsa_tensor_t* kv_cache, const int32_t* pos,
+                           int32_t topk, dsa_tensor_t* out, dsa_tensor_t* sel_idx, dsa_stream_t stream,
+                           void* workspace, size_t workspace_bytes)
+{
+    return decode_ws(q, q_idx, w_idx, k_idx_cache, kv_cache, pos, topk, nullptr, out, sel_idx, stream, workspace,
+                     workspace_bytes);
+}
+
+dsa_status_t dsa_decode_sink_ws(const dsa_tensor_t* q, const dsa_tensor_t* q_idx, const dsa_tensor_t* w_idx,
+                                const dsa_tensor_t* k_idx_cache, const dsa_tensor_t* kv_cache, const int32_t* pos,
+                                int32_t topk, const float* sink, dsa_tensor_t* out, dsa_tensor_t* sel_idx,
+                                dsa_stream_t stream, void* workspace, size_t workspace_bytes)
+{
+    if (!sink) return fail(DSA_ERR_INVALID_ARG, "sink: null");
+    return decode_ws(q, q_idx, w_idx, k_idx_cache, kv_cache, pos, topk, sink, out, sel_idx, stream, workspace,
+                     workspace_bytes);
+}
+
+void dsa_set_short_context_bypass(int32_t enable) { g_bypass.store(enable != 0 ? 1 : 0); }
+
+dsa_status_t dsa_swa_decode(const dsa_tensor_t* q, const dsa_tensor_t* kv_cache, const int32_t* pos, int32_t window,
+                            const float* sink, dsa_tensor_t* out, dsa_stream_t stream_, void* workspace,
+                            size_t workspace_bytes)
+{
+    t_last_error.clear();
+    if (!q) return fail(DSA_ERR_INVALID_ARG, "q: null");
+    Shape sh;
+    sh.T = static_cast<int>(q->shape[0]);
+    dsa_status_t st = check_T(q->shape[0]);
+    if (st) return st;
+    const int64_t qd[3] = {sh.T, kH, kD};
+    if ((st = check_contig(q, "q", DSA_BF16, 3, qd))) return st;
+    if ((st = check_kv(kv_cache, sh))) return st;
+    if (window < 1 || window > kMaxTopk) return fail(DSA_ERR_INVALID_ARG, "window = %d outside [1, %d]", window, kMaxTopk);
+    if ((st = check_contig(out, "out", DSA_BF16, 3, qd))) return st;
+    if (!pos) return fail(DSA_ERR_INVALID_ARG, "pos: null");
+    for (int t = 0; t < sh.T; ++t)
+        if (pos[t] < 0 || pos[t] >= sh.L) return fail(DSA_ERR_INVALID_ARG, "pos[%d] = %d outside [0, L)", t, pos[t]);
+    if (sink && !aligned16(sink)) return fail(DSA_ERR_INVALID_ARG, "sink: not 16-byte aligned");
+    const Layout l = layout(sh.T, sh.L);
+    if ((st = check_ws(workspace, workspace_bytes, l))) return st;
+    DeviceInfo dev;
+    if ((st = device_info(dev))) return st;
+    StepParams p{};
+    p.phases = kPhaseSelectPos | kPhaseAttend;
+    p.grid = grid_blocks(dev, false);
+    set_pos(p, pos, sh.T);
+    p.L = static_cast<int32_t>(sh.L);
+    p.topk = window;
+    p.window = window;
+    p.sel = at<int32_t>(workspace, l.list);   // the window's positions live in the candidate-list region
+    p.sel_ld = window;
+    p.q = static_cast<const uint16_t*>(q->data);
+    p.kv = static_cast<const uint16_t*>(kv_cache->data);
+    p.kv_ld = sh.kv_ld;
+    p.sink = sink;
+    p.out = static_cast<uint16_t*>(out->data);
+    p.err = dev.err;
+    attn_params(p, workspace, l, window);
+    CUtensorMap none;
+    std::memset(&none, 0, sizeof none);
+    return launch(none, none, p, false, workspace, l, reinterpret_cast<cudaStream_t>(stream_));
 }
 
 dsa_status_t dsa_decode(const dsa_tensor_t* q, const dsa_tensor_t* q_idx, const dsa_tensor_t* w_idx,

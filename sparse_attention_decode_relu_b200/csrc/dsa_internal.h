@@ -30,6 +30,7 @@ enum : int {
     kPhaseRanges = 2,   // per-block key ranges of caller-provided scores
     kPhaseTopk = 4,     // histogram, candidates, ordered emission
     kPhaseAttend = 8,   // split attention + merge
+    kPhaseSelectPos = 16,   // selection by position: the last `window` visible positions
 };
 
 struct StepParams {
@@ -64,6 +65,7 @@ struct StepParams {
     int32_t rows_per_split;  // multiple of 16, <= kMaxRowsPerSplit
     int32_t nsplit;
     const float* sink;       // [64] or nullptr
+    int32_t window;          // kPhaseSelectPos: positions selected per query (<= topk)
     float* po;               // [T][nsplit][64][128] partial outputs
     float2* pml;             // [T][nsplit][64] (max in log2 units, sum)
     uint16_t* out;           // [T][64][128] bf16

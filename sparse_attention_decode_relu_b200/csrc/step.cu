@@ -1108,6 +1108,25 @@ __device__ void phase_emit(const StepParams& p, uint8_t* smem, uint64_t* ring_fu
     }
 }
 
+// Selection by position (no scoring): query t takes the last min(n_t, window)
+// visible positions, ascending, then -1 padding to topk.  With window = topk and
+// n_t <= topk for every query this is exactly the top-k (everything is
+// selected), so the scoring phases can be skipped; with a small window it is
+// sliding-window attention.
+__device__ void phase_select_pos(const StepParams& p)
+{
+    const int64_t total = (int64_t)p.T * p.topk;
+    for (int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x; i < total; i += (int64_t)gridDim.x * kThreads) {
+        const int t = static_cast<int>(i / p.topk), j = static_cast<int>(i % p.topk);
+        int pos_t = 0;
+#pragma unroll
+        for (int k = 0; k < kMaxT; ++k)
+            if (k == t) pos_t = p.pos[k];
+        const int cnt = min(pos_t + 1, p.window);
+        p.sel[(int64_t)t * p.sel_ld + j] = j < cnt ? pos_t + 1 - cnt + j : -1;
+    }
+}
+
 // ==================================================================================
 // Phase 5: sparse attention per (query t, row split).  Warp 4 gathers whole
 // 2 KiB token rows (K then V of the 4 groups) by bulk async copy into a 6-stage
@@ -1425,8 +1444,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ok) phase_emit(p, smem, bars + kStreamBar, seq, res, scratch);
         stamp(p, 7);
     }
+    if (p.phases & kPhaseSelectPos) phase_select_pos(p);
     if (p.phases & kPhaseAttend) {
-        if (p.phases & (kPhaseIndex | kPhaseTopk)) ok = gb.sync(&ok_s) && ok;
+        if (p.phases & (kPhaseIndex | kPhaseTopk | kPhaseSelectPos)) ok = gb.sync(&ok_s) && ok;
         stamp(p, 8);
         if (ok) phase_attend(p, smem, bars);
         stamp(p, 9);

@@ -59,6 +59,12 @@ def lib():
             L.dsa_decode.argtypes = [T, T, T, T, T, P, ctypes.c_int32, T, T, P]
             L.dsa_decode_ws.restype = st
             L.dsa_decode_ws.argtypes = [T, T, T, T, T, P, ctypes.c_int32, T, T, P, P, ctypes.c_size_t]
+            L.dsa_decode_sink_ws.restype = st
+            L.dsa_decode_sink_ws.argtypes = [T, T, T, T, T, P, ctypes.c_int32, P, T, T, P, P, ctypes.c_size_t]
+            L.dsa_set_short_context_bypass.restype = None
+            L.dsa_set_short_context_bypass.argtypes = [ctypes.c_int32]
+            L.dsa_swa_decode.restype = st
+            L.dsa_swa_decode.argtypes = [T, T, P, ctypes.c_int32, P, T, P, P, ctypes.c_size_t]
             L.dsa_index_scores.restype = st
             L.dsa_index_scores.argtypes = [T, T, T, P, P, ctypes.c_int64, P]
             L.dsa_topk_from_scores.restype = st
@@ -143,13 +149,42 @@ def dsa_decode(q, q_idx, w_idx, k_idx_cache, kv_cache, pos, topk, out, sel_idx, 
                             ctypes.byref(o[1]), _stream(stream)))
 
 
+def _sink_ptr(sink):
+    if sink is None:
+        return None
+    if not sink.is_cuda or sink.dtype != torch.float32 or sink.numel() != 64 or not sink.is_contiguous():
+        raise ValueError("sink must be a contiguous float32 CUDA tensor of 64 logits")
+    return sink.data_ptr()
+
+
 def dsa_decode_ws(q, q_idx, w_idx, k_idx_cache, kv_cache, pos, topk, out, sel_idx, workspace, stream=None, *,
-                  k_scale=None):
+                  k_scale=None, sink=None):
+    """dsa_decode_ws, or dsa_decode_sink_ws when a sink is given."""
     a = [_desc(q), _desc(q_idx), _desc(w_idx), _desc(k_idx_cache, k_scale), _desc(kv_cache)]
     o = [_desc(out), _desc(sel_idx)]
-    _check(lib().dsa_decode_ws(*[ctypes.byref(x) for x in a], _pos(pos), int(topk), ctypes.byref(o[0]),
-                               ctypes.byref(o[1]), _stream(stream), workspace.data_ptr(),
-                               workspace.numel() * workspace.element_size()))
+    ws = (workspace.data_ptr(), workspace.numel() * workspace.element_size())
+    if sink is None:
+        _check(lib().dsa_decode_ws(*[ctypes.byref(x) for x in a], _pos(pos), int(topk), ctypes.byref(o[0]),
+                                   ctypes.byref(o[1]), _stream(stream), *ws))
+    else:
+        _check(lib().dsa_decode_sink_ws(*[ctypes.byref(x) for x in a], _pos(pos), int(topk), _sink_ptr(sink),
+                                        ctypes.byref(o[0]), ctypes.byref(o[1]), _stream(stream), *ws))
+
+
+def dsa_decode_sink_ws(q, q_idx, w_idx, k_idx_cache, kv_cache, pos, topk, sink, out, sel_idx, workspace,
+                       stream=None, *, k_scale=None):
+    dsa_decode_ws(q, q_idx, w_idx, k_idx_cache, kv_cache, pos, topk, out, sel_idx, workspace, stream,
+                  k_scale=k_scale, sink=sink)
+
+
+def dsa_set_short_context_bypass(enable: bool):
+    lib().dsa_set_short_context_bypass(1 if enable else 0)
+
+
+def dsa_swa_decode(q, kv_cache, pos, window, out, workspace, stream=None, *, sink=None):
+    _check(lib().dsa_swa_decode(ctypes.byref(_desc(q)), ctypes.byref(_desc(kv_cache)), _pos(pos), int(window),
+                                _sink_ptr(sink), ctypes.byref(_desc(out)), _stream(stream), workspace.data_ptr(),
+                                workspace.numel() * workspace.element_size()))
 
 
 def dsa_index_scores(q_idx, w_idx, k_idx_cache, pos, scores, stream=None, *, k_scale=None):
@@ -185,10 +220,8 @@ def dsa_topk_from_scores_noalloc(scores, L, pos, topk, sel_idx, stream=None):
 def dsa_sparse_attn(q, kv_cache, sel_idx, pos, out, workspace, stream=None, *, sink=None):
     d = [_desc(q), _desc(kv_cache), _desc(sel_idx)]
     o = _desc(out)
-    if sink is not None and (not sink.is_cuda or sink.dtype != torch.float32 or sink.numel() != 64):
-        raise ValueError("sink must be a float32 CUDA tensor of 64 logits")
-    _check(lib().dsa_sparse_attn(*[ctypes.byref(x) for x in d], _pos(pos),
-                                 None if sink is None else sink.data_ptr(), ctypes.byref(o), _stream(stream),
+    _check(lib().dsa_sparse_attn(*[ctypes.byref(x) for x in d], _pos(pos), _sink_ptr(sink), ctypes.byref(o),
+                                 _stream(stream),
                                  workspace.data_ptr(), workspace.numel() * workspace.element_size()))
 
 

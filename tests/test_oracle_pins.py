@@ -344,3 +344,33 @@ def test_planted_margin_full_size(orc):
     sel = orc.topk(s, w.pos, 2048)
     for t in range(w.T):
         assert np.array_equal(sel[t], w.planted)
+
+
+@pytest.mark.parametrize("window,with_sink", [(128, False), (128, True), (1, False), (300, True)])
+def test_window_attention_matches_band_mask(orc, window, with_sink):
+    """Sliding-window attention equals dense attention under a band mask
+    pos - window < s <= pos (torch, built here from the mask, not from the
+    oracle's selection), with the sink as an extra zero-valued key."""
+    rng = np.random.default_rng(50 + window)
+    T, L = 3, 260
+    q = synth.f32_to_bf16_bits(rng.standard_normal((T, 64, 128), dtype=np.float32))
+    kv = synth.f32_to_bf16_bits(rng.standard_normal((L, 2, 4, 128), dtype=np.float32))
+    pos = np.array([259, 100, 5], np.int32)
+    sink = rng.standard_normal(64).astype(np.float32) if with_sink else None
+    got = orc.swa_decode(q, kv, pos, window, sink=sink)
+    qd = torch.from_numpy(synth.bf16_bits_to_f32(q).astype(np.float64))
+    kd = torch.from_numpy(synth.bf16_bits_to_f32(kv).astype(np.float64))
+    K, V = kd[:, 0].permute(1, 0, 2), kd[:, 1].permute(1, 0, 2)
+    s = torch.arange(L)
+    for t in range(T):
+        mask = (s <= int(pos[t])) & (s > int(pos[t]) - window)
+        z = torch.einsum("ghd,gld->ghl", qd[t].reshape(4, 16, 128), K) / math.sqrt(128)
+        z = z.masked_fill(~mask[None, None, :], -math.inf)
+        if sink is not None:
+            z = torch.cat([z, torch.from_numpy(sink.astype(np.float64)).reshape(4, 16, 1)], dim=-1)
+        p = torch.softmax(z, dim=-1)[..., :L]
+        ref = torch.einsum("ghl,gld->ghd", p, V).reshape(64, 128).numpy()
+        np.testing.assert_allclose(got[t], ref, rtol=1e-11, atol=1e-12)
+    sel = orc.window_select(pos, window)
+    n = min(6, window)   # query 2 sees positions 0..5
+    assert sel[2, :n].tolist() == list(range(6 - n, 6)) and np.all(sel[2, n:] == -1)
