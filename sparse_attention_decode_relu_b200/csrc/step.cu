@@ -166,6 +166,22 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t& total,
     return before + x - v;
 }
 
+// Sum over the block in a fixed order (warp tree, then warps 0..7); the
+// barriers also order the shared-memory writes made before the call.
+__device__ __forceinline__ float block_sum_f(float v, uint32_t* scratch)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    __syncthreads();
+    if ((threadIdx.x & 31) == 0) scratch[threadIdx.x >> 5] = __float_as_uint(v);
+    __syncthreads();
+    float s = 0.f;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) s += __uint_as_float(scratch[w]);
+    __syncthreads();
+    return s;
+}
+
 __device__ __forceinline__ uint32_t block_sum(uint32_t v, uint32_t* scratch)
 {
     uint32_t total;
@@ -322,10 +338,18 @@ __device__ void phase_index(const CUtensorMap& kmap, const CUtensorMap& smap, co
     if (warp == 0) tmem_alloc(tmem_slot, kTmemCols);
     // The indexer queries as the B operand: row r = t*16 + j, 16-byte chunk c at
     // r*128 + (c ^ (r & 7))*16 (the 128B swizzle); rows >= T*16 are never read.
-    for (int i = tid; i < T * kHI * 8; i += kThreads) {
-        const int r = i >> 3, c = i & 7;
-        const uint4 v = __ldg(reinterpret_cast<const uint4*>(p.q_idx) + i);
-        *reinterpret_cast<uint4*>(qsw + r * 128 + ((c ^ (r & 7)) << 4)) = v;
+    {
+        uint4 v[kMaxT * kHI * 8 / kThreads];   // every load in flight before the first store
+#pragma unroll
+        for (int u = 0; u < kMaxT * kHI * 8 / kThreads; ++u) {
+            const int i = tid + u * kThreads;
+            v[u] = i < T * kHI * 8 ? __ldg(reinterpret_cast<const uint4*>(p.q_idx) + i) : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int u = 0; u < kMaxT * kHI * 8 / kThreads; ++u) {
+            const int i = tid + u * kThreads, r = i >> 3, c = i & 7;
+            if (i < T * kHI * 8) *reinterpret_cast<uint4*>(qsw + r * 128 + ((c ^ (r & 7)) << 4)) = v[u];
+        }
     }
     // Counters the top-k phases accumulate into start at zero.
     for (int i = blockIdx.x * kThreads + tid; i < p.zero_words; i += gridDim.x * kThreads) p.zero[i] = 0u;
@@ -714,7 +738,13 @@ __device__ Cut query_cut(const StepParams& p, int t, uint32_t* h, uint32_t* res,
     query_range(p, t, lo, hi, scratch);
     const int shift = range_shift(lo, hi);
     const uint32_t* gh = p.hist + (int64_t)t * kHistBins;
-    for (int b = threadIdx.x; b < kHistBins; b += kThreads) h[b] = __ldcg(gh + b);
+    {
+        uint32_t v[kHistBins / kThreads];   // every load in flight before the first use
+#pragma unroll
+        for (int i = 0; i < kHistBins / kThreads; ++i) v[i] = __ldcg(gh + threadIdx.x + i * kThreads);
+#pragma unroll
+        for (int i = 0; i < kHistBins / kThreads; ++i) h[threadIdx.x + i * kThreads] = v[i];
+    }
     __syncthreads();
     find_from_top<kHistBins>(h, static_cast<uint32_t>(p.topk), res, scratch);
     Cut cu{lo, hi, 0u};
@@ -963,7 +993,19 @@ __device__ void phase_emit(const StepParams& p, uint8_t* smem, uint64_t* ring_fu
         for (int c = tid; c < it.c; c += kThreads) before += __ldcg(above + c);
         const bool fits = m <= static_cast<uint32_t>(kInCap);
         if (fits)
-            for (uint32_t j = tid; j < m; j += kThreads) in[j] = __ldcg(glist + j);
+            for (uint32_t j0 = 0; j0 < m; j0 += 8 * kThreads) {   // eight loads in flight per thread
+                uint2 v[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const uint32_t j = j0 + u * kThreads + tid;
+                    v[u] = j < m ? __ldcg(glist + j) : make_uint2(0u, 0u);
+                }
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const uint32_t j = j0 + u * kThreads + tid;
+                    if (j < m) in[j] = v[u];
+                }
+            }
         if (tid == 0) nval = 0;
         __syncthreads();
         uint32_t nin = 0;   // keys inside the threshold bin, gathered in vals
@@ -1179,7 +1221,17 @@ __device__ void phase_attend(const StepParams& p, uint8_t* smem, uint64_t* bars)
         if (warp == kConsumers) {
             // producer: validate the selected rows, gather them whole
             const int32_t* selrow = p.sel + (int64_t)t * p.sel_ld + r0;
-            for (int j = lane; j < r1 - r0; j += 32) sel_s[j] = __ldcg(selrow + j);
+            {
+                int32_t v[kMaxRowsPerSplit / 32];   // every load in flight before the first store
+#pragma unroll
+                for (int u = 0; u < kMaxRowsPerSplit / 32; ++u) {
+                    const int j = lane + u * 32;
+                    v[u] = j < r1 - r0 ? __ldcg(selrow + j) : -1;
+                }
+#pragma unroll
+                for (int u = 0; u < kMaxRowsPerSplit / 32; ++u)
+                    if (lane + u * 32 < r1 - r0) sel_s[lane + u * 32] = v[u];
+            }
             __syncwarp();
             for (int k = 0; k < ntile; ++k) {
                 const int kk = phase_base + k;
@@ -1345,47 +1397,72 @@ __device__ void phase_attend(const StepParams& p, uint8_t* smem, uint64_t* bars)
 __device__ void phase_merge(const StepParams& p, uint8_t* smem, uint32_t* scratch)
 {
     float* part = reinterpret_cast<float*>(smem);   // [4][128] partial sums + [4] denominators
+    float* wsp = part + 4 * kD + 4;                 // [kMaxAttnItems] weight of each split
     const int items = p.T * kH;
-    const int grp = threadIdx.x >> 6, d2 = threadIdx.x & 63;
+    const int tid = threadIdx.x, grp = tid >> 6, d2 = tid & 63;
     for (int r = 0;; ++r) {
         const int i = item_of(r);
         if (i >= items) break;
         const int t = i / kH, h = i % kH;
         const float2* ml = p.pml + (int64_t)t * p.nsplit * kH + h;
-        // running max over all splits (each thread reads a quarter, then combine)
-        float M = -INFINITY;
-        for (int s = grp; s < p.nsplit; s += 4) M = fmaxf(M, __ldcg(ml + (int64_t)s * kH).x);
-        if (d2 == 0) scratch[grp] = __float_as_uint(M);
-        __syncthreads();
-        M = fmaxf(fmaxf(__uint_as_float(scratch[0]), __uint_as_float(scratch[1])),
-                  fmaxf(__uint_as_float(scratch[2]), __uint_as_float(scratch[3])));
-        float sink = -INFINITY;
-        if (p.sink != nullptr) {
-            sink = p.sink[h] * kLog2e;
-            M = fmaxf(M, sink);
+        // (max, sum) of every split, one load per thread, then the running max
+        float2 mv[kMaxAttnItems / kThreads];
+#pragma unroll
+        for (int u = 0; u < kMaxAttnItems / kThreads; ++u) {
+            const int s = tid + u * kThreads;
+            mv[u] = s < p.nsplit ? __ldcg(ml + (int64_t)s * kH) : make_float2(-INFINITY, 0.f);
         }
-        float den = 0.f, ax = 0.f, ay = 0.f;
-#pragma unroll 4
-        for (int s = grp; s < p.nsplit; s += 4) {
-            const float2 v = __ldcg(ml + (int64_t)s * kH);
-            if (v.x == -INFINITY) continue;
-            const float w = exp2f(v.x - M);
-            den += w * v.y;
-            const float2 o = __ldcg(reinterpret_cast<const float2*>(
-                p.po + (((int64_t)t * p.nsplit + s) * kH + h) * kD + 2 * d2));
-            ax += w * o.x;
-            ay += w * o.y;
+        float M = -INFINITY;
+#pragma unroll
+        for (int u = 0; u < kMaxAttnItems / kThreads; ++u) M = fmaxf(M, mv[u].x);
+        float sink = -INFINITY;
+        if (p.sink != nullptr) sink = p.sink[h] * kLog2e;
+        M = fmaxf(M, sink);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+        if ((tid & 31) == 0) scratch[tid >> 5] = __float_as_uint(M);
+        __syncthreads();
+        M = __uint_as_float(scratch[0]);
+#pragma unroll
+        for (int w = 1; w < kWarps; ++w) M = fmaxf(M, __uint_as_float(scratch[w]));
+        // split weights (0 for a split without rows) and this thread's share of the denominator
+        float den = 0.f;
+#pragma unroll
+        for (int u = 0; u < kMaxAttnItems / kThreads; ++u) {
+            const int s = tid + u * kThreads;
+            if (s < p.nsplit) {
+                const float w = mv[u].x == -INFINITY ? 0.f : exp2f(mv[u].x - M);
+                wsp[s] = w;
+                den += w * mv[u].y;
+            }
+        }
+        __syncthreads();
+        // numerator: group g takes splits g, g+4, ...; eight loads in flight per thread
+        float ax = 0.f, ay = 0.f;
+        const float2* po = reinterpret_cast<const float2*>(p.po + ((int64_t)t * p.nsplit * kH + h) * kD) + d2;
+        for (int s0 = grp; s0 < p.nsplit; s0 += 32) {
+            float2 ov[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int s = s0 + 4 * u;
+                ov[u] = (s < p.nsplit && wsp[s] > 0.f) ? __ldcg(po + (int64_t)s * kH * (kD / 2)) : make_float2(0.f, 0.f);
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int s = s0 + 4 * u;
+                const float w = s < p.nsplit ? wsp[s] : 0.f;
+                ax = fmaf(w, ov[u].x, ax);
+                ay = fmaf(w, ov[u].y, ay);
+            }
         }
         part[grp * kD + 2 * d2] = ax;
         part[grp * kD + 2 * d2 + 1] = ay;
-        if (d2 == 0) part[4 * kD + grp] = den;
-        __syncthreads();
+        den = block_sum_f(den, scratch);
         if (grp == 0) {
-            float dd = (p.sink != nullptr && M != -INFINITY) ? exp2f(sink - M) : 0.f;
+            float dd = den + ((p.sink != nullptr && M != -INFINITY) ? exp2f(sink - M) : 0.f);
             float x = 0.f, y = 0.f;
 #pragma unroll
             for (int g = 0; g < 4; ++g) {
-                dd += part[4 * kD + g];
                 x += part[g * kD + 2 * d2];
                 y += part[g * kD + 2 * d2 + 1];
             }
