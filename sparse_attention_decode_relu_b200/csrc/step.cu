@@ -290,8 +290,8 @@ constexpr uint32_t kTmemCols = 256;        // two accumulator buffers of 128 col
 constexpr int kMmaBar = 40;                // the two MMA-completion mbarriers
 constexpr int kTileBytesBf16 = kKeyTile * kDI * 2;   // 16 KiB, one 128 x 64 bf16 operand tile
 static_assert(kIdxStages * kTileBytesBf16 + 2 * kTileBytesBf16 + kTileBytesBf16 + kMaxT * kHI * 4 +
-                  (kIdxStages + 2) * kKeyTile * 4 <= kDataBytes, "indexer buffers fit the data region");
-static_assert(kMmaBar + 2 <= kBarSlots && kIdxStages + 1 <= 8, "indexer mbarriers fit");
+                  (kIdxStages + 4) * kKeyTile * 4 <= kDataBytes, "indexer buffers fit the data region");
+static_assert(kMmaBar + 6 <= kBarSlots && kIdxStages + 1 <= 8, "indexer mbarriers fit");
 
 template <bool FP8>
 __device__ void phase_index(const CUtensorMap& kmap, const CUtensorMap& smap, const StepParams& p, uint8_t* smem,
@@ -303,10 +303,12 @@ __device__ void phase_index(const CUtensorMap& kmap, const CUtensorMap& smap, co
     uint8_t* qsw = cvt + (FP8 ? 2 * kTileBytesBf16 : 0);                   // [128 rows][128 B] queries
     float* w_s = reinterpret_cast<float*>(qsw + kTileBytesBf16);           // [8][16]
     float* sc_s = w_s + kMaxT * kHI;                                       // [kIdxStages][128] scales
-    float* scl = sc_s + kIdxStages * kKeyTile;                             // [2][128] scales of the TMEM tiles
-    uint64_t* full = bars;                  // [kIdxStages]
+    float* scl = sc_s + kIdxStages * kKeyTile;                             // [2 halves][2][128] tile scales
+    uint64_t* full = bars;                  // [kIdxStages] key tile landed
     uint64_t* setup = bars + kIdxStages;
-    uint64_t* mmab = bars + kMmaBar;        // [2]
+    uint64_t* mmab = bars + kMmaBar;        // [2] MMAs of the tile in TMEM buffer b complete
+    uint64_t* convb = mmab + 2;             // [2] every thread is done with the raw tile of buffer b
+    uint64_t* tfree = mmab + 4;             // [2] every thread is done reading TMEM buffer b
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int T = p.T;
@@ -325,8 +327,11 @@ __device__ void phase_index(const CUtensorMap& kmap, const CUtensorMap& smap, co
         prefetch_tmap(&kmap);
         if (scaled) prefetch_tmap(&smap);
         for (int s = 0; s <= kIdxStages; ++s) mbar_init(&bars[s], 1);
-        mbar_init(&mmab[0], 1);
-        mbar_init(&mmab[1], 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&mmab[b], 1);
+            mbar_init(&convb[b], kThreads);
+            mbar_init(&tfree[b], kThreads);
+        }
         fence_mbar_init();
         mbar_arrive_expect_tx(setup, T * kHI * 4);
         bulk_g2s(w_s, p.w, T * kHI * 4, setup);
@@ -380,61 +385,62 @@ __device__ void phase_index(const CUtensorMap& kmap, const CUtensorMap& smap, co
     const uint32_t idesc = umma_idesc_bf16(kKeyTile, T * kHI);
     const uint64_t bdesc = umma_desc_sw128(smem_u32(qsw));
 
-    int mma_issued = 0, mma_done = 0;
-    // Epilogue of local tile e: wait for its MMA, then scores from TMEM buffer e & 1.
+    int mma_issued = 0, mma_done = 0;   // (thread 0) tiles whose MMAs were issued / waited for
+    float* my_scl = scl + half * 2 * kKeyTile;   // this half's copy: written and read by the same thread
+    // Epilogue of local tile e: wait for its MMAs, then scores from TMEM buffer e & 1.
     auto epilogue = [&](int e) -> bool {
         const int b = e & 1;
-        const bool okm = __syncthreads_and(mbar_wait(&mmab[b], (e >> 1) & 1, p.err));
-        mma_done = e + 1;
+        if (!mbar_wait(&mmab[b], (e >> 1) & 1, p.err)) return false;
         tc_fence_after();
-        if (okm && qa < qb) {
+        if (qa < qb) {
             const int s = tile_of(e) * kKeyTile + row;
-            const float scale = scl[b * kKeyTile + row];
-            const uint32_t tbase = tmem + static_cast<uint32_t>((quad * 32) << 16) + b * 128;
-            // Two queries per TMEM load; the 16-head sum as four interleaved partial
-            // sums over heads {j, j+4, j+8, j+12}, combined in a fixed order.
+            const float scale = my_scl[b * kKeyTile + row];
+            const uint32_t tbase = tmem + static_cast<uint32_t>((quad * 32) << 16) + b * 128 + qa * kHI;
+            // Up to four queries: two TMEM loads in flight, one wait; the 16-head sum as
+            // four interleaved partial sums over heads {j, j+4, j+8, j+12}, combined in
+            // a fixed order.
+            uint32_t r[2][32];
+            tmem_ld32_nowait(tbase, r[0]);
+            if (qb - qa > 2) tmem_ld32_nowait(tbase + 2 * kHI, r[1]);
+            tmem_ld_wait();
 #pragma unroll
-            for (int u0 = 0; u0 < 4; u0 += 2) {
-                const int t0 = qa + u0;
-                if (t0 < qb) {
-                    uint32_t r[32];
-                    tmem_ld32_nowait(tbase + t0 * kHI, r);
-                    tmem_ld_wait();
+            for (int u = 0; u < 4; ++u) {
+                const int t = qa + u;
+                if (t < qb) {
+                    const float4* w4 = reinterpret_cast<const float4*>(w_s + t * kHI);
+                    const float* v = reinterpret_cast<const float*>(&r[u >> 1][(u & 1) * 16]);
+                    float part[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        const int u = u0 + h, t = t0 + h;
-                        if (t < qb) {
-                            const float4* w4 = reinterpret_cast<const float4*>(w_s + t * kHI);
-                            float part[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                            for (int g4 = 0; g4 < 4; ++g4) {
-                                const float4 w = w4[g4];
-                                const float* v = reinterpret_cast<const float*>(r + h * 16 + g4 * 4);
-                                part[0] = fmaf(fmaxf(v[0], 0.f), w.x, part[0]);
-                                part[1] = fmaf(fmaxf(v[1], 0.f), w.y, part[1]);
-                                part[2] = fmaf(fmaxf(v[2], 0.f), w.z, part[2]);
-                                part[3] = fmaf(fmaxf(v[3], 0.f), w.w, part[3]);
-                            }
-                            const float acc = ((part[0] + part[1]) + (part[2] + part[3])) * scale;
-                            if (s < p.L) {
-                                if (s <= pos_q[u]) {
-                                    p.scores[(int64_t)t * p.ld + s] = acc;
-                                    const uint32_t k = score_key(acc);
-                                    klo[u] = min(klo[u], k);
-                                    khi[u] = max(khi[u], k);
-                                } else {
-                                    p.scores[(int64_t)t * p.ld + s] = -INFINITY;
-                                }
-                            }
+                    for (int g4 = 0; g4 < 4; ++g4) {
+                        const float4 w = w4[g4];
+                        part[0] = fmaf(fmaxf(v[g4 * 4 + 0], 0.f), w.x, part[0]);
+                        part[1] = fmaf(fmaxf(v[g4 * 4 + 1], 0.f), w.y, part[1]);
+                        part[2] = fmaf(fmaxf(v[g4 * 4 + 2], 0.f), w.z, part[2]);
+                        part[3] = fmaf(fmaxf(v[g4 * 4 + 3], 0.f), w.w, part[3]);
+                    }
+                    const float acc = ((part[0] + part[1]) + (part[2] + part[3])) * scale;
+                    if (s < p.L) {
+                        if (s <= pos_q[u]) {
+                            p.scores[(int64_t)t * p.ld + s] = acc;
+                            const uint32_t k = score_key(acc);
+                            klo[u] = min(klo[u], k);
+                            khi[u] = max(khi[u], k);
+                        } else {
+                            p.scores[(int64_t)t * p.ld + s] = -INFINITY;
                         }
                     }
                 }
             }
         }
         tc_fence_before();
-        return okm;
+        mbar_arrive(&tfree[b]);
+        return true;
     };
 
+    // Steady state without block-wide barriers: every thread widens its share of
+    // tile it and signals convb; thread 0 issues tile it's MMAs once every share is
+    // in and the epilogue of tile it - 2 has released the TMEM buffer; every thread
+    // then runs the epilogue of tile it - 1.
     bool aborted = __syncthreads_or(!ok);
     int it = 0;
     for (; !aborted; ++it) {
@@ -442,20 +448,20 @@ __device__ void phase_index(const CUtensorMap& kmap, const CUtensorMap& smap, co
         const bool have = tile < ntiles;
         if (have) {
             const int stage = it % kIdxStages;
-            ok = mbar_wait(&full[stage], (it / kIdxStages) & 1, p.err);
-            if (__syncthreads_or(!ok)) {
+            const int b = it & 1;
+            if (!mbar_wait(&full[stage], (it / kIdxStages) & 1, p.err)) {
                 aborted = true;
                 break;
             }
-            const int b = it & 1;
+            if (qa < qb) my_scl[b * kKeyTile + row] = scaled ? sc_s[stage * kKeyTile + row] : 1.0f;
             uint32_t a_addr;
             if constexpr (FP8) {
                 // Widen 128 x 64 E4M3 codes to bf16 (exact) in the 128B-swizzled layout.
                 const uint8_t* raw = ring + stage * raw_bytes;
                 uint8_t* dst = cvt + b * kTileBytesBf16;
 #pragma unroll
-                for (int r = 0; r < 2; ++r) {
-                    const int chunk = tid + r * kThreads;
+                for (int rr = 0; rr < 2; ++rr) {
+                    const int chunk = tid + rr * kThreads;
                     const int kr = chunk >> 2, piece = chunk & 3;
                     const uint4 v = *reinterpret_cast<const uint4*>(raw + kr * 64 + piece * 16);
                     const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
@@ -474,32 +480,39 @@ __device__ void phase_index(const CUtensorMap& kmap, const CUtensorMap& smap, co
             } else {
                 a_addr = smem_u32(ring + stage * raw_bytes);
             }
-            if (tid < kKeyTile) scl[b * kKeyTile + tid] = scaled ? sc_s[stage * kKeyTile + tid] : 1.0f;
-            tc_fence_before();
-            __syncthreads();   // operands ready; the epilogue of local tile it - 2 is done with buffer b
+            mbar_arrive(&convb[b]);   // this thread is done with the raw stage (scale copy, widening)
             if (tid == 0) {
-                tc_fence_after();
-                const uint64_t adesc = umma_desc_sw128(a_addr);
+                bool okw = true;
+                okw = mbar_wait(&convb[b], (it >> 1) & 1, p.err);
+                if (okw && it >= 2) okw = mbar_wait(&tfree[b], ((it >> 1) - 1) & 1, p.err);
+                if (okw) {
+                    tc_fence_after();
+                    const uint64_t adesc = umma_desc_sw128(a_addr);
 #pragma unroll
-                for (int k = 0; k < kDI / 16; ++k)
-                    tc_mma_bf16(tmem + b * 128, adesc + 2 * k, bdesc + 2 * k, idesc, k > 0 ? 1u : 0u);
-                tc_commit(&mmab[b]);
-                if constexpr (FP8) {   // the raw tile is consumed: refill its stage now
-                    const int next = tile_of(it + kIdxStages);
-                    if (next < ntiles) {
-                        load_tile(stage, next);
-                        ++issued;
+                    for (int k = 0; k < kDI / 16; ++k)
+                        tc_mma_bf16(tmem + b * 128, adesc + 2 * k, bdesc + 2 * k, idesc, k > 0 ? 1u : 0u);
+                    tc_commit(&mmab[b]);
+                    ++mma_issued;
+                    if constexpr (FP8) {   // every share of the raw tile is consumed: refill its stage now
+                        const int next = tile_of(it + kIdxStages);
+                        if (next < ntiles) {
+                            load_tile(stage, next);
+                            ++issued;
+                        }
                     }
+                } else {
+                    aborted = true;
                 }
             }
-            ++mma_issued;
+            if (aborted) break;
         }
         if (it > 0) {
             if (!epilogue(it - 1)) {
                 aborted = true;
                 break;
             }
-            if constexpr (!FP8) {   // the MMA of local tile it - 1 is complete: refill its stage
+            if (tid == 0) mma_done = it;
+            if constexpr (!FP8) {   // the MMAs of local tile it - 1 are complete: refill its stage
                 const int next = tile_of(it - 1 + kIdxStages);
                 if (tid == 0 && next < ntiles) {
                     load_tile((it - 1) % kIdxStages, next);
@@ -509,12 +522,14 @@ __device__ void phase_index(const CUtensorMap& kmap, const CUtensorMap& smap, co
         }
         if (!have) break;
     }
-    if (aborted) {   // let copies and MMAs still in flight land before the smem and TMEM are reused
-        if (tid == 0) {
-            mbar_wait(setup, 0, p.err);
-            for (int k = it; k < issued; ++k) mbar_wait(&full[k % kIdxStages], (k / kIdxStages) & 1, p.err);
-            for (int e = mma_done; e < mma_issued; ++e) mbar_wait(&mmab[e & 1], (e >> 1) & 1, p.err);
-        }
+    // A wait that ran out (error bit set) ends the loop for that thread; the others
+    // run into bounded waits and stop too.  Copies and MMAs still in flight land
+    // before the shared memory and TMEM are reused.
+    aborted = __syncthreads_or(aborted);
+    if (aborted && tid == 0) {
+        mbar_wait(setup, 0, p.err);
+        for (int k = it; k < issued; ++k) mbar_wait(&full[k % kIdxStages], (k / kIdxStages) & 1, p.err);
+        for (int e = mma_done; e < mma_issued; ++e) mbar_wait(&mmab[e & 1], (e >> 1) & 1, p.err);
     }
     tc_fence_before();
     __syncthreads();
