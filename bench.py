@@ -138,7 +138,10 @@ class Clocks:
                 **({"error": self.err} if self.err else {})}
 
 
-def dist_setup(n):
+def dist_setup(n, backend="nccl"):
+    """One process per GPU (torchrun sets RANK / WORLD_SIZE / LOCAL_RANK); every
+    rank runs an independent replica of the step.  backend "gloo" (CPU, no
+    device) serves the host-side tests."""
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -149,29 +152,41 @@ def dist_setup(n):
 
         import torch.distributed as dist
 
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
-    else:
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif backend == "nccl":
         torch.cuda.set_device(0)
     return rank, world, local
 
 
-def reduce_max(x, world):
+def reduce_max(x, world, device="cuda"):
+    """The maximum of x over all ranks (the slowest replica sets the step time)."""
     if world == 1:
         return x
     import torch.distributed as dist
 
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
 
-def barrier(world):
+def barrier(world, cuda=True):
     if world > 1:
         import torch.distributed as dist
 
         dist.barrier()
-    torch.cuda.synchronize()
+    if cuda:
+        torch.cuda.synchronize()
+
+
+def whole_job_gbs(bytes_per_step, ms_max, world):
+    """Weak scaling: every rank moves bytes_per_step per step; the job's rate is
+    the bytes of all ranks over the slowest rank's step time."""
+    return world * bytes_per_step / (ms_max * 1e-3) / 1e9
 
 
 def swa_bytes(w, window):
@@ -357,7 +372,7 @@ def main():
     phase_us = {k: round(v / args.steps, 2) for k, v in phase_sum.items()}
 
     ab = swa_bytes(w, args.window) if args.op == "swa" else algorithmic_bytes(w, sel.cpu().numpy())
-    value = world * ab["step"] / (ms * 1e-3) / 1e9
+    value = whole_job_gbs(ab["step"], ms, world)
 
     # End to end through the public API: per step the query-side inputs come from
     # pinned host memory and the outputs go back to it; the caches stay resident.
@@ -395,7 +410,7 @@ def main():
         stream.synchronize()
         e_times.append(a.elapsed_time(b))
     e_ms = reduce_max(statistics.mean(e_times), world)
-    e2e = {"value": round(world * ab["step"] / (e_ms * 1e-3) / 1e9, 3), "unit": "GB/s",
+    e2e = {"value": round(whole_job_gbs(ab["step"], e_ms, world), 3), "unit": "GB/s",
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e_ms, 4)}
 
     # Roofline of the step kernel (the only kernel: every phase of the step runs in
