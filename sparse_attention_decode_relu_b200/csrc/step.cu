@@ -1409,7 +1409,10 @@ __device__ void phase_attend(const StepParams& p, uint8_t* smem, uint64_t* bars)
 // Phase 6: merge the splits of each (query, head) in split order.  Thread
 // (g, d) sums splits g, g+4, ... for dims 2d, 2d+1; the four partial sums are
 // then added in a fixed order.
-__device__ void phase_merge(const StepParams& p, uint8_t* smem, uint32_t* scratch)
+// Phase 6 for one or two queries (many splits per head): one block per (query,
+// head); four thread groups share the splits, with every split's (max, sum) in
+// one load per thread and eight partial-output loads in flight per thread.
+__device__ void phase_merge_block(const StepParams& p, uint8_t* smem, uint32_t* scratch)
 {
     float* part = reinterpret_cast<float*>(smem);   // [4][128] partial sums + [4] denominators
     float* wsp = part + 4 * kD + 4;                 // [kMaxAttnItems] weight of each split
@@ -1488,6 +1491,94 @@ __device__ void phase_merge(const StepParams& p, uint8_t* smem, uint32_t* scratc
     }
 }
 
+// Phase 6 for three or more queries: one warp per item (query t, head h, half of
+// the 128 dims): every split's (max, sum) with one load per lane and split, the
+// running max and the denominator by warp shuffles, the weighted partial outputs
+// with sixteen loads in flight per lane, all in a fixed order.  A sink joins the
+// denominator with no value row.
+constexpr int kMergeSplitsSmem = 512;      // split weights a warp keeps in shared memory (>= nsplit)
+static_assert(kWarps * 2 * kMergeSplitsSmem * 4 <= kDataBytes, "merge weights fit");
+static_assert(kMaxAttnItems <= kMergeSplitsSmem, "every split has a weight slot");
+
+__device__ void phase_merge(const StepParams& p, uint8_t* smem, uint32_t* /*scratch*/)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    float* wsp = reinterpret_cast<float*>(smem) + warp * 2 * kMergeSplitsSmem;   // this warp's split weights
+    float* lsp = wsp + kMergeSplitsSmem;                                            // and split sums
+    const int P = 2;                              // shares of the 128 dims per (t, h)
+    const int dpl = kD / (32 * P);                // dims per lane: 1 or 2
+    const int items = p.T * kH * P;
+    const int ns = p.nsplit;
+    for (int i = blockIdx.x * kWarps + warp; i < items; i += gridDim.x * kWarps) {
+        const int t = i / (kH * P), h = (i / P) % kH, part = i % P;
+        const float2* ml = p.pml + (int64_t)t * ns * kH + h;
+        float M = -INFINITY;
+        for (int s0 = 0; s0 < ns; s0 += 32 * 4) {   // four (max, sum) loads in flight per lane
+            float2 v[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int s = s0 + u * 32 + lane;
+                v[u] = s < ns ? __ldcg(ml + (int64_t)s * kH) : make_float2(-INFINITY, 0.f);
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int s = s0 + u * 32 + lane;
+                if (s < ns) {
+                    wsp[s] = v[u].x;   // the split's max for now, its weight below
+                    lsp[s] = v[u].y;
+                }
+                M = fmaxf(M, v[u].x);
+            }
+        }
+        const float sink = p.sink != nullptr ? p.sink[h] * kLog2e : -INFINITY;
+        M = fmaxf(M, sink);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+        float den = 0.f;
+        for (int s = lane; s < ns; s += 32) {
+            const float m = wsp[s];
+            const float w = m == -INFINITY ? 0.f : exp2f(m - M);
+            den += w * lsp[s];
+            wsp[s] = w;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+        __syncwarp();
+        // numerator for this lane's dims, splits in order, sixteen loads in flight
+        const int d0 = part * (kD / P) + lane * dpl;
+        const float* po = p.po + ((int64_t)t * ns * kH + h) * kD + d0;
+        float x0 = 0.f, x1 = 0.f;
+        for (int s0 = 0; s0 < ns; s0 += 16) {
+            float2 o[16];
+#pragma unroll
+            for (int u = 0; u < 16; ++u) {
+                const int s = s0 + u;
+                const bool use = s < ns && wsp[s] > 0.f;
+                const float* src = po + (int64_t)s * kH * kD;
+                o[u] = !use ? make_float2(0.f, 0.f)
+                            : (dpl == 2 ? __ldcg(reinterpret_cast<const float2*>(src)) : make_float2(__ldcg(src), 0.f));
+            }
+#pragma unroll
+            for (int u = 0; u < 16; ++u) {
+                const int s = s0 + u;
+                const float w = s < ns ? wsp[s] : 0.f;
+                x0 = fmaf(w, o[u].x, x0);
+                x1 = fmaf(w, o[u].y, x1);
+            }
+        }
+        const float dd = den + ((p.sink != nullptr && M != -INFINITY) ? exp2f(sink - M) : 0.f);
+        const float inv = dd > 0.f ? 1.0f / dd : 0.f;
+        uint16_t* dst = p.out + ((int64_t)t * kH + h) * kD + d0;
+        if (dpl == 2) {
+            *reinterpret_cast<uint32_t*>(dst) = pack_bf16(x0 * inv, x1 * inv);
+        } else {
+            const __nv_bfloat16 b = __float2bfloat16_rn(x0 * inv);
+            *reinterpret_cast<__nv_bfloat16*>(dst) = b;
+        }
+        __syncwarp();
+    }
+}
+
 // ==================================================================================
 template <bool FP8>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -1544,7 +1635,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         stamp(p, 9);
         ok = gb.sync(&ok_s) && ok;
         stamp(p, 10);
-        if (ok) phase_merge(p, smem, scratch);
+        if (ok) {
+            if (p.T <= 2)
+                phase_merge_block(p, smem, scratch);
+            else
+                phase_merge(p, smem, scratch);
+        }
         stamp(p, 11);
     }
     if (p.bar_ctrl != nullptr) barrier_exit(p);
