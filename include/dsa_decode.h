@@ -141,6 +141,20 @@ DSA_API dsa_status_t dsa_decode_sink_ws(const dsa_tensor_t *q, const dsa_tensor_
                                         const float *sink, dsa_tensor_t *out, dsa_tensor_t *sel_idx,
                                         dsa_stream_t stream, void *workspace, size_t workspace_bytes);
 
+/* dsa_decode_ws with the query positions in device memory: pos_device is int32
+ * [T] (T = q's first dimension), read by the kernel at launch, so one CUDA graph
+ * of the step serves every decode position (write the next positions into the
+ * buffer, replay).  The work is split over the whole cache [0, L) instead of the
+ * positions known on the host, and the short-context bypass does not apply.  A
+ * position outside [0, L) is clamped and flags DSA_ERR_DEVICE (bit 16).  sink is
+ * NULL or as in dsa_decode_sink_ws.  NaiveAI research page, "The execution
+ * model": rounds of the decoding loop advance on the device without the host. */
+DSA_API dsa_status_t dsa_decode_devpos_ws(const dsa_tensor_t *q, const dsa_tensor_t *q_idx,
+                                          const dsa_tensor_t *w_idx, const dsa_tensor_t *k_idx_cache,
+                                          const dsa_tensor_t *kv_cache, const int32_t *pos_device, int32_t topk,
+                                          const float *sink, dsa_tensor_t *out, dsa_tensor_t *sel_idx,
+                                          dsa_stream_t stream, void *workspace, size_t workspace_bytes);
+
 /* Short-context bypass (on by default): when every query of a step sees at most
  * topk positions (pos[t] + 1 <= topk), the top-k selects everything, so the step
  * skips the indexer and the selection and takes the visible positions directly.

@@ -17,6 +17,7 @@ enum : uint32_t {
     ERR_BAD_INDEX = 1u << 1,      // a selected index outside [0, pos[t]]
     ERR_TOPK_STATE = 1u << 2,     // top-k bookkeeping inconsistent (bad input scores)
     ERR_WORKSPACE_STATE = 1u << 3,  // workspace control words were not zero at launch
+    ERR_BAD_POS = 1u << 4,          // a query position in device memory outside [0, L) (clamped)
 };
 
 // Every spin on an mbarrier gives up after this many SM clocks (~1 s).

@@ -443,10 +443,15 @@ static std::atomic<int> g_bypass{1};
 static dsa_status_t decode_ws(const dsa_tensor_t* q, const dsa_tensor_t* q_idx, const dsa_tensor_t* w_idx,
                        const dsa_tensor_t* k_idx_cache, const dsa_tensor_t* kv_cache, const int32_t* pos, int32_t topk,
                        const float* sink, dsa_tensor_t* out, dsa_tensor_t* sel_idx, dsa_stream_t stream_,
-                       void* workspace, size_t workspace_bytes)
+                       void* workspace, size_t workspace_bytes, const int32_t* pos_device = nullptr)
 {
     t_last_error.clear();
     Shape sh;
+    const int32_t zeros[kMaxT] = {0, 0, 0, 0, 0, 0, 0, 0};   // stand-in host positions for a device pos
+    if (pos_device) {
+        if (reinterpret_cast<uintptr_t>(pos_device) & 3u) return fail(DSA_ERR_INVALID_ARG, "pos_device: not 4-byte aligned");
+        pos = zeros;
+    }
     dsa_status_t st = check_decode_args(q, q_idx, w_idx, k_idx_cache, kv_cache, pos, topk, out, sel_idx, sh);
     if (st) return st;
     if (sink && !aligned16(sink)) return fail(DSA_ERR_INVALID_ARG, "sink: not 16-byte aligned");
@@ -461,7 +466,10 @@ static dsa_status_t decode_ws(const dsa_tensor_t* q, const dsa_tensor_t* q_idx, 
     p.phases = kPhaseIndex | kPhaseTopk | kPhaseAttend;
     p.grid = grid_blocks(dev, sh.fp8);
     set_pos(p, pos, sh.T);
-    if (g_bypass.load() && p.n_max <= topk) {
+    if (pos_device) {   // positions are read at launch: split the work over the whole cache
+        p.pos_dev = pos_device;
+        p.n_max = static_cast<int32_t>(sh.L);
+    } else if (g_bypass.load() && p.n_max <= topk) {
         p.phases = kPhaseSelectPos | kPhaseAttend;
         p.window = topk;
     }
@@ -508,6 +516,16 @@ dsa_status_t dsa_decode_sink_ws(const dsa_tensor_t* q, const dsa_tensor_t* q_idx
 }
 
 void dsa_set_short_context_bypass(int32_t enable) { g_bypass.store(enable != 0 ? 1 : 0); }
+
+dsa_status_t dsa_decode_devpos_ws(const dsa_tensor_t* q, const dsa_tensor_t* q_idx, const dsa_tensor_t* w_idx,
+                                  const dsa_tensor_t* k_idx_cache, const dsa_tensor_t* kv_cache,
+                                  const int32_t* pos_device, int32_t topk, const float* sink, dsa_tensor_t* out,
+                                  dsa_tensor_t* sel_idx, dsa_stream_t stream, void* workspace, size_t workspace_bytes)
+{
+    if (!pos_device) return fail(DSA_ERR_INVALID_ARG, "pos_device: null");
+    return decode_ws(q, q_idx, w_idx, k_idx_cache, kv_cache, nullptr, topk, sink, out, sel_idx, stream, workspace,
+                     workspace_bytes, pos_device);
+}
 
 dsa_status_t dsa_swa_decode(const dsa_tensor_t* q, const dsa_tensor_t* kv_cache, const int32_t* pos, int32_t window,
                             const float* sink, dsa_tensor_t* out, dsa_stream_t stream_, void* workspace,
@@ -712,7 +730,7 @@ dsa_status_t dsa_device_status(dsa_stream_t stream_)
         e = cudaMemcpyToSymbol(g_err_word, &zero, sizeof zero);
         if (e != cudaSuccess) return cuda_fail(e, "clear device error word");
         return fail(DSA_ERR_DEVICE, "device error word 0x%x (1: wait timeout, 2: bad selected index, 4: top-k state, "
-                    "8: workspace control words not zero at launch)",
+                    "8: workspace control words not zero at launch, 16: device query position outside [0, L))",
                     word);
     }
     return DSA_OK;

@@ -38,6 +38,7 @@ struct StepParams {
     int32_t grid;            // blocks (one per SM, all co-resident)
     int32_t T, L, n_max, topk;
     int32_t pos[kMaxT];
+    const int32_t* pos_dev;  // nullptr, or pos [T] in device memory read at launch (then n_max = L here)
     // indexer
     const uint16_t* q_idx;   // [T][16][64] bf16
     const float* w;          // [T][16]

@@ -125,6 +125,14 @@ __device__ __forceinline__ void barrier_exit(const StepParams& p)
     }
 }
 
+// The query positions of this launch (from the launch parameters, or read from
+// device memory at launch) and the furthest visible position + 1.
+struct PosView {
+    int32_t pos[kMaxT];
+    int32_t n_max;
+};
+__shared__ PosView g_qpos;
+
 // Phase-boundary timestamp (when the caller asked for a trace).
 __device__ __forceinline__ void stamp(const StepParams& p, int slot)
 {
@@ -312,7 +320,7 @@ __device__ void phase_index(const CUtensorMap& kmap, const CUtensorMap& smap, co
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int T = p.T;
-    const int ntiles = (p.n_max + kKeyTile - 1) / kKeyTile;
+    const int ntiles = (g_qpos.n_max + kKeyTile - 1) / kKeyTile;
     const bool scaled = p.scale != nullptr;
     const uint32_t tile_tx = raw_bytes + (scaled ? kKeyTile * 4 : 0);
     auto tile_of = [&](int it) { return blockIdx.x + it * static_cast<int>(gridDim.x); };
@@ -378,7 +386,7 @@ __device__ void phase_index(const CUtensorMap& kmap, const CUtensorMap& smap, co
         pos_q[u] = -1;
 #pragma unroll
         for (int i = 0; i < kMaxT; ++i)
-            if (i == qa + u) pos_q[u] = p.pos[i];
+            if (i == qa + u) pos_q[u] = g_qpos.pos[i];
         klo[u] = 0xFFFFFFFFu;
         khi[u] = 0u;
     }
@@ -577,7 +585,7 @@ __device__ void phase_ranges(const StepParams& p, uint32_t* scratch)
 {
     for (int i = blockIdx.x * kThreads + threadIdx.x; i < p.zero_words; i += gridDim.x * kThreads) p.zero[i] = 0u;
     for (int t = 0; t < p.T; ++t) {
-        const int n = p.pos[t] + 1;
+        const int n = g_qpos.pos[t] + 1;
         uint32_t lo = 0xFFFFFFFFu, hi = 0u;
         const float* row = p.scores + (int64_t)t * p.ld;
         for (int s = blockIdx.x * kThreads + threadIdx.x; s < n; s += gridDim.x * kThreads) {
@@ -670,7 +678,7 @@ __device__ __forceinline__ Item topk_item(const StepParams& p, int i)
     int pos_t = 0;
 #pragma unroll
     for (int k = 0; k < kMaxT; ++k)
-        if (k == it.t) pos_t = p.pos[k];
+        if (k == it.t) pos_t = g_qpos.pos[k];
     it.n = pos_t + 1;
     it.s0 = min(it.n, it.c * p.chunk);
     it.s1 = min(it.n, it.s0 + p.chunk);
@@ -1178,7 +1186,7 @@ __device__ void phase_select_pos(const StepParams& p)
         int pos_t = 0;
 #pragma unroll
         for (int k = 0; k < kMaxT; ++k)
-            if (k == t) pos_t = p.pos[k];
+            if (k == t) pos_t = g_qpos.pos[k];
         const int cnt = min(pos_t + 1, p.window);
         p.sel[(int64_t)t * p.sel_ld + j] = j < cnt ? pos_t + 1 - cnt + j : -1;
     }
@@ -1221,7 +1229,7 @@ __device__ void phase_attend(const StepParams& p, uint8_t* smem, uint64_t* bars)
         int pos_t = 0;
 #pragma unroll
         for (int k = 0; k < kMaxT; ++k)
-            if (k == t) pos_t = p.pos[k];
+            if (k == t) pos_t = g_qpos.pos[k];
         const int rows_t = min(p.rows, pos_t + 1);
         const int r0 = split * p.rows_per_split;
         const int r1 = min(r0 + p.rows_per_split, rows_t);
@@ -1584,6 +1592,30 @@ template <bool FP8>
 __global__ void __launch_bounds__(kThreads, 1)
     step_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap smap, const StepParams p)
 {
+    // Query positions: from the launch, or read from device memory (pos_dev) so
+    // that one CUDA graph of the step serves every decode position.  A position
+    // outside [0, L) is clamped and flagged.
+    if (threadIdx.x < 32) {
+        int v = 0;
+        if (threadIdx.x < p.T) {
+            v = p.pos[threadIdx.x < kMaxT ? threadIdx.x : 0];
+            if (p.pos_dev != nullptr) {
+                v = __ldcg(p.pos_dev + threadIdx.x);
+                if (v < 0 || v >= p.L) {
+                    if (blockIdx.x == 0) atomicOr(p.err, ERR_BAD_POS);
+                    v = min(max(v, 0), p.L - 1);
+                }
+            }
+            g_qpos.pos[threadIdx.x] = v;
+        } else if (threadIdx.x < kMaxT) {
+            g_qpos.pos[threadIdx.x] = 0;
+        }
+        int n = threadIdx.x < p.T ? v + 1 : 0;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) n = max(n, __shfl_xor_sync(0xffffffffu, n, o));
+        if (threadIdx.x == 0) g_qpos.n_max = p.pos_dev != nullptr ? n : p.n_max;
+    }
+    __syncthreads();
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kBarOffset);

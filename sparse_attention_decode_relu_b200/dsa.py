@@ -61,6 +61,8 @@ def lib():
             L.dsa_decode_ws.argtypes = [T, T, T, T, T, P, ctypes.c_int32, T, T, P, P, ctypes.c_size_t]
             L.dsa_decode_sink_ws.restype = st
             L.dsa_decode_sink_ws.argtypes = [T, T, T, T, T, P, ctypes.c_int32, P, T, T, P, P, ctypes.c_size_t]
+            L.dsa_decode_devpos_ws.restype = st
+            L.dsa_decode_devpos_ws.argtypes = [T, T, T, T, T, P, ctypes.c_int32, P, T, T, P, P, ctypes.c_size_t]
             L.dsa_set_short_context_bypass.restype = None
             L.dsa_set_short_context_bypass.argtypes = [ctypes.c_int32]
             L.dsa_swa_decode.restype = st
@@ -175,6 +177,18 @@ def dsa_decode_sink_ws(q, q_idx, w_idx, k_idx_cache, kv_cache, pos, topk, sink, 
                        stream=None, *, k_scale=None):
     dsa_decode_ws(q, q_idx, w_idx, k_idx_cache, kv_cache, pos, topk, out, sel_idx, workspace, stream,
                   k_scale=k_scale, sink=sink)
+
+
+def dsa_decode_devpos_ws(q, q_idx, w_idx, k_idx_cache, kv_cache, pos_device, topk, out, sel_idx, workspace,
+                         stream=None, *, k_scale=None, sink=None):
+    """The step with query positions read from pos_device (int32 CUDA tensor [T]) at launch."""
+    if not pos_device.is_cuda or pos_device.dtype != torch.int32 or pos_device.numel() != q.shape[0]:
+        raise ValueError("pos_device must be an int32 CUDA tensor with one position per query")
+    a = [_desc(q), _desc(q_idx), _desc(w_idx), _desc(k_idx_cache, k_scale), _desc(kv_cache)]
+    o = [_desc(out), _desc(sel_idx)]
+    _check(lib().dsa_decode_devpos_ws(*[ctypes.byref(x) for x in a], pos_device.data_ptr(), int(topk),
+                                      _sink_ptr(sink), ctypes.byref(o[0]), ctypes.byref(o[1]), _stream(stream),
+                                      workspace.data_ptr(), workspace.numel() * workspace.element_size()))
 
 
 def dsa_set_short_context_bypass(enable: bool):

@@ -90,3 +90,61 @@ def test_short_context_bypass_is_exact(name):
     for t in range(w.T):
         s = res[0][1][t].cpu().numpy()
         assert s[: n[t]].tolist() == list(range(n[t])) and np.all(s[n[t]:] == -1)
+
+
+def test_device_positions_replay_one_graph_across_steps():
+    """One CUDA graph of the step with positions in device memory serves several
+    decode positions: each replay equals the host-position entry point bit for
+    bit and the oracle's selection exactly (integer inputs)."""
+    w = synth.config("sweep_L16384_T8_int")
+    d = dsa.to_device(w)
+    T, L, k = w.T, w.L, w.topk
+    ws = dsa.workspace(T, L, k)
+    pos_dev = torch.tensor(w.pos, dtype=torch.int32, device="cuda")
+    out = torch.empty((T, 64, 128), dtype=torch.bfloat16, device="cuda")
+    sel = torch.empty((T, k), dtype=torch.int32, device="cuda")
+    s = torch.cuda.Stream()
+
+    def step():
+        dsa.dsa_decode_devpos_ws(d["q"], d["q_idx"], d["w_idx"], d["k_idx"], d["kv"], pos_dev, k, out, sel, ws,
+                                 k_scale=d["k_scale"])
+
+    with torch.cuda.stream(s):
+        step()
+    s.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        step()
+    for positions in (w.pos, w.pos - 3000, np.array([16383, 100, 5000, 2047, 2048, 9000, 16000, 0], np.int32)):
+        pos_dev.copy_(torch.from_numpy(positions.astype(np.int32)))
+        torch.cuda.synchronize()
+        g.replay()
+        torch.cuda.synchronize()
+        dsa.dsa_device_status()
+        ref_o, ref_s = dsa.decode(d["q"], d["q_idx"], d["w_idx"], d["k_idx"], d["kv"], positions, k,
+                                  k_scale=d["k_scale"], ws=dsa.workspace(T, L, k))
+        dsa.dsa_device_status()
+        assert torch.equal(sel, ref_s) and torch.equal(out.view(torch.int16), ref_o.view(torch.int16))
+        o_ora, s_ora = oracle.decode(w.q, w.q_idx, w.w_idx, w.k_idx, w.k_scale, w.kv, positions, k)
+        assert np.array_equal(sel.cpu().numpy(), s_ora)
+        check_attention(out.double().cpu().numpy(), o_ora, f"device positions {positions.tolist()}")
+    del g
+
+
+def test_device_position_out_of_range_is_clamped_and_flagged():
+    w = synth.config("tiny_decode")
+    d = dsa.to_device(w)
+    ws = dsa.workspace(w.T, w.L, w.topk)
+    out = torch.empty((1, 64, 128), dtype=torch.bfloat16, device="cuda")
+    sel = torch.empty((1, w.topk), dtype=torch.int32, device="cuda")
+    pos_dev = torch.tensor([w.L + 5], dtype=torch.int32, device="cuda")
+    dsa.dsa_decode_devpos_ws(d["q"], d["q_idx"], d["w_idx"], d["k_idx"], d["kv"], pos_dev, w.topk, out, sel, ws,
+                             k_scale=d["k_scale"])
+    with pytest.raises(dsa.DsaError) as e:
+        dsa.dsa_device_status()
+    assert e.value.status == dsa.ERR_DEVICE and "0x10" in str(e.value)
+    # clamped to the last position: the same result as pos = L - 1
+    ref_o, ref_s = dsa.decode(d["q"], d["q_idx"], d["w_idx"], d["k_idx"], d["kv"], [w.L - 1], w.topk,
+                              k_scale=d["k_scale"], ws=ws)
+    dsa.dsa_device_status()
+    assert torch.equal(sel, ref_s)
