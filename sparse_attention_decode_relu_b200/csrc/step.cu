@@ -133,6 +133,17 @@ struct PosView {
 };
 __shared__ PosView g_qpos;
 
+// Position of query k: the launch parameter (constant bank), or the view filled
+// from device memory at launch.
+__device__ __forceinline__ int query_pos(const StepParams& p, int k)
+{
+    return p.pos_dev != nullptr ? g_qpos.pos[k] : p.pos[k];
+}
+__device__ __forceinline__ int visible_max(const StepParams& p)
+{
+    return p.pos_dev != nullptr ? g_qpos.n_max : p.n_max;
+}
+
 // Phase-boundary timestamp (when the caller asked for a trace).
 __device__ __forceinline__ void stamp(const StepParams& p, int slot)
 {
@@ -320,7 +331,7 @@ __device__ void phase_index(const CUtensorMap& kmap, const CUtensorMap& smap, co
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int T = p.T;
-    const int ntiles = (g_qpos.n_max + kKeyTile - 1) / kKeyTile;
+    const int ntiles = (visible_max(p) + kKeyTile - 1) / kKeyTile;
     const bool scaled = p.scale != nullptr;
     const uint32_t tile_tx = raw_bytes + (scaled ? kKeyTile * 4 : 0);
     auto tile_of = [&](int it) { return blockIdx.x + it * static_cast<int>(gridDim.x); };
@@ -386,7 +397,7 @@ __device__ void phase_index(const CUtensorMap& kmap, const CUtensorMap& smap, co
         pos_q[u] = -1;
 #pragma unroll
         for (int i = 0; i < kMaxT; ++i)
-            if (i == qa + u) pos_q[u] = g_qpos.pos[i];
+            if (i == qa + u) pos_q[u] = query_pos(p, i);
         klo[u] = 0xFFFFFFFFu;
         khi[u] = 0u;
     }
@@ -585,7 +596,7 @@ __device__ void phase_ranges(const StepParams& p, uint32_t* scratch)
 {
     for (int i = blockIdx.x * kThreads + threadIdx.x; i < p.zero_words; i += gridDim.x * kThreads) p.zero[i] = 0u;
     for (int t = 0; t < p.T; ++t) {
-        const int n = g_qpos.pos[t] + 1;
+        const int n = query_pos(p, t) + 1;
         uint32_t lo = 0xFFFFFFFFu, hi = 0u;
         const float* row = p.scores + (int64_t)t * p.ld;
         for (int s = blockIdx.x * kThreads + threadIdx.x; s < n; s += gridDim.x * kThreads) {
@@ -678,7 +689,7 @@ __device__ __forceinline__ Item topk_item(const StepParams& p, int i)
     int pos_t = 0;
 #pragma unroll
     for (int k = 0; k < kMaxT; ++k)
-        if (k == it.t) pos_t = g_qpos.pos[k];
+        if (k == it.t) pos_t = query_pos(p, k);
     it.n = pos_t + 1;
     it.s0 = min(it.n, it.c * p.chunk);
     it.s1 = min(it.n, it.s0 + p.chunk);
@@ -1186,7 +1197,7 @@ __device__ void phase_select_pos(const StepParams& p)
         int pos_t = 0;
 #pragma unroll
         for (int k = 0; k < kMaxT; ++k)
-            if (k == t) pos_t = g_qpos.pos[k];
+            if (k == t) pos_t = query_pos(p, k);
         const int cnt = min(pos_t + 1, p.window);
         p.sel[(int64_t)t * p.sel_ld + j] = j < cnt ? pos_t + 1 - cnt + j : -1;
     }
@@ -1229,7 +1240,7 @@ __device__ void phase_attend(const StepParams& p, uint8_t* smem, uint64_t* bars)
         int pos_t = 0;
 #pragma unroll
         for (int k = 0; k < kMaxT; ++k)
-            if (k == t) pos_t = g_qpos.pos[k];
+            if (k == t) pos_t = query_pos(p, k);
         const int rows_t = min(p.rows, pos_t + 1);
         const int r0 = split * p.rows_per_split;
         const int r1 = min(r0 + p.rows_per_split, rows_t);
@@ -1592,30 +1603,27 @@ template <bool FP8>
 __global__ void __launch_bounds__(kThreads, 1)
     step_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap smap, const StepParams p)
 {
-    // Query positions: from the launch, or read from device memory (pos_dev) so
-    // that one CUDA graph of the step serves every decode position.  A position
-    // outside [0, L) is clamped and flagged.
-    if (threadIdx.x < 32) {
-        int v = 0;
-        if (threadIdx.x < p.T) {
-            v = p.pos[threadIdx.x < kMaxT ? threadIdx.x : 0];
-            if (p.pos_dev != nullptr) {
+    // Query positions read from device memory (pos_dev), so that one CUDA graph of
+    // the step serves every decode position.  A position outside [0, L) is clamped
+    // and flagged.
+    if (p.pos_dev != nullptr) {
+        if (threadIdx.x < 32) {
+            int v = 0;
+            if (threadIdx.x < p.T) {
                 v = __ldcg(p.pos_dev + threadIdx.x);
                 if (v < 0 || v >= p.L) {
                     if (blockIdx.x == 0) atomicOr(p.err, ERR_BAD_POS);
                     v = min(max(v, 0), p.L - 1);
                 }
             }
-            g_qpos.pos[threadIdx.x] = v;
-        } else if (threadIdx.x < kMaxT) {
-            g_qpos.pos[threadIdx.x] = 0;
-        }
-        int n = threadIdx.x < p.T ? v + 1 : 0;
+            if (threadIdx.x < kMaxT) g_qpos.pos[threadIdx.x] = v;
+            int n = threadIdx.x < p.T ? v + 1 : 0;
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) n = max(n, __shfl_xor_sync(0xffffffffu, n, o));
-        if (threadIdx.x == 0) g_qpos.n_max = p.pos_dev != nullptr ? n : p.n_max;
+            for (int o = 16; o > 0; o >>= 1) n = max(n, __shfl_xor_sync(0xffffffffu, n, o));
+            if (threadIdx.x == 0) g_qpos.n_max = n;
+        }
+        __syncthreads();
     }
-    __syncthreads();
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kBarOffset);
