@@ -6,18 +6,22 @@
 // bounded grid barrier between phases, so no kernel boundary (launch latency,
 // ramp, drain) separates the stages:
 //
-//   1 index   : ReLU indexer scan over the key cache (TMA tiles, tensor cores),
-//               fp32 scores plus each block's per-query key range
+//   1 index   : ReLU indexer scan over the key cache: TMA key tiles,
+//               tcgen05.mma with fp32 accumulators in TMEM, fp32 scores plus
+//               each block's per-query key range
 //   2 hist    : first radix pass of the top-k, per (query, chunk) work item:
 //               4096 bins over the query's key range, summed in global memory
-//   3 extract : the bin holding the topk-th key; every key in that bin goes to
-//               the query's candidate list, keys above it are counted per chunk
-//   4 emit    : tau and the tie count from the candidate list (small), then
-//               each chunk writes its selected positions in order
+//   3 extract : the bin holding the topk-th key; every key at or above that bin
+//               goes to the query's candidate list, keys above it are counted
+//               per chunk
+//   4 emit    : each chunk block finds tau and the tie cut among the keys inside
+//               the bin and writes its selected positions in order
+//   (or)      : selection by position: the last W visible positions (the
+//               short-context bypass with W = topk, sliding-window decode)
 //   5 attend  : gathered sparse attention per (query, row split): whole K/V rows
 //               by bulk async copy, tensor-core QK and PV, online softmax;
 //               partial (max, sum, output) states to global memory
-//   6 merge   : per (query, head group), the splits merged in a fixed order
+//   6 merge   : per (query, head), the splits merged in a fixed order
 //
 // Stage entry points run a sub-range of the phases.  Every reduction is either
 // integer or in a fixed order, so results are bitwise reproducible.
@@ -1524,8 +1528,7 @@ __device__ void phase_merge(const StepParams& p, uint8_t* smem, uint32_t* /*scra
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     float* wsp = reinterpret_cast<float*>(smem) + warp * 2 * kMergeSplitsSmem;   // this warp's split weights
     float* lsp = wsp + kMergeSplitsSmem;                                            // and split sums
-    const int P = 2;                              // shares of the 128 dims per (t, h)
-    const int dpl = kD / (32 * P);                // dims per lane: 1 or 2
+    constexpr int P = 2;                          // halves of the 128 dims per (t, h); two dims per lane
     const int items = p.T * kH * P;
     const int ns = p.nsplit;
     for (int i = blockIdx.x * kWarps + warp; i < items; i += gridDim.x * kWarps) {
@@ -1564,7 +1567,7 @@ __device__ void phase_merge(const StepParams& p, uint8_t* smem, uint32_t* /*scra
         for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
         __syncwarp();
         // numerator for this lane's dims, splits in order, sixteen loads in flight
-        const int d0 = part * (kD / P) + lane * dpl;
+        const int d0 = part * (kD / P) + lane * 2;
         const float* po = p.po + ((int64_t)t * ns * kH + h) * kD + d0;
         float x0 = 0.f, x1 = 0.f;
         for (int s0 = 0; s0 < ns; s0 += 16) {
@@ -1572,10 +1575,8 @@ __device__ void phase_merge(const StepParams& p, uint8_t* smem, uint32_t* /*scra
 #pragma unroll
             for (int u = 0; u < 16; ++u) {
                 const int s = s0 + u;
-                const bool use = s < ns && wsp[s] > 0.f;
-                const float* src = po + (int64_t)s * kH * kD;
-                o[u] = !use ? make_float2(0.f, 0.f)
-                            : (dpl == 2 ? __ldcg(reinterpret_cast<const float2*>(src)) : make_float2(__ldcg(src), 0.f));
+                o[u] = (s < ns && wsp[s] > 0.f) ? __ldcg(reinterpret_cast<const float2*>(po + (int64_t)s * kH * kD))
+                                                : make_float2(0.f, 0.f);
             }
 #pragma unroll
             for (int u = 0; u < 16; ++u) {
@@ -1587,13 +1588,7 @@ __device__ void phase_merge(const StepParams& p, uint8_t* smem, uint32_t* /*scra
         }
         const float dd = den + ((p.sink != nullptr && M != -INFINITY) ? exp2f(sink - M) : 0.f);
         const float inv = dd > 0.f ? 1.0f / dd : 0.f;
-        uint16_t* dst = p.out + ((int64_t)t * kH + h) * kD + d0;
-        if (dpl == 2) {
-            *reinterpret_cast<uint32_t*>(dst) = pack_bf16(x0 * inv, x1 * inv);
-        } else {
-            const __nv_bfloat16 b = __float2bfloat16_rn(x0 * inv);
-            *reinterpret_cast<__nv_bfloat16*>(dst) = b;
-        }
+        *reinterpret_cast<uint32_t*>(p.out + ((int64_t)t * kH + h) * kD + d0) = pack_bf16(x0 * inv, x1 * inv);
         __syncwarp();
     }
 }
