@@ -119,3 +119,33 @@ def test_validation_null_and_mismatch():
     assert st == dsa.ERR_INVALID_ARG and "null" in err
     L = dsa.lib()
     assert L.dsa_status_str(4) == b"device-side anomaly"
+
+
+def test_new_entry_points_validate_before_launch():
+    """Sliding-window decode, the step with a sink and the step with device
+    positions reject bad arguments on the host, before any launch."""
+    L = dsa.lib()
+    r = ctypes.byref
+    q, qi, w, k, kv, pos, topk, out, sel = _args()
+    # sliding-window decode: window outside [1, 2048]
+    for bad in (0, 2049):
+        st = L.dsa_swa_decode(r(q), r(kv), pos, bad, None, r(out), None, 0x100000, 1 << 40)
+        assert st == dsa.ERR_INVALID_ARG and "window" in L.dsa_last_error().decode()
+    # sliding-window decode: a sink that is not 16-byte aligned
+    st = L.dsa_swa_decode(r(q), r(kv), pos, 128, 0x10004, r(out), None, 0x100000, 1 << 40)
+    assert st == dsa.ERR_INVALID_ARG and "sink" in L.dsa_last_error().decode()
+    # the step with a sink: the sink is required
+    st = L.dsa_decode_sink_ws(r(q), r(qi), r(w), r(k), r(kv), pos, topk, None, r(out), r(sel), None, 0x100000,
+                              1 << 40)
+    assert st == dsa.ERR_INVALID_ARG and "sink" in L.dsa_last_error().decode()
+    # the step with device positions: null or misaligned position array
+    st = L.dsa_decode_devpos_ws(r(q), r(qi), r(w), r(k), r(kv), None, topk, None, r(out), r(sel), None, 0x100000,
+                                1 << 40)
+    assert st == dsa.ERR_INVALID_ARG and "pos_device" in L.dsa_last_error().decode()
+    st = L.dsa_decode_devpos_ws(r(q), r(qi), r(w), r(k), r(kv), 0x10002, topk, None, r(out), r(sel), None,
+                                0x100000, 1 << 40)
+    assert st == dsa.ERR_INVALID_ARG and "pos_device" in L.dsa_last_error().decode()
+    # ... and the other arguments are still checked (topk out of range)
+    st = L.dsa_decode_devpos_ws(r(q), r(qi), r(w), r(k), r(kv), 0x10000, 4096, None, r(out), r(sel), None, 0x100000,
+                                1 << 40)
+    assert st == dsa.ERR_INVALID_ARG and "topk" in L.dsa_last_error().decode()
