@@ -13,9 +13,9 @@
  *      2,048 tokens.  Query t sits at position pos[t] and may select
  *      s in [0, pos[t]].  If pos[t] + 1 <= topk every visible position is
  *      selected; otherwise the topk largest scores, equal scores going to the
- *      lower position, which makes the result unique.  "NaiveRT > Why
- *      single-stream speed matters for RL" requires bitwise-identical results
- *      run to run; every kernel here is deterministic.
+ *      lower position, which makes the result unique.  "AI-Centered R&D in
+ *      Practice" requires bitwise-identical results run to run; every kernel
+ *      here is deterministic.
  *   3. Sparse attention.  "Hybrid SWA-DSA Architecture": GQA with four KV
  *      groups; "NaiveRT > Optimizing inside the kernel": eight query heads
  *      per GPU under TP8, i.e. 64 query heads.  For head h (group g = h / 16)

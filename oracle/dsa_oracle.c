@@ -10,8 +10,8 @@
  *     full history; the backbone attends only to a selected subset.
  *   - "Technical Details > Hybrid SWA-DSA Architecture": DSA selects the top
  *     2,048 tokens; GQA with four KV groups; the indexer has 16 query heads.
- *   - "NaiveRT > Why single-stream speed matters for RL": results must be
- *     bitwise-deterministic, which fixes a unique tie rule for the selection.
+ *   - "AI-Centered R&D in Practice": results must be bitwise-deterministic,
+ *     which fixes a unique tie rule for the selection.
  *   - "NaiveRT > Optimizing inside the kernel": eight query heads per GPU under
  *     TP8, i.e. 64 backbone query heads in total.
  * The pages do not print the indexer formula.  Reading taken (the standard
