@@ -75,6 +75,21 @@ def peaks():
         return 6650.0, "fallback"
 
 
+def bf16_peak():
+    """Measured dense bf16 tensor-core throughput (TFLOP/s, burst), or the fallback."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    except Exception:
+        return 1590.0, "fallback"
+
+
+def indexer_flops(w):
+    """Algorithmic multiply-adds x 2 of the indexer: every visible key against the
+    T x 16 query heads over 64 dims."""
+    return 2 * 16 * 64 * w.T * (int(w.pos.max()) + 1)
+
+
 def algorithmic_bytes(w, sel):
     """Bytes the method must move per step: the indexer key cache up to the
     furthest visible position, each unique selected K/V row once, per-query
@@ -421,6 +436,16 @@ def main():
             "frac": round(achieved / peak, 4), "peak_source": which, "traffic": profiled_traffic(w.name) if args.op == "step" else None,
             "algorithmic_bytes": ab["step"]}
 
+    # The indexer's tensor-core rate (tcgen05.mma), over its in-kernel phase time.
+    tensor = None
+    bypassed = (not args.no_bypass) and int(w.pos.max()) + 1 <= topk   # no indexer phase then
+    if args.op == "step" and not bypassed and phase_us.get("indexer", 0) > 0:
+        tpk, tsrc = bf16_peak()
+        tf = indexer_flops(w) / (phase_us["indexer"] * 1e-6) / 1e12
+        tensor = {"phase": "indexer", "flops_per_step": indexer_flops(w), "phase_us": phase_us["indexer"],
+                  "tflops": round(tf, 2), "peak": tpk, "unit": "TFLOP/s", "frac": round(tf / tpk, 4),
+                  "peak_source": tsrc}
+
     line = {
         "metric": METRIC, "value": round(value, 3), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms, 5), "us_per_step": round(ms * 1e3, 2),
@@ -436,6 +461,7 @@ def main():
         "frac_of_peak_hbm": round(ab["step"] / (ms * 1e-3) / 1e9 / peak, 4),
         "phase_us": phase_us,
         "roofline": roof,
+        "tensor": tensor,
         "e2e": e2e,
         "gpu_launches": int(kernels_per_step * args.steps),
         "clocks": clk,
