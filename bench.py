@@ -281,6 +281,8 @@ def main():
                     help="step: the DSA decode/verify step; swa: sliding-window decode on the same q / K/V")
     ap.add_argument("--window", type=int, default=128, help="window of --op swa")
     ap.add_argument("--no-bypass", action="store_true", help="score and select even when every query sees <= topk")
+    ap.add_argument("--pos", choices=["host", "device"], default="host",
+                    help="device: query positions in device memory (dsa_decode_devpos_ws), one graph for every position")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
@@ -315,9 +317,14 @@ def main():
     grid = dsa.dsa_step_grid(w.key_dtype == "fp8")
     trace = torch.zeros(grid * 32, dtype=torch.int64, device=dev)
 
+    pos_dev = torch.tensor(w.pos, dtype=torch.int32, device=dev)
+
     def step():
         if args.op == "swa":
             dsa.dsa_swa_decode(d["q"], d["kv"], w.pos, args.window, out, ws)
+        elif args.pos == "device":
+            dsa.dsa_decode_devpos_ws(d["q"], d["q_idx"], d["w_idx"], d["k_idx"], d["kv"], pos_dev, topk, out, sel, ws,
+                                     k_scale=d["k_scale"])
         else:
             dsa.dsa_decode_ws(d["q"], d["q_idx"], d["w_idx"], d["k_idx"], d["kv"], d["pos"], topk, out, sel, ws,
                               k_scale=d["k_scale"])
@@ -395,7 +402,8 @@ def main():
     dev_in = {k: torch.empty_like(d[k]) for k in h_in}
     h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
     h_sel = torch.empty(sel.shape, dtype=sel.dtype).pin_memory()
-    h2d = sum(v.numel() * v.element_size() for v in h_in.values())
+    h_pos = torch.tensor(w.pos, dtype=torch.int32).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in h_in.values()) + (h_pos.numel() * 4 if args.pos == "device" else 0)
     d2h = h_out.numel() * h_out.element_size() + (0 if args.op == "swa" else h_sel.numel() * h_sel.element_size())
 
     def e2e_step():
@@ -404,6 +412,10 @@ def main():
                 dev_in[k].copy_(h_in[k], non_blocking=True)
             if args.op == "swa":
                 dsa.dsa_swa_decode(dev_in["q"], d["kv"], w.pos, args.window, out, ws)
+            elif args.pos == "device":
+                pos_dev.copy_(h_pos, non_blocking=True)
+                dsa.dsa_decode_devpos_ws(dev_in["q"], dev_in["q_idx"], dev_in["w_idx"], d["k_idx"], d["kv"], pos_dev,
+                                         topk, out, sel, ws, k_scale=d["k_scale"])
             else:
                 dsa.dsa_decode_ws(dev_in["q"], dev_in["q_idx"], dev_in["w_idx"], d["k_idx"], d["kv"], d["pos"], topk,
                                   out, sel, ws, k_scale=d["k_scale"])
@@ -433,12 +445,12 @@ def main():
     peak, which = peaks()
     achieved = ab["step"] / (ms * 1e-3) / 1e9
     roof = {"kernel": "step_kernel", "bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-            "frac": round(achieved / peak, 4), "peak_source": which, "traffic": profiled_traffic(w.name) if args.op == "step" else None,
+            "frac": round(achieved / peak, 4), "peak_source": which, "traffic": profiled_traffic(w.name) if args.op == "step" and args.pos == "host" else None,
             "algorithmic_bytes": ab["step"]}
 
     # The indexer's tensor-core rate (tcgen05.mma), over its in-kernel phase time.
     tensor = None
-    bypassed = (not args.no_bypass) and int(w.pos.max()) + 1 <= topk   # no indexer phase then
+    bypassed = (not args.no_bypass and args.pos == "host") and int(w.pos.max()) + 1 <= topk   # no indexer phase then
     if args.op == "step" and not bypassed and phase_us.get("indexer", 0) > 0:
         tpk, tsrc = bf16_peak()
         tf = indexer_flops(w) / (phase_us["indexer"] * 1e-6) / 1e12
@@ -451,10 +463,12 @@ def main():
         "warmup": args.warmup, "ms_per_step": round(ms, 5), "us_per_step": round(ms * 1e3, 2),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": w.name, "op": args.op, **({"window": args.window} if args.op == "swa" else {}),
-                   "short_context_bypass": not args.no_bypass,
+                   "short_context_bypass": not args.no_bypass, "positions": args.pos,
                    "L": L, "T": T, "topk": topk, "key_dtype": w.key_dtype, "recipe": w.recipe,
                    "seed": w.seed, "parallelism": f"replicas{world}", "l2": "flushed before every step (write 2x L2, then read another 2x L2: cold and clean)",
-                   "timing": "CUDA-graph replay of " + ("dsa_swa_decode" if args.op == "swa" else "dsa_decode_ws") +
+                   "timing": "CUDA-graph replay of " + ("dsa_swa_decode" if args.op == "swa" else
+                                                          "dsa_decode_devpos_ws" if args.pos == "device" else
+                                                          "dsa_decode_ws") +
                              ", CUDA events per step",
                    "algorithmic_bytes_per_step": ab["step"], "unique_kv_rows": ab["unique_rows"],
                    "gathered_kv_rows": ab["gathered_rows"]},
