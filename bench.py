@@ -206,12 +206,12 @@ def whole_job_gbs(bytes_per_step, ms_max, world):
 
 def swa_bytes(w, window):
     """Sliding-window decode: each unique K/V row of the windows once, plus the
-    queries and outputs."""
-    import oracle
-
-    sel = oracle.window_select(w.pos, window)
-    uniq = np.unique(sel[sel >= 0]).size
-    return {"step": uniq * 2048 + w.T * 2 * 64 * 128 * 2, "unique_rows": uniq, "gathered_rows": int((sel >= 0).sum())}
+    queries and outputs.  Query t reads positions [pos_t + 1 - n_t, pos_t] with
+    n_t = min(pos_t + 1, window)."""
+    rows = [np.arange(int(p) + 1 - min(int(p) + 1, window), int(p) + 1) for p in w.pos]
+    uniq = np.unique(np.concatenate(rows)).size
+    gathered = sum(r.size for r in rows)
+    return {"step": uniq * 2048 + w.T * 2 * 64 * 128 * 2, "unique_rows": uniq, "gathered_rows": gathered}
 
 
 def oracle_step(w, op, window):
@@ -223,9 +223,35 @@ def oracle_step(w, op, window):
     return oracle.decode(w.q, w.q_idx, w.w_idx, w.k_idx, w.k_scale, w.kv, w.pos, w.topk)
 
 
+def cpu_model():
+    """The host CPU's model name and logical core count."""
+    name = "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    name = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return name, os.cpu_count()
+
+
+def one_query(w):
+    """The workload restricted to its last query (the same caches): the bounded
+    sample of the one-thread oracle timing."""
+    import copy
+
+    s = copy.copy(w)
+    t = w.T - 1
+    s.T, s.q, s.q_idx, s.w_idx, s.pos = 1, w.q[t:t + 1], w.q_idx[t:t + 1], w.w_idx[t:t + 1], w.pos[t:t + 1]
+    return s
+
+
 def cpu_baseline(w, budget_s=15.0, op="step", window=128):
     """The oracle as it stands, on this host's cores, over whole steps of the same
-    workload until about budget_s seconds have passed."""
+    workload until about budget_s seconds have passed (mean step time); then one
+    thread on a bounded sample: the step of the workload's last query alone."""
     import oracle
 
     times = []
@@ -236,7 +262,32 @@ def cpu_baseline(w, budget_s=15.0, op="step", window=128):
         times.append(time.perf_counter() - t0)
         if time.perf_counter() > t_end or len(times) >= 50:
             break
-    return statistics.median(times), len(times), sel, oracle.threads()
+    cores = oracle.threads()
+    w1 = one_query(w)
+    oracle.set_threads(1)
+    try:
+        t1 = []
+        t_end = time.perf_counter() + budget_s / 3
+        while True:
+            t0 = time.perf_counter()
+            _, sel1 = oracle_step(w1, op, window)
+            t1.append(time.perf_counter() - t0)
+            if time.perf_counter() > t_end or len(t1) >= 20:
+                break
+    finally:
+        oracle.set_threads(cores)
+    return {"mean_s": statistics.mean(times), "steps": len(times), "sel": sel, "cores": cores,
+            "one_thread_mean_s": statistics.mean(t1), "one_thread_steps": len(t1), "one_thread_sel": sel1,
+            "one_thread_workload": w1}
+
+
+def workload_config(w, args):
+    """The workload's identity (the same in both arms)."""
+    c = {"workload": w.name, "op": args.op, "L": w.L, "T": w.T, "topk": w.topk, "key_dtype": w.key_dtype,
+         "recipe": w.recipe, "seed": w.seed}
+    if args.op == "swa":
+        c["window"] = args.window
+    return c
 
 
 def run_reference(args, w, rank, world):
@@ -259,10 +310,10 @@ def run_reference(args, w, rank, world):
         "impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "GB/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(t * 1e3, 3), "us_per_step": round(t * 1e6, 1),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name, "op": args.op, "L": w.L, "T": w.T, "topk": w.topk, "key_dtype": w.key_dtype,
-                   "recipe": w.recipe, "seed": w.seed},
+        "config": workload_config(w, args),
+        "run": {"timing": "wall clock per whole oracle step, mean", "cpu": cpu_model()[0], "nproc": cpu_model()[1]},
         "cpu_baseline": {"value": round(value, 3), "unit": "GB/s", "cores": oracle.threads(), "kind": "oracle",
-                         "sample": f"whole steps of {w.name} (fp64 C oracle, OpenMP), {args.steps} timed"},
+                         "sample": f"whole steps of {w.name} (fp64 C oracle, OpenMP), {args.steps} timed, mean"},
         "e2e": {"value": round(value, 3), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -273,9 +324,11 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--config", default="verify_block")
+    ap.add_argument("--config", default="verify_1m",
+                    help="workload name (default: the 1M-context 8-token verify block, the largest single-GPU case)")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end leg (profiling runs)")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--op", choices=["step", "swa"], default="step",
                     help="step: the DSA decode/verify step; swa: sliding-window decode on the same q / K/V")
@@ -396,49 +449,66 @@ def main():
     ab = swa_bytes(w, args.window) if args.op == "swa" else algorithmic_bytes(w, sel.cpu().numpy())
     value = whole_job_gbs(ab["step"], ms, world)
 
-    # End to end through the public API: per step the query-side inputs come from
-    # pinned host memory and the outputs go back to it; the caches stay resident.
-    h_in = {k: d[k].cpu().pin_memory() for k in (("q",) if args.op == "swa" else ("q", "q_idx", "w_idx"))}
-    dev_in = {k: torch.empty_like(d[k]) for k in h_in}
-    h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    h_sel = torch.empty(sel.shape, dtype=sel.dtype).pin_memory()
-    h_pos = torch.tensor(w.pos, dtype=torch.int32).pin_memory()
-    h2d = sum(v.numel() * v.element_size() for v in h_in.values()) + (h_pos.numel() * 4 if args.pos == "device" else 0)
-    d2h = h_out.numel() * h_out.element_size() + (0 if args.op == "swa" else h_sel.numel() * h_sel.element_size())
+    # End to end through the public API, as a serving loop would run it: one CUDA
+    # graph holds, per step, the host->device copies of the step's query-side
+    # inputs and positions from pinned host memory, the step with positions in
+    # device memory (dsa_decode_devpos_ws; dsa_swa_decode for --op swa), and the
+    # device->host copies of the outputs.  The caches stay resident.
+    e2e = None
+    if not args.no_e2e:
+        h_in = {k: d[k].cpu().pin_memory() for k in (("q",) if args.op == "swa" else ("q", "q_idx", "w_idx"))}
+        dev_in = {k: torch.empty_like(d[k]) for k in h_in}
+        h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        h_sel = torch.empty(sel.shape, dtype=sel.dtype).pin_memory()
+        h_pos = torch.tensor(w.pos, dtype=torch.int32).pin_memory()
+        e_pos = torch.empty_like(pos_dev)
+        h2d = sum(v.numel() * v.element_size() for v in h_in.values()) + (0 if args.op == "swa" else h_pos.numel() * 4)
+        d2h = h_out.numel() * h_out.element_size() + (0 if args.op == "swa" else h_sel.numel() * h_sel.element_size())
 
-    def e2e_step():
-        with torch.cuda.stream(stream):
+        def e2e_step():
             for k in h_in:
                 dev_in[k].copy_(h_in[k], non_blocking=True)
             if args.op == "swa":
                 dsa.dsa_swa_decode(dev_in["q"], d["kv"], w.pos, args.window, out, ws)
-            elif args.pos == "device":
-                pos_dev.copy_(h_pos, non_blocking=True)
-                dsa.dsa_decode_devpos_ws(dev_in["q"], dev_in["q_idx"], dev_in["w_idx"], d["k_idx"], d["kv"], pos_dev,
-                                         topk, out, sel, ws, k_scale=d["k_scale"])
             else:
-                dsa.dsa_decode_ws(dev_in["q"], dev_in["q_idx"], dev_in["w_idx"], d["k_idx"], d["kv"], d["pos"], topk,
-                                  out, sel, ws, k_scale=d["k_scale"])
+                e_pos.copy_(h_pos, non_blocking=True)
+                dsa.dsa_decode_devpos_ws(dev_in["q"], dev_in["q_idx"], dev_in["w_idx"], d["k_idx"], d["kv"], e_pos,
+                                         topk, out, sel, ws, k_scale=d["k_scale"])
             h_out.copy_(out, non_blocking=True)
             if args.op != "swa":
                 h_sel.copy_(sel, non_blocking=True)
 
-    for _ in range(args.warmup):
-        e2e_step()
-    stream.synchronize()
-    e_times = []
-    for _ in range(args.steps):
-        flush_l2()
-        torch.cuda.current_stream().synchronize()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        e2e_step()
-        b.record(stream)
+        with torch.cuda.stream(stream):
+            e2e_step()   # eager once (first-call set-up outside the capture)
         stream.synchronize()
-        e_times.append(a.elapsed_time(b))
-    e_ms = reduce_max(statistics.mean(e_times), world)
-    e2e = {"value": round(whole_job_gbs(ab["step"], e_ms, world), 3), "unit": "GB/s",
-           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e_ms, 4)}
+        e_graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(e_graph, stream=stream):
+            e2e_step()
+        for _ in range(args.warmup):
+            with torch.cuda.stream(stream):
+                e_graph.replay()
+        stream.synchronize()
+        e_times = []
+        for _ in range(args.steps):
+            flush_l2()
+            torch.cuda.current_stream().synchronize()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            with torch.cuda.stream(stream):
+                a.record(stream)
+                e_graph.replay()
+                b.record(stream)
+            stream.synchronize()
+            e_times.append(a.elapsed_time(b))
+        dsa.dsa_device_status(stream)
+        if args.op != "swa":   # the host copies hold the step's results
+            assert torch.equal(h_sel, sel.cpu()), "end-to-end selection differs from the device-timed step"
+        e_ms = reduce_max(statistics.mean(e_times), world)
+        e2e = {"value": round(whole_job_gbs(ab["step"], e_ms, world), 3), "unit": "GB/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e_ms, 4),
+               "timing": "CUDA-graph replay of H2D copies + " +
+                         ("dsa_swa_decode" if args.op == "swa" else "dsa_decode_devpos_ws") +
+                         " + D2H copies, CUDA events per step, mean"}
+        del e_graph
 
     # Roofline of the step kernel (the only kernel: every phase of the step runs in
     # one cooperative launch), timed by the events around each graph replay.
@@ -462,16 +532,15 @@ def main():
         "metric": METRIC, "value": round(value, 3), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms, 5), "us_per_step": round(ms * 1e3, 2),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": w.name, "op": args.op, **({"window": args.window} if args.op == "swa" else {}),
-                   "short_context_bypass": not args.no_bypass, "positions": args.pos,
-                   "L": L, "T": T, "topk": topk, "key_dtype": w.key_dtype, "recipe": w.recipe,
-                   "seed": w.seed, "parallelism": f"replicas{world}", "l2": "flushed before every step (write 2x L2, then read another 2x L2: cold and clean)",
-                   "timing": "CUDA-graph replay of " + ("dsa_swa_decode" if args.op == "swa" else
-                                                          "dsa_decode_devpos_ws" if args.pos == "device" else
-                                                          "dsa_decode_ws") +
-                             ", CUDA events per step",
-                   "algorithmic_bytes_per_step": ab["step"], "unique_kv_rows": ab["unique_rows"],
-                   "gathered_kv_rows": ab["gathered_rows"]},
+        "config": workload_config(w, args),
+        "run": {"short_context_bypass": not args.no_bypass, "positions": args.pos,
+                "parallelism": f"replicas{world}",
+                "l2": "flushed before every step (write 2x L2, then read another 2x L2: cold and clean)",
+                "timing": "CUDA-graph replay of " + ("dsa_swa_decode" if args.op == "swa" else
+                                                       "dsa_decode_devpos_ws" if args.pos == "device" else
+                                                       "dsa_decode_ws") + ", CUDA events per step, mean",
+                "algorithmic_bytes_per_step": ab["step"], "unique_kv_rows": ab["unique_rows"],
+                "gathered_kv_rows": ab["gathered_rows"], "cpu": cpu_model()[0], "nproc": cpu_model()[1]},
         "frac_of_peak_hbm": round(ab["step"] / (ms * 1e-3) / 1e9 / peak, 4),
         "phase_us": phase_us,
         "roofline": roof,
@@ -481,10 +550,19 @@ def main():
         "clocks": clk,
     }
     if rank == 0 and not args.no_cpu_baseline:
-        t_cpu, n_cpu, _, cores = cpu_baseline(w, args.cpu_budget, args.op, args.window)
-        line["cpu_baseline"] = {"value": round(ab["step"] / t_cpu / 1e9, 4), "unit": "GB/s", "cores": cores,
-                                "kind": "oracle", "us_per_step": round(t_cpu * 1e6, 1),
-                                "sample": f"{n_cpu} whole steps of {w.name}, median"}
+        cb = cpu_baseline(w, args.cpu_budget, args.op, args.window)
+        w1 = cb["one_thread_workload"]
+        ab1 = swa_bytes(w1, args.window) if args.op == "swa" else algorithmic_bytes(w1, cb["one_thread_sel"])
+        cpu, nproc = cpu_model()
+        line["cpu_baseline"] = {
+            "value": round(ab["step"] / cb["mean_s"] / 1e9, 4), "unit": "GB/s", "cores": cb["cores"],
+            "kind": "oracle", "us_per_step": round(cb["mean_s"] * 1e6, 1),
+            "sample": f"{cb['steps']} whole steps of {w.name} on {cb['cores']} OpenMP threads, mean",
+            "cpu": cpu, "nproc": nproc,
+            "one_thread": {"value": round(ab1["step"] / cb["one_thread_mean_s"] / 1e9, 4), "unit": "GB/s",
+                           "cores": 1, "us_per_step": round(cb["one_thread_mean_s"] * 1e6, 1),
+                           "sample": f"{cb['one_thread_steps']} steps of the last query of {w.name} alone "
+                                     f"(T = 1, pos = {int(w1.pos[0])}), mean"}}
     if rank == 0:
         print(json.dumps(line), flush=True)
     del graph

@@ -176,14 +176,20 @@ DSA_API dsa_status_t dsa_swa_decode(const dsa_tensor_t *q, const dsa_tensor_t *k
 
 /* Stage 1 alone: scores [T][ld] f32 (ld >= L, a multiple of 4).  scores[t][s] is
  * I[t,s] for s <= pos[t] and -inf for s > pos[t].  The sum is taken in fp32
- * (tensor-core dot products, then a fixed-order weighted sum over heads). */
+ * (tensor-core dot products, then a fixed-order weighted sum over heads).
+ * NaiveAI research page, "Technical Details > Model Architecture": the
+ * lightweight indexer scores every cached position (it still scans the full
+ * history); "Hybrid SWA-DSA Architecture": 16 indexer query heads. */
 DSA_API dsa_status_t dsa_index_scores(const dsa_tensor_t *q_idx, const dsa_tensor_t *w_idx,
                               const dsa_tensor_t *k_idx_cache, const int32_t *pos, float *scores,
                               int64_t ld, dsa_stream_t stream);
 
 /* Stage 2 alone: causal top-k of caller scores [T][ld] (f32, ld >= L, a multiple
  * of 4; entries s > pos[t] are ignored).  -0 and +0 compare equal.  Writes sel_idx
- * [T][sel_ld] (sel_ld >= topk).  Workspace: dsa_workspace_bytes(T, L, topk). */
+ * [T][sel_ld] (sel_ld >= topk).  Workspace: dsa_workspace_bytes(T, L, topk).
+ * NaiveAI research page, "Hybrid SWA-DSA Architecture": DSA keeps the top
+ * 2,048 positions of the indexer's scores; "AI-Centered R&D in Practice":
+ * bitwise-reproducible results, hence the lower-position tie rule. */
 DSA_API dsa_status_t dsa_topk_from_scores(const float *scores, int32_t T, int64_t L, int64_t ld,
                                   const int32_t *pos, int32_t topk, int32_t *sel_idx, int64_t sel_ld,
                                   dsa_stream_t stream, void *workspace, size_t workspace_bytes);
@@ -212,7 +218,10 @@ DSA_API dsa_status_t dsa_topk_from_scores_noalloc(const float *scores, int32_t T
  * (entries < 0 are skipped; an entry outside [0, pos[t]] is skipped and flags
  * DSA_ERR_DEVICE).  `sink` is NULL or a per-head logit [64] f32 (device) that
  * joins each head's softmax denominator with no value row (an attention sink).
- * Workspace: dsa_workspace_bytes(T, L, topk). */
+ * Workspace: dsa_workspace_bytes(T, L, topk).  NaiveAI research page,
+ * "Technical Details > Model Architecture": the backbone attends only to the
+ * selected subset; "Hybrid SWA-DSA Architecture": GQA with four KV groups and
+ * a sink bias. */
 DSA_API dsa_status_t dsa_sparse_attn(const dsa_tensor_t *q, const dsa_tensor_t *kv_cache,
                              const dsa_tensor_t *sel_idx, const int32_t *pos, const float *sink,
                              dsa_tensor_t *out, dsa_stream_t stream, void *workspace,
@@ -238,6 +247,21 @@ DSA_API uint64_t dsa_launch_count(void);
  * selection, events[3] after the attention and events[4] at the end of the
  * call.  n == 0 disables; any other n is ignored. */
 DSA_API void dsa_set_stage_events(void *const *events, int32_t n);
+
+/* Failure-detection test hook for the calling host thread (one launch only).
+ * The next step-kernel launch from this thread that uses grid barriers makes
+ * each of them wait for one arrival more than its grid makes: a block that
+ * never comes.  Every wait then runs into its bound after limit_cycles SM clocks
+ * (1000 <= limit_cycles <= 2e9, the normal bound), sets the wait-timeout bit
+ * (1) of the device error word and skips the work that depended on the
+ * barrier; the launch still ends normally and leaves the workspace control
+ * words at zero, so the next call runs as usual.  Only waits between blocks are
+ * affected; waits for a block's own copies in flight keep their normal bound.
+ * NaiveAI research page, "NaiveRT > A DSA layer: from 29 kernels to one": the
+ * single cooperative kernel depends on synchronisation between its CTAs, which
+ * is what a bounded wait guards.  Returns DSA_ERR_INVALID_ARG for a limit
+ * outside the range. */
+DSA_API dsa_status_t dsa_debug_fail_next_barriers(int64_t limit_cycles);
 
 /* Profiling hook for the calling host thread: when device_buffer is not NULL,
  * every launch records, per block b and slot k < 32, the GPU global timer (ns)

@@ -12,6 +12,7 @@
 #include <cuda_runtime.h>
 
 #include "../../include/dsa_decode.h"
+#include "common.cuh"
 #include "dsa_internal.h"
 
 namespace dsa {
@@ -24,6 +25,7 @@ thread_local std::string t_last_error;
 thread_local void* t_stage_events[5] = {nullptr, nullptr, nullptr, nullptr, nullptr};
 thread_local bool t_stage_events_on = false;
 thread_local unsigned long long* t_trace = nullptr;
+thread_local long long t_fail_barriers = 0;   // > 0: the next launch's grid barriers wait for a block that never comes
 std::atomic<uint64_t> g_launches{0};
 
 dsa_status_t fail(dsa_status_t st, const char* fmt, ...)
@@ -295,6 +297,7 @@ void topk_params(StepParams& p, void* ws, const Layout& l)
     p.hist = at<uint32_t>(ws, l.hist);
     p.list_n = at<uint32_t>(ws, l.list_n);
     p.list = at<uint2>(ws, l.list);
+    p.list_ld = l.ld;
     p.above = at<uint32_t>(ws, l.above);
     p.cuts = at<uint32_t>(ws, l.cuts);
     p.mm = at<uint2>(ws, l.mm);
@@ -333,6 +336,13 @@ dsa_status_t launch(const CUtensorMap& map, const CUtensorMap& smap, StepParams&
     // creation on, and every launch leaves them zero.
     if (p.phases & (kPhaseTopk | kPhaseAttend)) p.bar_ctrl = at<uint32_t>(ws, l.ctrl);
     p.trace = t_trace;
+    p.barrier_limit = kWaitLimitCycles;
+    p.barrier_extra = 0;
+    if (t_fail_barriers > 0 && p.bar_ctrl != nullptr) {   // one launch only
+        p.barrier_limit = t_fail_barriers;
+        p.barrier_extra = 1;
+        t_fail_barriers = 0;
+    }
     if ((e = launch_step(&map, &smap, p, fp8, stream)) != cudaSuccess) return cuda_fail(e, "step launch");
     g_launches += 1;
     return DSA_OK;
@@ -417,7 +427,6 @@ dsa_status_t run_topk_stage(const float* scores, int32_t T, int64_t L, int64_t l
     p.sel_ld = sel_ld;
     p.err = dev.err;
     topk_params(p, ws, l);
-    p.list = at<uint2>(ws, l.list);
     CUtensorMap none;
     std::memset(&none, 0, sizeof none);
     return launch(none, none, p, false, ws, l, stream);
@@ -751,6 +760,16 @@ const char* dsa_status_str(dsa_status_t s)
 const char* dsa_last_error(void) { return t_last_error.c_str(); }
 
 uint64_t dsa_launch_count(void) { return g_launches.load(); }
+
+dsa_status_t dsa_debug_fail_next_barriers(int64_t limit_cycles)
+{
+    t_last_error.clear();
+    if (limit_cycles < 1000 || limit_cycles > kWaitLimitCycles)
+        return fail(DSA_ERR_INVALID_ARG, "limit_cycles = %lld outside [1000, %lld]", (long long)limit_cycles,
+                    (long long)kWaitLimitCycles);
+    t_fail_barriers = limit_cycles;
+    return DSA_OK;
+}
 
 void dsa_set_step_trace(void* device_buffer) { t_trace = static_cast<unsigned long long*>(device_buffer); }
 

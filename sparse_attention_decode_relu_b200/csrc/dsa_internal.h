@@ -50,7 +50,8 @@ struct StepParams {
     int32_t mm_slots;
     uint32_t* hist;          // [T][kHistBins]
     uint32_t* list_n;        // [kMaxT] candidates per query
-    uint2* list;             // [T][ld] (key, position) candidates
+    uint2* list;             // [T][list_ld] (key, position) candidates
+    int64_t list_ld;         // candidate-list row stride (the workspace's, not the caller's score stride)
     uint32_t* above;         // [T][kMaxChunksStep] keys above the threshold bin, per chunk
     uint32_t* cuts;          // [kMaxT][4]: threshold bin (cut, ctop) and #keys above it, per query
     uint32_t* zero;          // words phase 1 clears (hist, list_n)
@@ -73,6 +74,8 @@ struct StepParams {
     // control
     unsigned long long* trace;   // [grid][kTraceSlots] globaltimer stamps at phase boundaries, or nullptr
     uint32_t* bar_ctrl;      // grid barrier arrival counter (zero at launch)
+    int64_t barrier_limit;   // SM clocks a grid-barrier wait spins before it gives up
+    uint32_t barrier_extra;  // arrivals a grid barrier waits for beyond the grid (0; 1 = a block that never comes)
     uint32_t* err;
 };
 

@@ -68,6 +68,8 @@ struct GridBarrier {
     uint32_t* count;
     uint32_t* err;
     uint32_t next;     // count value that ends the next barrier
+    long long limit;   // SM clocks a wait spins before it gives up
+    uint32_t extra;    // arrivals waited for beyond the grid's own (0 except under the fault hook)
     uint32_t c0 = 0, x0 = 0;   // (thread 0) both words as this block first saw them
     bool bad = false;          // (thread 0) they were not zero at launch
 
@@ -95,11 +97,11 @@ struct GridBarrier {
             }
             bool ok = !bad;
             if (ok) {
-                const uint32_t target = next;
+                const uint32_t target = next + extra;
                 asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(count) : "memory");
                 const long long t0 = clock64();
                 while (ld_acquire(count) < target) {
-                    if (clock64() - t0 > kWaitLimitCycles) {
+                    if (clock64() - t0 > limit) {
                         atomicOr(err, ERR_WAIT_TIMEOUT);
                         ok = false;
                         break;
@@ -819,7 +821,7 @@ __device__ void phase_extract(const StepParams& p, uint8_t* smem, uint64_t* ring
             reinterpret_cast<uint4*>(p.cuts)[it.t] = make_uint4(cu.cut, cu.ctop, cu.above, 0u);
         if (threadIdx.x == 0) nstage = 0;
         __syncthreads();
-        uint2* list = p.list + (int64_t)it.t * p.ld;
+        uint2* list = p.list + (int64_t)it.t * p.list_ld;
         // Move the staged candidates to the list (all threads; nstage is uniform here).
         auto flush = [&]() {
             const uint32_t n = min(nstage, static_cast<uint32_t>(kStageCap));
@@ -1024,7 +1026,7 @@ __device__ void phase_emit(const StepParams& p, uint8_t* smem, uint64_t* ring_fu
         const uint32_t m = __ldcg(p.list_n + it.t);
         const uint4 cq = __ldcg(reinterpret_cast<const uint4*>(p.cuts) + it.t);
         const Cut cu{cq.x, cq.y, cq.z};
-        const uint2* glist = p.list + (int64_t)it.t * p.ld;
+        const uint2* glist = p.list + (int64_t)it.t * p.list_ld;
         const uint32_t* above = p.above + (int64_t)it.t * kMaxChunksStep;
         // keys above the bin in the chunks before this one
         uint32_t before = 0;
@@ -1627,7 +1629,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __shared__ int ok_s;
     __shared__ uint32_t tmem_slot;
 
-    GridBarrier gb{p.bar_ctrl, p.err, gridDim.x};
+    GridBarrier gb{p.bar_ctrl, p.err, gridDim.x, p.barrier_limit, p.barrier_extra};
 
     if (threadIdx.x == 0) {
         mbar_init(bars + 24, 1);

@@ -83,6 +83,8 @@ def lib():
             L.dsa_status_str.argtypes = [st]
             L.dsa_last_error.restype = ctypes.c_char_p
             L.dsa_launch_count.restype = ctypes.c_uint64
+            L.dsa_debug_fail_next_barriers.restype = st
+            L.dsa_debug_fail_next_barriers.argtypes = [ctypes.c_int64]
             L.dsa_set_step_trace.restype = None
             L.dsa_set_step_trace.argtypes = [P]
             L.dsa_step_grid.restype = ctypes.c_int32
@@ -221,7 +223,7 @@ def dsa_topk_from_scores(scores, L, pos, topk, sel_idx, workspace, stream=None):
 
 def dsa_topk_from_scores_noalloc(scores, L, pos, topk, sel_idx, stream=None):
     """dsa_topk_from_scores with the library's static scratch instead of a
-    workspace (T <= 8, L <= 65536; concurrent calls on the GPU race)."""
+    workspace (T <= 8, L <= 262144; concurrent calls on the GPU race)."""
     if scores.dtype != torch.float32 or scores.dim() != 2 or scores.stride(1) != 1:
         raise ValueError("scores must be float32 [T][ld] with unit inner stride")
     if sel_idx.dtype != torch.int32 or sel_idx.stride(1) != 1:
@@ -241,6 +243,12 @@ def dsa_sparse_attn(q, kv_cache, sel_idx, pos, out, workspace, stream=None, *, s
 
 def dsa_device_status(stream=None):
     _check(lib().dsa_device_status(_stream(stream)))
+
+
+def dsa_debug_fail_next_barriers(limit_cycles: int):
+    """Test hook: the next step launch from this thread waits at every grid
+    barrier for a block that never comes, giving up after limit_cycles."""
+    _check(lib().dsa_debug_fail_next_barriers(int(limit_cycles)))
 
 
 def dsa_launch_count() -> int:

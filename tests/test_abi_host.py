@@ -149,3 +149,10 @@ def test_new_entry_points_validate_before_launch():
     st = L.dsa_decode_devpos_ws(r(q), r(qi), r(w), r(k), r(kv), 0x10000, 4096, None, r(out), r(sel), None, 0x100000,
                                 1 << 40)
     assert st == dsa.ERR_INVALID_ARG and "topk" in L.dsa_last_error().decode()
+
+
+def test_barrier_fault_hook_validates_its_limit():
+    L = dsa.lib()
+    for bad in (0, 999, 2_000_000_001, -5):
+        assert L.dsa_debug_fail_next_barriers(bad) == dsa.ERR_INVALID_ARG
+    assert b"limit_cycles" in L.dsa_last_error()

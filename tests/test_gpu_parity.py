@@ -34,9 +34,12 @@ SMALL = [
     ("ragged_fp8_T3", dict(L=2999, T=3, key_dtype="fp8", recipe="normal", seed=42, pos=np.array([2998, 2500, 10]))),
     ("ragged_fp8_T8_int", dict(L=5000, T=8, key_dtype="fp8", recipe="int", seed=43)),
     ("sweep_L2200_T8", None),
+    ("sweep_L2200_T1", None),
     ("sweep_L2200_T1_int", None),
     ("sweep_L200_T8", None),
+    ("sweep_L200_T1", None),
     ("sweep_L16384_T1", None),
+    ("sweep_L16384_T8", None),
     ("verify_block", None),
     ("verify_block_int", None),
     ("long_decode", None),
@@ -102,9 +105,9 @@ def test_small_topk(topk):
     check_attention(out, ref_out, f"topk={topk}")
 
 
-def _topk_gpu(scores_np, pos, topk):
+def _topk_gpu(scores_np, pos, topk, ld=None):
     T, L = scores_np.shape
-    ld = round_up(L, 4)
+    ld = ld or round_up(L, 4)
     s = torch.full((T, ld), float("nan"), dtype=torch.float32, device="cuda")
     s[:, :L] = torch.from_numpy(scores_np.astype(np.float32)).cuda()
     sel = torch.empty((T, topk), dtype=torch.int32, device="cuda")
@@ -142,6 +145,19 @@ def test_topk_stage_exact(case):
     s = s.astype(np.float32).astype(np.float64)
     pos = np.array([L - 1, L // 2, 3000], np.int32)
     assert np.array_equal(_topk_gpu(s, pos, k), oracle.topk(s, pos, k))
+
+
+def test_topk_stage_wide_score_stride():
+    """A score row stride far above the workspace's own row length: the
+    candidate lists keep the workspace's stride (every score tied, so every
+    visible position is a candidate)."""
+    T, L, k = 8, 40000, 2048
+    s = np.full((T, L), 1.25)
+    pos = np.array([L - 1 - 977 * t for t in range(T)], np.int32)
+    ld = round_up(L, 64) + 64
+    got = _topk_gpu(s, pos, k, ld=ld)
+    assert np.array_equal(got, oracle.topk(s, pos, k))
+    assert np.array_equal(got, _topk_gpu(s, pos, k))
 
 
 def test_topk_stage_many_chunks():
@@ -231,7 +247,7 @@ def test_graph_capture_replays_the_step():
 
 
 @pytest.mark.slow
-@pytest.mark.parametrize("name", ["sweep_L262144_T8", "sweep_L262144_T1_int"])
+@pytest.mark.parametrize("name", ["sweep_L262144_T8", "sweep_L262144_T1", "sweep_L262144_T1_int"])
 def test_sweep_256k(name):
     w = synth.config(name)
     d = dsa.to_device(w)
@@ -297,3 +313,26 @@ def test_workspace_control_words_left_zero_and_checked():
     ws[: dsa.WS_CTRL_BYTES].zero_()
     o2, s2 = gpu_decode(w, d, ws=ws)
     assert np.array_equal(s2, ref_s) and np.array_equal(o2, ref_o)
+
+
+def test_barrier_wait_timeout_is_reported_and_recovers():
+    """Failure detection of the single cooperative kernel: with the test hook,
+    every grid barrier of one launch waits for a block that never comes.  Each
+    bounded wait runs out (about 1 ms here), the launch reports the wait-timeout
+    bit alone, leaves the workspace control words at zero, and the next call on
+    the same workspace matches the oracle again."""
+    w = synth.config("tiny_decode")   # 4096 positions, one query: every phase and barrier runs
+    d = dsa.to_device(w)
+    ws = dsa.workspace(w.T, w.L, w.topk)
+    ref_o, ref_s = gpu_decode(w, d, ws=ws)
+    dsa.dsa_debug_fail_next_barriers(2_000_000)
+    dsa.decode(d["q"], d["q_idx"], d["w_idx"], d["k_idx"], d["kv"], d["pos"], w.topk, k_scale=d["k_scale"], ws=ws)
+    with pytest.raises(dsa.DsaError) as e:
+        dsa.dsa_device_status()
+    assert e.value.status == dsa.ERR_DEVICE and "word 0x1 " in str(e.value)
+    assert int(ws[: dsa.WS_CTRL_BYTES].count_nonzero()) == 0
+    o2, s2 = gpu_decode(w, d, ws=ws)   # the hook covered one launch only
+    assert np.array_equal(s2, ref_s) and np.array_equal(o2, ref_o)
+    ora_o, ora_s = oracle.decode(w.q, w.q_idx, w.w_idx, w.k_idx, w.k_scale, w.kv, w.pos, w.topk)
+    assert np.array_equal(s2, ora_s)
+    check_attention(o2, ora_o, "after a timed-out launch")

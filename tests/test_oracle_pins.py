@@ -177,6 +177,62 @@ def test_indexer_integer_inputs_give_exact_integers(orc):
     assert s.max() < 2 ** 24
 
 
+# ---------------------------------------------------------------- error-band magnitude
+def test_index_magnitude_hand_worked(orc):
+    """The magnitude sum M = scale * sum_j |w_j| * sum_d |q_jd k_d| of the
+    hand-worked example, worked out by hand in the fixture (bf16 and E4M3 keys,
+    with and without per-token scales, an invisible position)."""
+    d, q_idx, w, k = _hand()
+    pos = np.array([int(d["pos"][0])], np.int32)
+    scale = np.array([float(v) for v in d["scale"]], np.float32)
+    for keys, ones in ((synth.f32_to_bf16_bits(k), None), (synth.f32_to_e4m3_codes(k), np.ones(len(k), np.float32))):
+        assert orc.index_magnitude(q_idx, w, keys, ones, pos)[0].tolist() == [float(v) for v in d["magnitude"]]
+        m4 = orc.index_magnitude(q_idx, w, keys, ones, np.array([4], np.int32))
+        assert m4[0].tolist() == [float(v) for v in d["magnitude_pos4"]]
+    e4 = synth.f32_to_e4m3_codes(k)
+    got = orc.index_magnitude(q_idx, w, e4, scale, pos)[0].tolist()
+    assert got == [float(v) for v in d["magnitude_scaled"]]
+
+
+@pytest.mark.parametrize("fp8", [False, True])
+def test_index_magnitude_matches_numpy(orc, fp8):
+    """Against a numpy restatement on dequantised inputs: |w| @ (|Q| |K8|^T),
+    times the per-token scale; negative weights count by their absolute value,
+    scales are not uniform, invisible positions give 0."""
+    rng = np.random.default_rng(31 + fp8)
+    T, L = 3, 333
+    q_idx, w, keys, scale = _rand_idx(rng, T, L, fp8)
+    w = (w * 2 - 1).astype(np.float32)   # mixed signs
+    pos = np.array([L - 1, 200, 0], np.int32)
+    got = orc.index_magnitude(q_idx, w, keys, scale, pos)
+    Q = np.abs(synth.bf16_bits_to_f32(q_idx).astype(np.float64))
+    K8 = np.abs(_dequant(keys, None))
+    ref = np.einsum("tj,tjs->ts", np.abs(w.astype(np.float64)), np.einsum("tjd,sd->tjs", Q, K8))
+    if scale is not None:
+        ref = ref * scale.astype(np.float64)[None, :]
+    ref[np.arange(L)[None, :] > pos[:, None]] = 0.0
+    np.testing.assert_allclose(got, ref, rtol=1e-12, atol=0)
+
+
+def test_index_magnitude_bounds_the_score(orc):
+    """|I| <= M always (triangle inequality, ReLU is 1-Lipschitz through 0), with
+    equality when every query, key and weight is non-negative (then nothing is
+    cancelled or clipped)."""
+    rng = np.random.default_rng(33)
+    T, L = 2, 250
+    q_idx, w, keys, scale = _rand_idx(rng, T, L, True)
+    w = (w * 2 - 1).astype(np.float32)
+    pos = np.full(T, L - 1, np.int32)
+    s = orc.index_scores(q_idx, w, keys, scale, pos)
+    m = orc.index_magnitude(q_idx, w, keys, scale, pos)
+    assert np.all(np.abs(s) <= m * (1 + 1e-12))
+    qp = synth.f32_to_bf16_bits(rng.random((T, 16, 64), dtype=np.float32))
+    wp = rng.random((T, 16), dtype=np.float32)
+    kp = synth.f32_to_e4m3_codes(rng.random((L, 64), dtype=np.float32) * 3)
+    np.testing.assert_allclose(orc.index_scores(qp, wp, kp, scale, pos), orc.index_magnitude(qp, wp, kp, scale, pos),
+                               rtol=1e-13, atol=0)
+
+
 # ---------------------------------------------------------------- top-k
 def _brute_topk(scores, pos, k):
     T = scores.shape[0]

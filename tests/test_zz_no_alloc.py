@@ -12,33 +12,38 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 from sparse_attention_decode_relu_b200 import dsa
 
 pytestmark = pytest.mark.gpu
 
 
-def _scores(rng, T, L, kind):
+def _scores(rng, T, L, kind, ld=None):
     if kind == "ties":
         s = rng.integers(0, 50, size=(T, L)).astype(np.float32)
+    elif kind == "equal":
+        s = np.full((T, L), 0.5, np.float32)
     else:
         s = rng.standard_normal((T, L)).astype(np.float32)
-    ld = (L + 3) // 4 * 4
+    ld = ld or (L + 3) // 4 * 4
     out = torch.zeros((T, ld), dtype=torch.float32, device="cuda")
     out[:, :L] = torch.from_numpy(s).cuda()
-    return out
+    return out, s.astype(np.float64)
 
 
 @pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")
 def test_noalloc_topk_matches_workspace_entry_two_calls_in_a_row():
     rng = np.random.default_rng(2024)
-    # The first two calls take the multi-block path that works in the scratch array
-    # (the second finds the first one's leftovers there); 40000 scores per query
-    # take the cluster path that needs none.
-    cases = [(8, 262144, 2048, "ties", [262143 - i for i in range(8)]),
-             (3, 200000, 777, "normal", [199999, 1000, 150000]),
-             (3, 40000, 777, "normal", [39999, 1000, 20000])]
-    for T, L, k, kind, pos in cases:
-        scores = _scores(rng, T, L, kind)
+    # Every call works in the one scratch array: the second finds the first
+    # one's leftovers there, the third checks a shorter context on the same
+    # scratch after two larger calls, and the last gives the scores a row
+    # stride far beyond the scratch's own row length.
+    cases = [(8, 262144, 2048, "ties", [262143 - i for i in range(8)], None),
+             (3, 200000, 777, "normal", [199999, 1000, 150000], None),
+             (3, 40000, 777, "normal", [39999, 1000, 20000], None),
+             (8, 40000, 2048, "equal", [39999 - 977 * i for i in range(8)], 40000 + 64 + 64)]
+    for T, L, k, kind, pos, ld in cases:
+        scores, s_np = _scores(rng, T, L, kind, ld)
         ref = torch.full((T, k), -7, dtype=torch.int32, device="cuda")
         ws = dsa.workspace(T, L, k)
         dsa.dsa_topk_from_scores(scores, L, pos, k, ref, ws)
@@ -46,6 +51,7 @@ def test_noalloc_topk_matches_workspace_entry_two_calls_in_a_row():
         dsa.dsa_topk_from_scores_noalloc(scores, L, pos, k, got)
         dsa.dsa_device_status()
         assert torch.equal(got, ref), (T, L, k, kind)
+        assert np.array_equal(got.cpu().numpy(), oracle.topk(s_np, np.array(pos, np.int32), k)), (T, L, k, kind)
 
 
 @pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")
