@@ -413,20 +413,20 @@ def main():
         return s0.elapsed_time(s1)
 
     def phases():
-        """Phase spans of the last replay, from the in-kernel stamps."""
+        """Phase spans of the last replay, from the in-kernel stamps (a phase runs
+        from its earliest start stamp to its latest end stamp over the blocks that
+        stamped it)."""
         t = trace.view(grid, 32).cpu().numpy().astype(np.int64)
-        # phase k runs from its start stamp (earliest block) to its end stamp (latest block)
-        spans = {}
-        for name, a, b in (("indexer", 0, 1), ("topk_hist", 2, 3), ("topk_extract", 4, 5), ("topk_emit", 6, 7),
-                           ("attention", 8, 9), ("merge", 10, 11)):
-            spans[name] = (t[:, b].max() - t[:, a].min()) / 1e3
-        spans["kernel"] = (t[:, 30].max() - t[:, 0].min()) / 1e3
+
+        def span(a, b):
+            sa, sb = t[:, a][t[:, a] > 0], t[:, b][t[:, b] > 0]
+            return (sb.max() - sa.min()) / 1e3 if sa.size and sb.size else 0.0
+
+        spans = {"indexer": span(0, 1), "barrier": span(1, 2), "topk_extract": span(2, 3),
+                 "topk_select": span(4, 5), "attention": span(6, 7), "merge": span(8, 9)}
+        spans["kernel"] = span(0, 30)
         spans["sm_mhz_in_kernel"] = float((t[0, 29] - t[0, 28]) / max(1, t[0, 30] - t[0, 0]) * 1e3)
         spans["start_skew"] = (t[:, 0].max() - t[:, 0].min()) / 1e3
-        emitting = t[:, 13] > 0   # blocks that selected and compacted a chunk
-        if emitting.any():
-            for name, a, b in (("emit_load", 6, 12), ("emit_select", 12, 13), ("emit_out", 13, 7)):
-                spans[name] = (t[emitting, b] - t[emitting, a]).max() / 1e3
         return spans
 
     for _ in range(args.warmup):

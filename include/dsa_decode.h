@@ -102,14 +102,18 @@ typedef struct {
  * All device base addresses must be 16-byte aligned. */
 
 /* Bytes of workspace dsa_decode_ws needs for these sizes (0 if they are invalid).
- * Workspace contract (dsa_decode_ws, dsa_topk_from_scores, dsa_sparse_attn): the
- * caller owns the memory; its first DSA_WS_CTRL_BYTES bytes are grid-barrier
- * control words that must be zero before the workspace's first use (one
- * cudaMemsetAsync when it is created); every call leaves them zero again, so
- * later calls need no reset.  A launch that finds them non-zero flags
- * DSA_ERR_DEVICE (bit 8 of the error word).  One workspace serves one call at a
- * time: calls that may overlap on the GPU need separate workspaces. */
-#define DSA_WS_CTRL_BYTES 256
+ * Workspace contract (dsa_decode_ws, dsa_topk_from_scores, dsa_sparse_attn and
+ * the other calls that take a workspace): the caller owns the memory; its first
+ * DSA_WS_CTRL_BYTES bytes are the control region -- grid-barrier words,
+ * per-query flags and a launch counter in the first 1024 bytes, then two radix
+ * histograms that successive launches alternate between -- which must be zero
+ * before the workspace's first use (one cudaMemsetAsync when it is created).  Every call leaves it ready for the next one (barrier and
+ * per-query words back at zero, the histogram the next call uses cleared), so
+ * later calls need no reset.  A launch that finds the grid-barrier words
+ * (bytes 0..3 and 128..131) non-zero flags DSA_ERR_DEVICE (bit 8 of the error
+ * word).  One workspace serves one call at a time: calls that may overlap on the
+ * GPU need separate workspaces. */
+#define DSA_WS_CTRL_BYTES 263168
 DSA_API size_t dsa_workspace_bytes(int32_t T, int64_t L, int32_t topk);
 
 /* The whole step: indexer scan, causal top-k, sparse attention.  Takes its
@@ -200,7 +204,7 @@ DSA_API dsa_status_t dsa_topk_from_scores(const float *scores, int32_t T, int64_
  * capture or a real-time decode loop that forbids allocation after start-up,
  * or a host whose device memory is entirely owned by another allocator.  The
  * paper has no counterpart; this is an interface choice of this library.
- * Its scratch is a static device array of about 17.0 MB inside libdsa.so; every
+ * Its scratch is a static device array of about 17.3 MB inside libdsa.so; every
  * GPU that loads the library holds it until the process exits.
  *   - Limits: T <= 8 and L <= 262144 scores per query; larger L returns
  *     DSA_ERR_INVALID_ARG (say "exceeds the no-allocation scratch limit").
@@ -266,10 +270,10 @@ DSA_API dsa_status_t dsa_debug_fail_next_barriers(int64_t limit_cycles);
 /* Profiling hook for the calling host thread: when device_buffer is not NULL,
  * every launch records, per block b and slot k < 32, the GPU global timer (ns)
  * into ((uint64_t*)device_buffer)[b * 32 + k] at the phase boundaries of the
- * step: 0 start, 1 indexer scan done, 2/3 histogram start/end, 4/5 candidate
- * extraction, 6/7 ordered emission, 8/9 split attention, 10/11 merge, 12-15
- * inside the emission, 30 end; slots 28/29 hold the SM clock counter at start
- * and end.  The buffer must hold dsa_step_grid(...) * 32 entries.  NULL
+ * step: 0 start, 1 indexer scan done, 2/3 candidate extraction (after the
+ * grid barrier), 4/5 the per-query selection (blocks 0..T-1 only), 6 first
+ * attention item starts (after its query's selection), 7 attention done, 8/9
+ * merge, 30 end; slots 28/29 hold the SM clock counter at start and end.  The buffer must hold dsa_step_grid(...) * 32 entries.  NULL
  * disables. */
 DSA_API void dsa_set_step_trace(void *device_buffer);
 

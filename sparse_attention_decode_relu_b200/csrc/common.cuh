@@ -6,8 +6,9 @@
 #include <cstdint>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
-#include <cuda_fp8.h>
 #include <cuda_runtime.h>
+
+#include "dsa_internal.h"
 
 namespace dsa {
 
@@ -20,8 +21,7 @@ enum : uint32_t {
     ERR_BAD_POS = 1u << 4,          // a query position in device memory outside [0, L) (clamped)
 };
 
-// Every spin on an mbarrier gives up after this many SM clocks (~1 s).
-constexpr long long kWaitLimitCycles = 2000000000LL;
+// Every spin on an mbarrier gives up after kWaitLimitCycles SM clocks (~1 s).
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p)
 {
@@ -93,23 +93,23 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
         : "memory");
 }
 
-// 2-D tiled tensor copy global -> shared through a tensor map (TMA).
-__device__ __forceinline__ void tma_load_2d(void* dst, const void* tmap, int32_t x, int32_t y, uint64_t* bar)
+// L2 cache policy for data read once (streamed): evict first.
+__device__ __forceinline__ uint64_t l2_evict_first_policy()
 {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
-        "[%4];" ::"r"(smem_u32(dst)),
-        "l"(tmap), "r"(x), "r"(y), "r"(smem_u32(bar))
-        : "memory");
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
 }
 
-// 1-D tiled tensor copy global -> shared through a tensor map (TMA).
-__device__ __forceinline__ void tma_load_1d(void* dst, const void* tmap, int32_t x, uint64_t* bar)
+// 2-D tiled tensor copy global -> shared through a tensor map (TMA), with an L2
+// cache policy.
+__device__ __forceinline__ void tma_load_2d_hint(void* dst, const void* tmap, int32_t x, int32_t y, uint64_t* bar,
+                                                 uint64_t policy)
 {
     asm volatile(
-        "cp.async.bulk.tensor.1d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2}], [%3];" ::"r"(
-            smem_u32(dst)),
-        "l"(tmap), "r"(x), "r"(smem_u32(bar))
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1, "
+        "{%2, %3}], [%4], %5;" ::"r"(smem_u32(dst)),
+        "l"(tmap), "r"(x), "r"(y), "r"(smem_u32(bar)), "l"(policy)
         : "memory");
 }
 
@@ -155,16 +155,6 @@ __device__ __forceinline__ uint32_t score_key(float f)
     uint32_t b = __float_as_uint(f);
     if ((b & 0x7FFFFFFFu) == 0u) b = 0u;
     return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
-}
-
-// Two E4M3 codes (low byte first) -> two bf16 packed in a uint32.  Exact: every
-// E4M3 value is representable in fp16, fp32 and bf16.
-__device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint16_t two)
-{
-    __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(two), __NV_E4M3);
-    __half2 hh = *reinterpret_cast<__half2*>(&h);
-    float2 f = __half22float2(hh);
-    return pack_bf16(f.x, f.y);
 }
 
 // ---- fifth-generation tensor cores (tcgen05) and tensor memory -----------------
@@ -239,5 +229,53 @@ __device__ __forceinline__ void tmem_ld32_nowait(uint32_t taddr, uint32_t (&r)[3
 }
 
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// 32 consecutive 32-bit columns of this warp's 32 TMEM lanes from registers
+// (lane i of the warp writes row lane-base + i); see tmem_st_wait.
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32])
+{
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+        "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]),
+        "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]),
+        "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// D[tmem] (+)= A[tmem] * B[smem]^T: the A operand (M = 128 rows, one row per
+// TMEM lane, K packed two bf16 per 32-bit column) is read from tensor memory.
+__device__ __forceinline__ void tc_mma_bf16_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                                   uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Four E4M3 codes (byte i = element i) -> two bf16x2 words {e0, e1}, {e2, e3},
+// exactly.  Each code's low seven bits (exponent and mantissa) go to bits 4..10
+// of a 16-bit lane and its sign to bit 15: read as bf16 that is the code's value
+// times 2^-120 for every code, subnormal codes included (the bf16 exponent field
+// takes the E4M3 one unchanged, whose bias is 7 against bf16's 127).  One bf16
+// multiply by 2^120, exact, restores the value.
+__device__ __forceinline__ void e4m3x4_to_bf16x4(uint32_t w, uint32_t& lo, uint32_t& hi)
+{
+    const uint32_t x0 = __byte_perm(w, 0u, 0x1404);   // byte 1 of each 16-bit lane: e0, e1
+    const uint32_t x1 = __byte_perm(w, 0u, 0x3424);   // e2, e3
+    const uint32_t y0 = ((x0 >> 4) & 0x07F007F0u) | (x0 & 0x80008000u);
+    const uint32_t y1 = ((x1 >> 4) & 0x07F007F0u) | (x1 & 0x80008000u);
+    const __nv_bfloat162 k = __floats2bfloat162_rn(0x1p120f, 0x1p120f);
+    __nv_bfloat162 a = __hmul2(*reinterpret_cast<const __nv_bfloat162*>(&y0), k);
+    __nv_bfloat162 b = __hmul2(*reinterpret_cast<const __nv_bfloat162*>(&y1), k);
+    lo = *reinterpret_cast<uint32_t*>(&a);
+    hi = *reinterpret_cast<uint32_t*>(&b);
+}
 
 }  // namespace dsa

@@ -182,13 +182,13 @@ dsa_status_t check_sel(const dsa_tensor_t* sel, int T, int32_t topk)
 }
 
 // ------------------------------------------------------------------ workspace
-// Device workspace of one step: barrier words, the top-k counters the indexer
-// clears, per-block key ranges, per-chunk counts, fp32 scores, candidate lists,
-// and the attention splits' partial states.
+// Device workspace of one step: the control region (barrier and per-query
+// words, two radix histograms), per-query cuts, per-sub-segment candidate
+// counts, candidate lists, fp32 scores, and the attention splits' partial
+// states.
 struct Layout {
     int64_t ld = 0;            // score / candidate row stride (elements)
-    size_t ctrl = 0, hist = 0, list_n = 0, zero_bytes = 0;
-    size_t mm = 0, above = 0, cuts = 0, scores = 0, list = 0, po = 0, pml = 0;
+    size_t ctrl = 0, cuts = 0, seg_n = 0, scores = 0, list = 0, po = 0, pml = 0;
     size_t total = 0;
 };
 
@@ -207,17 +207,13 @@ Layout layout(int T, int64_t L, bool with_scores = true, bool with_attn = true)
         return at;
     };
     l.ctrl = take(kWsCtrlBytes);
-    l.hist = take(sizeof(uint32_t) * ((size_t)T * kHistBins + kMaxT));
-    l.list_n = l.hist + sizeof(uint32_t) * (size_t)T * kHistBins;
-    l.zero_bytes = sizeof(uint32_t) * ((size_t)T * kHistBins + kMaxT);
-    l.mm = take(sizeof(uint2) * (size_t)kMaxGrid * kMaxT);
-    l.above = take(sizeof(uint32_t) * (size_t)kMaxT * kMaxChunksStep);
     l.cuts = take(sizeof(uint32_t) * 4 * kMaxT);
+    l.seg_n = take(sizeof(uint32_t) * (size_t)kMaxT * kMaxSeg);
     l.list = take(sizeof(uint2) * (size_t)T * l.ld);
     if (with_scores) l.scores = take(sizeof(float) * (size_t)T * l.ld);
     if (with_attn) {
-        l.po = take(sizeof(float) * (size_t)kMaxAttnItems * kH * kD);
-        l.pml = take(sizeof(float2) * (size_t)kMaxAttnItems * kH);
+        l.po = take(sizeof(float) * (size_t)kMaxT * kG * kMaxSplitsTG * 16 * kD);
+        l.pml = take(sizeof(float2) * (size_t)kMaxT * kG * kMaxSplitsTG * 16);
     }
     l.total = off;
     return l;
@@ -249,9 +245,10 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
     return fn;
 }
 
-// TMA descriptors of the indexer key cache (128-key tiles; bf16 rows land
-// 128B-swizzled) and of its per-token scales (128 per tile).
-dsa_status_t encode_key_maps(const dsa_tensor_t* k, const Shape& sh, CUtensorMap& map, CUtensorMap& smap)
+// TMA descriptor of the indexer key cache: 128-key tiles; bf16 rows land
+// 128B-swizzled (the MMA's shared-memory operand layout), E4M3 rows 64B-swizzled
+// (conflict-free row reads for the widening).
+dsa_status_t encode_key_map(const dsa_tensor_t* k, const Shape& sh, CUtensorMap& map)
 {
     auto enc = encode_fn();
     if (!enc) return fail(DSA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
@@ -261,20 +258,9 @@ dsa_status_t encode_key_maps(const dsa_tensor_t* k, const Shape& sh, CUtensorMap
     const cuuint32_t estr[2] = {1, 1};
     CUresult r = enc(&map, sh.fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, k->data, dims,
                      strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                     sh.fp8 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B,
+                     sh.fp8 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(DSA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
-    std::memset(&smap, 0, sizeof smap);
-    if (k->scale) {
-        const cuuint64_t sdims[1] = {static_cast<cuuint64_t>(sh.L)};
-        const cuuint64_t sstr[1] = {static_cast<cuuint64_t>(sh.L * 4)};
-        const cuuint32_t sbox[1] = {static_cast<cuuint32_t>(kKeyTile)};
-        const cuuint32_t sestr[1] = {1};
-        r = enc(&smap, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 1, const_cast<float*>(k->scale), sdims, sstr, sbox, sestr,
-                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-        if (r != CUDA_SUCCESS) return fail(DSA_ERR_CUDA, "cuTensorMapEncodeTiled (scale) failed (%d)", static_cast<int>(r));
-    }
     return DSA_OK;
 }
 
@@ -291,59 +277,57 @@ int grid_blocks(const DeviceInfo& dev, bool fp8)
     return g;
 }
 
-// Fill the top-k part of the parameters (work split, workspace pointers).
+// Fill the top-k part of the parameters (work split, workspace pointers): one
+// extraction item per (query, chunk) and block, chunks a multiple of 256
+// positions so that each warp's eighth starts 128-byte aligned.
 void topk_params(StepParams& p, void* ws, const Layout& l)
 {
-    p.hist = at<uint32_t>(ws, l.hist);
-    p.list_n = at<uint32_t>(ws, l.list_n);
+    p.cuts = at<uint32_t>(ws, l.cuts);
+    p.seg_n = at<uint32_t>(ws, l.seg_n);
     p.list = at<uint2>(ws, l.list);
     p.list_ld = l.ld;
-    p.above = at<uint32_t>(ws, l.above);
-    p.cuts = at<uint32_t>(ws, l.cuts);
-    p.mm = at<uint2>(ws, l.mm);
-    p.mm_slots = p.grid;
-    p.zero = at<uint32_t>(ws, l.hist);
-    p.zero_words = static_cast<int32_t>(l.zero_bytes / 4);
     int nchunk = p.grid / p.T;
     if (nchunk < 1) nchunk = 1;
     if (nchunk > kMaxChunksStep) nchunk = kMaxChunksStep;
-    int64_t chunk = round_up((p.n_max + nchunk - 1) / nchunk, 4);
-    if (chunk < 4) chunk = 4;
+    int64_t chunk = round_up((p.n_max + nchunk - 1) / nchunk, 256);
+    if (chunk < 256) chunk = 256;
     p.chunk = static_cast<int32_t>(chunk);
     p.nchunk = static_cast<int32_t>((p.n_max + chunk - 1) / chunk);
     if (p.nchunk < 1) p.nchunk = 1;
 }
 
-void attn_params(StepParams& p, void* ws, const Layout& l, int32_t topk)
+// Attention work split: items (query, KV group, row split), about one per
+// block; splits of a multiple of 16 rows, at most kMaxRowsPerSplit rows and
+// kMaxSplitsTG splits per (query, group).
+void attn_params(StepParams& p, void* ws, const Layout& l, int32_t rows)
 {
-    int64_t nsplit = p.grid / p.T;
-    if (nsplit * p.T > kMaxAttnItems) nsplit = kMaxAttnItems / p.T;
+    int64_t nsplit = p.grid / (p.T * kG);
+    if (nsplit > kMaxSplitsTG) nsplit = kMaxSplitsTG;
     if (nsplit < 1) nsplit = 1;
-    int64_t rps = round_up((topk + nsplit - 1) / nsplit, 16);
+    int64_t rps = round_up((rows + nsplit - 1) / nsplit, 16);
     if (rps > kMaxRowsPerSplit) rps = kMaxRowsPerSplit;
-    p.rows = topk;
+    p.rows = rows;
     p.rows_per_split = static_cast<int32_t>(rps);
-    p.nsplit = static_cast<int32_t>((topk + rps - 1) / rps);
+    p.nsplit = static_cast<int32_t>((rows + rps - 1) / rps);
     p.po = at<float>(ws, l.po);
     p.pml = at<float2>(ws, l.pml);
 }
 
-dsa_status_t launch(const CUtensorMap& map, const CUtensorMap& smap, StepParams& p, bool fp8, void* ws,
-                    const Layout& l, cudaStream_t stream)
+dsa_status_t launch(const CUtensorMap& map, StepParams& p, bool fp8, void* ws, const Layout& l, cudaStream_t stream)
 {
     cudaError_t e;
-    // Grid barriers are used: their control words are zero from the workspace's
-    // creation on, and every launch leaves them zero.
-    if (p.phases & (kPhaseTopk | kPhaseAttend)) p.bar_ctrl = at<uint32_t>(ws, l.ctrl);
+    // Every launch with a workspace uses its control region: zero from the
+    // workspace's creation on, and each launch leaves it ready for the next.
+    p.ctrl = ws != nullptr ? at<uint32_t>(ws, l.ctrl) : nullptr;
     p.trace = t_trace;
     p.barrier_limit = kWaitLimitCycles;
     p.barrier_extra = 0;
-    if (t_fail_barriers > 0 && p.bar_ctrl != nullptr) {   // one launch only
+    if (t_fail_barriers > 0 && p.ctrl != nullptr) {   // one launch only
         p.barrier_limit = t_fail_barriers;
         p.barrier_extra = 1;
         t_fail_barriers = 0;
     }
-    if ((e = launch_step(&map, &smap, p, fp8, stream)) != cudaSuccess) return cuda_fail(e, "step launch");
+    if ((e = launch_step(&map, p, fp8, stream)) != cudaSuccess) return cuda_fail(e, "step launch");
     g_launches += 1;
     return DSA_OK;
 }
@@ -377,13 +361,13 @@ dsa_status_t check_decode_args(const dsa_tensor_t* q, const dsa_tensor_t* q_idx,
 // ------------------------------------------------------------------ no-allocation top-k
 // Scratch for dsa_topk_from_scores_noalloc: a file-scope device array, so that
 // entry point never allocates.  Sized for T <= 8 queries and L <= 262144 scores
-// per query: barrier words, the top-k counters, per-block key ranges, per-chunk
-// counts and the candidate lists (about 17.0 MB per device, held until the
-// process exits).
+// per query: the control region (barrier words, two radix histograms), cuts,
+// per-sub-segment counts and the candidate lists (about 17.3 MB per device,
+// held until the process exits).  Static device memory starts zeroed, which is
+// the state the control region needs before its first use.
 constexpr int64_t kNoAllocMaxL = 262144;
-constexpr size_t kNoAllocBytes = ru256(kWsCtrlBytes) + ru256(sizeof(uint32_t) * ((size_t)kMaxT * kHistBins + kMaxT)) +
-                                 ru256(sizeof(uint2) * (size_t)kMaxGrid * kMaxT) +
-                                 ru256(sizeof(uint32_t) * (size_t)kMaxT * kMaxChunksStep) + ru256(sizeof(uint32_t) * 4 * kMaxT) +
+constexpr size_t kNoAllocBytes = ru256(kWsCtrlBytes) + ru256(sizeof(uint32_t) * 4 * kMaxT) +
+                                 ru256(sizeof(uint32_t) * (size_t)kMaxT * kMaxSeg) +
                                  ru256(sizeof(uint2) * (size_t)kMaxT * ((kNoAllocMaxL + 63) / 64 * 64));
 
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocBytes];
@@ -416,7 +400,7 @@ dsa_status_t run_topk_stage(const float* scores, int32_t T, int64_t L, int64_t l
     dsa_status_t st = device_info(dev);
     if (st) return st;
     StepParams p{};
-    p.phases = kPhaseRanges | kPhaseTopk;
+    p.phases = kPhaseHistScores | kPhaseTopk;
     p.grid = grid_blocks(dev, false);
     set_pos(p, pos, T);
     p.L = static_cast<int32_t>(L);
@@ -429,7 +413,7 @@ dsa_status_t run_topk_stage(const float* scores, int32_t T, int64_t L, int64_t l
     topk_params(p, ws, l);
     CUtensorMap none;
     std::memset(&none, 0, sizeof none);
-    return launch(none, none, p, false, ws, l, stream);
+    return launch(none, p, false, ws, l, stream);
 }
 
 }  // namespace
@@ -469,8 +453,8 @@ static dsa_status_t decode_ws(const dsa_tensor_t* q, const dsa_tensor_t* q_idx, 
     DeviceInfo dev;
     if ((st = device_info(dev))) return st;
     cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
-    CUtensorMap map, smap;
-    if ((st = encode_key_maps(k_idx_cache, sh, map, smap))) return st;
+    CUtensorMap map;
+    if ((st = encode_key_map(k_idx_cache, sh, map))) return st;
     StepParams p{};
     p.phases = kPhaseIndex | kPhaseTopk | kPhaseAttend;
     p.grid = grid_blocks(dev, sh.fp8);
@@ -500,7 +484,7 @@ static dsa_status_t decode_ws(const dsa_tensor_t* q, const dsa_tensor_t* q_idx, 
     topk_params(p, workspace, l);
     attn_params(p, workspace, l, topk);
     stage_event(0, stream);
-    st = launch(map, smap, p, sh.fp8, workspace, l, stream);
+    st = launch(map, p, sh.fp8, workspace, l, stream);
     for (int i = 1; i < 5; ++i) stage_event(i, stream);
     return st;
 }
@@ -577,7 +561,7 @@ dsa_status_t dsa_swa_decode(const dsa_tensor_t* q, const dsa_tensor_t* kv_cache,
     attn_params(p, workspace, l, window);
     CUtensorMap none;
     std::memset(&none, 0, sizeof none);
-    return launch(none, none, p, false, workspace, l, reinterpret_cast<cudaStream_t>(stream_));
+    return launch(none, p, false, workspace, l, reinterpret_cast<cudaStream_t>(stream_));
 }
 
 dsa_status_t dsa_decode(const dsa_tensor_t* q, const dsa_tensor_t* q_idx, const dsa_tensor_t* w_idx,
@@ -615,8 +599,8 @@ dsa_status_t dsa_index_scores(const dsa_tensor_t* q_idx, const dsa_tensor_t* w_i
     if (ld < sh.L || ld % 4) return fail(DSA_ERR_INVALID_ARG, "scores: ld = %lld must be >= L and a multiple of 4", (long long)ld);
     DeviceInfo dev;
     if ((st = device_info(dev))) return st;
-    CUtensorMap map, smap;
-    if ((st = encode_key_maps(k_idx_cache, sh, map, smap))) return st;
+    CUtensorMap map;
+    if ((st = encode_key_map(k_idx_cache, sh, map))) return st;
     StepParams p{};
     p.phases = kPhaseIndex;
     p.grid = grid_blocks(dev, sh.fp8);
@@ -629,7 +613,7 @@ dsa_status_t dsa_index_scores(const dsa_tensor_t* q_idx, const dsa_tensor_t* w_i
     p.ld = ld;
     p.err = dev.err;
     const Layout l{};
-    return launch(map, smap, p, sh.fp8, nullptr, l, reinterpret_cast<cudaStream_t>(stream_));
+    return launch(map, p, sh.fp8, nullptr, l, reinterpret_cast<cudaStream_t>(stream_));
 }
 
 dsa_status_t dsa_topk_from_scores(const float* scores, int32_t T, int64_t L, int64_t ld, const int32_t* pos,
@@ -723,7 +707,7 @@ dsa_status_t dsa_sparse_attn(const dsa_tensor_t* q, const dsa_tensor_t* kv_cache
     attn_params(p, workspace, l, topk);
     CUtensorMap none;
     std::memset(&none, 0, sizeof none);
-    return launch(none, none, p, false, workspace, l, reinterpret_cast<cudaStream_t>(stream_));
+    return launch(none, p, false, workspace, l, reinterpret_cast<cudaStream_t>(stream_));
 }
 
 dsa_status_t dsa_device_status(dsa_stream_t stream_)

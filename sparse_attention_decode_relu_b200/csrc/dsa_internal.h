@@ -14,23 +14,43 @@ constexpr int kHI = 16, kDI = 64;          // indexer heads, indexer dim
 constexpr int kMaxT = 8;
 constexpr int kMaxTopk = 2048;
 constexpr int kKeyTile = 128;              // keys per indexer tile
-constexpr int kHistBins = 4096;            // first-level radix bins (top 12 key bits)
+constexpr int kHistBins = 4096;            // first radix level: the top 12 bits of a score key
+constexpr int kHistShift = 20;             // key >> kHistShift is the bin
 
-constexpr int kMaxRowsPerSplit = 256;       // selected rows one attention work item gathers
+constexpr int kMaxRowsPerSplit = 512;       // selected rows one attention work item gathers
+constexpr int kMaxSplitsTG = 16;            // attention row splits per (query, KV group)
 constexpr int kMaxChunksStep = 1024;        // top-k chunks per query (<= grid)
+constexpr int kSegPerChunk = 8;             // candidate sub-segments per chunk (one per warp)
+constexpr int kMaxSeg = kMaxChunksStep * kSegPerChunk;
 constexpr int kMaxGrid = 1024;              // blocks of the step kernel
-constexpr int kMaxAttnItems = 512;          // (query, split) attention work items
 constexpr int kTraceSlots = 32;             // phase-boundary stamps per block
-constexpr int kBarCtrlBytes = 128;          // grid barrier arrival counter (its own line)
-constexpr int kWsCtrlBytes = kBarCtrlBytes + 128;  // + the exit counter: workspace bytes [0, 256)
+
+// Workspace control region.  Words (uint32) of the first 1024 bytes:
+//   0          grid-barrier arrival count      (own 128-byte line)
+//   32         exit count                      (own line)
+//   64         launch epoch (never reset; selects the histogram buffer)
+//   96 + t     extraction items of query t that are done
+//   128 + t    query t's selection is written
+//   160 + 4t+g attention splits of (query t, KV group g) that are done
+// then two global histograms [2][kMaxT][kHistBins] u32.  Every word but the
+// epoch is zero again when a launch ends; launch e uses histogram e & 1 and
+// clears histogram (e + 1) & 1 for the next one.  The whole region must be zero
+// before a workspace's first use.
+constexpr int kCtrlWordExit = 32, kCtrlWordEpoch = 64, kCtrlWordArrive = 96, kCtrlWordReady = 128,
+              kCtrlWordDone = 160;
+constexpr int kCtrlBytes = 1024;
+constexpr int kHistWords = kMaxT * kHistBins;                 // one histogram buffer
+constexpr int kWsCtrlBytes = kCtrlBytes + 2 * kHistWords * 4;  // must be zero before first use
+
+constexpr long long kWaitLimitCycles = 2000000000LL;   // every spin gives up after this many SM clocks (~1 s)
 
 // Phases of the step kernel.
 enum : int {
-    kPhaseIndex = 1,    // indexer scan (scores + per-block key ranges)
-    kPhaseRanges = 2,   // per-block key ranges of caller-provided scores
-    kPhaseTopk = 4,     // histogram, candidates, ordered emission
-    kPhaseAttend = 8,   // split attention + merge
-    kPhaseSelectPos = 16,   // selection by position: the last `window` visible positions
+    kPhaseIndex = 1,       // indexer scan (scores; with a workspace also the first radix histogram)
+    kPhaseHistScores = 2,  // first radix histogram of caller-provided scores
+    kPhaseTopk = 4,        // candidate extraction, per-query selection
+    kPhaseAttend = 8,      // split attention + merge
+    kPhaseSelectPos = 16,  // selection by position: the last `window` visible positions
 };
 
 struct StepParams {
@@ -46,17 +66,11 @@ struct StepParams {
     float* scores;           // [T][ld]
     int64_t ld;
     // top-k
-    uint2* mm;               // [grid][kMaxT] per-block (min, max) key of visible scores
-    int32_t mm_slots;
-    uint32_t* hist;          // [T][kHistBins]
-    uint32_t* list_n;        // [kMaxT] candidates per query
-    uint2* list;             // [T][list_ld] (key, position) candidates
+    uint32_t* cuts;          // [kMaxT][4]: threshold-bin key, #keys above the bin
+    uint32_t* seg_n;         // [kMaxT][kMaxSeg] candidates per sub-segment
+    uint2* list;             // [T][list_ld] (key, position): sub-segment (c, w) starts at c*chunk + w*chunk/8
     int64_t list_ld;         // candidate-list row stride (the workspace's, not the caller's score stride)
-    uint32_t* above;         // [T][kMaxChunksStep] keys above the threshold bin, per chunk
-    uint32_t* cuts;          // [kMaxT][4]: threshold bin (cut, ctop) and #keys above it, per query
-    uint32_t* zero;          // words phase 1 clears (hist, list_n)
-    int32_t zero_words;
-    int32_t chunk, nchunk;   // top-k work items: nchunk chunks of `chunk` positions per query
+    int32_t chunk, nchunk;   // extraction items: nchunk chunks of `chunk` positions per query (chunk % 256 == 0)
     int32_t* sel;            // [T][sel_ld]
     int64_t sel_ld;
     // attention
@@ -65,23 +79,22 @@ struct StepParams {
     int64_t kv_ld;
     int32_t rows;            // selected rows per query to read (= topk)
     int32_t rows_per_split;  // multiple of 16, <= kMaxRowsPerSplit
-    int32_t nsplit;
+    int32_t nsplit;          // row splits per (query, KV group), <= kMaxSplitsTG
     const float* sink;       // [64] or nullptr
     int32_t window;          // kPhaseSelectPos: positions selected per query (<= topk)
-    float* po;               // [T][nsplit][64][128] partial outputs
-    float2* pml;             // [T][nsplit][64] (max in log2 units, sum)
+    float* po;               // [T][4][nsplit][16][128] partial outputs per (query, group, split)
+    float2* pml;             // [T][4][nsplit][16] (max in log2 units, sum)
     uint16_t* out;           // [T][64][128] bf16
     // control
     unsigned long long* trace;   // [grid][kTraceSlots] globaltimer stamps at phase boundaries, or nullptr
-    uint32_t* bar_ctrl;      // grid barrier arrival counter (zero at launch)
-    int64_t barrier_limit;   // SM clocks a grid-barrier wait spins before it gives up
-    uint32_t barrier_extra;  // arrivals a grid barrier waits for beyond the grid (0; 1 = a block that never comes)
+    uint32_t* ctrl;          // workspace control region (kWsCtrlBytes), or nullptr (indexer stage alone)
+    int64_t barrier_limit;   // SM clocks a wait between blocks spins before it gives up
+    uint32_t barrier_extra;  // arrivals such a wait needs beyond the real ones (0; 1 = a block that never comes)
     uint32_t* err;
 };
 
 int step_smem_bytes();
 int step_max_blocks(bool fp8);
-cudaError_t launch_step(const CUtensorMap* kmap, const CUtensorMap* smap, const StepParams& p, bool fp8,
-                        cudaStream_t s);
+cudaError_t launch_step(const CUtensorMap* kmap, const StepParams& p, bool fp8, cudaStream_t s);
 
 }  // namespace dsa

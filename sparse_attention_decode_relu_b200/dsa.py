@@ -20,7 +20,8 @@ from . import build as _build
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_DEVICE = 0, 1, 2, 3, 4
 BF16, FP8_E4M3, F32, I32 = 0, 1, 2, 3
-WS_CTRL_BYTES = 256   # DSA_WS_CTRL_BYTES: leading workspace bytes that must be zero before first use
+WS_CTRL_BYTES = 263168   # DSA_WS_CTRL_BYTES: leading workspace bytes that must be zero before first use
+WS_WORDS_ZERO_AFTER_CALL = [0, 32] + list(range(96, 104)) + list(range(128, 136))   # int32 words a call leaves at 0
 
 _lock = threading.Lock()
 _lib = None
@@ -279,7 +280,7 @@ def workspace(T: int, L: int, topk: int, device=None) -> torch.Tensor:
     if n == 0:
         raise DsaError(ERR_INVALID_ARG, "invalid sizes for a workspace")
     ws = torch.empty(n, dtype=torch.uint8, device=device or "cuda")
-    ws[:WS_CTRL_BYTES].zero_()   # grid-barrier control words start at zero; calls keep them so
+    ws[:WS_CTRL_BYTES].zero_()   # the control region starts at zero; every call leaves it ready for the next
     return ws
 
 

@@ -63,6 +63,33 @@ def test_indexer_scores(name, kw):
         assert np.array_equal(gs, os_)   # every score is an exact fp32 integer or half-integer
 
 
+def test_indexer_decodes_every_e4m3_code():
+    """Every finite E4M3 code (subnormals and both zeros included) widened by the
+    indexer, at every dim position: key row s holds one code at dim s % 64 (twice,
+    at two dim offsets); the queries are +1 and -1 on every dim of head 0, so the
+    scores are ReLU(+-value) of each code, exact in fp32."""
+    codes = np.array([c for c in range(256) if c not in (0x7F, 0xFF)], np.uint8)
+    L = 2 * len(codes)
+    k = np.zeros((L, 64), np.uint8)
+    for s in range(L):
+        k[s, (s + 7 * (s >= len(codes))) % 64] = codes[s % len(codes)]
+    w = synth.make_workload("codes", L=L, T=2, key_dtype="fp8", recipe="int", seed=5)
+    w.k_idx = k
+    w.k_scale = np.ones(L, np.float32)
+    qf = np.zeros((2, 16, 64), np.float32)
+    qf[0, 0, :] = 1.0
+    qf[1, 0, :] = -1.0
+    w.q_idx = synth.f32_to_bf16_bits(qf)
+    w.w_idx = np.zeros((2, 16), np.float32)
+    w.w_idx[:, 0] = 1.0
+    w.pos = np.array([L - 1, L - 1], np.int32)
+    d = dsa.to_device(w, with_kv=False)
+    gs = gpu_scores(w, d)
+    os_ = oracle.index_scores(w.q_idx, w.w_idx, w.k_idx, w.k_scale, w.pos)
+    assert np.array_equal(gs, os_)
+    assert (gs > 0).sum() == 2 * 2 * 126   # 126 positive and 126 negative non-zero codes, twice
+
+
 @pytest.mark.parametrize("name,kw", SMALL, ids=[s[0] for s in SMALL])
 def test_decode_step(name, kw):
     w = _workload(name, kw)
@@ -295,15 +322,24 @@ def test_verify_1m_integer_twin_selection():
     assert np.array_equal(sel.cpu().numpy(), oracle.topk(os_, w.pos, w.topk))
 
 
+def _ctrl_words_zero(ws):
+    words = ws[:1024].view(torch.int32)
+    return all(int(words[i]) == 0 for i in dsa.WS_WORDS_ZERO_AFTER_CALL)
+
+
 def test_workspace_control_words_left_zero_and_checked():
-    """Each launch leaves the workspace's grid-barrier control words at zero, so a
-    workspace needs zeroing only once; a launch that finds them non-zero reports
-    it (device error word) and skips the work that depends on the barrier."""
+    """Each launch leaves the workspace's grid-barrier and per-query words at zero
+    (and advances its launch counter), so a workspace needs zeroing only once; a
+    launch that finds the barrier words non-zero reports it (device error word)
+    and skips the work that depends on the barrier."""
     w = synth.config("tiny_decode")
     d = dsa.to_device(w)
     ws = dsa.workspace(w.T, w.L, w.topk)
     ref_o, ref_s = gpu_decode(w, d, ws=ws)
-    assert int(ws[: dsa.WS_CTRL_BYTES].count_nonzero()) == 0
+    assert _ctrl_words_zero(ws)
+    assert int(ws[:1024].view(torch.int32)[64]) == 1   # one launch so far
+    o1, s1 = gpu_decode(w, d, ws=ws)                    # the other histogram buffer, same result
+    assert np.array_equal(s1, ref_s) and np.array_equal(o1, ref_o) and _ctrl_words_zero(ws)
     ws[:4].view(torch.int32).fill_(1 << 16)       # an arrival count no launch can start from
     out, sel = dsa.decode(d["q"], d["q_idx"], d["w_idx"], d["k_idx"], d["kv"], d["pos"], w.topk,
                           k_scale=d["k_scale"], ws=ws)
@@ -330,7 +366,7 @@ def test_barrier_wait_timeout_is_reported_and_recovers():
     with pytest.raises(dsa.DsaError) as e:
         dsa.dsa_device_status()
     assert e.value.status == dsa.ERR_DEVICE and "word 0x1 " in str(e.value)
-    assert int(ws[: dsa.WS_CTRL_BYTES].count_nonzero()) == 0
+    assert _ctrl_words_zero(ws)
     o2, s2 = gpu_decode(w, d, ws=ws)   # the hook covered one launch only
     assert np.array_equal(s2, ref_s) and np.array_equal(o2, ref_o)
     ora_o, ora_s = oracle.decode(w.q, w.q_idx, w.w_idx, w.k_idx, w.k_scale, w.kv, w.pos, w.topk)
