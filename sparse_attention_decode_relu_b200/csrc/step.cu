@@ -335,9 +335,11 @@ constexpr uint32_t kACol = kAccBufs * 128;   // first column of the A buffers
 constexpr int kTileBytesBf16 = kKeyTile * kDI * 2;   // 16 KiB, one 128 x 64 bf16 operand tile
 constexpr int kHistFlushTiles = 256;         // an epilogue warp flushes its share of the 16-bit counters this often
 static_assert(kACol + kABufs * 32 <= kTmemCols, "tensor memory budget");
-static_assert(kRawStagesF8 * kKeyTile * kDI + kTileBytesBf16 + kMaxT * kHI * 4 + kHistWords * 2 <= kDataBytes,
+static_assert(kRawStagesF8 * kKeyTile * kDI + kTileBytesBf16 + kMaxT * kHI * 4 + kHistWords * 2 + 4 * 32 * kMaxT * 4 <=
+                  kDataBytes,
               "FP8 indexer buffers fit the data region");
-static_assert(kRawStagesBf * kTileBytesBf16 + kTileBytesBf16 + kMaxT * kHI * 4 + kHistWords * 2 <= kDataBytes,
+static_assert(kRawStagesBf * kTileBytesBf16 + kTileBytesBf16 + kMaxT * kHI * 4 + kHistWords * 2 + 4 * 32 * kMaxT * 4 <=
+                  kDataBytes,
               "bf16 indexer buffers fit the data region");
 
 // The block's 16-bit counters (two per word) added to the launch's histogram.
@@ -363,6 +365,7 @@ __device__ void phase_index(const CUtensorMap& kmap, const StepParams& p, uint8_
     uint8_t* qsw = smem + S * raw_bytes;                                // [128 rows][128 B] queries (B operand)
     float* w_s = reinterpret_cast<float*>(qsw + kTileBytesBf16);        // [8][16]
     uint32_t* hs = reinterpret_cast<uint32_t*>(w_s + kMaxT * kHI);      // [8][2048]: two 16-bit counters per word
+    uint32_t* hstage = hs + kHistWords / 2;                             // [4 warps][32 keys][8 queries] bins
     uint64_t* raw_full = bars + kBarRawFull;
     uint64_t* raw_empty = bars + kBarRawEmpty;
     uint64_t* a_full = bars + kBarAFull;
@@ -557,6 +560,9 @@ __device__ void phase_index(const CUtensorMap& kmap, const StepParams& p, uint8_
             }
             tc_fence_after();
             const uint32_t tbase = tmem + lane_base + cb * 128;
+            uint32_t bins[kMaxT];   // histogram bin of each query's score (~0u: not counted)
+#pragma unroll
+            for (int k = 0; k < kMaxT; ++k) bins[k] = ~0u;
             // Queries in groups of four: two 32-column loads in flight, one wait.
 #pragma unroll
             for (int g = 0; g < kMaxT / 4; ++g) {
@@ -574,29 +580,44 @@ __device__ void phase_index(const CUtensorMap& kmap, const StepParams& p, uint8_
                     for (int u = 0; u < 4; ++u) {
                         const int t = g * 4 + u;
                         if (t < T) {
+                            // Four partial sums over heads {j, j+4, j+8, j+12}, j < 4, as two packed
+                            // fp32 FMAs per four heads, combined in a fixed order.
                             const float4* w4 = reinterpret_cast<const float4*>(w_s + t * kHI);
                             const float* v = reinterpret_cast<const float*>(&r[u >> 1][(u & 1) * 16]);
-                            float part[4] = {0.f, 0.f, 0.f, 0.f};
+                            float2 p01 = make_float2(0.f, 0.f), p23 = make_float2(0.f, 0.f);
 #pragma unroll
                             for (int g4 = 0; g4 < 4; ++g4) {
                                 const float4 w = w4[g4];
-                                part[0] = fmaf(fmaxf(v[g4 * 4 + 0], 0.f), w.x, part[0]);
-                                part[1] = fmaf(fmaxf(v[g4 * 4 + 1], 0.f), w.y, part[1]);
-                                part[2] = fmaf(fmaxf(v[g4 * 4 + 2], 0.f), w.z, part[2]);
-                                part[3] = fmaf(fmaxf(v[g4 * 4 + 3], 0.f), w.w, part[3]);
+                                p01 = __ffma2_rn(make_float2(fmaxf(v[g4 * 4 + 0], 0.f), fmaxf(v[g4 * 4 + 1], 0.f)),
+                                                 make_float2(w.x, w.y), p01);
+                                p23 = __ffma2_rn(make_float2(fmaxf(v[g4 * 4 + 2], 0.f), fmaxf(v[g4 * 4 + 3], 0.f)),
+                                                 make_float2(w.z, w.w), p23);
                             }
-                            const float acc = ((part[0] + part[1]) + (part[2] + part[3])) * scale;
+                            const float acc = ((p01.x + p01.y) + (p23.x + p23.y)) * scale;
                             if (s < p.L) {
                                 const bool vis = s <= pos_q[t];
                                 p.scores[(int64_t)t * p.ld + s] = vis ? acc : -INFINITY;
-                                if (hist && vis) {
-                                    const uint32_t bin = score_key(acc) >> kHistShift;
-                                    atomicAdd(&hs[t * (kHistBins / 2) + (bin >> 1)], 1u << ((bin & 1) << 4));
-                                }
+                                if (vis) bins[t] = score_key(acc) >> kHistShift;
                             }
                         }
                     }
                 }
+            }
+            if (hist) {
+                // Count the bins through a transpose in shared memory: lane l then adds key
+                // (4i + l/8)'s bin of query l % 8 in round i, so one atomic instruction spreads
+                // over eight query histograms instead of one (far fewer address conflicts).
+                uint32_t* st = hstage + quad * 32 * kMaxT;
+                *reinterpret_cast<uint4*>(st + lane * kMaxT) = make_uint4(bins[0], bins[1], bins[2], bins[3]);
+                *reinterpret_cast<uint4*>(st + lane * kMaxT + 4) = make_uint4(bins[4], bins[5], bins[6], bins[7]);
+                __syncwarp();
+                uint32_t* hq = hs + (lane & (kMaxT - 1)) * (kHistBins / 2);
+#pragma unroll
+                for (int i = 0; i < kMaxT; ++i) {
+                    const uint32_t bin = st[i * 32 + lane];
+                    if (bin != ~0u) atomicAdd(&hq[bin >> 1], 1u << ((bin & 1) << 4));
+                }
+                __syncwarp();
             }
             if (hist && (e + 1) % kHistFlushTiles == 0) {
                 // 16-bit counters: this warp moves its quarter of them to the global
@@ -653,7 +674,8 @@ __device__ void phase_hist_scores(const StepParams& p, uint8_t* smem)
         if (n <= p.topk) continue;
         for (int b = tid; b < kHistBins; b += kThreads) h[b] = 0u;
         __syncthreads();
-        const int64_t s0 = min((int64_t)n, (int64_t)blockIdx.x * per), s1 = min((int64_t)n, s0 + per);
+        // this block's slice [s0, s1): s0 is a multiple of 4 unless the slice is empty
+        const int64_t s0 = (int64_t)blockIdx.x * per, s1 = min((int64_t)n, s0 + per);
         const float4* row = reinterpret_cast<const float4*>(p.scores + (int64_t)t * p.ld);
         bool nan = false;
         for (int64_t q0 = s0 / 4; q0 * 4 < s1; q0 += 4 * kThreads) {
@@ -669,7 +691,7 @@ __device__ void phase_hist_scores(const StepParams& p, uint8_t* smem)
                 const float f[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
 #pragma unroll
                 for (int k = 0; k < 4; ++k)
-                    if (s + k < s1) {
+                    if (s + k >= s0 && s + k < s1) {
                         nan |= f[k] != f[k];
                         atomicAdd(&h[score_key(f[k]) >> kHistShift], 1u);
                     }
@@ -831,11 +853,29 @@ __device__ void phase_select(const StepParams& p, uint8_t* smem, uint32_t* res, 
             uint32_t nsel = 0;
             if (m <= static_cast<uint32_t>(kSelCap)) {
                 // ---- the candidates fit in shared memory ----
+                // Entry j's sub-segment is the last k with off[k] <= j (binary search); eight
+                // independent loads in flight per thread.
                 uint2* ent = reinterpret_cast<uint2*>(smem + kSelEntOff);
-                for (int k = warp; k < nseg; k += kWarps) {
-                    const uint32_t o = off[k], cnt = seg_cnt(k);
-                    const uint2* src = glist + seg_start(p, k);
-                    for (uint32_t j = lane; j < cnt; j += 32) ent[o + j] = __ldcg(src + j);
+                for (uint32_t j0 = 0; j0 < m; j0 += 8 * kThreads) {
+                    uint2 v[8];
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        const uint32_t j = j0 + u * kThreads + tid;
+                        v[u] = make_uint2(0u, 0u);
+                        if (j < m) {
+                            int a = 0, b = nseg - 1;   // off[a] <= j < off[b + 1]
+                            while (a < b) {
+                                const int mid = (a + b + 1) >> 1;
+                                if (off[mid] <= j) a = mid; else b = mid - 1;
+                            }
+                            v[u] = __ldcg(glist + seg_start(p, a) + (j - off[a]));
+                        }
+                    }
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        const uint32_t j = j0 + u * kThreads + tid;
+                        if (j < m) ent[j] = v[u];
+                    }
                 }
                 __syncthreads();
 #pragma unroll 1
@@ -963,8 +1003,9 @@ __device__ void phase_select_pos(const StepParams& p)
 // When the step selected the rows itself, an item starts as soon as its query's
 // selection is flagged; with selection by position the rows follow from the
 // query position directly.  Warp 4 gathers the selected rows' K and V of group
-// g (two 256-byte pieces per row) by bulk async copy into a ring of 16-row
-// tiles; consumer warps 0-3 take the tiles in turn: the 16 query heads of the
+// g (two 256-byte pieces per row, one row per warp instruction of 16-byte
+// asynchronous copies) into a ring of 16-row tiles; consumer warps 0-3 take the
+// tiles in turn: the 16 query heads of the
 // group are the 16 rows of an m16n8k16 tile (QK and PV on the tensor cores,
 // online softmax in the exp2 domain).  The four warps' states are merged in
 // shared memory, in warp order, into the item's partial (max, sum, output),
@@ -1003,7 +1044,7 @@ __device__ void phase_attend(const StepParams& p, uint8_t* smem, uint64_t* bars,
     int phase_base = 0;   // tiles this block has gathered so far (mbarrier phase bookkeeping)
     if (tid == 0) {
         for (int s = 0; s < kAttStagesG; ++s) {
-            mbar_init(&full[s], 1);
+            mbar_init(&full[s], 33);   // the producer's 32 lanes' copies landed + its row indices written
             mbar_init(&empty[s], 1);
         }
         fence_mbar_init();
@@ -1072,24 +1113,19 @@ __device__ void phase_attend(const StepParams& p, uint8_t* smem, uint64_t* bars,
                     }
                     rowidx[stage * kTileRows + lane] = valid ? s : -1;
                 }
-                const uint32_t vmask = __ballot_sync(0xffffffffu, valid);
-                // Rows with nothing to load get a zero V row, so P = 0 never meets stale data.
-                uint32_t none = ~vmask & 0xFFFFu;
-                while (none) {
-                    const int z = __ffs(none) - 1;
-                    none &= none - 1;
-                    uint4* v = reinterpret_cast<uint4*>(dst + (kTileRows + z) * kGPitch);
-                    if (lane < 16) v[lane] = make_uint4(0u, 0u, 0u, 0u);
+                // Row i: lanes 0-15 copy its K_g piece, lanes 16-31 its V_g piece, 16 bytes each.
+                // A row with nothing to load is zero-filled (no read), so P = 0 never meets
+                // stale data.
+                const int half = lane >> 4, c16 = lane & 15;
+#pragma unroll 4
+                for (int i = 0; i < kTileRows; ++i) {
+                    const int si = __shfl_sync(0xffffffffu, valid ? s : -1, i);
+                    const uint16_t* src = si >= 0 ? p.kv + (int64_t)si * p.kv_ld + half * kG * kD + g * kD + c16 * 8 : p.kv;
+                    cp_async16(dst + (half * kTileRows + i) * kGPitch + c16 * 16, src, si >= 0 ? 16u : 0u);
                 }
-                fence_proxy_async_smem();
+                cp_async_mbar_arrive(&full[stage]);
                 __syncwarp();
-                if (lane == 0) mbar_arrive_expect_tx(&full[stage], __popc(vmask) * 2 * kD * 2);
-                __syncwarp();
-                if (valid) {
-                    const uint16_t* rowp = p.kv + (int64_t)s * p.kv_ld + g * kD;
-                    bulk_g2s(dst + lane * kGPitch, rowp, kD * 2, &full[stage]);
-                    bulk_g2s(dst + (kTileRows + lane) * kGPitch, rowp + kG * kD, kD * 2, &full[stage]);
-                }
+                if (lane == 0) mbar_arrive(&full[stage]);   // the row indices above are written
             }
         } else if (warp < kConsumers) {
             uint32_t qa[8][4];
@@ -1180,9 +1216,7 @@ __device__ void phase_attend(const StepParams& p, uint8_t* smem, uint64_t* bars,
         }
         if (__syncthreads_or(failed)) {
             // A bounded wait ran out: let the copies in flight land; the partial is empty.
-            if (tid == kProducer * 32)
-                for (int k = max(0, ntile - kAttStagesG); k < ntile; ++k)
-                    mbar_wait(&full[(phase_base + k) % kAttStagesG], ((phase_base + k) / kAttStagesG) & 1, p.err);
+            if (warp == kProducer) asm volatile("cp.async.wait_all;" ::: "memory");
             __syncthreads();
             m0 = m1 = -INFINITY;
             l0 = l1 = 0.f;
