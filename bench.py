@@ -214,12 +214,22 @@ def swa_bytes(w, window):
     return {"step": uniq * 2048 + w.T * 2 * 64 * 128 * 2, "unique_rows": uniq, "gathered_rows": gathered}
 
 
+def index_bytes(w):
+    """The indexer stage alone: the key cache up to the furthest visible
+    position, the per-query indexer inputs, and the fp32 scores it writes."""
+    n_max = int(w.pos.max()) + 1
+    step = n_max * KEY_BYTES[w.key_dtype] + w.T * (16 * 64 * 2 + 16 * 4) + w.T * w.L * 4
+    return {"step": step, "unique_rows": 0, "gathered_rows": 0}
+
+
 def oracle_step(w, op, window):
     """One step of the oracle (test infrastructure) for this workload and op."""
     import oracle
 
     if op == "swa":
         return oracle.swa_decode(w.q, w.kv, w.pos, window), oracle.window_select(w.pos, window)
+    if op == "index":
+        return oracle.index_scores(w.q_idx, w.w_idx, w.k_idx, w.k_scale, w.pos), None
     return oracle.decode(w.q, w.q_idx, w.w_idx, w.k_idx, w.k_scale, w.kv, w.pos, w.topk)
 
 
@@ -303,7 +313,8 @@ def run_reference(args, w, rank, world):
         t0 = time.perf_counter()
         _, sel = oracle_step(w, args.op, args.window)
         times.append(time.perf_counter() - t0)
-    ab = swa_bytes(w, args.window) if args.op == "swa" else algorithmic_bytes(w, sel)
+    ab = (swa_bytes(w, args.window) if args.op == "swa" else index_bytes(w) if args.op == "index"
+          else algorithmic_bytes(w, sel))
     t = statistics.mean(times)
     value = ab["step"] / t / 1e9
     line = {
@@ -330,8 +341,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end leg (profiling runs)")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
-    ap.add_argument("--op", choices=["step", "swa"], default="step",
-                    help="step: the DSA decode/verify step; swa: sliding-window decode on the same q / K/V")
+    ap.add_argument("--op", choices=["step", "swa", "index"], default="step",
+                    help="step: the DSA decode/verify step; swa: sliding-window decode on the same q / K/V; "
+                         "index: the indexer stage alone (dsa_index_scores)")
     ap.add_argument("--window", type=int, default=128, help="window of --op swa")
     ap.add_argument("--no-bypass", action="store_true", help="score and select even when every query sees <= topk")
     ap.add_argument("--pos", choices=["host", "device"], default="host",
@@ -351,8 +363,9 @@ def main():
     dsa.dsa_set_short_context_bypass(not args.no_bypass)
     rank, world, local = dist_setup(args.gpus)
     dev = torch.device("cuda", torch.cuda.current_device())
-    d = dsa.to_device(w, device=dev)
+    d = dsa.to_device(w, device=dev, with_kv=args.op != "index")
     T, L, topk = w.T, w.L, w.topk
+    scores = torch.empty((T, (L + 3) // 4 * 4), dtype=torch.float32, device=dev) if args.op == "index" else None
     ws = dsa.workspace(T, L, topk, device=dev)
     out = torch.empty((T, 64, 128), dtype=torch.bfloat16, device=dev)
     sel = torch.empty((T, topk), dtype=torch.int32, device=dev)
@@ -373,7 +386,9 @@ def main():
     pos_dev = torch.tensor(w.pos, dtype=torch.int32, device=dev)
 
     def step():
-        if args.op == "swa":
+        if args.op == "index":
+            dsa.dsa_index_scores(d["q_idx"], d["w_idx"], d["k_idx"], w.pos, scores, k_scale=d["k_scale"])
+        elif args.op == "swa":
             dsa.dsa_swa_decode(d["q"], d["kv"], w.pos, args.window, out, ws)
         elif args.pos == "device":
             dsa.dsa_decode_devpos_ws(d["q"], d["q_idx"], d["w_idx"], d["k_idx"], d["kv"], pos_dev, topk, out, sel, ws,
@@ -446,7 +461,8 @@ def main():
     ms = reduce_max(statistics.mean(totals), world)
     phase_us = {k: round(v / args.steps, 2) for k, v in phase_sum.items()}
 
-    ab = swa_bytes(w, args.window) if args.op == "swa" else algorithmic_bytes(w, sel.cpu().numpy())
+    ab = (swa_bytes(w, args.window) if args.op == "swa" else index_bytes(w) if args.op == "index"
+          else algorithmic_bytes(w, sel.cpu().numpy()))
     value = whole_job_gbs(ab["step"], ms, world)
 
     # End to end through the public API, as a serving loop would run it: one CUDA
@@ -455,7 +471,7 @@ def main():
     # device memory (dsa_decode_devpos_ws; dsa_swa_decode for --op swa), and the
     # device->host copies of the outputs.  The caches stay resident.
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and args.op != "index":
         h_in = {k: d[k].cpu().pin_memory() for k in (("q",) if args.op == "swa" else ("q", "q_idx", "w_idx"))}
         dev_in = {k: torch.empty_like(d[k]) for k in h_in}
         h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
@@ -515,13 +531,15 @@ def main():
     peak, which = peaks()
     achieved = ab["step"] / (ms * 1e-3) / 1e9
     roof = {"kernel": "step_kernel", "bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-            "frac": round(achieved / peak, 4), "peak_source": which, "traffic": profiled_traffic(w.name) if args.op == "step" and args.pos == "host" else None,
+            "frac": round(achieved / peak, 4), "peak_source": which,
+            "traffic": profiled_traffic(w.name if args.op == "step" else f"{w.name}:{args.op}") if args.pos == "host" else None,
             "algorithmic_bytes": ab["step"]}
 
     # The indexer's tensor-core rate (tcgen05.mma), over its in-kernel phase time.
     tensor = None
-    bypassed = (not args.no_bypass and args.pos == "host") and int(w.pos.max()) + 1 <= topk   # no indexer phase then
-    if args.op == "step" and not bypassed and phase_us.get("indexer", 0) > 0:
+    bypassed = (args.op == "step" and not args.no_bypass and args.pos == "host"
+                and int(w.pos.max()) + 1 <= topk)   # no indexer phase then
+    if args.op in ("step", "index") and not bypassed and phase_us.get("indexer", 0) > 0:
         tpk, tsrc = bf16_peak()
         tf = indexer_flops(w) / (phase_us["indexer"] * 1e-6) / 1e12
         tensor = {"phase": "indexer", "flops_per_step": indexer_flops(w), "phase_us": phase_us["indexer"],
@@ -537,6 +555,7 @@ def main():
                 "parallelism": f"replicas{world}",
                 "l2": "flushed before every step (write 2x L2, then read another 2x L2: cold and clean)",
                 "timing": "CUDA-graph replay of " + ("dsa_swa_decode" if args.op == "swa" else
+                                                       "dsa_index_scores" if args.op == "index" else
                                                        "dsa_decode_devpos_ws" if args.pos == "device" else
                                                        "dsa_decode_ws") + ", CUDA events per step, mean",
                 "algorithmic_bytes_per_step": ab["step"], "unique_kv_rows": ab["unique_rows"],
@@ -549,7 +568,7 @@ def main():
         "gpu_launches": int(kernels_per_step * args.steps),
         "clocks": clk,
     }
-    if rank == 0 and not args.no_cpu_baseline:
+    if rank == 0 and not args.no_cpu_baseline and args.op != "index":
         cb = cpu_baseline(w, args.cpu_budget, args.op, args.window)
         w1 = cb["one_thread_workload"]
         ab1 = swa_bytes(w1, args.window) if args.op == "swa" else algorithmic_bytes(w1, cb["one_thread_sel"])

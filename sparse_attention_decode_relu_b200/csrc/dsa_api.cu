@@ -212,8 +212,8 @@ Layout layout(int T, int64_t L, bool with_scores = true, bool with_attn = true)
     l.list = take(sizeof(uint2) * (size_t)T * l.ld);
     if (with_scores) l.scores = take(sizeof(float) * (size_t)T * l.ld);
     if (with_attn) {
-        l.po = take(sizeof(float) * (size_t)kMaxT * kG * kMaxSplitsTG * 16 * kD);
-        l.pml = take(sizeof(float2) * (size_t)kMaxT * kG * kMaxSplitsTG * 16);
+        l.po = take(sizeof(float) * (size_t)kMaxT * kMaxSplitsQ * kH * kD);
+        l.pml = take(sizeof(float2) * (size_t)kMaxT * kMaxSplitsQ * kH);
     }
     l.total = off;
     return l;
@@ -296,13 +296,14 @@ void topk_params(StepParams& p, void* ws, const Layout& l)
     if (p.nchunk < 1) p.nchunk = 1;
 }
 
-// Attention work split: items (query, KV group, row split), about one per
-// block; splits of a multiple of 16 rows, at most kMaxRowsPerSplit rows and
-// kMaxSplitsTG splits per (query, group).
+// Attention work split: items (query, row split), about one per block; splits
+// of a multiple of 16 rows, at least kMinRowsPerSplit (so at most kMaxSplitsQ
+// per query) and at most kMaxRowsPerSplit.
 void attn_params(StepParams& p, void* ws, const Layout& l, int32_t rows)
 {
-    int64_t nsplit = p.grid / (p.T * kG);
-    if (nsplit > kMaxSplitsTG) nsplit = kMaxSplitsTG;
+    int64_t nsplit = p.grid / p.T;
+    const int64_t most = (rows + kMinRowsPerSplit - 1) / kMinRowsPerSplit;
+    if (nsplit > most) nsplit = most;
     if (nsplit < 1) nsplit = 1;
     int64_t rps = round_up((rows + nsplit - 1) / nsplit, 16);
     if (rps > kMaxRowsPerSplit) rps = kMaxRowsPerSplit;

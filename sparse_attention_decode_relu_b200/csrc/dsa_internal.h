@@ -18,7 +18,8 @@ constexpr int kHistBins = 4096;            // first radix level: the top 12 bits
 constexpr int kHistShift = 20;             // key >> kHistShift is the bin
 
 constexpr int kMaxRowsPerSplit = 512;       // selected rows one attention work item gathers
-constexpr int kMaxSplitsTG = 16;            // attention row splits per (query, KV group)
+constexpr int kMaxSplitsQ = 32;             // attention row splits per query
+constexpr int kMinRowsPerSplit = 64;        // (so that topk <= 2048 rows make at most kMaxSplitsQ splits)
 constexpr int kMaxChunksStep = 1024;        // top-k chunks per query (<= grid)
 constexpr int kSegPerChunk = 8;             // candidate sub-segments per chunk (one per warp)
 constexpr int kMaxSeg = kMaxChunksStep * kSegPerChunk;
@@ -31,7 +32,7 @@ constexpr int kTraceSlots = 32;             // phase-boundary stamps per block
 //   64         launch epoch (never reset; selects the histogram buffer)
 //   96 + t     extraction items of query t that are done
 //   128 + t    query t's selection is written
-//   160 + 4t+g attention splits of (query t, KV group g) that are done
+//   160 + t    attention splits of query t that are done
 // then two global histograms [2][kMaxT][kHistBins] u32.  Every word but the
 // epoch is zero again when a launch ends; launch e uses histogram e & 1 and
 // clears histogram (e + 1) & 1 for the next one.  The whole region must be zero
@@ -79,11 +80,11 @@ struct StepParams {
     int64_t kv_ld;
     int32_t rows;            // selected rows per query to read (= topk)
     int32_t rows_per_split;  // multiple of 16, <= kMaxRowsPerSplit
-    int32_t nsplit;          // row splits per (query, KV group), <= kMaxSplitsTG
+    int32_t nsplit;          // row splits per query, <= kMaxSplitsQ
     const float* sink;       // [64] or nullptr
     int32_t window;          // kPhaseSelectPos: positions selected per query (<= topk)
-    float* po;               // [T][4][nsplit][16][128] partial outputs per (query, group, split)
-    float2* pml;             // [T][4][nsplit][16] (max in log2 units, sum)
+    float* po;               // [T][nsplit][64][128] partial outputs per (query, split)
+    float2* pml;             // [T][nsplit][64] (max in log2 units, sum)
     uint16_t* out;           // [T][64][128] bf16
     // control
     unsigned long long* trace;   // [grid][kTraceSlots] globaltimer stamps at phase boundaries, or nullptr

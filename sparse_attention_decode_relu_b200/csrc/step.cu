@@ -17,11 +17,12 @@
 //               flag per query
 //   (or)      : selection by position: the last W visible positions (the
 //               short-context bypass with W = topk, sliding-window decode)
-//   4 attend  : gathered sparse attention per (query, KV group, row split),
-//               each item starting as soon as its query's selection is
-//               flagged: the group's K and V rows by bulk async copy,
-//               tensor-core QK and PV, online softmax; the last split of a
-//               (query, group) to finish merges the splits in a fixed order
+//   4 attend  : gathered sparse attention per (query, row split), each item
+//               starting as soon as its query's selection is flagged: whole
+//               K/V rows by bulk async copy, tensor-core QK and PV, online
+//               softmax; partial (max, sum, output) states to global memory
+//   5 merge   : per (query, head), the splits merged in a fixed order, as soon
+//               as every split of the query is done
 //
 // Stage entry points run a sub-range of the phases.  Every reduction is either
 // integer or in a fixed order, so results are bitwise reproducible.
@@ -140,7 +141,7 @@ __device__ __forceinline__ void barrier_exit(const StepParams& p)
             for (int t = 0; t < kMaxT; ++t) {
                 p.ctrl[kCtrlWordArrive + t] = 0u;
                 p.ctrl[kCtrlWordReady + t] = 0u;
-                for (int g = 0; g < kG; ++g) p.ctrl[kCtrlWordDone + t * kG + g] = 0u;
+                p.ctrl[kCtrlWordDone + t] = 0u;
             }
             p.ctrl[kCtrlWordEpoch] += 1u;
             __threadfence();
@@ -215,6 +216,26 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t& total,
     return before + x - v;
 }
 
+// Exclusive prefix maximum over the block (thread order; 0 for thread 0).
+__device__ __forceinline__ uint32_t block_excl_max(uint32_t v, uint32_t* scratch)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    uint32_t x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x = max(x, y);
+    }
+    if (lane == 31) scratch[warp] = x;
+    __syncthreads();
+    uint32_t before = 0;
+    for (int w = 0; w < warp; ++w) before = max(before, scratch[w]);
+    const uint32_t prev = __shfl_up_sync(0xffffffffu, x, 1);
+    if (lane > 0) before = max(before, prev);
+    __syncthreads();
+    return before;
+}
+
 // In-place exclusive prefix sum of a[0, n) in shared memory (each thread scans
 // a contiguous run); returns the total.
 __device__ uint32_t block_scan_array(uint32_t* a, int n, uint32_t* scratch)
@@ -251,31 +272,58 @@ __device__ __forceinline__ uint32_t bin_top(uint32_t start, int shift, uint32_t 
     return (start > 0xFFFFFFFFu - width) ? hi : min(hi, start + width);
 }
 
-// Bin b of an NB-bin histogram in shared memory holding the need-th largest
-// entry: #(bins > b) < need <= #(bins >= b).  res = {b, #(bins > b), found}.
-template <int NB>
-__device__ void find_from_top(const uint32_t* h, uint32_t need, uint32_t* res, uint32_t* scratch)
+// Bin b of a kHistBins-bin histogram in shared memory holding the need-th
+// largest entry: #(bins > b) < need <= #(bins >= b).  res = {b, #(bins > b),
+// found}.  The bins form 128 chunks of 32; every warp sums its chunks (lane l
+// reads bin 32c + l: no bank conflicts); warp 0 then scans the chunk sums from
+// the top, and the chosen chunk's bins from the top.
+__device__ void find_from_top(const uint32_t* h, uint32_t need, uint32_t* res)
 {
-    constexpr int PER = NB / kThreads;
-    const int top = NB - PER * threadIdx.x;   // thread 0 owns the highest bins
-    uint32_t cnt[PER];
-    uint32_t sum = 0;
-#pragma unroll
-    for (int i = 0; i < PER; ++i) {
-        cnt[i] = h[top - 1 - i];
-        sum += cnt[i];
+    constexpr int kChunks = kHistBins / 32;
+    __shared__ uint32_t csum[kChunks];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    for (int c = warp; c < kChunks; c += kWarps) {
+        const uint32_t v = __reduce_add_sync(0xffffffffu, h[c * 32 + lane]);
+        if (lane == 0) csum[c] = v;
     }
-    if (threadIdx.x == 0) res[2] = 0;
-    uint32_t total;
-    uint32_t run = block_excl_scan(sum, total, scratch);
+    __syncthreads();
+    if (warp == 0) {
+        // lane l takes chunks 127 - 4l .. 124 - 4l, i.e. from the top
+        uint32_t cs[4], sum = 0;
 #pragma unroll
-    for (int i = 0; i < PER; ++i) {
-        if (run < need && run + cnt[i] >= need) {
-            res[0] = static_cast<uint32_t>(top - 1 - i);
-            res[1] = run;
-            res[2] = 1;
+        for (int j = 0; j < 4; ++j) {
+            cs[j] = csum[kChunks - 1 - 4 * lane - j];
+            sum += cs[j];
         }
-        run += cnt[i];
+        const uint32_t incl = warp_incl_scan(sum);
+        uint32_t run = incl - sum;
+        int chunk = -1;
+        uint32_t before = 0;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            if (run < need && run + cs[j] >= need) {
+                chunk = kChunks - 1 - 4 * lane - j;
+                before = run;
+            }
+            run += cs[j];
+        }
+        const uint32_t who = __ballot_sync(0xffffffffu, chunk >= 0);
+        if (who) {
+            const int src = __ffs(who) - 1;
+            chunk = __shfl_sync(0xffffffffu, chunk, src);
+            before = __shfl_sync(0xffffffffu, before, src);
+            const int bin = chunk * 32 + 31 - lane;   // lane l: the chunk's bins from the top
+            const uint32_t v = h[bin];
+            const uint32_t vi = warp_incl_scan(v);
+            const uint32_t ex = before + vi - v;
+            if (ex < need && ex + v >= need) {
+                res[0] = static_cast<uint32_t>(bin);
+                res[1] = ex;
+                res[2] = 1;
+            }
+        } else if (lane == 0) {
+            res[2] = 0;
+        }
     }
     __syncthreads();
 }
@@ -297,7 +345,7 @@ __device__ void radix_pass(ForEach for_each_key, uint32_t& lo, uint32_t& hi, uin
         if (k >= l0 && k <= h0) atomicAdd(&h[(k - l0) >> shift], 1u);
     });
     __syncthreads();
-    find_from_top<kHistBins>(h, need, res, scratch);
+    find_from_top(h, need, res);
     if (!res[2]) {
         if (threadIdx.x == 0) atomicOr(err, ERR_TOPK_STATE);
         res[0] = 0;
@@ -311,21 +359,22 @@ __device__ void radix_pass(ForEach for_each_key, uint32_t& lo, uint32_t& hi, uin
 }
 
 // ==================================================================================
-// Phase 1: indexer scan on the fifth-generation tensor cores, warp-specialised.
-// A tile of 128 keys is the M side of tcgen05.mma kind::f16 (bf16 operands,
-// fp32 accumulators in tensor memory), the T x 16 indexer query heads the N
-// side (16..128), the 64 dims K (four K = 16 steps).  Roles:
-//   warps 0-3  FP8 keys: widen the E4M3 tile (TMA, 64-byte swizzle) row by row
-//              (one key per thread) into bf16 and store it into a tensor-memory
-//              A buffer; bf16 keys arrive from TMA already as the shared-memory
-//              A operand (128-byte swizzle).  Warp 0's lane 0 issues the TMA
-//              loads, warp 1's lane 0 the MMAs.
-//   warps 4-7  epilogue: each thread owns one key (a TMEM lane): ReLU, head
-//              weights, a fixed-order sum over the 16 heads, the per-token
-//              scale; the fp32 score goes to global memory and its key to the
-//              block's per-query histogram (16-bit counters in shared memory).
+// Phase 1: indexer scan on the fifth-generation tensor cores.  A tile of 128
+// keys is the M side of tcgen05.mma kind::f16 (bf16 operands, fp32 accumulators
+// in tensor memory), the T x 16 indexer query heads the N side (16..128), the 64
+// dims K (four K = 16 steps).  The eight warps are alike: warps w and w + 4 own
+// the same 32 key rows (TMEM lanes), and per tile each
+//   - (FP8 keys) widens its half of every row's 64 E4M3 codes (TMA tile with a
+//     64-byte swizzle) exactly into bf16, straight into 16 columns of the
+//     tile's tensor-memory A buffer (bf16 keys arrive from TMA already as the
+//     shared-memory A operand, 128-byte swizzle);
+//   - runs the epilogue of the previous tile for its half of the queries: ReLU,
+//     head weights, a fixed-order sum over the 16 heads, the per-token scale;
+//     the fp32 score goes to global memory and its key's top bits to the
+//     block's per-query histogram (16-bit counters in shared memory).
+// Warp 0's lane 0 also refills the TMA ring, warp 1's lane 0 issues the MMAs.
 // Tensor memory: three accumulator buffers of 128 columns and four A buffers of
-// 32 columns, all 512 columns.  mbarriers chain the roles; nothing waits on a
+// 32 columns, all 512 columns.  mbarriers chain the steps; nothing waits on a
 // block-wide barrier inside the loop.
 // ==================================================================================
 constexpr int kRawStagesF8 = 8, kRawStagesBf = 6;
@@ -365,7 +414,7 @@ __device__ void phase_index(const CUtensorMap& kmap, const StepParams& p, uint8_
     uint8_t* qsw = smem + S * raw_bytes;                                // [128 rows][128 B] queries (B operand)
     float* w_s = reinterpret_cast<float*>(qsw + kTileBytesBf16);        // [8][16]
     uint32_t* hs = reinterpret_cast<uint32_t*>(w_s + kMaxT * kHI);      // [8][2048]: two 16-bit counters per word
-    uint32_t* hstage = hs + kHistWords / 2;                             // [4 warps][32 keys][8 queries] bins
+    uint32_t* hstage = hs + kHistWords / 2;                             // [8 warps][32 keys][4 queries] bins
     uint64_t* raw_full = bars + kBarRawFull;
     uint64_t* raw_empty = bars + kBarRawEmpty;
     uint64_t* a_full = bars + kBarAFull;
@@ -375,7 +424,10 @@ __device__ void phase_index(const CUtensorMap& kmap, const StepParams& p, uint8_
     uint64_t* setup = bars + kBarSetup;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quad = warp & 3, half = warp >> 2;     // TMEM lane quarter; which half of the row / queries
     const int T = p.T;
+    const int Th = (T + 1) >> 1;                     // queries per half
+    const int qa = min(T, half * Th), qb = min(T, qa + Th);   // this warp's queries [qa, qb)
     const int ntiles = (visible_max(p) + kKeyTile - 1) / kKeyTile;
     const int nloc = ntiles > static_cast<int>(blockIdx.x) ? (ntiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
     const bool hist = g_view.hist != nullptr;
@@ -387,20 +439,20 @@ __device__ void phase_index(const CUtensorMap& kmap, const StepParams& p, uint8_
         tma_load_2d_hint(ring + stage * raw_bytes, &kmap, 0, tile_of(it) * kKeyTile, &raw_full[stage], stream_policy);
     };
 
-    int issued = 0;   // (warp 0 lane 0) key tiles requested
+    int issued = 0;   // (thread 0) key tiles requested
     if (tid == 0) {
         prefetch_tmap(&kmap);
         for (int s = 0; s < S; ++s) {
             mbar_init(&raw_full[s], 1);
-            mbar_init(&raw_empty[s], FP8 ? 4 : 1);   // four converter warps, or the MMA commit
+            mbar_init(&raw_empty[s], FP8 ? kWarps : 1);   // every warp's half rows read, or the MMA commit
         }
         for (int b = 0; b < kABufs; ++b) {
-            mbar_init(&a_full[b], 4);
+            mbar_init(&a_full[b], kWarps);
             mbar_init(&a_empty[b], 1);
         }
         for (int b = 0; b < kAccBufs; ++b) {
             mbar_init(&acc_full[b], 1);
-            mbar_init(&acc_empty[b], 4);
+            mbar_init(&acc_empty[b], kWarps);
         }
         mbar_init(setup, 1);
         fence_mbar_init();
@@ -433,13 +485,16 @@ __device__ void phase_index(const CUtensorMap& kmap, const StepParams& p, uint8_
     const uint32_t tmem = *tmem_slot;
     const uint32_t idesc = umma_idesc_bf16(kKeyTile, T * kHI);
     const uint64_t bdesc = umma_desc_sw128(smem_u32(qsw));
-    const int quad = warp & 3;                       // TMEM lane quarter of this warp
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
-    bool aborted = false;
+    const int row = quad * 32 + lane;                // this thread's key row of every tile
     int mma_issued = 0;                              // (warp 1 lane 0)
+    bool aborted = __any_sync(0xffffffffu, !mbar_wait(setup, 0, p.err));   // warp-uniform from here on
+    int pos_q[4];                                    // positions of this warp's queries
+#pragma unroll
+    for (int u = 0; u < 4; ++u) pos_q[u] = qa + u < qb ? query_pos_rt(p, qa + u) : -1;
 
     // MMAs of local tile it into accumulator buffer it % 3 (one thread).
-    auto issue_mma = [&](int it, uint32_t a_src) -> bool {
+    auto issue_mma = [&](int it) -> bool {
         const int ab = it % kABufs, cb = it % kAccBufs;
         if constexpr (FP8) {
             if (!mbar_wait(&a_full[ab], (it / kABufs) & 1, p.err)) return false;
@@ -450,12 +505,12 @@ __device__ void phase_index(const CUtensorMap& kmap, const StepParams& p, uint8_
         tc_fence_after();
         const uint32_t d = tmem + cb * 128;
         if constexpr (FP8) {
+            const uint32_t a = tmem + kACol + ab * 32;
 #pragma unroll
-            for (int k = 0; k < kDI / 16; ++k)
-                tc_mma_bf16_tmem_a(d, a_src + k * 8, bdesc + 2 * k, idesc, k > 0 ? 1u : 0u);
+            for (int k = 0; k < kDI / 16; ++k) tc_mma_bf16_tmem_a(d, a + k * 8, bdesc + 2 * k, idesc, k > 0 ? 1u : 0u);
             tc_commit(&a_empty[ab]);
         } else {
-            const uint64_t adesc = umma_desc_sw128(a_src);
+            const uint64_t adesc = umma_desc_sw128(smem_u32(ring + (it % S) * raw_bytes));
 #pragma unroll
             for (int k = 0; k < kDI / 16; ++k) tc_mma_bf16(d, adesc + 2 * k, bdesc + 2 * k, idesc, k > 0 ? 1u : 0u);
             tc_commit(&raw_empty[it % S]);
@@ -465,177 +520,137 @@ __device__ void phase_index(const CUtensorMap& kmap, const StepParams& p, uint8_
         return true;
     };
 
-    if (warp < 4) {
-        if constexpr (FP8) {
-            // ---- converters (one key row per thread), producer and MMA lanes ----
-            const int row = quad * 32 + lane;
-            for (int it = 0; it < nloc; ++it) {
-                const int stage = it % S, ab = it % kABufs;
-                bool ok = it < kABufs || mbar_wait(&a_empty[ab], ((it / kABufs) - 1) & 1, p.err);
-                ok = ok && mbar_wait(&raw_full[stage], (it / S) & 1, p.err);
-                if (__any_sync(0xffffffffu, !ok)) {
-                    aborted = true;
-                    break;
-                }
-                // Row `row` of the tile: 64 codes, 16-byte chunk c stored at chunk c ^ ((row >> 1) & 3).
-                const uint8_t* src = ring + stage * raw_bytes + row * 64;
-                uint4 v[4];
+    // FP8: this warp's half of key row `row` (32 codes, two 16-byte chunks stored at
+    // chunk c ^ ((row >> 1) & 3)) widened into 16 columns of the tile's A buffer.
+    auto convert = [&](int it) -> bool {
+        const int stage = it % S, ab = it % kABufs;
+        bool ok = it < kABufs || mbar_wait(&a_empty[ab], ((it / kABufs) - 1) & 1, p.err);
+        ok = ok && mbar_wait(&raw_full[stage], (it / S) & 1, p.err);
+        if (__any_sync(0xffffffffu, !ok)) return false;
+        const uint8_t* src = ring + stage * raw_bytes + row * 64;
+        uint4 v[2];
 #pragma unroll
-                for (int c = 0; c < 4; ++c)
-                    v[c] = *reinterpret_cast<const uint4*>(src + ((c ^ ((row >> 1) & 3)) << 4));
-                uint32_t r[32];
+        for (int c = 0; c < 2; ++c)
+            v[c] = *reinterpret_cast<const uint4*>(src + (((2 * half + c) ^ ((row >> 1) & 3)) << 4));
+        uint32_t r[16];
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    e4m3x4_to_bf16x4(v[c].x, r[8 * c + 0], r[8 * c + 1]);
-                    e4m3x4_to_bf16x4(v[c].y, r[8 * c + 2], r[8 * c + 3]);
-                    e4m3x4_to_bf16x4(v[c].z, r[8 * c + 4], r[8 * c + 5]);
-                    e4m3x4_to_bf16x4(v[c].w, r[8 * c + 6], r[8 * c + 7]);
+        for (int c = 0; c < 2; ++c) {
+            e4m3x4_to_bf16x4(v[c].x, r[8 * c + 0], r[8 * c + 1]);
+            e4m3x4_to_bf16x4(v[c].y, r[8 * c + 2], r[8 * c + 3]);
+            e4m3x4_to_bf16x4(v[c].z, r[8 * c + 4], r[8 * c + 5]);
+            e4m3x4_to_bf16x4(v[c].w, r[8 * c + 6], r[8 * c + 7]);
+        }
+        tmem_st16(tmem + lane_base + kACol + ab * 32 + half * 16, r);
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+            mbar_arrive(&a_full[ab]);
+            mbar_arrive(&raw_empty[stage]);
+        }
+        return true;
+    };
+
+    // Epilogue of local tile e for this warp's queries: ReLU, head weights, a
+    // fixed-order head sum, the per-token scale; scores to global memory, keys'
+    // top bits counted in the block's histogram.
+    auto epilogue = [&](int e) -> bool {
+        const int cb = e % kAccBufs;
+        const int s = tile_of(e) * kKeyTile + row;
+        const float scale = (p.scale != nullptr && s < p.L) ? __ldg(p.scale + s) : 1.0f;
+        if (__any_sync(0xffffffffu, !mbar_wait(&acc_full[cb], (e / kAccBufs) & 1, p.err))) return false;
+        tc_fence_after();
+        uint32_t r[2][32];
+        if (qa < qb) {
+            const uint32_t tbase = tmem + lane_base + cb * 128 + qa * kHI;
+            tmem_ld32_nowait(tbase, r[0]);
+            if (qb - qa > 2) tmem_ld32_nowait(tbase + 32, r[1]);
+            tmem_ld_wait();
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[cb]);   // this warp is done with the buffer
+        uint32_t bins[4] = {~0u, ~0u, ~0u, ~0u};    // histogram bin of each query's score (~0u: none)
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int t = qa + u;
+            if (t < qb) {
+                // Four partial sums over heads {j, j+4, j+8, j+12}, j < 4, as two packed
+                // fp32 FMAs per four heads, combined in a fixed order.
+                const float4* w4 = reinterpret_cast<const float4*>(w_s + t * kHI);
+                const float* v = reinterpret_cast<const float*>(&r[u >> 1][(u & 1) * 16]);
+                float2 p01 = make_float2(0.f, 0.f), p23 = make_float2(0.f, 0.f);
+#pragma unroll
+                for (int g4 = 0; g4 < 4; ++g4) {
+                    const float4 w = w4[g4];
+                    p01 = __ffma2_rn(make_float2(fmaxf(v[g4 * 4 + 0], 0.f), fmaxf(v[g4 * 4 + 1], 0.f)),
+                                     make_float2(w.x, w.y), p01);
+                    p23 = __ffma2_rn(make_float2(fmaxf(v[g4 * 4 + 2], 0.f), fmaxf(v[g4 * 4 + 3], 0.f)),
+                                     make_float2(w.z, w.w), p23);
                 }
-                tmem_st32(tmem + lane_base + kACol + ab * 32, r);
-                tmem_st_wait();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive(&a_full[ab]);
-                    mbar_arrive(&raw_empty[stage]);
-                }
-                bool bad = false;
-                if (warp == 0 && lane == 0 && issued < nloc) {
-                    // the stage is free once all four converter warps have read it
-                    if (mbar_wait(&raw_empty[stage], (it / S) & 1, p.err)) {
-                        load_tile(issued);
-                        ++issued;
-                    } else {
-                        bad = true;
-                    }
-                }
-                if (warp == 1 && lane == 0 && !issue_mma(it, tmem + kACol + ab * 32)) bad = true;
-                if (__any_sync(0xffffffffu, bad)) {
-                    aborted = true;
-                    break;
+                const float acc = ((p01.x + p01.y) + (p23.x + p23.y)) * scale;
+                if (s < p.L) {
+                    const bool vis = s <= pos_q[u];
+                    p.scores[(int64_t)t * p.ld + s] = vis ? acc : -INFINITY;
+                    if (vis) bins[u] = score_key(acc) >> kHistShift;
                 }
             }
-        } else {
-            // ---- bf16 keys: a producer lane and an MMA lane ----
-            if (warp == 0 && lane == 0) {
-                for (; issued < nloc; ++issued) {
-                    if (!mbar_wait(&raw_empty[issued % S], ((issued / S) - 1) & 1, p.err)) {
-                        aborted = true;
-                        break;
-                    }
+        }
+        if (hist && qa < qb) {
+            // The bins through a transpose in shared memory: in round i lane l adds key
+            // (8i + l/4)'s bin of query qa + l % 4, so one atomic instruction spreads over
+            // four query histograms.
+            uint32_t* st = hstage + warp * 32 * 4;
+            *reinterpret_cast<uint4*>(st + lane * 4) = make_uint4(bins[0], bins[1], bins[2], bins[3]);
+            __syncwarp();
+            uint32_t* hq = hs + (qa + (lane & 3)) * (kHistBins / 2);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const uint32_t bin = st[i * 32 + lane];
+                if (bin != ~0u) atomicAdd(&hq[bin >> 1], 1u << ((bin & 1) << 4));
+            }
+            __syncwarp();
+        }
+        if (hist && (e + 1) % kHistFlushTiles == 0) {
+            // 16-bit counters: this warp moves its eighth of them to the global histogram
+            // (atomic exchange, so concurrent increments are kept) well before any can
+            // overflow: the warps are at most a tile or two apart, so between two flushes
+            // of a word it takes at most (kHistFlushTiles + kAccBufs) * 128 < 65536 counts.
+            const int words = T * (kHistBins / 2), w0 = warp * words / kWarps, w1 = (warp + 1) * words / kWarps;
+            for (int i = w0 + lane; i < w1; i += 32) {
+                const uint32_t v = atomicExch(&hs[i], 0u);
+                if (v) {
+                    uint32_t* gh = g_view.hist + (i / (kHistBins / 2)) * kHistBins + 2 * (i % (kHistBins / 2));
+                    if (v & 0xFFFFu) atomicAdd(gh, v & 0xFFFFu);
+                    if (v >> 16) atomicAdd(gh + 1, v >> 16);
+                }
+            }
+        }
+        return true;
+    };
+
+    // Every warp: widen tile it (FP8), then the epilogue of tile it - 1.  Warp 0's
+    // lane 0 refills the ring one tile behind; warp 1's lane 0 issues tile it's MMAs.
+    for (int it = 0; it <= nloc && !aborted; ++it) {
+        if (it < nloc) {
+            bool bad = false;
+            if constexpr (FP8) bad = !convert(it);
+            if (!bad && warp == 0 && lane == 0 && it >= 1 && issued < nloc) {
+                const int prev = it - 1;   // its stage is free once it has been read (FP8) or its MMAs are done
+                if (mbar_wait(&raw_empty[prev % S], (prev / S) & 1, p.err)) {
                     load_tile(issued);
+                    ++issued;
+                } else {
+                    bad = true;
                 }
-            } else if (warp == 1 && lane == 0) {
-                for (int it = 0; it < nloc; ++it)
-                    if (!issue_mma(it, smem_u32(ring + (it % S) * raw_bytes))) {
-                        aborted = true;
-                        break;
-                    }
             }
-        }
-    } else {
-        // ---- epilogue: key row `row`, every query of the launch ----
-        const int row = quad * 32 + lane;
-        aborted = !mbar_wait(setup, 0, p.err);
-        int pos_q[kMaxT];
-#pragma unroll
-        for (int k = 0; k < kMaxT; ++k) pos_q[k] = k < T ? query_pos(p, k) : -1;
-        const bool scaled = p.scale != nullptr;
-        float scale_next = 1.0f;
-        if (scaled && nloc > 0) {
-            const int s = tile_of(0) * kKeyTile + row;
-            scale_next = s < p.L ? __ldg(p.scale + s) : 1.0f;
-        }
-        for (int e = 0; e < nloc && !aborted; ++e) {
-            const int cb = e % kAccBufs;
-            const int s = tile_of(e) * kKeyTile + row;
-            const float scale = scale_next;
-            if (scaled && e + 1 < nloc) {   // next tile's scale, in flight during this tile
-                const int s2 = tile_of(e + 1) * kKeyTile + row;
-                scale_next = s2 < p.L ? __ldg(p.scale + s2) : 1.0f;
-            }
-            if (__any_sync(0xffffffffu, !mbar_wait(&acc_full[cb], (e / kAccBufs) & 1, p.err))) {
+            if (!bad && warp == 1 && lane == 0 && !issue_mma(it)) bad = true;
+            if (__any_sync(0xffffffffu, bad)) {
                 aborted = true;
                 break;
             }
-            tc_fence_after();
-            const uint32_t tbase = tmem + lane_base + cb * 128;
-            uint32_t bins[kMaxT];   // histogram bin of each query's score (~0u: not counted)
-#pragma unroll
-            for (int k = 0; k < kMaxT; ++k) bins[k] = ~0u;
-            // Queries in groups of four: two 32-column loads in flight, one wait.
-#pragma unroll
-            for (int g = 0; g < kMaxT / 4; ++g) {
-                if (g * 4 < T) {
-                    uint32_t r[2][32];
-                    tmem_ld32_nowait(tbase + g * 64, r[0]);
-                    if (g * 4 + 2 < T) tmem_ld32_nowait(tbase + g * 64 + 32, r[1]);
-                    tmem_ld_wait();
-                    if (g * 4 + 4 >= T) {   // the last load of this buffer is done: release it
-                        tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(&acc_empty[cb]);
-                    }
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const int t = g * 4 + u;
-                        if (t < T) {
-                            // Four partial sums over heads {j, j+4, j+8, j+12}, j < 4, as two packed
-                            // fp32 FMAs per four heads, combined in a fixed order.
-                            const float4* w4 = reinterpret_cast<const float4*>(w_s + t * kHI);
-                            const float* v = reinterpret_cast<const float*>(&r[u >> 1][(u & 1) * 16]);
-                            float2 p01 = make_float2(0.f, 0.f), p23 = make_float2(0.f, 0.f);
-#pragma unroll
-                            for (int g4 = 0; g4 < 4; ++g4) {
-                                const float4 w = w4[g4];
-                                p01 = __ffma2_rn(make_float2(fmaxf(v[g4 * 4 + 0], 0.f), fmaxf(v[g4 * 4 + 1], 0.f)),
-                                                 make_float2(w.x, w.y), p01);
-                                p23 = __ffma2_rn(make_float2(fmaxf(v[g4 * 4 + 2], 0.f), fmaxf(v[g4 * 4 + 3], 0.f)),
-                                                 make_float2(w.z, w.w), p23);
-                            }
-                            const float acc = ((p01.x + p01.y) + (p23.x + p23.y)) * scale;
-                            if (s < p.L) {
-                                const bool vis = s <= pos_q[t];
-                                p.scores[(int64_t)t * p.ld + s] = vis ? acc : -INFINITY;
-                                if (vis) bins[t] = score_key(acc) >> kHistShift;
-                            }
-                        }
-                    }
-                }
-            }
-            if (hist) {
-                // Count the bins through a transpose in shared memory: lane l then adds key
-                // (4i + l/8)'s bin of query l % 8 in round i, so one atomic instruction spreads
-                // over eight query histograms instead of one (far fewer address conflicts).
-                uint32_t* st = hstage + quad * 32 * kMaxT;
-                *reinterpret_cast<uint4*>(st + lane * kMaxT) = make_uint4(bins[0], bins[1], bins[2], bins[3]);
-                *reinterpret_cast<uint4*>(st + lane * kMaxT + 4) = make_uint4(bins[4], bins[5], bins[6], bins[7]);
-                __syncwarp();
-                uint32_t* hq = hs + (lane & (kMaxT - 1)) * (kHistBins / 2);
-#pragma unroll
-                for (int i = 0; i < kMaxT; ++i) {
-                    const uint32_t bin = st[i * 32 + lane];
-                    if (bin != ~0u) atomicAdd(&hq[bin >> 1], 1u << ((bin & 1) << 4));
-                }
-                __syncwarp();
-            }
-            if (hist && (e + 1) % kHistFlushTiles == 0) {
-                // 16-bit counters: this warp moves its quarter of them to the global
-                // histogram (atomic exchange, so concurrent increments are kept)
-                // well before any can overflow.  No barrier: the epilogue warps are
-                // at most kAccBufs tiles apart, so between two flushes of a word it
-                // takes at most (kHistFlushTiles + kAccBufs) * 128 < 65536 counts.
-                const int words = T * (kHistBins / 2), q0 = quad * words / 4, q1 = (quad + 1) * words / 4;
-                for (int i = q0 + lane; i < q1; i += 32) {
-                    const uint32_t v = atomicExch(&hs[i], 0u);
-                    if (v) {
-                        uint32_t* gh = g_view.hist + (i / (kHistBins / 2)) * kHistBins + 2 * (i % (kHistBins / 2));
-                        if (v & 0xFFFFu) atomicAdd(gh, v & 0xFFFFu);
-                        if (v >> 16) atomicAdd(gh + 1, v >> 16);
-                    }
-                }
-            }
         }
+        if (it >= 1 && !epilogue(it - 1)) aborted = true;
     }
     // A wait that ran out (error bit set) ends the loop for that warp; the others
     // run into bounded waits and stop too.  Copies and MMAs still in flight land
@@ -743,7 +758,7 @@ __device__ void phase_extract(const StepParams& p, uint8_t* smem, uint64_t* bars
         fence_mbar_init();
         fence_proxy_async_smem();   // earlier generic writes to the ring region come first
         __syncthreads();
-        find_from_top<kHistBins>(h, static_cast<uint32_t>(p.topk), res, scratch);
+        find_from_top(h, static_cast<uint32_t>(p.topk), res);
         uint32_t cut = 0u;
         if (res[2]) {
             cut = res[0] << kHistShift;
@@ -814,9 +829,12 @@ __device__ void phase_extract(const StepParams& p, uint8_t* smem, uint64_t* bars
 constexpr int kSelHOff = 0;                              // [kHistBins] select bins
 constexpr int kSelOffOff = kHistBins * 4;                // [kMaxSeg] sub-segment offsets
 constexpr int kSelEntOff = kSelOffOff + kMaxSeg * 4;     // candidates (key, position)
-constexpr int kSelCap = (kDataBytes - kSelEntOff) / 8;
+constexpr int kSelCap = (kDataBytes - kSelEntOff) / 10 / 256 * 256;   // with a 16-bit sub-segment index each
+constexpr int kSelSegOff = kSelEntOff + kSelCap * 8;     // [kSelCap] sub-segment of each candidate
 constexpr int kSelGOff = kSelEntOff + kMaxSeg * 4;       // (global path) second per-sub-segment array
-static_assert(kSelCap >= 4096 && kSelGOff + kMaxSeg * 4 <= kDataBytes, "selection buffers fit");
+static_assert(kSelCap >= 4096 && kSelSegOff + kSelCap * 2 <= kDataBytes && kSelGOff + kMaxSeg * 4 <= kDataBytes,
+              "selection buffers fit");
+static_assert(kMaxSeg <= 65536, "sub-segment indices fit 16 bits");
 
 __device__ __forceinline__ int seg_start(const StepParams& p, int i)
 {
@@ -853,9 +871,29 @@ __device__ void phase_select(const StepParams& p, uint8_t* smem, uint32_t* res, 
             uint32_t nsel = 0;
             if (m <= static_cast<uint32_t>(kSelCap)) {
                 // ---- the candidates fit in shared memory ----
-                // Entry j's sub-segment is the last k with off[k] <= j (binary search); eight
-                // independent loads in flight per thread.
+                // Entry j's sub-segment: every non-empty sub-segment writes its index at its
+                // first slot, then a running maximum fills the slots in between.  The loads
+                // are then independent: eight in flight per thread.
                 uint2* ent = reinterpret_cast<uint2*>(smem + kSelEntOff);
+                uint16_t* segof = reinterpret_cast<uint16_t*>(smem + kSelSegOff);
+                for (uint32_t j = tid; j < m; j += kThreads) segof[j] = 0;
+                __syncthreads();
+                for (int k = tid; k < nseg; k += kThreads)
+                    if (seg_cnt(k)) segof[off[k]] = static_cast<uint16_t>(k);
+                __syncthreads();
+                {
+                    const uint32_t per = (m + kThreads - 1) / kThreads;
+                    const uint32_t j0 = min(m, tid * per), j1 = min(m, j0 + per);
+                    uint32_t run = 0;
+                    for (uint32_t j = j0; j < j1; ++j) run = max(run, static_cast<uint32_t>(segof[j]));
+                    const uint32_t before = block_excl_max(run, scratch);
+                    run = before;
+                    for (uint32_t j = j0; j < j1; ++j) {
+                        run = max(run, static_cast<uint32_t>(segof[j]));
+                        segof[j] = static_cast<uint16_t>(run);
+                    }
+                }
+                __syncthreads();
                 for (uint32_t j0 = 0; j0 < m; j0 += 8 * kThreads) {
                     uint2 v[8];
 #pragma unroll
@@ -863,12 +901,8 @@ __device__ void phase_select(const StepParams& p, uint8_t* smem, uint32_t* res, 
                         const uint32_t j = j0 + u * kThreads + tid;
                         v[u] = make_uint2(0u, 0u);
                         if (j < m) {
-                            int a = 0, b = nseg - 1;   // off[a] <= j < off[b + 1]
-                            while (a < b) {
-                                const int mid = (a + b + 1) >> 1;
-                                if (off[mid] <= j) a = mid; else b = mid - 1;
-                            }
-                            v[u] = __ldcg(glist + seg_start(p, a) + (j - off[a]));
+                            const int k = segof[j];
+                            v[u] = __ldcg(glist + seg_start(p, k) + (j - off[k]));
                         }
                     }
 #pragma unroll
@@ -999,40 +1033,29 @@ __device__ void phase_select_pos(const StepParams& p)
 }
 
 // ==================================================================================
-// Phase 4: sparse attention, one work item per (query t, KV group g, row split).
-// When the step selected the rows itself, an item starts as soon as its query's
+// Phase 4: sparse attention, one work item per (query t, row split).  When the
+// step selected the rows itself, an item starts as soon as its query's
 // selection is flagged; with selection by position the rows follow from the
-// query position directly.  Warp 4 gathers the selected rows' K and V of group
-// g (two 256-byte pieces per row, one row per warp instruction of 16-byte
-// asynchronous copies) into a ring of 16-row tiles; consumer warps 0-3 take the
-// tiles in turn: the 16 query heads of the
-// group are the 16 rows of an m16n8k16 tile (QK and PV on the tensor cores,
-// online softmax in the exp2 domain).  The four warps' states are merged in
-// shared memory, in warp order, into the item's partial (max, sum, output),
-// which goes to global memory.  The last item of a (query, group) to finish
-// merges the group's splits in split order (with the sink, if any) and writes
-// the output: no grid barrier.
+// query position directly.  Warp 4 gathers whole 2 KiB token rows (K then V of
+// the 4 groups) by bulk async copy into a 6-stage ring of 16-row tiles; warp
+// g < 4 owns KV group g, i.e. query heads 16g .. 16g+15 -- the 16 rows of an
+// m16n8k16 tile, so nothing is padded.  Online softmax in the exp2 domain; the
+// partial (max, sum, output) of every head goes to global memory and the item
+// raises its query's done counter.
 // ==================================================================================
-constexpr int kAttStagesG = 16;
-constexpr int kGPitch = 272;                       // 256-byte rows padded: conflict-free ldmatrix
-constexpr int kGTileBytes = 2 * kTileRows * kGPitch;   // K rows, then V rows
-constexpr int kGRingBytes = kAttStagesG * kGTileBytes;
-constexpr int kGRowIdxOff = kGRingBytes;                          // [stage][16] row index (-1: none)
-constexpr int kGSelOff = kGRowIdxOff + kAttStagesG * kTileRows * 4;   // [kMaxRowsPerSplit] the item's rows
-constexpr int kGRedOff = kGSelOff + kMaxRowsPerSplit * 4;            // [4 warps][16][128] f32 + [4][16] m, l
-constexpr int kGRedBytes = 4 * kTileRows * kD * 4 + 2 * 4 * kTileRows * 4;
-static_assert(kGRedOff + kGRedBytes <= kDataBytes, "attention buffers fit");
-static_assert(kBarAttEmpty + kAttStagesG <= kBarSlots, "attention mbarriers fit");
+constexpr int kAttStages = 6;
+constexpr int kRowBytes = 2048;
+constexpr int kPitch = 2064;                                     // bank-conflict-free ldmatrix rows
+constexpr int kRowIdxOff = kAttStages * kTileRows * kPitch;      // [stage][16] row index (-1: none)
+constexpr int kSelSOff = kRowIdxOff + kAttStages * kTileRows * 4;   // [kMaxRowsPerSplit] the item's rows
+static_assert(kSelSOff + kMaxRowsPerSplit * 4 <= kDataBytes, "attention buffers fit");
+static_assert(kBarAttEmpty + kAttStages <= kBarSlots, "attention mbarriers fit");
 
 __device__ void phase_attend(const StepParams& p, uint8_t* smem, uint64_t* bars, bool wait_sel, int* ok_s)
 {
     uint8_t* ring = smem;
-    int32_t* rowidx = reinterpret_cast<int32_t*>(smem + kGRowIdxOff);
-    int32_t* sel_s = reinterpret_cast<int32_t*>(smem + kGSelOff);
-    float* red_o = reinterpret_cast<float*>(smem + kGRedOff);       // [4][16][128]
-    float* red_m = red_o + 4 * kTileRows * kD;                        // [4][16]
-    float* red_l = red_m + 4 * kTileRows;                             // [4][16]
-    __shared__ int last_s;
+    int32_t* rowidx = reinterpret_cast<int32_t*>(smem + kRowIdxOff);
+    int32_t* sel_s = reinterpret_cast<int32_t*>(smem + kSelSOff);
     uint64_t* full = bars + kBarAttFull;
     uint64_t* empty = bars + kBarAttEmpty;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -1041,22 +1064,20 @@ __device__ void phase_attend(const StepParams& p, uint8_t* smem, uint64_t* bars,
     const float sm_scale = kLog2e * rsqrtf(static_cast<float>(kD));
     const bool by_pos = (p.phases & kPhaseSelectPos) != 0;
 
-    int phase_base = 0;   // tiles this block has gathered so far (mbarrier phase bookkeeping)
+    int phase_base = 0;   // tiles consumed by this block so far (mbarrier phase bookkeeping)
     if (tid == 0) {
-        for (int s = 0; s < kAttStagesG; ++s) {
-            mbar_init(&full[s], 33);   // the producer's 32 lanes' copies landed + its row indices written
-            mbar_init(&empty[s], 1);
+        for (int s = 0; s < kAttStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], kConsumers);
         }
         fence_mbar_init();
     }
     __syncthreads();
 
-    const int items = p.T * kG * p.nsplit;
-    bool merged_any = false;
     for (int r = 0;; ++r) {
         const int i = item_of(r);
-        if (i >= items) break;
-        const int t = i / (kG * p.nsplit), g = (i / p.nsplit) % kG, split = i % p.nsplit;
+        if (i >= p.T * p.nsplit) break;
+        const int t = i / p.nsplit, split = i % p.nsplit;
         const int pos_t = query_pos_rt(p, t);
         bool sel_ok = true;
         if (wait_sel) {   // the query's selection is written (phase 3 flags it)
@@ -1077,7 +1098,7 @@ __device__ void phase_attend(const StepParams& p, uint8_t* smem, uint64_t* bars,
         for (int k = 0; k < 16; ++k) oacc[k][0] = oacc[k][1] = oacc[k][2] = oacc[k][3] = 0.f;
 
         if (warp == kProducer) {
-            // the item's rows: validated, then gathered K_g and V_g piece by piece
+            // producer: the item's rows, validated, then gathered whole
             if (by_pos) {
                 const int cnt = min(pos_t + 1, p.window);   // row j of the window: pos_t + 1 - cnt + j
                 for (int j = lane; j < r1 - r0; j += 32) sel_s[j] = pos_t + 1 - cnt + r0 + j;
@@ -1096,12 +1117,12 @@ __device__ void phase_attend(const StepParams& p, uint8_t* smem, uint64_t* bars,
             __syncwarp();
             for (int k = 0; k < ntile; ++k) {
                 const int kk = phase_base + k;
-                const int stage = kk % kAttStagesG;
-                if (kk >= kAttStagesG && !mbar_wait(&empty[stage], ((kk / kAttStagesG) - 1) & 1, p.err)) {
+                const int stage = kk % kAttStages;
+                if (kk >= kAttStages && !mbar_wait(&empty[stage], ((kk / kAttStages) - 1) & 1, p.err)) {
                     failed = true;
                     break;
                 }
-                uint8_t* dst = ring + stage * kGTileBytes;
+                uint8_t* dst = ring + stage * kTileRows * kPitch;
                 int s = -1;
                 bool valid = false;
                 if (lane < kTileRows) {
@@ -1113,23 +1134,26 @@ __device__ void phase_attend(const StepParams& p, uint8_t* smem, uint64_t* bars,
                     }
                     rowidx[stage * kTileRows + lane] = valid ? s : -1;
                 }
-                // Row i: lanes 0-15 copy its K_g piece, lanes 16-31 its V_g piece, 16 bytes each.
-                // A row with nothing to load is zero-filled (no read), so P = 0 never meets
-                // stale data.
-                const int half = lane >> 4, c16 = lane & 15;
-#pragma unroll 4
-                for (int i = 0; i < kTileRows; ++i) {
-                    const int si = __shfl_sync(0xffffffffu, valid ? s : -1, i);
-                    const uint16_t* src = si >= 0 ? p.kv + (int64_t)si * p.kv_ld + half * kG * kD + g * kD + c16 * 8 : p.kv;
-                    cp_async16(dst + (half * kTileRows + i) * kGPitch + c16 * 16, src, si >= 0 ? 16u : 0u);
+                const uint32_t vmask = __ballot_sync(0xffffffffu, valid);
+                // Rows with nothing to load get a zero V half, so P = 0 never meets stale data.
+                uint32_t none = ~vmask & 0xFFFFu;
+                while (none) {
+                    const int z = __ffs(none) - 1;
+                    none &= none - 1;
+                    uint4* v = reinterpret_cast<uint4*>(dst + z * kPitch + kRowBytes / 2);
+                    v[lane] = make_uint4(0u, 0u, 0u, 0u);
+                    v[lane + 32] = make_uint4(0u, 0u, 0u, 0u);
                 }
-                cp_async_mbar_arrive(&full[stage]);
+                fence_proxy_async_smem();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&full[stage]);   // the row indices above are written
+                if (lane == 0) mbar_arrive_expect_tx(&full[stage], __popc(vmask) * kRowBytes);
+                __syncwarp();
+                if (valid) bulk_g2s(dst + lane * kPitch, p.kv + (int64_t)s * p.kv_ld, kRowBytes, &full[stage]);
             }
         } else if (warp < kConsumers) {
+            const int grp = warp;
             uint32_t qa[8][4];
-            const uint16_t* qbp = p.q + ((int64_t)t * kH + g * 16) * kD;
+            const uint16_t* qbp = p.q + ((int64_t)t * kH + grp * 16) * kD;
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
                 qa[kk][0] = __ldg(reinterpret_cast<const uint32_t*>(qbp + gq * kD + kk * 16 + 2 * c));
@@ -1137,14 +1161,14 @@ __device__ void phase_attend(const StepParams& p, uint8_t* smem, uint64_t* bars,
                 qa[kk][2] = __ldg(reinterpret_cast<const uint32_t*>(qbp + gq * kD + kk * 16 + 8 + 2 * c));
                 qa[kk][3] = __ldg(reinterpret_cast<const uint32_t*>(qbp + (gq + 8) * kD + kk * 16 + 8 + 2 * c));
             }
-            for (int k = warp; k < ntile; k += kConsumers) {
+            for (int k = 0; k < ntile; ++k) {
                 const int kk0 = phase_base + k;
-                const int stage = kk0 % kAttStagesG;
-                if (!mbar_wait(&full[stage], (kk0 / kAttStagesG) & 1, p.err)) {
+                const int stage = kk0 % kAttStages;
+                if (!mbar_wait(&full[stage], (kk0 / kAttStages) & 1, p.err)) {
                     failed = true;
                     break;
                 }
-                const uint32_t base = smem_u32(ring + stage * kGTileBytes);
+                const uint32_t base = smem_u32(ring + stage * kTileRows * kPitch);
                 const int32_t* ridx = rowidx + stage * kTileRows;
                 float sacc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
                 float sodd[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
@@ -1155,7 +1179,7 @@ __device__ void phase_attend(const StepParams& p, uint8_t* smem, uint64_t* bars,
                         const int key = nt * 8 + (lane & 7);
                         const int dim = kk2 * 32 + (lane >> 3) * 8;
                         uint32_t b0, b1, b2, b3;
-                        ldsm_x4(base + key * kGPitch + dim * 2, b0, b1, b2, b3);
+                        ldsm_x4(base + key * kPitch + grp * 256 + dim * 2, b0, b1, b2, b3);
                         mma_bf16_16816(sacc[nt], qa[2 * kk2], b0, b1);
                         mma_bf16_16816(sodd[nt], qa[2 * kk2 + 1], b2, b3);
                     }
@@ -1206,7 +1230,7 @@ __device__ void phase_attend(const StepParams& p, uint8_t* smem, uint64_t* bars,
                     const int key = (lane & 7) + 8 * ((lane >> 3) & 1);
                     const int dim = nd2 * 16 + 8 * (lane >> 4);
                     uint32_t v0, v1, v2, v3;
-                    ldsm_x4_t(base + (kTileRows + key) * kGPitch + dim * 2, v0, v1, v2, v3);
+                    ldsm_x4_t(base + key * kPitch + kRowBytes / 2 + grp * 256 + dim * 2, v0, v1, v2, v3);
                     mma_bf16_16816(oacc[2 * nd2], pa, v0, v1);
                     mma_bf16_16816(oacc[2 * nd2 + 1], pa, v2, v3);
                 }
@@ -1216,128 +1240,89 @@ __device__ void phase_attend(const StepParams& p, uint8_t* smem, uint64_t* bars,
         }
         if (__syncthreads_or(failed)) {
             // A bounded wait ran out: let the copies in flight land; the partial is empty.
-            if (warp == kProducer) asm volatile("cp.async.wait_all;" ::: "memory");
+            if (tid == kProducer * 32)
+                for (int k = max(0, ntile - kAttStages); k < ntile; ++k)
+                    mbar_wait(&full[(phase_base + k) % kAttStages], ((phase_base + k) / kAttStages) & 1, p.err);
             __syncthreads();
             m0 = m1 = -INFINITY;
             l0 = l1 = 0.f;
 #pragma unroll
             for (int k = 0; k < 16; ++k) oacc[k][0] = oacc[k][1] = oacc[k][2] = oacc[k][3] = 0.f;
         }
-        // the four consumer warps' states into shared memory
         if (warp < kConsumers) {
             l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
             l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
             l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
             l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+            const int h0 = warp * 16 + gq, h1 = h0 + 8;
+            const int64_t part = (int64_t)t * p.nsplit + split;
             if (c == 0) {
-                red_m[warp * 16 + gq] = m0;
-                red_m[warp * 16 + gq + 8] = m1;
-                red_l[warp * 16 + gq] = l0;
-                red_l[warp * 16 + gq + 8] = l1;
+                p.pml[part * kH + h0] = make_float2(m0, l0);
+                p.pml[part * kH + h1] = make_float2(m1, l1);
             }
-            float* o0 = red_o + (warp * 16 + gq) * kD;
-            float* o1 = red_o + (warp * 16 + gq + 8) * kD;
+            float* o0 = p.po + (part * kH + h0) * kD;
+            float* o1 = p.po + (part * kH + h1) * kD;
 #pragma unroll
             for (int nd = 0; nd < 16; ++nd) {
                 *reinterpret_cast<float2*>(o0 + nd * 8 + 2 * c) = make_float2(oacc[nd][0], oacc[nd][1]);
                 *reinterpret_cast<float2*>(o1 + nd * 8 + 2 * c) = make_float2(oacc[nd][2], oacc[nd][3]);
             }
         }
-        __syncthreads();
-        // the item's partial: thread (head h, dims 8d .. 8d+7) combines the warps in order
-        const int64_t part = ((int64_t)t * kG + g) * p.nsplit + split;
-        {
-            const int h = tid >> 4, d8 = (tid & 15) * 8;
-            float M = -INFINITY;
-#pragma unroll
-            for (int w = 0; w < kConsumers; ++w) M = fmaxf(M, red_m[w * 16 + h]);
-            float l = 0.f, o[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int w = 0; w < kConsumers; ++w) {
-                const float mw = red_m[w * 16 + h];
-                const float a = mw == -INFINITY ? 0.f : exp2f(mw - M);
-                l = fmaf(a, red_l[w * 16 + h], l);
-                const float4 x = *reinterpret_cast<const float4*>(red_o + (w * 16 + h) * kD + d8);
-                const float4 y = *reinterpret_cast<const float4*>(red_o + (w * 16 + h) * kD + d8 + 4);
-                o[0] = fmaf(a, x.x, o[0]);
-                o[1] = fmaf(a, x.y, o[1]);
-                o[2] = fmaf(a, x.z, o[2]);
-                o[3] = fmaf(a, x.w, o[3]);
-                o[4] = fmaf(a, y.x, o[4]);
-                o[5] = fmaf(a, y.y, o[5]);
-                o[6] = fmaf(a, y.z, o[6]);
-                o[7] = fmaf(a, y.w, o[7]);
-            }
-            float* dst = p.po + (part * kTileRows + h) * kD + d8;
-            *reinterpret_cast<float4*>(dst) = make_float4(o[0], o[1], o[2], o[3]);
-            *reinterpret_cast<float4*>(dst + 4) = make_float4(o[4], o[5], o[6], o[7]);
-            if ((tid & 15) == 0) p.pml[part * kTileRows + h] = make_float2(M, l);
-        }
-        __syncthreads();
-        if (tid == 0) {
-            __threadfence();
-            uint32_t old;
-            asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;"
-                         : "=r"(old)
-                         : "l"(p.ctrl + kCtrlWordDone + t * kG + g)
-                         : "memory");
-            last_s = old == static_cast<uint32_t>(p.nsplit) - 1u;
-        }
-        __syncthreads();
-        if (last_s) {
-            // every split of (t, g) is in: merge them in split order
-            if (!merged_any) stamp(p, 8);
-            merged_any = true;
-            const int h = tid >> 4, d8 = (tid & 15) * 8;
-            const int64_t p0 = ((int64_t)t * kG + g) * p.nsplit;
-            float2 ml[kMaxSplitsTG];   // every split's (max, sum) for head h: one load each, all in flight
-#pragma unroll
-            for (int s = 0; s < kMaxSplitsTG; ++s)
-                ml[s] = s < p.nsplit ? __ldcg(p.pml + (p0 + s) * kTileRows + h) : make_float2(-INFINITY, 0.f);
-            const float sink = p.sink != nullptr ? p.sink[g * 16 + h] * kLog2e : -INFINITY;
-            float M = sink;
-#pragma unroll
-            for (int s = 0; s < kMaxSplitsTG; ++s) M = fmaxf(M, ml[s].x);
-            float den = (p.sink != nullptr && M != -INFINITY) ? exp2f(sink - M) : 0.f;
-            float o[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int s0 = 0; s0 < kMaxSplitsTG; s0 += 8) {
-                float4 ox[8], oy[8];   // eight splits' outputs in flight
-#pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    const int s = s0 + u;
-                    const float* src = p.po + ((p0 + s) * kTileRows + h) * kD + d8;
-                    const bool in = s < p.nsplit && ml[s].x != -INFINITY;
-                    ox[u] = in ? __ldcg(reinterpret_cast<const float4*>(src)) : make_float4(0.f, 0.f, 0.f, 0.f);
-                    oy[u] = in ? __ldcg(reinterpret_cast<const float4*>(src + 4)) : make_float4(0.f, 0.f, 0.f, 0.f);
-                }
-#pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    const int s = s0 + u;
-                    const float a = ml[s].x == -INFINITY ? 0.f : exp2f(ml[s].x - M);
-                    den = fmaf(a, ml[s].y, den);
-                    o[0] = fmaf(a, ox[u].x, o[0]);
-                    o[1] = fmaf(a, ox[u].y, o[1]);
-                    o[2] = fmaf(a, ox[u].z, o[2]);
-                    o[3] = fmaf(a, ox[u].w, o[3]);
-                    o[4] = fmaf(a, oy[u].x, o[4]);
-                    o[5] = fmaf(a, oy[u].y, o[5]);
-                    o[6] = fmaf(a, oy[u].z, o[6]);
-                    o[7] = fmaf(a, oy[u].w, o[7]);
-                }
-            }
-            const float inv = den > 0.f ? 1.0f / den : 0.f;
-            uint4 packed;
-            packed.x = pack_bf16(o[0] * inv, o[1] * inv);
-            packed.y = pack_bf16(o[2] * inv, o[3] * inv);
-            packed.z = pack_bf16(o[4] * inv, o[5] * inv);
-            packed.w = pack_bf16(o[6] * inv, o[7] * inv);
-            *reinterpret_cast<uint4*>(p.out + ((int64_t)t * kH + g * 16 + h) * kD + d8) = packed;
-        }
         phase_base += ntile;
         __syncthreads();
+        if (tid == 0) red_release_add(p.ctrl + kCtrlWordDone + t, 1u);   // this split of query t is written
     }
-    if (merged_any) stamp(p, 9);
+}
+
+// ==================================================================================
+// Phase 5: merge the splits of each (query, head) in split order, one warp per
+// item (query t, head h, half of the 128 dims), starting once every split of
+// its query is done (its counter; no grid barrier).  Lane s loads split s's
+// (max, sum); every lane loads all splits' outputs for its two dims, all loads
+// in flight at once; the max, the weights and the denominator come by warp
+// shuffles, the sink joins the denominator with no value row.
+// ==================================================================================
+__device__ void phase_merge(const StepParams& p)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    constexpr int P = 2;                          // halves of the 128 dims per (t, h); two dims per lane
+    const int items = p.T * kH * P;
+    const int ns = p.nsplit;                      // <= kMaxSplitsQ
+    for (int i = blockIdx.x * kWarps + warp; i < items; i += gridDim.x * kWarps) {
+        const int t = i / (kH * P), h = (i / P) % kH, part = i % P;
+        int ok = 1;
+        if (lane == 0) ok = wait_counter(p, p.ctrl + kCtrlWordDone + t, static_cast<uint32_t>(ns)) ? 1 : 0;
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) continue;
+        const float2* ml = p.pml + (int64_t)t * ns * kH + h;
+        const int d0 = part * (kD / P) + lane * 2;
+        const float* po = p.po + ((int64_t)t * ns * kH + h) * kD + d0;
+        const float2 mine = lane < ns ? __ldcg(ml + (int64_t)lane * kH) : make_float2(-INFINITY, 0.f);
+        float2 o[kMaxSplitsQ];
+#pragma unroll
+        for (int s = 0; s < kMaxSplitsQ; ++s)
+            o[s] = s < ns ? __ldcg(reinterpret_cast<const float2*>(po + (int64_t)s * kH * kD)) : make_float2(0.f, 0.f);
+        const float sink = p.sink != nullptr ? p.sink[h] * kLog2e : -INFINITY;
+        float M = fmaxf(mine.x, sink);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+        const float wmine = mine.x == -INFINITY ? 0.f : exp2f(mine.x - M);
+        float den = wmine * mine.y;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) den += __shfl_xor_sync(0xffffffffu, den, off);
+        float x0 = 0.f, x1 = 0.f;
+#pragma unroll
+        for (int s = 0; s < kMaxSplitsQ; ++s) {   // splits in order
+            const float w = __shfl_sync(0xffffffffu, wmine, s);
+            if (s < ns) {
+                x0 = fmaf(w, o[s].x, x0);
+                x1 = fmaf(w, o[s].y, x1);
+            }
+        }
+        const float dd = den + ((p.sink != nullptr && M != -INFINITY) ? exp2f(sink - M) : 0.f);
+        const float inv = dd > 0.f ? 1.0f / dd : 0.f;
+        *reinterpret_cast<uint32_t*>(p.out + ((int64_t)t * kH + h) * kD + d0) = pack_bf16(x0 * inv, x1 * inv);
+    }
 }
 
 // ==================================================================================
@@ -1388,8 +1373,8 @@ __global__ void __launch_bounds__(kThreads, 1) step_kernel(const __grid_constant
     GridBarrier gb{p.ctrl, gridDim.x};
     // Stamps (when tracing): 0 start, 1 indexer done, 2 extraction start (after
     // the barrier), 3 extraction done, 4/5 selection (blocks < T), 6 first
-    // attention item starts, 7 attention done, 8/9 first merge this block does
-    // starts / its last one ends, 30 end; 28/29 SM clock.
+    // attention item starts, 7 this block's attention items done, 9 its merge
+    // items done, 30 end; 28/29 SM clock.
     bool ok = true;
     if (p.ctrl != nullptr) gb.enter();
     stamp(p, 0);
@@ -1415,6 +1400,9 @@ __global__ void __launch_bounds__(kThreads, 1) step_kernel(const __grid_constant
     if (p.phases & kPhaseAttend) {
         if (ok) phase_attend(p, smem, bars, (p.phases & kPhaseTopk) != 0, &ok_s);
         stamp(p, 7);
+        if (ok) phase_merge(p);
+        __syncthreads();
+        stamp(p, 9);
     }
     if (p.ctrl != nullptr) barrier_exit(p);
     if (p.trace != nullptr && threadIdx.x == 0) {
