@@ -67,7 +67,7 @@ struct StepParams {
     float* scores;           // [T][ld]
     int64_t ld;
     // top-k
-    uint32_t* cuts;          // [kMaxT][4]: threshold-bin key, #keys above the bin
+    uint32_t* cuts;          // [kMaxT][4]: lowest candidate key, #keys above the selection range, its top key
     uint32_t* seg_n;         // [kMaxT][kMaxSeg] candidates per sub-segment
     uint2* list;             // [T][list_ld] (key, position): sub-segment (c, w) starts at c*chunk + w*chunk/8
     int64_t list_ld;         // candidate-list row stride (the workspace's, not the caller's score stride)

@@ -26,6 +26,8 @@
 //
 // Stage entry points run a sub-range of the phases.  Every reduction is either
 // integer or in a fixed order, so results are bitwise reproducible.
+#include <type_traits>
+
 #include "common.cuh"
 #include "dsa_internal.h"
 
@@ -44,8 +46,7 @@ constexpr int kBarSlots = 96;             // mbarriers (8 bytes each) after the 
 constexpr int kStepSmem = 1024 + kBarOffset + kBarSlots * 8;
 
 // mbarrier slots of each phase (disjoint, so no phase re-initialises another's)
-constexpr int kBarRawFull = 0, kBarRawEmpty = 8, kBarAFull = 16, kBarAEmpty = 20, kBarAccFull = 24,
-              kBarAccEmpty = 27, kBarSetup = 30;
+constexpr int kBarRawFull = 0, kBarShare = 16, kBarAccFull = 24, kBarSetup = 30;
 constexpr int kBarExtract = 32;           // [8 warps][4 stages]
 constexpr int kBarAttFull = 64, kBarAttEmpty = 80;
 
@@ -363,33 +364,49 @@ __device__ void radix_pass(ForEach for_each_key, uint32_t& lo, uint32_t& hi, uin
 // keys is the M side of tcgen05.mma kind::f16 (bf16 operands, fp32 accumulators
 // in tensor memory), the T x 16 indexer query heads the N side (16..128), the 64
 // dims K (four K = 16 steps).  The eight warps are alike: warps w and w + 4 own
-// the same 32 key rows (TMEM lanes), and per tile each
-//   - (FP8 keys) widens its half of every row's 64 E4M3 codes (TMA tile with a
-//     64-byte swizzle) exactly into bf16, straight into 16 columns of the
-//     tile's tensor-memory A buffer (bf16 keys arrive from TMA already as the
-//     shared-memory A operand, 128-byte swizzle);
-//   - runs the epilogue of the previous tile for its half of the queries: ReLU,
-//     head weights, a fixed-order sum over the 16 heads, the per-token scale;
-//     the fp32 score goes to global memory and its key's top bits to the
-//     block's per-query histogram (16-bit counters in shared memory).
-// Warp 0's lane 0 also refills the TMA ring, warp 1's lane 0 issues the MMAs.
-// Tensor memory: three accumulator buffers of 128 columns and four A buffers of
-// 32 columns, all 512 columns.  mbarriers chain the steps; nothing waits on a
-// block-wide barrier inside the loop.
+// the same 32 key rows (TMEM lanes 32 (w % 4) ..), and warp w works on
+//   - (FP8 keys) half of every such row's 64 E4M3 codes (TMA tile with a 64-byte
+//     swizzle), widened exactly into bf16 straight into 16 columns of the tile's
+//     tensor-memory A buffer; bf16 keys arrive from TMA already as the
+//     shared-memory A operand (128-byte swizzle);
+//   - the epilogue of its half of the queries: ReLU, head weights, a fixed-order
+//     sum over the 16 heads, the per-token scale; the fp32 score goes to global
+//     memory, and each thread keeps the largest key it has seen per query.
+// Every warp marks its share of a tile done on an mbarrier; tile j's MMAs (and
+// the TMA refill of the stage they free) are issued by warp j % 8, at the end of
+// its iteration two tiles earlier, so that the issue (a thread blocks while the
+// tensor core takes the instructions) rotates over the warps and its wait for
+// the other shares is long satisfied.  Otherwise warps wait only for data: a
+// TMA stage to land, an accumulator to be complete.  Tensor memory: three
+// accumulator buffers of 128 columns and four A buffers of 32 columns.
+//
+// First radix pass.  Each (thread, query) pair sees a fixed set of positions
+// (its key row of each of the block's tiles); the block histogram of top-12-bit
+// bins counts one key per pair, the largest.  Those counts are a lower bound:
+// the bin b* where they first reach topk from the top has at least topk keys at
+// or above it, i.e. b* <= the bin of the topk-th largest key.  The selection
+// then radix-selects among all keys of bin >= b*.  With 148 x 128 pairs per
+// query, b* sits near the top 2048 / 18944 of the pair maxima, so for scores
+// without heavy ties the candidates number little more than topk.
 // ==================================================================================
 constexpr int kRawStagesF8 = 8, kRawStagesBf = 6;
 constexpr int kAccBufs = 3, kABufs = 4;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kACol = kAccBufs * 128;   // first column of the A buffers
 constexpr int kTileBytesBf16 = kKeyTile * kDI * 2;   // 16 KiB, one 128 x 64 bf16 operand tile
-constexpr int kHistFlushTiles = 256;         // an epilogue warp flushes its share of the 16-bit counters this often
+constexpr int kIdxCounters = 16;             // shared words: counters and issue marks
 static_assert(kACol + kABufs * 32 <= kTmemCols, "tensor memory budget");
-static_assert(kRawStagesF8 * kKeyTile * kDI + kTileBytesBf16 + kMaxT * kHI * 4 + kHistWords * 2 + 4 * 32 * kMaxT * 4 <=
+static_assert(kRawStagesF8 * kKeyTile * kDI + kTileBytesBf16 + kMaxT * kHI * 4 + kHistWords * 2 + kIdxCounters * 4 <=
                   kDataBytes,
               "FP8 indexer buffers fit the data region");
-static_assert(kRawStagesBf * kTileBytesBf16 + kTileBytesBf16 + kMaxT * kHI * 4 + kHistWords * 2 + 4 * 32 * kMaxT * 4 <=
+static_assert(kRawStagesBf * kTileBytesBf16 + kTileBytesBf16 + kMaxT * kHI * 4 + kHistWords * 2 + kIdxCounters * 4 <=
                   kDataBytes,
               "bf16 indexer buffers fit the data region");
+
+__device__ __forceinline__ void red_max_shared(uint32_t* a, uint32_t v)
+{
+    asm volatile("red.shared::cta.max.u32 [%0], %1;" ::"r"(smem_u32(a)), "r"(v) : "memory");
+}
 
 // The block's 16-bit counters (two per word) added to the launch's histogram.
 __device__ __forceinline__ void flush_hist16(const uint32_t* hs, int T)
@@ -404,65 +421,180 @@ __device__ __forceinline__ void flush_hist16(const uint32_t* hs, int T)
     }
 }
 
+// Everything a warp of the indexer needs.
+struct IndexCtx {
+    uint8_t* ring;           // [S][raw tile]
+    uint8_t* qsw;            // the B operand
+    const float* w_s;        // [8][16] head weights
+    uint32_t* hs;            // [8][2048] two 16-bit counters per word
+    uint32_t* cnt;           // [0] loads issued; [1] MMA groups issued (for the drain after an abort)
+    uint64_t* raw_full;
+    uint64_t* acc_full;
+    uint64_t* share;         // [kABufs or kAccBufs]: every warp's share of a tile done
+    const CUtensorMap* kmap;
+    uint64_t policy;
+    uint32_t tmem, idesc;
+    uint64_t bdesc;
+    int nloc;                // tiles of this block
+    int qa, nq;              // this warp's queries [qa, qa + nq)
+};
+
+template <bool FP8>
+struct IndexTile {
+    static constexpr int S = FP8 ? kRawStagesF8 : kRawStagesBf;
+    static constexpr int kRawBytes = kKeyTile * kDI * (FP8 ? 1 : 2);
+    static constexpr int kShareBufs = FP8 ? kABufs : kAccBufs;   // share barriers cycled by tile
+    __device__ static int tile_of(int j) { return blockIdx.x + j * static_cast<int>(gridDim.x); }
+
+    // TMA of local tile j into its ring stage (one thread).
+    __device__ static void load(const IndexCtx& c, int j)
+    {
+        const int stage = j % S;
+        mbar_arrive_expect_tx(&c.raw_full[stage], kRawBytes);
+        tma_load_2d_hint(c.ring + stage * kRawBytes, c.kmap, 0, tile_of(j) * kKeyTile, &c.raw_full[stage], c.policy);
+        red_max_shared(&c.cnt[0], static_cast<uint32_t>(j + 1));
+    }
+    // MMAs of local tile j into accumulator buffer j % 3, committed to its barrier (one thread).
+    __device__ static void mma(const IndexCtx& c, int j)
+    {
+        const uint32_t d = c.tmem + (j % kAccBufs) * 128;
+        if constexpr (FP8) {
+            const uint32_t a = c.tmem + kACol + (j % kABufs) * 32;
+#pragma unroll
+            for (int k = 0; k < kDI / 16; ++k) tc_mma_bf16_tmem_a(d, a + k * 8, c.bdesc + 2 * k, c.idesc, k > 0 ? 1u : 0u);
+        } else {
+            const uint64_t adesc = umma_desc_sw128(smem_u32(c.ring + (j % S) * kRawBytes));
+#pragma unroll
+            for (int k = 0; k < kDI / 16; ++k) tc_mma_bf16(d, adesc + 2 * k, c.bdesc + 2 * k, c.idesc, k > 0 ? 1u : 0u);
+        }
+        tc_commit(&c.acc_full[j % kAccBufs]);
+        red_max_shared(&c.cnt[1], static_cast<uint32_t>(j + 1));
+    }
+    // This warp's share of tile j is done (FP8: its A columns written; bf16: tile
+    // j's accumulator read).
+    __device__ static void done(const IndexCtx& c, int j, int lane)
+    {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&c.share[j % kShareBufs]);
+    }
+    // Issue tile j's MMAs once every share is in (FP8: of tile j; bf16: of tile
+    // j - 3, whose accumulator buffer it reuses, and tile j's data has landed),
+    // and refill the stage freed (FP8: tile j's, with tile j + S; bf16: tile j -
+    // 3's, with tile j - 3 + S).  One thread; false if a wait ran out.
+    __device__ static bool issue(const IndexCtx& c, int j, uint32_t* err)
+    {
+        const int f = FP8 ? j : j - kAccBufs;   // the tile whose shares free what tile j needs
+        if (!mbar_wait(&c.share[f % kShareBufs], (f / kShareBufs) & 1, err)) return false;
+        if constexpr (!FP8) {
+            if (!mbar_wait(&c.raw_full[j % S], (j / S) & 1, err)) return false;
+        }
+        tc_fence_after();
+        mma(c, j);
+        if (f + S < c.nloc) load(c, f + S);
+        return true;
+    }
+    // FP8: this warp's half of its 32 key rows of tile j widened into the A buffer.
+    // False if the wait for the data ran out.
+    __device__ static bool convert(const IndexCtx& c, int j, int row, int half, uint32_t lane_base, uint32_t* err)
+    {
+        const int stage = j % S;
+        if (__any_sync(0xffffffffu, !mbar_wait(&c.raw_full[stage], (j / S) & 1, err))) return false;
+        const uint8_t* src = c.ring + stage * kRawBytes + row * 64;   // 16-byte chunk q stored at q ^ ((row >> 1) & 3)
+        uint4 v[2];
+#pragma unroll
+        for (int q = 0; q < 2; ++q) v[q] = *reinterpret_cast<const uint4*>(src + (((2 * half + q) ^ ((row >> 1) & 3)) << 4));
+        uint32_t r[16];
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+            e4m3x4_to_bf16x4(v[q].x, r[8 * q + 0], r[8 * q + 1]);
+            e4m3x4_to_bf16x4(v[q].y, r[8 * q + 2], r[8 * q + 3]);
+            e4m3x4_to_bf16x4(v[q].z, r[8 * q + 4], r[8 * q + 5]);
+            e4m3x4_to_bf16x4(v[q].w, r[8 * q + 6], r[8 * q + 7]);
+        }
+        tmem_st16(c.tmem + lane_base + kACol + (j % kABufs) * 32 + half * 16, r);
+        tmem_st_wait();
+        return true;
+    }
+};
+
+// Math of one tile for this warp's queries (NQ >= nq of them, a compile-time
+// bound so that the code is straight-line) from the accumulator registers.
+template <int NQ>
+__device__ __forceinline__ void index_math(const IndexCtx& c, const StepParams& p, const uint32_t (&r)[NQ > 2 ? 2 : 1][32],
+                                           int s, float scale, const int (&pos_q)[4], uint32_t (&kmax)[4])
+{
+    float4 w[NQ][4];
+#pragma unroll
+    for (int u = 0; u < NQ; ++u)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) w[u][k] = reinterpret_cast<const float4*>(c.w_s + (c.qa + u) * kHI)[k];
+#pragma unroll
+    for (int u = 0; u < NQ; ++u) {
+        // Four partial sums over heads {j, j+4, j+8, j+12}, j < 4, as two packed fp32
+        // FMAs per four heads, combined in a fixed order.
+        const float* v = reinterpret_cast<const float*>(&r[u >> 1][(u & 1) * 16]);
+        float2 p01 = make_float2(0.f, 0.f), p23 = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int g4 = 0; g4 < 4; ++g4) {
+            p01 = __ffma2_rn(make_float2(fmaxf(v[g4 * 4 + 0], 0.f), fmaxf(v[g4 * 4 + 1], 0.f)),
+                             make_float2(w[u][g4].x, w[u][g4].y), p01);
+            p23 = __ffma2_rn(make_float2(fmaxf(v[g4 * 4 + 2], 0.f), fmaxf(v[g4 * 4 + 3], 0.f)),
+                             make_float2(w[u][g4].z, w[u][g4].w), p23);
+        }
+        const float acc = ((p01.x + p01.y) + (p23.x + p23.y)) * scale;
+        if (u < c.nq && s < p.L) {
+            const bool vis = s <= pos_q[u];
+            p.scores[(int64_t)(c.qa + u) * p.ld + s] = vis ? acc : -INFINITY;
+            if (vis) kmax[u] = max(kmax[u], score_key(acc));
+        }
+    }
+}
+
 template <bool FP8>
 __device__ void phase_index(const CUtensorMap& kmap, const StepParams& p, uint8_t* smem, uint64_t* bars,
                             uint32_t* tmem_slot)
 {
-    constexpr int S = FP8 ? kRawStagesF8 : kRawStagesBf;
-    constexpr int raw_bytes = kKeyTile * kDI * (FP8 ? 1 : 2);
-    uint8_t* ring = smem;                                               // [S][raw_bytes]
-    uint8_t* qsw = smem + S * raw_bytes;                                // [128 rows][128 B] queries (B operand)
-    float* w_s = reinterpret_cast<float*>(qsw + kTileBytesBf16);        // [8][16]
-    uint32_t* hs = reinterpret_cast<uint32_t*>(w_s + kMaxT * kHI);      // [8][2048]: two 16-bit counters per word
-    uint32_t* hstage = hs + kHistWords / 2;                             // [8 warps][32 keys][4 queries] bins
-    uint64_t* raw_full = bars + kBarRawFull;
-    uint64_t* raw_empty = bars + kBarRawEmpty;
-    uint64_t* a_full = bars + kBarAFull;
-    uint64_t* a_empty = bars + kBarAEmpty;
-    uint64_t* acc_full = bars + kBarAccFull;
-    uint64_t* acc_empty = bars + kBarAccEmpty;
-    uint64_t* setup = bars + kBarSetup;
-
+    using Tile = IndexTile<FP8>;
+    constexpr int S = Tile::S;
+    constexpr int raw_bytes = Tile::kRawBytes;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int quad = warp & 3, half = warp >> 2;     // TMEM lane quarter; which half of the row / queries
     const int T = p.T;
-    const int Th = (T + 1) >> 1;                     // queries per half
-    const int qa = min(T, half * Th), qb = min(T, qa + Th);   // this warp's queries [qa, qb)
     const int ntiles = (visible_max(p) + kKeyTile - 1) / kKeyTile;
-    const int nloc = ntiles > static_cast<int>(blockIdx.x) ? (ntiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
-    const bool hist = g_view.hist != nullptr;
-    auto tile_of = [&](int it) { return blockIdx.x + it * static_cast<int>(gridDim.x); };
-    const uint64_t stream_policy = l2_evict_first_policy();   // keys are read once; the scores stay in L2
-    auto load_tile = [&](int it) {
-        const int stage = it % S;
-        mbar_arrive_expect_tx(&raw_full[stage], raw_bytes);
-        tma_load_2d_hint(ring + stage * raw_bytes, &kmap, 0, tile_of(it) * kKeyTile, &raw_full[stage], stream_policy);
-    };
 
-    int issued = 0;   // (thread 0) key tiles requested
+    IndexCtx c;
+    c.ring = smem;
+    c.qsw = smem + S * raw_bytes;
+    c.w_s = reinterpret_cast<const float*>(c.qsw + kTileBytesBf16);
+    c.hs = reinterpret_cast<uint32_t*>(c.qsw + kTileBytesBf16 + kMaxT * kHI * 4);
+    c.cnt = c.hs + kHistWords / 2;
+    c.raw_full = bars + kBarRawFull;
+    c.acc_full = bars + kBarAccFull;
+    c.share = bars + kBarShare;
+    c.kmap = &kmap;
+    c.policy = l2_evict_first_policy();   // keys are read once; the scores stay in L2
+    c.nloc = ntiles > static_cast<int>(blockIdx.x) ? (ntiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+    c.qa = half == 0 ? 0 : (T + 1) >> 1;
+    c.nq = half == 0 ? (T + 1) >> 1 : T >> 1;
+    const bool hist = g_view.hist != nullptr;
+    uint64_t* setup = bars + kBarSetup;
+    float* w_s = const_cast<float*>(c.w_s);
+
     if (tid == 0) {
         prefetch_tmap(&kmap);
-        for (int s = 0; s < S; ++s) {
-            mbar_init(&raw_full[s], 1);
-            mbar_init(&raw_empty[s], FP8 ? kWarps : 1);   // every warp's half rows read, or the MMA commit
-        }
-        for (int b = 0; b < kABufs; ++b) {
-            mbar_init(&a_full[b], kWarps);
-            mbar_init(&a_empty[b], 1);
-        }
-        for (int b = 0; b < kAccBufs; ++b) {
-            mbar_init(&acc_full[b], 1);
-            mbar_init(&acc_empty[b], kWarps);
-        }
+        for (int s = 0; s < S; ++s) mbar_init(&c.raw_full[s], 1);
+        for (int b = 0; b < kAccBufs; ++b) mbar_init(&c.acc_full[b], 1);
+        for (int b = 0; b < Tile::kShareBufs; ++b) mbar_init(&c.share[b], kWarps);
         mbar_init(setup, 1);
         fence_mbar_init();
         mbar_arrive_expect_tx(setup, T * kHI * 4);
         bulk_g2s(w_s, p.w, T * kHI * 4, setup);
-        for (; issued < S && issued < nloc; ++issued) load_tile(issued);
     }
+    if (tid < kIdxCounters) c.cnt[tid] = 0u;
     if (warp == 0) tmem_alloc(tmem_slot, kTmemCols);
-    // The indexer queries as the B operand: row r = t*16 + j, 16-byte chunk c at
-    // r*128 + (c ^ (r & 7))*16 (the 128B swizzle); rows >= T*16 are never read.
+    // The indexer queries as the B operand: row r = t*16 + j, 16-byte chunk k at
+    // r*128 + (k ^ (r & 7))*16 (the 128B swizzle); rows >= T*16 are never read.
     {
         uint4 v[kMaxT * kHI * 8 / kThreads];   // every load in flight before the first store
 #pragma unroll
@@ -472,203 +604,145 @@ __device__ void phase_index(const CUtensorMap& kmap, const StepParams& p, uint8_
         }
 #pragma unroll
         for (int u = 0; u < kMaxT * kHI * 8 / kThreads; ++u) {
-            const int i = tid + u * kThreads, r = i >> 3, c = i & 7;
-            if (i < T * kHI * 8) *reinterpret_cast<uint4*>(qsw + r * 128 + ((c ^ (r & 7)) << 4)) = v[u];
+            const int i = tid + u * kThreads, r = i >> 3, k = i & 7;
+            if (i < T * kHI * 8) *reinterpret_cast<uint4*>(c.qsw + r * 128 + ((k ^ (r & 7)) << 4)) = v[u];
         }
     }
     if (hist)
-        for (int i = tid; i < kHistWords / 2; i += kThreads) hs[i] = 0u;
+        for (int i = tid; i < kHistWords / 2; i += kThreads) c.hs[i] = 0u;
     fence_proxy_async_smem();   // the queries are read by the tensor cores (async proxy)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
-    const uint32_t idesc = umma_idesc_bf16(kKeyTile, T * kHI);
-    const uint64_t bdesc = umma_desc_sw128(smem_u32(qsw));
+    c.tmem = *tmem_slot;
+    c.idesc = umma_idesc_bf16(kKeyTile, T * kHI);
+    c.bdesc = umma_desc_sw128(smem_u32(c.qsw));
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
     const int row = quad * 32 + lane;                // this thread's key row of every tile
-    int mma_issued = 0;                              // (warp 1 lane 0)
-    bool aborted = __any_sync(0xffffffffu, !mbar_wait(setup, 0, p.err));   // warp-uniform from here on
+    bool aborted = false;
+    if (tid == 0) {
+        for (int j = 0; j < S && j < c.nloc; ++j) Tile::load(c, j);
+        if constexpr (!FP8) {   // the first accumulator buffers are free: their MMAs go out as the data lands
+            for (int j = 0; j < kAccBufs && j < c.nloc && !aborted; ++j) {
+                aborted = !mbar_wait(&c.raw_full[j], 0, p.err);
+                if (!aborted) Tile::mma(c, j);
+            }
+        }
+    }
+    aborted = __any_sync(0xffffffffu, aborted || !mbar_wait(setup, 0, p.err));   // warp-uniform from here on
     int pos_q[4];                                    // positions of this warp's queries
 #pragma unroll
-    for (int u = 0; u < 4; ++u) pos_q[u] = qa + u < qb ? query_pos_rt(p, qa + u) : -1;
+    for (int u = 0; u < 4; ++u) pos_q[u] = u < c.nq ? query_pos_rt(p, c.qa + u) : -1;
+    uint32_t kmax[4] = {0u, 0u, 0u, 0u};             // largest key seen per query (0: none)
 
-    // MMAs of local tile it into accumulator buffer it % 3 (one thread).
-    auto issue_mma = [&](int it) -> bool {
-        const int ab = it % kABufs, cb = it % kAccBufs;
+    auto run = [&](auto nq_tag) {
+        constexpr int NQ = decltype(nq_tag)::value;
+        const bool scaled = p.scale != nullptr;
+        float scale_next = 1.0f;
+        if (NQ > 0 && scaled && c.nloc > 0) {
+            const int s = Tile::tile_of(0) * kKeyTile + row;
+            scale_next = s < p.L ? __ldg(p.scale + s) : 1.0f;
+        }
+        // Tile j's MMAs go out from warp j % 8 at the end of its iteration j - 2 (FP8:
+        // tiles 0 and 1 here; bf16: tiles 0..2 went out with the first loads).
+        auto issue_by_me = [&](int j) -> bool {
+            bool ok = true;
+            if (j < c.nloc && (FP8 || j >= kAccBufs) && warp == j % kWarps && lane == 0) ok = Tile::issue(c, j, p.err);
+            return !__any_sync(0xffffffffu, !ok);
+        };
         if constexpr (FP8) {
-            if (!mbar_wait(&a_full[ab], (it / kABufs) & 1, p.err)) return false;
-        } else {
-            if (!mbar_wait(&raw_full[it % S], (it / S) & 1, p.err)) return false;
-        }
-        if (it >= kAccBufs && !mbar_wait(&acc_empty[cb], ((it / kAccBufs) - 1) & 1, p.err)) return false;
-        tc_fence_after();
-        const uint32_t d = tmem + cb * 128;
-        if constexpr (FP8) {
-            const uint32_t a = tmem + kACol + ab * 32;
-#pragma unroll
-            for (int k = 0; k < kDI / 16; ++k) tc_mma_bf16_tmem_a(d, a + k * 8, bdesc + 2 * k, idesc, k > 0 ? 1u : 0u);
-            tc_commit(&a_empty[ab]);
-        } else {
-            const uint64_t adesc = umma_desc_sw128(smem_u32(ring + (it % S) * raw_bytes));
-#pragma unroll
-            for (int k = 0; k < kDI / 16; ++k) tc_mma_bf16(d, adesc + 2 * k, bdesc + 2 * k, idesc, k > 0 ? 1u : 0u);
-            tc_commit(&raw_empty[it % S]);
-        }
-        tc_commit(&acc_full[cb]);
-        ++mma_issued;
-        return true;
-    };
-
-    // FP8: this warp's half of key row `row` (32 codes, two 16-byte chunks stored at
-    // chunk c ^ ((row >> 1) & 3)) widened into 16 columns of the tile's A buffer.
-    auto convert = [&](int it) -> bool {
-        const int stage = it % S, ab = it % kABufs;
-        bool ok = it < kABufs || mbar_wait(&a_empty[ab], ((it / kABufs) - 1) & 1, p.err);
-        ok = ok && mbar_wait(&raw_full[stage], (it / S) & 1, p.err);
-        if (__any_sync(0xffffffffu, !ok)) return false;
-        const uint8_t* src = ring + stage * raw_bytes + row * 64;
-        uint4 v[2];
-#pragma unroll
-        for (int c = 0; c < 2; ++c)
-            v[c] = *reinterpret_cast<const uint4*>(src + (((2 * half + c) ^ ((row >> 1) & 3)) << 4));
-        uint32_t r[16];
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-            e4m3x4_to_bf16x4(v[c].x, r[8 * c + 0], r[8 * c + 1]);
-            e4m3x4_to_bf16x4(v[c].y, r[8 * c + 2], r[8 * c + 3]);
-            e4m3x4_to_bf16x4(v[c].z, r[8 * c + 4], r[8 * c + 5]);
-            e4m3x4_to_bf16x4(v[c].w, r[8 * c + 6], r[8 * c + 7]);
-        }
-        tmem_st16(tmem + lane_base + kACol + ab * 32 + half * 16, r);
-        tmem_st_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) {
-            mbar_arrive(&a_full[ab]);
-            mbar_arrive(&raw_empty[stage]);
-        }
-        return true;
-    };
-
-    // Epilogue of local tile e for this warp's queries: ReLU, head weights, a
-    // fixed-order head sum, the per-token scale; scores to global memory, keys'
-    // top bits counted in the block's histogram.
-    auto epilogue = [&](int e) -> bool {
-        const int cb = e % kAccBufs;
-        const int s = tile_of(e) * kKeyTile + row;
-        const float scale = (p.scale != nullptr && s < p.L) ? __ldg(p.scale + s) : 1.0f;
-        if (__any_sync(0xffffffffu, !mbar_wait(&acc_full[cb], (e / kAccBufs) & 1, p.err))) return false;
-        tc_fence_after();
-        uint32_t r[2][32];
-        if (qa < qb) {
-            const uint32_t tbase = tmem + lane_base + cb * 128 + qa * kHI;
-            tmem_ld32_nowait(tbase, r[0]);
-            if (qb - qa > 2) tmem_ld32_nowait(tbase + 32, r[1]);
-            tmem_ld_wait();
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&acc_empty[cb]);   // this warp is done with the buffer
-        uint32_t bins[4] = {~0u, ~0u, ~0u, ~0u};    // histogram bin of each query's score (~0u: none)
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int t = qa + u;
-            if (t < qb) {
-                // Four partial sums over heads {j, j+4, j+8, j+12}, j < 4, as two packed
-                // fp32 FMAs per four heads, combined in a fixed order.
-                const float4* w4 = reinterpret_cast<const float4*>(w_s + t * kHI);
-                const float* v = reinterpret_cast<const float*>(&r[u >> 1][(u & 1) * 16]);
-                float2 p01 = make_float2(0.f, 0.f), p23 = make_float2(0.f, 0.f);
-#pragma unroll
-                for (int g4 = 0; g4 < 4; ++g4) {
-                    const float4 w = w4[g4];
-                    p01 = __ffma2_rn(make_float2(fmaxf(v[g4 * 4 + 0], 0.f), fmaxf(v[g4 * 4 + 1], 0.f)),
-                                     make_float2(w.x, w.y), p01);
-                    p23 = __ffma2_rn(make_float2(fmaxf(v[g4 * 4 + 2], 0.f), fmaxf(v[g4 * 4 + 3], 0.f)),
-                                     make_float2(w.z, w.w), p23);
-                }
-                const float acc = ((p01.x + p01.y) + (p23.x + p23.y)) * scale;
-                if (s < p.L) {
-                    const bool vis = s <= pos_q[u];
-                    p.scores[(int64_t)t * p.ld + s] = vis ? acc : -INFINITY;
-                    if (vis) bins[u] = score_key(acc) >> kHistShift;
+            for (int j = 0; j < 2 && j < c.nloc && !aborted; ++j) {
+                aborted = !Tile::convert(c, j, row, half, lane_base, p.err);
+                if (!aborted) {
+                    Tile::done(c, j, lane);
+                    aborted = !issue_by_me(j);
                 }
             }
         }
-        if (hist && qa < qb) {
-            // The bins through a transpose in shared memory: in round i lane l adds key
-            // (8i + l/4)'s bin of query qa + l % 4, so one atomic instruction spreads over
-            // four query histograms.
-            uint32_t* st = hstage + warp * 32 * 4;
-            *reinterpret_cast<uint4*>(st + lane * 4) = make_uint4(bins[0], bins[1], bins[2], bins[3]);
-            __syncwarp();
-            uint32_t* hq = hs + (qa + (lane & 3)) * (kHistBins / 2);
+        for (int e = 0; e < c.nloc && !aborted; ++e) {
+            const int s = Tile::tile_of(e) * kKeyTile + row;
+            const float scale = scale_next;
+            if (NQ > 0 && scaled && e + 1 < c.nloc) {   // next tile's scale, in flight during this tile
+                const int s2 = Tile::tile_of(e + 1) * kKeyTile + row;
+                scale_next = s2 < p.L ? __ldg(p.scale + s2) : 1.0f;
+            }
+            // tile e's accumulator: wait, start the loads, then (FP8) widen tile e + 2
+            // while they are in flight
+            const int cb = e % kAccBufs;
+            if (__any_sync(0xffffffffu, !mbar_wait(&c.acc_full[cb], (e / kAccBufs) & 1, p.err))) {
+                aborted = true;
+                break;
+            }
+            tc_fence_after();
+            uint32_t r[NQ > 2 ? 2 : 1][32];
+            if constexpr (NQ > 0) {
+                const uint32_t tbase = c.tmem + lane_base + cb * 128 + c.qa * kHI;
+                tmem_ld32_nowait(tbase, r[0]);
+                if constexpr (NQ > 2) tmem_ld32_nowait(tbase + 32, r[1]);
+            }
+            if (FP8 && e + 2 < c.nloc) {
+                if (!Tile::convert(c, e + 2, row, half, lane_base, p.err)) {
+                    aborted = true;
+                    break;
+                }
+                Tile::done(c, e + 2, lane);
+            }
+            if constexpr (NQ > 0) {
+                tmem_ld_wait();
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const uint32_t bin = st[i * 32 + lane];
-                if (bin != ~0u) atomicAdd(&hq[bin >> 1], 1u << ((bin & 1) << 4));
+                for (int h = 0; h < (NQ > 2 ? 2 : 1); ++h)
+#pragma unroll
+                    for (int k = 0; k < 32; ++k) asm volatile("" : "+r"(r[h][k]));   // no use before the wait
+                index_math<NQ>(c, p, r, s, scale, pos_q, kmax);
             }
-            __syncwarp();
-        }
-        if (hist && (e + 1) % kHistFlushTiles == 0) {
-            // 16-bit counters: this warp moves its eighth of them to the global histogram
-            // (atomic exchange, so concurrent increments are kept) well before any can
-            // overflow: the warps are at most a tile or two apart, so between two flushes
-            // of a word it takes at most (kHistFlushTiles + kAccBufs) * 128 < 65536 counts.
-            const int words = T * (kHistBins / 2), w0 = warp * words / kWarps, w1 = (warp + 1) * words / kWarps;
-            for (int i = w0 + lane; i < w1; i += 32) {
-                const uint32_t v = atomicExch(&hs[i], 0u);
-                if (v) {
-                    uint32_t* gh = g_view.hist + (i / (kHistBins / 2)) * kHistBins + 2 * (i % (kHistBins / 2));
-                    if (v & 0xFFFFu) atomicAdd(gh, v & 0xFFFFu);
-                    if (v >> 16) atomicAdd(gh + 1, v >> 16);
-                }
-            }
-        }
-        return true;
-    };
-
-    // Every warp: widen tile it (FP8), then the epilogue of tile it - 1.  Warp 0's
-    // lane 0 refills the ring one tile behind; warp 1's lane 0 issues tile it's MMAs.
-    for (int it = 0; it <= nloc && !aborted; ++it) {
-        if (it < nloc) {
-            bool bad = false;
-            if constexpr (FP8) bad = !convert(it);
-            if (!bad && warp == 0 && lane == 0 && it >= 1 && issued < nloc) {
-                const int prev = it - 1;   // its stage is free once it has been read (FP8) or its MMAs are done
-                if (mbar_wait(&raw_empty[prev % S], (prev / S) & 1, p.err)) {
-                    load_tile(issued);
-                    ++issued;
-                } else {
-                    bad = true;
-                }
-            }
-            if (!bad && warp == 1 && lane == 0 && !issue_mma(it)) bad = true;
-            if (__any_sync(0xffffffffu, bad)) {
+            if constexpr (!FP8) Tile::done(c, e, lane);   // tile e's accumulator is read
+            if (!issue_by_me(e + 2)) {
                 aborted = true;
                 break;
             }
         }
-        if (it >= 1 && !epilogue(it - 1)) aborted = true;
+    };
+    if (c.nq > 2) {
+        run(std::integral_constant<int, 4>{});
+    } else if (c.nq == 2) {
+        run(std::integral_constant<int, 2>{});
+    } else if (c.nq == 1) {
+        run(std::integral_constant<int, 1>{});
+    } else {
+        run(std::integral_constant<int, 0>{});
     }
     // A wait that ran out (error bit set) ends the loop for that warp; the others
     // run into bounded waits and stop too.  Copies and MMAs still in flight land
-    // before the shared memory and tensor memory are reused.
+    // before the shared memory and tensor memory are reused: the last S loads and
+    // the last three MMA groups (every earlier one was waited for by an epilogue).
     aborted = __syncthreads_or(aborted);
     if (aborted) {
-        if (tid == 0)
-            for (int k = max(0, issued - S); k < issued; ++k) mbar_wait(&raw_full[k % S], (k / S) & 1, p.err);
-        if (tid == 32 && mma_issued > 0)
-            mbar_wait(&acc_full[(mma_issued - 1) % kAccBufs], ((mma_issued - 1) / kAccBufs) & 1, p.err);
+        if (tid == 0) {
+            const int li = static_cast<int>(c.cnt[0]);
+            for (int k = max(0, li - S); k < li; ++k) mbar_wait(&c.raw_full[k % S], (k / S) & 1, p.err);
+        }
+        if (tid == 32) {
+            const int mi = static_cast<int>(c.cnt[1]);
+            for (int k = max(0, mi - kAccBufs); k < mi; ++k)
+                mbar_wait(&c.acc_full[k % kAccBufs], (k / kAccBufs) & 1, p.err);
+        }
     }
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
         tc_fence_after();
-        tmem_dealloc(tmem, kTmemCols);
+        tmem_dealloc(c.tmem, kTmemCols);
     }
-    if (hist) flush_hist16(hs, T);   // the block's counters into the launch's histogram
+    if (hist) {
+        // one count per (thread, query): its largest key's bin
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+            if (u < c.nq && kmax[u] != 0u)
+                atomicAdd(&c.hs[(c.qa + u) * (kHistBins / 2) + (kmax[u] >> (kHistShift + 1))],
+                          1u << (((kmax[u] >> kHistShift) & 1u) << 4));
+        __syncthreads();
+        flush_hist16(c.hs, T);   // the block's counters into the launch's histogram
+    }
     // Positions no query can see (s >= n_max): -inf, as the stage contract states.
     const int64_t tail0 = (int64_t)ntiles * kKeyTile;
     for (int64_t s = tail0 + (int64_t)blockIdx.x * kThreads + tid; s < p.L; s += (int64_t)gridDim.x * kThreads)
@@ -759,13 +833,22 @@ __device__ void phase_extract(const StepParams& p, uint8_t* smem, uint64_t* bars
         fence_proxy_async_smem();   // earlier generic writes to the ring region come first
         __syncthreads();
         find_from_top(h, static_cast<uint32_t>(p.topk), res);
-        uint32_t cut = 0u;
+        // Exact histogram (caller scores): the candidates are the keys of the threshold
+        // bin and above, those above it all selected.  Indexer histogram of per-thread
+        // maxima (a lower bound): every key of bin >= b* is a candidate, to be
+        // radix-selected from the top; with fewer than topk counts, every visible key.
+        const bool bound = (p.phases & kPhaseIndex) != 0;
+        uint32_t cut = 0u, above = 0u, top = 0xFFFFFFFFu;
         if (res[2]) {
             cut = res[0] << kHistShift;
-        } else if (tid == 0) {   // histogram and scores disagree: cannot happen for consistent input
+            if (!bound) {
+                above = res[1];
+                top = bin_top(cut, kHistShift, 0xFFFFFFFFu);
+            }
+        } else if (!bound && tid == 0) {   // histogram and scores disagree: cannot happen for consistent input
             atomicOr(p.err, ERR_TOPK_STATE);
         }
-        if (c == 0 && tid == 0) reinterpret_cast<uint4*>(p.cuts)[t] = make_uint4(cut, res[2] ? res[1] : 0u, 0u, 0u);
+        if (c == 0 && tid == 0) reinterpret_cast<uint4*>(p.cuts)[t] = make_uint4(cut, above, top, 0u);
 
         const int R = p.chunk / kSegPerChunk;
         const int s0 = c * p.chunk + warp * R, s1 = min(s0 + R, n);
@@ -864,8 +947,8 @@ __device__ void phase_select(const StepParams& p, uint8_t* smem, uint32_t* res, 
             const uint4 cq = __ldcg(reinterpret_cast<const uint4*>(p.cuts) + t);
             __syncthreads();
             const uint32_t m = block_scan_array(off, nseg, scratch);   // off[k]: first slot of sub-segment k
-            uint32_t lo = cq.x, hi = bin_top(cq.x, kHistShift, 0xFFFFFFFFu);
-            uint32_t need = topk - cq.y;   // keys above the threshold bin are all taken
+            uint32_t lo = cq.x, hi = cq.z;   // the keys of [lo, hi] are radix-selected
+            uint32_t need = topk - cq.y;     // keys above hi are all taken
             const uint2* glist = p.list + (int64_t)t * p.list_ld;
             auto seg_cnt = [&](int k) { return (k + 1 < nseg ? off[k + 1] : m) - off[k]; };
             uint32_t nsel = 0;

@@ -27,12 +27,20 @@ def _custom(name, L, T, key_dtype, recipe, seed, pos=None, topk=2048):
 
 
 # Small and medium cases: several indexer tiles, ragged tails, both key formats,
-# T in {1, 3, 8}, queries at scattered positions.
+# T in {1, 3, 5, 6, 7, 8}, queries at scattered positions.
 SMALL = [
     ("tiny_decode", None),
     ("ragged_bf16_T3", dict(L=3001, T=3, key_dtype="bf16", recipe="normal", seed=41, pos=np.array([3000, 1500, 2047]))),
     ("ragged_fp8_T3", dict(L=2999, T=3, key_dtype="fp8", recipe="normal", seed=42, pos=np.array([2998, 2500, 10]))),
     ("ragged_fp8_T8_int", dict(L=5000, T=8, key_dtype="fp8", recipe="int", seed=43)),
+    # T = 5, 6, 7 (uneven query halves) at contexts where the fused first radix pass
+    # counts groups of 2, 4 and 8 keys
+    ("ragged_fp8_T6", dict(L=20000, T=6, key_dtype="fp8", recipe="normal", seed=44,
+                           pos=np.array([19999, 17000, 16383, 12000, 19000, 5000]))),
+    ("ragged_fp8_T5", dict(L=40000, T=5, key_dtype="fp8", recipe="normal", seed=45,
+                           pos=np.array([39999, 33000, 20000, 39000, 2100]))),
+    ("ragged_bf16_T7_int", dict(L=70001, T=7, key_dtype="bf16", recipe="int", seed=46,
+                                pos=np.array([70000, 69000, 65535, 40000, 70000, 1000, 66000]))),
     ("sweep_L2200_T8", None),
     ("sweep_L2200_T1", None),
     ("sweep_L2200_T1_int", None),
