@@ -329,7 +329,7 @@ dsa_status_t launch(const CUtensorMap& map, StepParams& p, bool fp8, void* ws, c
         t_fail_barriers = 0;
     }
     if ((e = launch_step(&map, p, fp8, stream)) != cudaSuccess) return cuda_fail(e, "step launch");
-    g_launches += 1;
+    g_launches += ((p.phases & kPhaseIndex) != 0) + ((p.phases & ~kPhaseIndex) != 0);   // indexer, cooperative kernel
     return DSA_OK;
 }
 

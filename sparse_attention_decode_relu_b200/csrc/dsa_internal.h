@@ -92,6 +92,7 @@ struct StepParams {
     int64_t barrier_limit;   // SM clocks a wait between blocks spins before it gives up
     uint32_t barrier_extra;  // arrivals such a wait needs beyond the real ones (0; 1 = a block that never comes)
     uint32_t* err;
+    int32_t hist_bound;      // the first radix histogram holds per-thread key maxima (a lower bound), not every key
 };
 
 int step_smem_bytes();

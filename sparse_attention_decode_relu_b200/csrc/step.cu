@@ -360,23 +360,26 @@ __device__ void radix_pass(ForEach for_each_key, uint32_t& lo, uint32_t& hi, uin
 }
 
 // ==================================================================================
-// Phase 1: indexer scan on the fifth-generation tensor cores.  A tile of 128
-// keys is the M side of tcgen05.mma kind::f16 (bf16 operands, fp32 accumulators
-// in tensor memory), the T x 16 indexer query heads the N side (16..128), the 64
-// dims K (four K = 16 steps).  The eight warps are alike: warps w and w + 4 own
-// the same 32 key rows (TMEM lanes 32 (w % 4) ..), and warp w works on
-//   - (FP8 keys) half of every such row's 64 E4M3 codes (TMA tile with a 64-byte
-//     swizzle), widened exactly into bf16 straight into 16 columns of the tile's
-//     tensor-memory A buffer; bf16 keys arrive from TMA already as the
-//     shared-memory A operand (128-byte swizzle);
-//   - the epilogue of its half of the queries: ReLU, head weights, a fixed-order
-//     sum over the 16 heads, the per-token scale; the fp32 score goes to global
-//     memory, and each thread keeps the largest key it has seen per query.
+// Phase 1: indexer scan on the fifth-generation tensor cores, a kernel of its own
+// (16 warps per SM: the per-tile work is a chain of latencies that four warps per
+// scheduler hide far better than two).  A tile of 128 keys is the M side of
+// tcgen05.mma kind::f16 (bf16 operands, fp32 accumulators in tensor memory), the
+// T x 16 indexer query heads the N side (16..128), the 64 dims K (four K = 16
+// steps).  The 16 warps are alike: warps w, w + 4, w + 8, w + 12 own the same 32
+// key rows (TMEM lanes 32 (w % 4) ..), and warp w, part p = w / 4, works on
+//   - (FP8 keys) the p-th quarter of every such row's 64 E4M3 codes (TMA tile
+//     with a 64-byte swizzle), widened exactly into bf16 straight into 8 columns
+//     of the tile's tensor-memory A buffer; bf16 keys arrive from TMA already as
+//     the shared-memory A operand (128-byte swizzle);
+//   - the epilogue of queries [p T / 4, (p + 1) T / 4): ReLU, head weights, a
+//     fixed-order sum over the 16 heads, the per-token scale; the fp32 score
+//     goes to global memory, and each thread keeps the largest key it has seen
+//     per query.
 // Every warp marks its share of a tile done on an mbarrier; tile j's MMAs (and
-// the TMA refill of the stage they free) are issued by warp j % 8, at the end of
-// its iteration two tiles earlier, so that the issue (a thread blocks while the
-// tensor core takes the instructions) rotates over the warps and its wait for
-// the other shares is long satisfied.  Otherwise warps wait only for data: a
+// the TMA refill of the stage they free) are issued by warp j % 16, at the end
+// of its iteration two tiles earlier, so that the issue (a thread blocks while
+// the tensor core takes the instructions) rotates over the warps and its wait
+// for the other shares is long satisfied.  Otherwise warps wait only for data: a
 // TMA stage to land, an accumulator to be complete.  Tensor memory: three
 // accumulator buffers of 128 columns and four A buffers of 32 columns.
 //
@@ -389,12 +392,16 @@ __device__ void radix_pass(ForEach for_each_key, uint32_t& lo, uint32_t& hi, uin
 // query, b* sits near the top 2048 / 18944 of the pair maxima, so for scores
 // without heavy ties the candidates number little more than topk.
 // ==================================================================================
+constexpr int kIdxThreads = 512;
+constexpr int kIdxWarps = kIdxThreads / 32;
+constexpr int kIdxParts = kIdxWarps / 4;     // warps per TMEM lane quarter
 constexpr int kRawStagesF8 = 8, kRawStagesBf = 6;
 constexpr int kAccBufs = 3, kABufs = 4;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kACol = kAccBufs * 128;   // first column of the A buffers
 constexpr int kTileBytesBf16 = kKeyTile * kDI * 2;   // 16 KiB, one 128 x 64 bf16 operand tile
-constexpr int kIdxCounters = 16;             // shared words: counters and issue marks
+constexpr int kIdxCounters = 16;             // shared words: issue marks
+static_assert(kIdxParts == 4 && kDI / kIdxParts == 16, "one 16-code chunk of a key row per warp");
 static_assert(kACol + kABufs * 32 <= kTmemCols, "tensor memory budget");
 static_assert(kRawStagesF8 * kKeyTile * kDI + kTileBytesBf16 + kMaxT * kHI * 4 + kHistWords * 2 + kIdxCounters * 4 <=
                   kDataBytes,
@@ -406,19 +413,6 @@ static_assert(kRawStagesBf * kTileBytesBf16 + kTileBytesBf16 + kMaxT * kHI * 4 +
 __device__ __forceinline__ void red_max_shared(uint32_t* a, uint32_t v)
 {
     asm volatile("red.shared::cta.max.u32 [%0], %1;" ::"r"(smem_u32(a)), "r"(v) : "memory");
-}
-
-// The block's 16-bit counters (two per word) added to the launch's histogram.
-__device__ __forceinline__ void flush_hist16(const uint32_t* hs, int T)
-{
-    for (int i = threadIdx.x; i < T * (kHistBins / 2); i += kThreads) {
-        const uint32_t v = hs[i];
-        if (v) {
-            uint32_t* gh = g_view.hist + (i / (kHistBins / 2)) * kHistBins + 2 * (i % (kHistBins / 2));
-            if (v & 0xFFFFu) atomicAdd(gh, v & 0xFFFFu);
-            if (v >> 16) atomicAdd(gh + 1, v >> 16);
-        }
-    }
 }
 
 // Everything a warp of the indexer needs.
@@ -494,59 +488,60 @@ struct IndexTile {
         if (f + S < c.nloc) load(c, f + S);
         return true;
     }
-    // FP8: this warp's half of its 32 key rows of tile j widened into the A buffer.
-    // False if the wait for the data ran out.
-    __device__ static bool convert(const IndexCtx& c, int j, int row, int half, uint32_t lane_base, uint32_t* err)
+    // FP8: this warp's quarter of its 32 key rows of tile j widened into the A
+    // buffer.  False if the wait for the data ran out.
+    __device__ static bool convert(const IndexCtx& c, int j, int row, int part, uint32_t lane_base, uint32_t* err)
     {
         const int stage = j % S;
         if (__any_sync(0xffffffffu, !mbar_wait(&c.raw_full[stage], (j / S) & 1, err))) return false;
-        const uint8_t* src = c.ring + stage * kRawBytes + row * 64;   // 16-byte chunk q stored at q ^ ((row >> 1) & 3)
-        uint4 v[2];
-#pragma unroll
-        for (int q = 0; q < 2; ++q) v[q] = *reinterpret_cast<const uint4*>(src + (((2 * half + q) ^ ((row >> 1) & 3)) << 4));
-        uint32_t r[16];
-#pragma unroll
-        for (int q = 0; q < 2; ++q) {
-            e4m3x4_to_bf16x4(v[q].x, r[8 * q + 0], r[8 * q + 1]);
-            e4m3x4_to_bf16x4(v[q].y, r[8 * q + 2], r[8 * q + 3]);
-            e4m3x4_to_bf16x4(v[q].z, r[8 * q + 4], r[8 * q + 5]);
-            e4m3x4_to_bf16x4(v[q].w, r[8 * q + 6], r[8 * q + 7]);
-        }
-        tmem_st16(c.tmem + lane_base + kACol + (j % kABufs) * 32 + half * 16, r);
+        // 16-byte chunk q of the row is stored at chunk q ^ ((row >> 1) & 3)
+        const uint4 v = *reinterpret_cast<const uint4*>(c.ring + stage * kRawBytes + row * 64 +
+                                                        ((part ^ ((row >> 1) & 3)) << 4));
+        uint32_t r[8];
+        e4m3x4_to_bf16x4(v.x, r[0], r[1]);
+        e4m3x4_to_bf16x4(v.y, r[2], r[3]);
+        e4m3x4_to_bf16x4(v.z, r[4], r[5]);
+        e4m3x4_to_bf16x4(v.w, r[6], r[7]);
+        tmem_st8(c.tmem + lane_base + kACol + (j % kABufs) * 32 + part * 8, r);
         tmem_st_wait();
         return true;
     }
 };
 
-// Math of one tile for this warp's queries (NQ >= nq of them, a compile-time
-// bound so that the code is straight-line) from the accumulator registers.
-template <int NQ>
-__device__ __forceinline__ void index_math(const IndexCtx& c, const StepParams& p, const uint32_t (&r)[NQ > 2 ? 2 : 1][32],
-                                           int s, float scale, const int (&pos_q)[4], uint32_t (&kmax)[4])
+// Math of one tile for this warp's queries (NQ of them, a compile-time count so
+// that the code is straight-line) from the accumulator registers.  w holds half
+// of each head weight: ReLU(x) w = (x + |x|) (w / 2) exactly (x + |x| is 2x or
+// +0, both exact; halving w is exact), so each head costs one add (with the
+// absolute value as an operand modifier) and half a packed FMA, all on the FMA
+// pipe, with the very rounding of fma(max(x, 0), w, acc).  FULL: every key of
+// the tile is in range and visible to the warp's queries (no per-key tests).
+template <int NQ, bool FULL>
+__device__ __forceinline__ void index_math(const StepParams& p, const uint32_t (&r)[32], const float4 (&w)[NQ][4],
+                                           int s, float scale, const int (&pos_q)[2], float* const (&out)[2],
+                                           float (&mx)[2])
 {
-    float4 w[NQ][4];
-#pragma unroll
-    for (int u = 0; u < NQ; ++u)
-#pragma unroll
-        for (int k = 0; k < 4; ++k) w[u][k] = reinterpret_cast<const float4*>(c.w_s + (c.qa + u) * kHI)[k];
 #pragma unroll
     for (int u = 0; u < NQ; ++u) {
         // Four partial sums over heads {j, j+4, j+8, j+12}, j < 4, as two packed fp32
         // FMAs per four heads, combined in a fixed order.
-        const float* v = reinterpret_cast<const float*>(&r[u >> 1][(u & 1) * 16]);
+        const float* v = reinterpret_cast<const float*>(&r[u * 16]);
         float2 p01 = make_float2(0.f, 0.f), p23 = make_float2(0.f, 0.f);
 #pragma unroll
         for (int g4 = 0; g4 < 4; ++g4) {
-            p01 = __ffma2_rn(make_float2(fmaxf(v[g4 * 4 + 0], 0.f), fmaxf(v[g4 * 4 + 1], 0.f)),
-                             make_float2(w[u][g4].x, w[u][g4].y), p01);
-            p23 = __ffma2_rn(make_float2(fmaxf(v[g4 * 4 + 2], 0.f), fmaxf(v[g4 * 4 + 3], 0.f)),
-                             make_float2(w[u][g4].z, w[u][g4].w), p23);
+            const float* x = v + g4 * 4;
+            p01 = __ffma2_rn(make_float2(x[0] + fabsf(x[0]), x[1] + fabsf(x[1])), make_float2(w[u][g4].x, w[u][g4].y),
+                             p01);
+            p23 = __ffma2_rn(make_float2(x[2] + fabsf(x[2]), x[3] + fabsf(x[3])), make_float2(w[u][g4].z, w[u][g4].w),
+                             p23);
         }
         const float acc = ((p01.x + p01.y) + (p23.x + p23.y)) * scale;
-        if (u < c.nq && s < p.L) {
+        if (FULL) {
+            out[u][s] = acc;
+            mx[u] = fmaxf(mx[u], acc);
+        } else if (s < p.L) {
             const bool vis = s <= pos_q[u];
-            p.scores[(int64_t)(c.qa + u) * p.ld + s] = vis ? acc : -INFINITY;
-            if (vis) kmax[u] = max(kmax[u], score_key(acc));
+            out[u][s] = vis ? acc : -INFINITY;
+            if (vis) mx[u] = fmaxf(mx[u], acc);
         }
     }
 }
@@ -559,7 +554,7 @@ __device__ void phase_index(const CUtensorMap& kmap, const StepParams& p, uint8_
     constexpr int S = Tile::S;
     constexpr int raw_bytes = Tile::kRawBytes;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int quad = warp & 3, half = warp >> 2;     // TMEM lane quarter; which half of the row / queries
+    const int quad = warp & 3, part = warp >> 2;     // TMEM lane quarter; which quarter of the row / queries
     const int T = p.T;
     const int ntiles = (visible_max(p) + kKeyTile - 1) / kKeyTile;
 
@@ -575,8 +570,8 @@ __device__ void phase_index(const CUtensorMap& kmap, const StepParams& p, uint8_
     c.kmap = &kmap;
     c.policy = l2_evict_first_policy();   // keys are read once; the scores stay in L2
     c.nloc = ntiles > static_cast<int>(blockIdx.x) ? (ntiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
-    c.qa = half == 0 ? 0 : (T + 1) >> 1;
-    c.nq = half == 0 ? (T + 1) >> 1 : T >> 1;
+    c.qa = part * T / kIdxParts;
+    c.nq = (part + 1) * T / kIdxParts - c.qa;        // 0, 1 or 2
     const bool hist = g_view.hist != nullptr;
     uint64_t* setup = bars + kBarSetup;
     float* w_s = const_cast<float*>(c.w_s);
@@ -585,7 +580,7 @@ __device__ void phase_index(const CUtensorMap& kmap, const StepParams& p, uint8_
         prefetch_tmap(&kmap);
         for (int s = 0; s < S; ++s) mbar_init(&c.raw_full[s], 1);
         for (int b = 0; b < kAccBufs; ++b) mbar_init(&c.acc_full[b], 1);
-        for (int b = 0; b < Tile::kShareBufs; ++b) mbar_init(&c.share[b], kWarps);
+        for (int b = 0; b < Tile::kShareBufs; ++b) mbar_init(&c.share[b], kIdxWarps);
         mbar_init(setup, 1);
         fence_mbar_init();
         mbar_arrive_expect_tx(setup, T * kHI * 4);
@@ -596,20 +591,20 @@ __device__ void phase_index(const CUtensorMap& kmap, const StepParams& p, uint8_
     // The indexer queries as the B operand: row r = t*16 + j, 16-byte chunk k at
     // r*128 + (k ^ (r & 7))*16 (the 128B swizzle); rows >= T*16 are never read.
     {
-        uint4 v[kMaxT * kHI * 8 / kThreads];   // every load in flight before the first store
+        uint4 v[kMaxT * kHI * 8 / kIdxThreads];   // every load in flight before the first store
 #pragma unroll
-        for (int u = 0; u < kMaxT * kHI * 8 / kThreads; ++u) {
-            const int i = tid + u * kThreads;
+        for (int u = 0; u < kMaxT * kHI * 8 / kIdxThreads; ++u) {
+            const int i = tid + u * kIdxThreads;
             v[u] = i < T * kHI * 8 ? __ldg(reinterpret_cast<const uint4*>(p.q_idx) + i) : make_uint4(0u, 0u, 0u, 0u);
         }
 #pragma unroll
-        for (int u = 0; u < kMaxT * kHI * 8 / kThreads; ++u) {
-            const int i = tid + u * kThreads, r = i >> 3, k = i & 7;
+        for (int u = 0; u < kMaxT * kHI * 8 / kIdxThreads; ++u) {
+            const int i = tid + u * kIdxThreads, r = i >> 3, k = i & 7;
             if (i < T * kHI * 8) *reinterpret_cast<uint4*>(c.qsw + r * 128 + ((k ^ (r & 7)) << 4)) = v[u];
         }
     }
     if (hist)
-        for (int i = tid; i < kHistWords / 2; i += kThreads) c.hs[i] = 0u;
+        for (int i = tid; i < kHistWords / 2; i += kIdxThreads) c.hs[i] = 0u;
     fence_proxy_async_smem();   // the queries are read by the tensor cores (async proxy)
     tc_fence_before();
     __syncthreads();
@@ -630,29 +625,43 @@ __device__ void phase_index(const CUtensorMap& kmap, const StepParams& p, uint8_
         }
     }
     aborted = __any_sync(0xffffffffu, aborted || !mbar_wait(setup, 0, p.err));   // warp-uniform from here on
-    int pos_q[4];                                    // positions of this warp's queries
+    int pos_q[2];                                    // positions of this warp's queries
+    float* out[2];                                   // their score rows
+    float mx[2] = {NAN, NAN};                        // largest score seen per query (NaN: none yet)
+    int pos_min = p.L;                               // tiles wholly below it and below L need no tests
 #pragma unroll
-    for (int u = 0; u < 4; ++u) pos_q[u] = u < c.nq ? query_pos_rt(p, c.qa + u) : -1;
-    uint32_t kmax[4] = {0u, 0u, 0u, 0u};             // largest key seen per query (0: none)
+    for (int u = 0; u < 2; ++u) {
+        pos_q[u] = u < c.nq ? query_pos_rt(p, c.qa + u) : -1;
+        out[u] = p.scores + (int64_t)min(c.qa + u, T - 1) * p.ld;
+        if (u < c.nq) pos_min = min(pos_min, pos_q[u] + 1);
+    }
 
     auto run = [&](auto nq_tag) {
         constexpr int NQ = decltype(nq_tag)::value;
+        float4 w[NQ > 0 ? NQ : 1][4];   // half of this warp's head weights, for every tile
+#pragma unroll
+        for (int u = 0; u < NQ; ++u)
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const float4 h = reinterpret_cast<const float4*>(c.w_s + (c.qa + u) * kHI)[k];
+                w[u][k] = make_float4(0.5f * h.x, 0.5f * h.y, 0.5f * h.z, 0.5f * h.w);
+            }
         const bool scaled = p.scale != nullptr;
         float scale_next = 1.0f;
         if (NQ > 0 && scaled && c.nloc > 0) {
             const int s = Tile::tile_of(0) * kKeyTile + row;
             scale_next = s < p.L ? __ldg(p.scale + s) : 1.0f;
         }
-        // Tile j's MMAs go out from warp j % 8 at the end of its iteration j - 2 (FP8:
+        // Tile j's MMAs go out from warp j % 16 at the end of its iteration j - 2 (FP8:
         // tiles 0 and 1 here; bf16: tiles 0..2 went out with the first loads).
         auto issue_by_me = [&](int j) -> bool {
             bool ok = true;
-            if (j < c.nloc && (FP8 || j >= kAccBufs) && warp == j % kWarps && lane == 0) ok = Tile::issue(c, j, p.err);
+            if (j < c.nloc && (FP8 || j >= kAccBufs) && warp == j % kIdxWarps && lane == 0) ok = Tile::issue(c, j, p.err);
             return !__any_sync(0xffffffffu, !ok);
         };
         if constexpr (FP8) {
             for (int j = 0; j < 2 && j < c.nloc && !aborted; ++j) {
-                aborted = !Tile::convert(c, j, row, half, lane_base, p.err);
+                aborted = !Tile::convert(c, j, row, part, lane_base, p.err);
                 if (!aborted) {
                     Tile::done(c, j, lane);
                     aborted = !issue_by_me(j);
@@ -674,14 +683,10 @@ __device__ void phase_index(const CUtensorMap& kmap, const StepParams& p, uint8_
                 break;
             }
             tc_fence_after();
-            uint32_t r[NQ > 2 ? 2 : 1][32];
-            if constexpr (NQ > 0) {
-                const uint32_t tbase = c.tmem + lane_base + cb * 128 + c.qa * kHI;
-                tmem_ld32_nowait(tbase, r[0]);
-                if constexpr (NQ > 2) tmem_ld32_nowait(tbase + 32, r[1]);
-            }
+            uint32_t r[32];
+            if constexpr (NQ > 0) tmem_ld32_nowait(c.tmem + lane_base + cb * 128 + c.qa * kHI, r);
             if (FP8 && e + 2 < c.nloc) {
-                if (!Tile::convert(c, e + 2, row, half, lane_base, p.err)) {
+                if (!Tile::convert(c, e + 2, row, part, lane_base, p.err)) {
                     aborted = true;
                     break;
                 }
@@ -690,10 +695,11 @@ __device__ void phase_index(const CUtensorMap& kmap, const StepParams& p, uint8_
             if constexpr (NQ > 0) {
                 tmem_ld_wait();
 #pragma unroll
-                for (int h = 0; h < (NQ > 2 ? 2 : 1); ++h)
-#pragma unroll
-                    for (int k = 0; k < 32; ++k) asm volatile("" : "+r"(r[h][k]));   // no use before the wait
-                index_math<NQ>(c, p, r, s, scale, pos_q, kmax);
+                for (int k = 0; k < 32; ++k) asm volatile("" : "+r"(r[k]));   // no use before the wait
+                if (Tile::tile_of(e) * kKeyTile + kKeyTile <= pos_min)
+                    index_math<NQ, true>(p, r, w, s, scale, pos_q, out, mx);
+                else
+                    index_math<NQ, false>(p, r, w, s, scale, pos_q, out, mx);
             }
             if constexpr (!FP8) Tile::done(c, e, lane);   // tile e's accumulator is read
             if (!issue_by_me(e + 2)) {
@@ -702,9 +708,7 @@ __device__ void phase_index(const CUtensorMap& kmap, const StepParams& p, uint8_
             }
         }
     };
-    if (c.nq > 2) {
-        run(std::integral_constant<int, 4>{});
-    } else if (c.nq == 2) {
+    if (c.nq == 2) {
         run(std::integral_constant<int, 2>{});
     } else if (c.nq == 1) {
         run(std::integral_constant<int, 1>{});
@@ -736,18 +740,26 @@ __device__ void phase_index(const CUtensorMap& kmap, const StepParams& p, uint8_
     if (hist) {
         // one count per (thread, query): its largest key's bin
 #pragma unroll
-        for (int u = 0; u < 4; ++u)
-            if (u < c.nq && kmax[u] != 0u)
-                atomicAdd(&c.hs[(c.qa + u) * (kHistBins / 2) + (kmax[u] >> (kHistShift + 1))],
-                          1u << (((kmax[u] >> kHistShift) & 1u) << 4));
+        for (int u = 0; u < 2; ++u)
+            if (u < c.nq && !isnan(mx[u])) {
+                const uint32_t k = score_key(mx[u]);
+                atomicAdd(&c.hs[(c.qa + u) * (kHistBins / 2) + (k >> (kHistShift + 1))], 1u << (((k >> kHistShift) & 1u) << 4));
+            }
         __syncthreads();
-        flush_hist16(c.hs, T);   // the block's counters into the launch's histogram
+        // the block's 16-bit counters (two per word) into the launch's histogram
+        for (int i = tid; i < T * (kHistBins / 2); i += kIdxThreads) {
+            const uint32_t v = c.hs[i];
+            if (v) {
+                uint32_t* gh = g_view.hist + (i / (kHistBins / 2)) * kHistBins + 2 * (i % (kHistBins / 2));
+                if (v & 0xFFFFu) atomicAdd(gh, v & 0xFFFFu);
+                if (v >> 16) atomicAdd(gh + 1, v >> 16);
+            }
+        }
     }
     // Positions no query can see (s >= n_max): -inf, as the stage contract states.
     const int64_t tail0 = (int64_t)ntiles * kKeyTile;
-    for (int64_t s = tail0 + (int64_t)blockIdx.x * kThreads + tid; s < p.L; s += (int64_t)gridDim.x * kThreads)
+    for (int64_t s = tail0 + (int64_t)blockIdx.x * kIdxThreads + tid; s < p.L; s += (int64_t)gridDim.x * kIdxThreads)
         for (int tt = 0; tt < T; ++tt) p.scores[(int64_t)tt * p.ld + s] = -INFINITY;
-    __syncthreads();
 }
 
 // Phase 1 for caller-provided scores: the histogram of their keys' top 12 bits,
@@ -837,7 +849,7 @@ __device__ void phase_extract(const StepParams& p, uint8_t* smem, uint64_t* bars
         // bin and above, those above it all selected.  Indexer histogram of per-thread
         // maxima (a lower bound): every key of bin >= b* is a candidate, to be
         // radix-selected from the top; with fewer than topk counts, every visible key.
-        const bool bound = (p.phases & kPhaseIndex) != 0;
+        const bool bound = p.hist_bound != 0;
         uint32_t cut = 0u, above = 0u, top = 0xFFFFFFFFu;
         if (res[2]) {
             cut = res[0] << kHistShift;
@@ -1409,26 +1421,15 @@ __device__ void phase_merge(const StepParams& p)
 }
 
 // ==================================================================================
-template <bool FP8>
-__global__ void __launch_bounds__(kThreads, 1) step_kernel(const __grid_constant__ CUtensorMap kmap, const StepParams p)
+// Launch view: the histogram buffer of this launch's epoch (when the launch
+// counts one), and the query positions when they come from device memory (so
+// that one CUDA graph of the step serves every decode position; a position
+// outside [0, L) is clamped and flagged).  Returns the epoch (thread 0).
+__device__ uint32_t init_launch_view(const StepParams& p, bool counts)
 {
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kBarOffset);
-    __shared__ uint32_t scratch[64];
-    __shared__ uint32_t res[3];
-    __shared__ int ok_s;
-    __shared__ uint32_t tmem_slot;
-    __shared__ uint32_t epoch_s;
-
-    // Launch view: the histogram buffer of this launch's epoch, and the query
-    // positions when they come from device memory (so that one CUDA graph of the
-    // step serves every decode position; a position outside [0, L) is clamped and
-    // flagged).
+    uint32_t e = 0u;
     if (threadIdx.x == 0) {
-        const uint32_t e = p.ctrl != nullptr ? *reinterpret_cast<volatile uint32_t*>(p.ctrl + kCtrlWordEpoch) : 0u;
-        epoch_s = e;
-        const bool counts = (p.phases & (kPhaseIndex | kPhaseHistScores)) && (p.phases & kPhaseTopk);
+        e = p.ctrl != nullptr ? *reinterpret_cast<volatile uint32_t*>(p.ctrl + kCtrlWordEpoch) : 0u;
         g_view.hist = counts && p.ctrl != nullptr ? p.ctrl + kCtrlBytes / 4 + (e & 1u) * kHistWords : nullptr;
     }
     if (p.pos_dev != nullptr && threadIdx.x < 32) {
@@ -1446,6 +1447,41 @@ __global__ void __launch_bounds__(kThreads, 1) step_kernel(const __grid_constant
         for (int o = 16; o > 0; o >>= 1) n = max(n, __shfl_xor_sync(0xffffffffu, n, o));
         if (threadIdx.x == 0) g_view.n_max = n;
     }
+    return e;
+}
+
+// The indexer stage as a kernel of its own: one block per SM, 16 warps.  With a
+// workspace it also counts the first radix pass into the launch's histogram.
+template <bool FP8>
+__global__ void __launch_bounds__(kIdxThreads, 1) index_kernel(const __grid_constant__ CUtensorMap kmap, const StepParams p)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kBarOffset);
+    __shared__ uint32_t tmem_slot;
+    init_launch_view(p, p.hist_bound != 0);
+    __syncthreads();
+    stamp(p, 0);
+    if (p.trace != nullptr && threadIdx.x == 0) p.trace[(int64_t)blockIdx.x * kTraceSlots + 28] = clock64();
+    phase_index<FP8>(kmap, p, smem, bars, &tmem_slot);
+    __syncthreads();
+    stamp(p, 1);
+}
+
+// Stages 2 and 3 (and the first radix pass of caller-provided scores): one
+// cooperative launch, one block per SM.
+__global__ void __launch_bounds__(kThreads, 1) step_kernel(const StepParams p)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kBarOffset);
+    __shared__ uint32_t scratch[64];
+    __shared__ uint32_t res[3];
+    __shared__ int ok_s;
+    __shared__ uint32_t epoch_s;
+
+    const uint32_t e = init_launch_view(p, (p.phases & kPhaseTopk) && (p.hist_bound || (p.phases & kPhaseHistScores)));
+    if (threadIdx.x == 0) epoch_s = e;
     __syncthreads();
     // The other histogram buffer starts the next launch at zero.
     if (p.ctrl != nullptr) {
@@ -1454,20 +1490,19 @@ __global__ void __launch_bounds__(kThreads, 1) step_kernel(const __grid_constant
     }
 
     GridBarrier gb{p.ctrl, gridDim.x};
-    // Stamps (when tracing): 0 start, 1 indexer done, 2 extraction start (after
-    // the barrier), 3 extraction done, 4/5 selection (blocks < T), 6 first
-    // attention item starts, 7 this block's attention items done, 9 its merge
-    // items done, 30 end; 28/29 SM clock.
+    // Stamps (when tracing): 0 start and 1 first stage done (the indexer kernel's
+    // when it ran), 2 extraction start (after the barrier), 3 extraction done, 4/5
+    // selection (blocks < T), 6 first attention item starts, 7 this block's
+    // attention items done, 9 its merge items done, 30 end; 28/29 SM clock.
     bool ok = true;
     if (p.ctrl != nullptr) gb.enter();
-    stamp(p, 0);
-    if (p.trace != nullptr && threadIdx.x == 0) p.trace[(int64_t)blockIdx.x * kTraceSlots + 28] = clock64();
-    if (p.phases & kPhaseIndex) {
-        phase_index<FP8>(kmap, p, smem, bars, &tmem_slot);
-    } else if (p.phases & kPhaseHistScores) {
-        phase_hist_scores(p, smem);
+    const bool own_first = !p.hist_bound;   // no indexer kernel ran before this one
+    if (own_first) {
+        stamp(p, 0);
+        if (p.trace != nullptr && threadIdx.x == 0) p.trace[(int64_t)blockIdx.x * kTraceSlots + 28] = clock64();
     }
-    stamp(p, 1);
+    if (p.phases & kPhaseHistScores) phase_hist_scores(p, smem);
+    if (own_first) stamp(p, 1);
     if (p.phases & kPhaseTopk) {
         ok = gb.sync(p, &ok_s);
         stamp(p, 2);
@@ -1494,7 +1529,7 @@ __global__ void __launch_bounds__(kThreads, 1) step_kernel(const __grid_constant
     }
 }
 
-bool g_configured[64][2] = {};
+bool g_configured[64][3] = {};
 
 }  // namespace
 
@@ -1504,11 +1539,28 @@ cudaError_t launch_step(const CUtensorMap* kmap, const StepParams& p, bool fp8, 
 {
     int dev = 0;
     cudaGetDevice(&dev);
-    auto kern = fp8 ? step_kernel<true> : step_kernel<false>;
-    if (dev >= 0 && dev < 64 && !g_configured[dev][fp8]) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kStepSmem);
+    const bool cache = dev >= 0 && dev < 64;
+    if (p.phases & kPhaseIndex) {
+        auto kern = fp8 ? index_kernel<true> : index_kernel<false>;
+        if (!cache || !g_configured[dev][fp8]) {
+            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kStepSmem);
+            if (e != cudaSuccess) return e;
+            if (cache) g_configured[dev][fp8] = true;
+        }
+        StepParams q = p;
+        q.hist_bound = (p.phases & kPhaseTopk) != 0 ? 1 : 0;
+        kern<<<p.grid, kIdxThreads, kStepSmem, s>>>(*kmap, q);
+        cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
-        g_configured[dev][fp8] = true;
+    }
+    StepParams q = p;
+    q.phases &= ~kPhaseIndex;
+    q.hist_bound = (p.phases & kPhaseIndex) != 0 && (p.phases & kPhaseTopk) != 0 ? 1 : 0;
+    if (q.phases == 0) return cudaSuccess;
+    if (!cache || !g_configured[dev][2]) {
+        cudaError_t e = cudaFuncSetAttribute(step_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kStepSmem);
+        if (e != cudaSuccess) return e;
+        if (cache) g_configured[dev][2] = true;
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(p.grid, 1, 1);
@@ -1520,17 +1572,18 @@ cudaError_t launch_step(const CUtensorMap* kmap, const StepParams& p, bool fp8, 
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, *kmap, p);
+    return cudaLaunchKernelEx(&cfg, step_kernel, q);
 }
 
 int step_max_blocks(bool fp8)
 {
+    (void)fp8;
     int dev = 0, sms = 0, n = 0;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    auto kern = fp8 ? step_kernel<true> : step_kernel<false>;
-    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kStepSmem);
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, kThreads, kStepSmem) != cudaSuccess || n < 1) n = 1;
+    cudaFuncSetAttribute(step_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kStepSmem);
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, step_kernel, kThreads, kStepSmem) != cudaSuccess || n < 1)
+        n = 1;
     cudaGetLastError();
     return sms * (n > 1 ? 1 : n);   // one block per SM
 }
