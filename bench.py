@@ -440,7 +440,8 @@ def main():
         spans = {"indexer": span(0, 1), "barrier": span(1, 2), "topk_extract": span(2, 3),
                  "topk_select": span(4, 5), "attention": span(6, 7), "merge": span(8, 9)}
         spans["kernel"] = span(0, 30)
-        spans["sm_mhz_in_kernel"] = float((t[0, 29] - t[0, 28]) / max(1, t[0, 30] - t[0, 0]) * 1e3)
+        # SM clock over the last kernel of the step (its own start: clock 27, time 31)
+        spans["sm_mhz_in_kernel"] = float((t[0, 29] - t[0, 27]) / max(1, t[0, 30] - t[0, 31]) * 1e3)
         spans["start_skew"] = (t[:, 0].max() - t[:, 0].min()) / 1e3
         return spans
 

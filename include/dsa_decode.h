@@ -270,11 +270,13 @@ DSA_API dsa_status_t dsa_debug_fail_next_barriers(int64_t limit_cycles);
 /* Profiling hook for the calling host thread: when device_buffer is not NULL,
  * every launch records, per block b and slot k < 32, the GPU global timer (ns)
  * into ((uint64_t*)device_buffer)[b * 32 + k] at the phase boundaries of the
- * step: 0 start, 1 indexer scan done, 2/3 candidate extraction (after the
- * grid barrier), 4/5 the per-query selection (blocks 0..T-1 only), 6 first
+ * step: 0 start, 1 indexer scan done (both from the indexer kernel when it
+ * runs), 31 start of the cooperative kernel, 2/3 candidate extraction (after
+ * its grid barrier), 4/5 the per-query selection (blocks 0..T-1 only), 6 first
  * attention item starts (after its query's selection), 7 attention done, 8/9
- * merge, 30 end; slots 28/29 hold the SM clock counter at start and end.  The buffer must hold dsa_step_grid(...) * 32 entries.  NULL
- * disables. */
+ * merge, 30 end; slots 28, 27 and 29 hold the SM clock counter at the start of
+ * the first kernel, at the start of the cooperative kernel and at the end.  The
+ * buffer must hold dsa_step_grid(...) * 32 entries.  NULL disables. */
 DSA_API void dsa_set_step_trace(void *device_buffer);
 
 /* Blocks of the step kernel on the current device (one per SM); 0 on error. */

@@ -1459,6 +1459,9 @@ __global__ void __launch_bounds__(kIdxThreads, 1) index_kernel(const __grid_cons
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kBarOffset);
     __shared__ uint32_t tmem_slot;
+    // the cooperative kernel that consumes the scores may be launched now: its
+    // blocks take the SMs this grid leaves and wait for its completion
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     init_launch_view(p, p.hist_bound != 0);
     __syncthreads();
     stamp(p, 0);
@@ -1493,9 +1496,17 @@ __global__ void __launch_bounds__(kThreads, 1) step_kernel(const StepParams p)
     // Stamps (when tracing): 0 start and 1 first stage done (the indexer kernel's
     // when it ran), 2 extraction start (after the barrier), 3 extraction done, 4/5
     // selection (blocks < T), 6 first attention item starts, 7 this block's
-    // attention items done, 9 its merge items done, 30 end; 28/29 SM clock.
+    // attention items done, 9 its merge items done, 30 end, 31 this kernel's
+    // start; SM clock: 28 first kernel's start, 27 this kernel's start, 29 end.
     bool ok = true;
     if (p.ctrl != nullptr) gb.enter();
+    // Launched as a programmatic dependent of the indexer kernel: everything above
+    // touches nothing that grid writes; its scores and histogram are read below.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (p.trace != nullptr && threadIdx.x == 0) {   // this kernel's own start: SM clock and time
+        p.trace[(int64_t)blockIdx.x * kTraceSlots + 27] = clock64();
+        stamp(p, 31);
+    }
     const bool own_first = !p.hist_bound;   // no indexer kernel ran before this one
     if (own_first) {
         stamp(p, 0);
@@ -1530,6 +1541,7 @@ __global__ void __launch_bounds__(kThreads, 1) step_kernel(const StepParams p)
 }
 
 bool g_configured[64][3] = {};
+bool g_no_pdl[64] = {};
 
 }  // namespace
 
@@ -1567,12 +1579,24 @@ cudaError_t launch_step(const CUtensorMap* kmap, const StepParams& p, bool fp8, 
     cfg.blockDim = dim3(kThreads, 1, 1);
     cfg.dynamicSmemBytes = kStepSmem;
     cfg.stream = s;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeCooperative;
     attr[0].val.cooperative = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, step_kernel, q);
+    // after the indexer kernel: a programmatic dependent launch (its launch overlaps
+    // the indexer's tail), unless the device turned that down once
+    const bool pdl = (p.phases & kPhaseIndex) != 0 && !(cache && g_no_pdl[dev]);
+    cfg.numAttrs = pdl ? 2 : 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, step_kernel, q);
+    if (e != cudaSuccess && pdl) {
+        cudaGetLastError();
+        if (cache) g_no_pdl[dev] = true;
+        cfg.numAttrs = 1;
+        e = cudaLaunchKernelEx(&cfg, step_kernel, q);
+    }
+    return e;
 }
 
 int step_max_blocks(bool fp8)
