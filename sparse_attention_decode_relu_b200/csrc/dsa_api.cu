@@ -184,11 +184,12 @@ dsa_status_t check_sel(const dsa_tensor_t* sel, int T, int32_t topk)
 // ------------------------------------------------------------------ workspace
 // Device workspace of one step: the control region (barrier and per-query
 // words, two radix histograms), per-query cuts, per-sub-segment candidate
-// counts, candidate lists, fp32 scores, and the attention splits' partial
-// states.
+// counts, candidate lists, fp32 scores with the largest key of each group of 32
+// positions, and the attention splits' partial states.
 struct Layout {
     int64_t ld = 0;            // score / candidate row stride (elements)
-    size_t ctrl = 0, cuts = 0, seg_n = 0, scores = 0, list = 0, po = 0, pml = 0;
+    int64_t gmax_ld = 0;       // group-maximum row stride (32-position groups)
+    size_t ctrl = 0, cuts = 0, seg_n = 0, scores = 0, gmax = 0, list = 0, po = 0, pml = 0;
     size_t total = 0;
 };
 
@@ -210,7 +211,11 @@ Layout layout(int T, int64_t L, bool with_scores = true, bool with_attn = true)
     l.cuts = take(sizeof(uint32_t) * 4 * kMaxT);
     l.seg_n = take(sizeof(uint32_t) * (size_t)kMaxT * kMaxSeg);
     l.list = take(sizeof(uint2) * (size_t)T * l.ld);
-    if (with_scores) l.scores = take(sizeof(float) * (size_t)T * l.ld);
+    if (with_scores) {
+        l.scores = take(sizeof(float) * (size_t)T * l.ld);
+        l.gmax_ld = round_up(L, kKeyTile) / 32;   // every group of the indexer's tiles
+        l.gmax = take(sizeof(uint32_t) * (size_t)T * l.gmax_ld);
+    }
     if (with_attn) {
         l.po = take(sizeof(float) * (size_t)kMaxT * kMaxSplitsQ * kH * kD);
         l.pml = take(sizeof(float2) * (size_t)kMaxT * kMaxSplitsQ * kH);
@@ -474,6 +479,8 @@ static dsa_status_t decode_ws(const dsa_tensor_t* q, const dsa_tensor_t* q_idx, 
     p.scale = k_idx_cache->scale;
     p.scores = at<float>(workspace, l.scores);
     p.ld = l.ld;
+    p.gmax = at<uint32_t>(workspace, l.gmax);
+    p.gmax_ld = l.gmax_ld;
     p.sel = static_cast<int32_t*>(sel_idx->data);
     p.sel_ld = sel_idx->stride[0];
     p.q = static_cast<const uint16_t*>(q->data);

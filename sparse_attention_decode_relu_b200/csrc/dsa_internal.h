@@ -93,6 +93,8 @@ struct StepParams {
     uint32_t barrier_extra;  // arrivals such a wait needs beyond the real ones (0; 1 = a block that never comes)
     uint32_t* err;
     int32_t hist_bound;      // the first radix histogram holds per-thread key maxima (a lower bound), not every key
+    uint32_t* gmax;          // [T][gmax_ld] largest key of each 32-position group (0: none visible), or nullptr
+    int64_t gmax_ld;
 };
 
 int step_smem_bytes();

@@ -126,26 +126,38 @@ struct GridBarrier {
     }
 };
 
-// Last block out resets every control word but the epoch, and advances the
-// epoch (which histogram buffer the next launch uses).
+// Every block counts itself out (a release add, no round trip); block 0 waits
+// for the whole grid, then resets every control word but the epoch and advances
+// the epoch (which histogram buffer the next launch uses).  A returning atomic
+// on one word from every block serialises for microseconds; this costs one
+// bounded wait in one block.  If that wait runs out the words stay as they are,
+// and the next launch on the workspace reports them.
 __device__ __forceinline__ void barrier_exit(const StepParams& p)
 {
     if (threadIdx.x == 0) {
-        uint32_t old;
-        asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;"
-                     : "=r"(old)
-                     : "l"(p.ctrl + kCtrlWordExit)
-                     : "memory");
-        if (old == gridDim.x - 1u) {
-            p.ctrl[0] = 0u;
-            p.ctrl[kCtrlWordExit] = 0u;
-            for (int t = 0; t < kMaxT; ++t) {
-                p.ctrl[kCtrlWordArrive + t] = 0u;
-                p.ctrl[kCtrlWordReady + t] = 0u;
-                p.ctrl[kCtrlWordDone + t] = 0u;
+        red_release_add(p.ctrl + kCtrlWordExit, 1u);
+        if (blockIdx.x == 0) {
+            const uint32_t* word = p.ctrl + kCtrlWordExit;
+            bool ok = ld_acquire(word) >= gridDim.x;
+            const long long t0 = clock64();
+            while (!ok) {
+                if (clock64() - t0 > kWaitLimitCycles) {   // (not shortened by the test hook)
+                    atomicOr(p.err, ERR_WAIT_TIMEOUT);
+                    break;
+                }
+                ok = ld_acquire(word) >= gridDim.x;
             }
-            p.ctrl[kCtrlWordEpoch] += 1u;
-            __threadfence();
+            if (ok) {
+                p.ctrl[0] = 0u;
+                p.ctrl[kCtrlWordExit] = 0u;
+                for (int t = 0; t < kMaxT; ++t) {
+                    p.ctrl[kCtrlWordArrive + t] = 0u;
+                    p.ctrl[kCtrlWordReady + t] = 0u;
+                    p.ctrl[kCtrlWordDone + t] = 0u;
+                }
+                p.ctrl[kCtrlWordEpoch] += 1u;
+                __threadfence();
+            }
         }
     }
 }
@@ -199,20 +211,25 @@ __device__ __forceinline__ uint32_t warp_incl_scan(uint32_t v)
 }
 
 // Exclusive prefix sum over the block (thread order); `total` gets the sum.
+// One barrier between the warp scans and every thread summing the eight warp
+// totals itself (two 16-byte reads), one more before scratch is reused.
+// scratch: 16-byte aligned.
 __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t& total, uint32_t* scratch)
 {
+    static_assert(kWarps == 8, "two 16-byte reads of warp totals");
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const uint32_t x = warp_incl_scan(v);
     if (lane == 31) scratch[warp] = x;
     __syncthreads();
-    if (warp == 0) {
-        const uint32_t w = lane < kWarps ? scratch[lane] : 0u;
-        const uint32_t wi = warp_incl_scan(w);
-        if (lane < kWarps) scratch[lane] = wi;
+    const uint4 a = reinterpret_cast<const uint4*>(scratch)[0], b = reinterpret_cast<const uint4*>(scratch)[1];
+    const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+    uint32_t before = 0, tot = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        tot += w[i];
+        before += i < warp ? w[i] : 0u;
     }
-    __syncthreads();
-    const uint32_t before = warp ? scratch[warp - 1] : 0u;
-    total = scratch[kWarps - 1];
+    total = tot;
     __syncthreads();
     return before + x - v;
 }
@@ -422,6 +439,8 @@ struct IndexCtx {
     const float* w_s;        // [8][16] head weights
     uint32_t* hs;            // [8][2048] two 16-bit counters per word
     uint32_t* cnt;           // [0] loads issued; [1] MMA groups issued (for the drain after an abort)
+    uint32_t* gmax;          // group maxima of the launch, or nullptr
+    int64_t gmax_ld;
     uint64_t* raw_full;
     uint64_t* acc_full;
     uint64_t* share;         // [kABufs or kAccBufs]: every warp's share of a tile done
@@ -518,7 +537,7 @@ struct IndexTile {
 template <int NQ, bool FULL>
 __device__ __forceinline__ void index_math(const StepParams& p, const uint32_t (&r)[32], const float4 (&w)[NQ][4],
                                            int s, float scale, const int (&pos_q)[2], float* const (&out)[2],
-                                           float (&mx)[2])
+                                           float (&mx)[2], uint32_t (&key)[2])
 {
 #pragma unroll
     for (int u = 0; u < NQ; ++u) {
@@ -535,13 +554,18 @@ __device__ __forceinline__ void index_math(const StepParams& p, const uint32_t (
                              p23);
         }
         const float acc = ((p01.x + p01.y) + (p23.x + p23.y)) * scale;
+        key[u] = 0u;
         if (FULL) {
             out[u][s] = acc;
             mx[u] = fmaxf(mx[u], acc);
+            key[u] = score_key(acc);
         } else if (s < p.L) {
             const bool vis = s <= pos_q[u];
             out[u][s] = vis ? acc : -INFINITY;
-            if (vis) mx[u] = fmaxf(mx[u], acc);
+            if (vis) {
+                mx[u] = fmaxf(mx[u], acc);
+                key[u] = score_key(acc);
+            }
         }
     }
 }
@@ -564,6 +588,8 @@ __device__ void phase_index(const CUtensorMap& kmap, const StepParams& p, uint8_
     c.w_s = reinterpret_cast<const float*>(c.qsw + kTileBytesBf16);
     c.hs = reinterpret_cast<uint32_t*>(c.qsw + kTileBytesBf16 + kMaxT * kHI * 4);
     c.cnt = c.hs + kHistWords / 2;
+    c.gmax = p.gmax;
+    c.gmax_ld = p.gmax_ld;
     c.raw_full = bars + kBarRawFull;
     c.acc_full = bars + kBarAccFull;
     c.share = bars + kBarShare;
@@ -696,10 +722,23 @@ __device__ void phase_index(const CUtensorMap& kmap, const StepParams& p, uint8_
                 tmem_ld_wait();
 #pragma unroll
                 for (int k = 0; k < 32; ++k) asm volatile("" : "+r"(r[k]));   // no use before the wait
+                uint32_t key[2];
                 if (Tile::tile_of(e) * kKeyTile + kKeyTile <= pos_min)
-                    index_math<NQ, true>(p, r, w, s, scale, pos_q, out, mx);
+                    index_math<NQ, true>(p, r, w, s, scale, pos_q, out, mx, key);
                 else
-                    index_math<NQ, false>(p, r, w, s, scale, pos_q, out, mx);
+                    index_math<NQ, false>(p, r, w, s, scale, pos_q, out, mx, key);
+                if (c.gmax != nullptr) {
+                    // the largest key of this warp's 32 positions per query (lane u stores
+                    // query u's): lets the extraction skip groups below its cut
+                    uint32_t mine = 0u;
+#pragma unroll
+                    for (int u = 0; u < NQ; ++u) {
+                        const uint32_t m = __reduce_max_sync(0xffffffffu, key[u]);
+                        if (lane == u) mine = m;
+                    }
+                    if (lane < NQ)
+                        c.gmax[(int64_t)(c.qa + lane) * c.gmax_ld + Tile::tile_of(e) * (kKeyTile / 32) + quad] = mine;
+                }
             }
             if constexpr (!FP8) Tile::done(c, e, lane);   // tile e's accumulator is read
             if (!issue_by_me(e + 2)) {
@@ -868,47 +907,197 @@ __device__ void phase_extract(const StepParams& p, uint8_t* smem, uint64_t* bars
         const float* row = p.scores + (int64_t)t * p.ld;
         float* ring = reinterpret_cast<float*>(smem) + warp * kXStages * kXPiece;
         uint2* out = p.list + (int64_t)t * p.list_ld + s0;
-        auto issue = [&](int j) {
-            const int a = s0 + j * kXPiece;
-            const uint32_t bytes = static_cast<uint32_t>((min(kXPiece, s1 - a) + 3) & ~3) * 4u;
-            mbar_arrive_expect_tx(&full[j % kXStages], bytes);
-            bulk_g2s(ring + (j % kXStages) * kXPiece, row + a, bytes, &full[j % kXStages]);
-        };
-        if (lane == 0)
-            for (int j = 0; j < min(np, kXStages); ++j) issue(j);
         uint32_t count = 0;
-        int j = 0;
-        for (; j < np; ++j) {
-            if (__any_sync(0xffffffffu, !mbar_wait(&full[j % kXStages], (j / kXStages) & 1, p.err))) break;
-            const float* buf = ring + (j % kXStages) * kXPiece;
-            const int a = s0 + j * kXPiece;
-#pragma unroll 2
-            for (int k = 0; k < kXPiece / 128; ++k) {
-                const int base = a + k * 128 + lane * 4;
-                const float4 f = *reinterpret_cast<const float4*>(buf + k * 128 + lane * 4);
-                const uint32_t key[4] = {score_key(f.x), score_key(f.y), score_key(f.z), score_key(f.w)};
-                uint32_t m = 0;
+        if (p.gmax != nullptr && bound) {
+            // Only the 32-position groups whose largest key reaches the cut are read:
+            // eight rounds of 32 group maxima in flight per lane, then the hit groups'
+            // scores four at a time, in position order.
+            const uint32_t* gm = p.gmax + (int64_t)t * p.gmax_ld;
+            for (int base = s0; base < s1; base += 8 * 32 * 32) {
+                uint32_t m[8];
 #pragma unroll
-                for (int q = 0; q < 4; ++q) m |= static_cast<uint32_t>(base + q < s1 && key[q] >= cut) << q;
-                if (__ballot_sync(0xffffffffu, m != 0u)) {
-                    const uint32_t my = __popc(m);
-                    const uint32_t incl = warp_incl_scan(my);
-                    uint32_t o = count + incl - my;
+                for (int k = 0; k < 8; ++k) {
+                    const int g = base + (k * 32 + lane) * 32;
+                    m[k] = g < s1 ? __ldcg(gm + g / 32) : 0u;
+                }
 #pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        if (m & (1u << q)) out[o++] = make_uint2(key[q], static_cast<uint32_t>(base + q));
-                    count += __shfl_sync(0xffffffffu, incl, 31);
+                for (int k = 0; k < 8; ++k) {
+                    const int g0 = base + k * 32 * 32;
+                    uint32_t hit = __ballot_sync(0xffffffffu, g0 + lane * 32 < s1 && m[k] >= cut);
+                    while (hit) {
+                        int b[4];
+                        int nb = 0;
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            b[u] = 0;
+                            if (hit) {
+                                b[u] = __ffs(hit) - 1;
+                                hit &= hit - 1u;
+                                nb = u + 1;
+                            }
+                        }
+                        float f[4];
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            const int sp = g0 + b[u] * 32 + lane;
+                            f[u] = (u < nb && sp < s1) ? __ldcg(row + sp) : -INFINITY;
+                        }
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            if (u < nb) {
+                                const int sp = g0 + b[u] * 32 + lane;
+                                const uint32_t key = score_key(f[u]);
+                                const bool take = sp < s1 && key >= cut;
+                                const uint32_t tb = __ballot_sync(0xffffffffu, take);
+                                if (take) out[count + __popc(tb & ((1u << lane) - 1u))] = make_uint2(key, static_cast<uint32_t>(sp));
+                                count += __popc(tb);
+                            }
+                        }
+                    }
                 }
             }
-            __syncwarp();
-            if (lane == 0 && j + kXStages < np) issue(j + kXStages);
+        } else {
+            auto issue = [&](int j) {
+                const int a = s0 + j * kXPiece;
+                const uint32_t bytes = static_cast<uint32_t>((min(kXPiece, s1 - a) + 3) & ~3) * 4u;
+                mbar_arrive_expect_tx(&full[j % kXStages], bytes);
+                bulk_g2s(ring + (j % kXStages) * kXPiece, row + a, bytes, &full[j % kXStages]);
+            };
+            if (lane == 0)
+                for (int j = 0; j < min(np, kXStages); ++j) issue(j);
+            int j = 0;
+            for (; j < np; ++j) {
+                if (__any_sync(0xffffffffu, !mbar_wait(&full[j % kXStages], (j / kXStages) & 1, p.err))) break;
+                const float* buf = ring + (j % kXStages) * kXPiece;
+                const int a = s0 + j * kXPiece;
+#pragma unroll 2
+                for (int k = 0; k < kXPiece / 128; ++k) {
+                    const int base = a + k * 128 + lane * 4;
+                    const float4 f = *reinterpret_cast<const float4*>(buf + k * 128 + lane * 4);
+                    const uint32_t key[4] = {score_key(f.x), score_key(f.y), score_key(f.z), score_key(f.w)};
+                    uint32_t m = 0;
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) m |= static_cast<uint32_t>(base + q < s1 && key[q] >= cut) << q;
+                    if (__ballot_sync(0xffffffffu, m != 0u)) {
+                        const uint32_t my = __popc(m);
+                        const uint32_t incl = warp_incl_scan(my);
+                        uint32_t o = count + incl - my;
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)
+                            if (m & (1u << q)) out[o++] = make_uint2(key[q], static_cast<uint32_t>(base + q));
+                        count += __shfl_sync(0xffffffffu, incl, 31);
+                    }
+                }
+                __syncwarp();
+                if (lane == 0 && j + kXStages < np) issue(j + kXStages);
+            }
+            if (j < np && lane == 0)   // a wait ran out: let the copies in flight land
+                for (int k = j; k < min(np, j + kXStages); ++k) mbar_wait(&full[k % kXStages], (k / kXStages) & 1, p.err);
         }
-        if (j < np && lane == 0)   // a wait ran out: let the copies in flight land
-            for (int k = j; k < min(np, j + kXStages); ++k) mbar_wait(&full[k % kXStages], (k / kXStages) & 1, p.err);
         if (lane == 0) p.seg_n[t * kMaxSeg + c * kSegPerChunk + warp] = count;
     }
     __syncthreads();
     if (tid == 0) red_release_add(p.ctrl + kCtrlWordArrive + t, 1u);
+}
+
+// Candidates held in registers by the selection: up to kSelReg per thread, a
+// contiguous run of the position-ordered list each.
+constexpr int kSelReg = 16;
+
+// One radix pass over the keys in registers (k[u], u < cnt, of every thread):
+// the bin of [lo, hi] (at most 4096 bins of width 2^shift) holding the need-th
+// largest key becomes the new [lo, hi]; need drops by the keys above that bin.
+// Thread i sums bins [4096 - 16 (i + 1), 4096 - 16 i), so one block-wide scan
+// in thread order counts from the top; the thread whose run holds the need-th
+// key finds the bin within its 16.
+__device__ void radix_pass_reg(const uint32_t (&k)[kSelReg], int cnt, uint32_t& lo, uint32_t& hi, uint32_t& need,
+                               uint32_t* h, uint32_t* res, uint32_t* scratch, uint32_t* err)
+{
+    static_assert(kHistBins == 16 * kThreads, "16 bins per thread");
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    // Narrow [lo, hi] to the keys actually in it first: candidate keys cluster in a
+    // few bins of a wide range, and same-address shared atomics serialise.
+    {
+        uint32_t mn = 0xFFFFFFFFu, mx = 0u;
+#pragma unroll
+        for (int u = 0; u < kSelReg; ++u)
+            if (u < cnt && k[u] >= lo && k[u] <= hi) {
+                mn = min(mn, k[u]);
+                mx = max(mx, k[u]);
+            }
+        mn = __reduce_min_sync(0xffffffffu, mn);
+        mx = __reduce_max_sync(0xffffffffu, mx);
+        if (lane == 0) {
+            scratch[32 + warp] = mn;
+            scratch[48 + warp] = mx;
+        }
+        __syncthreads();
+        mn = 0xFFFFFFFFu;
+        mx = 0u;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) {
+            mn = min(mn, scratch[32 + w]);
+            mx = max(mx, scratch[48 + w]);
+        }
+        if (mn <= mx) {   // else no key in range: the search below reports it
+            lo = mn;
+            hi = mx;
+        }
+    }
+    const int shift = range_shift(lo, hi);
+    for (int i = tid; i < kHistBins / 4; i += kThreads) reinterpret_cast<uint4*>(h)[i] = make_uint4(0u, 0u, 0u, 0u);
+    if (tid == 0) res[2] = 0u;
+    __syncthreads();
+#pragma unroll
+    for (int u = 0; u < kSelReg; ++u)
+        if (u < cnt && k[u] >= lo && k[u] <= hi) atomicAdd(&h[(k[u] - lo) >> shift], 1u);
+    __syncthreads();
+    const int b0 = kHistBins - 16 * (tid + 1);
+    uint32_t c[16];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const uint4 v = reinterpret_cast<const uint4*>(h + b0)[q];
+        c[4 * q] = v.x;
+        c[4 * q + 1] = v.y;
+        c[4 * q + 2] = v.z;
+        c[4 * q + 3] = v.w;
+    }
+    uint32_t sum = 0;
+#pragma unroll
+    for (int q = 0; q < 16; ++q) sum += c[q];
+    uint32_t total;
+    const uint32_t before = block_excl_scan(sum, total, scratch);   // keys in the bins above this thread's
+    if (before < need && before + sum >= need) {
+        uint32_t run = before;
+        int bin = -1;
+        uint32_t above = 0;
+#pragma unroll
+        for (int q = 15; q >= 0; --q) {
+            if (bin < 0 && run + c[q] >= need) {
+                bin = b0 + q;
+                above = run;
+            }
+            run += c[q];
+        }
+        res[0] = static_cast<uint32_t>(bin);
+        res[1] = above;
+        res[2] = 1u;
+    }
+    __syncthreads();
+    if (!res[2]) {   // fewer keys in [lo, hi] than needed: inconsistent candidates
+        if (tid == 0) atomicOr(err, ERR_TOPK_STATE);
+        __syncthreads();
+        if (tid == 0) {
+            res[0] = 0u;
+            res[1] = 0u;
+        }
+        __syncthreads();
+    }
+    const uint32_t nlo = lo + (res[0] << shift);
+    hi = bin_top(nlo, shift, hi);
+    lo = nlo;
+    need -= res[1];
+    __syncthreads();
 }
 
 // ==================================================================================
@@ -964,7 +1153,74 @@ __device__ void phase_select(const StepParams& p, uint8_t* smem, uint32_t* res, 
             const uint2* glist = p.list + (int64_t)t * p.list_ld;
             auto seg_cnt = [&](int k) { return (k + 1 < nseg ? off[k + 1] : m) - off[k]; };
             uint32_t nsel = 0;
-            if (m <= static_cast<uint32_t>(kSelCap)) {
+            if (m <= static_cast<uint32_t>(kSelReg * kThreads)) {
+                // ---- few candidates: a run of up to 16 per thread, in registers ----
+                // The list into shared memory in list order, one thread per sub-segment (its
+                // loads, 16 entries at a time, all in flight); then thread i takes entries
+                // [i per, (i + 1) per).
+                uint32_t* ckey = reinterpret_cast<uint32_t*>(smem + kSelEntOff);
+                uint32_t* cpos = ckey + kSelReg * kThreads;
+                for (int k = tid; k < nseg; k += kThreads) {
+                    const uint32_t cnt = seg_cnt(k), o = off[k];
+                    const uint4* src = reinterpret_cast<const uint4*>(glist + seg_start(p, k));
+                    for (uint32_t j = 0; j < cnt; j += 16) {
+                        uint4 v[8];
+#pragma unroll
+                        for (int u = 0; u < 8; ++u)
+                            v[u] = j + 2 * u < cnt ? __ldcg(src + j / 2 + u) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+                        for (int u = 0; u < 8; ++u) {
+                            const uint32_t e = j + 2 * u;
+                            if (e < cnt) {
+                                ckey[o + e] = v[u].x;
+                                cpos[o + e] = v[u].y;
+                            }
+                            if (e + 1 < cnt) {
+                                ckey[o + e + 1] = v[u].z;
+                                cpos[o + e + 1] = v[u].w;
+                            }
+                        }
+                    }
+                }
+                __syncthreads();
+                const uint32_t per = (m + kThreads - 1) / kThreads;
+                const uint32_t j0 = min(m, tid * per), j1 = min(m, j0 + per);
+                const int cnt = static_cast<int>(j1 - j0);
+                uint32_t key[kSelReg], pos[kSelReg];
+#pragma unroll
+                for (int u = 0; u < kSelReg; ++u) {
+                    key[u] = u < cnt ? ckey[j0 + u] : 0u;
+                    pos[u] = u < cnt ? cpos[j0 + u] : 0u;
+                }
+#pragma unroll 1
+                for (int pass = 0; pass < 4 && lo != hi; ++pass)
+                    radix_pass_reg(key, cnt, lo, hi, need, h, res, scratch, p.err);
+                const uint32_t tau = lo;
+                // ordered compaction: one block scan of (keys above tau, ties) counts, packed
+                // as 16 + 16 bits (m <= 4096); ties are taken lowest position first
+                uint32_t gt = 0, eq = 0;
+#pragma unroll
+                for (int u = 0; u < kSelReg; ++u)
+                    if (u < cnt) {
+                        gt += key[u] > tau;
+                        eq += key[u] == tau;
+                    }
+                uint32_t tot;
+                const uint32_t ex = block_excl_scan((gt << 16) | eq, tot, scratch);
+                uint32_t tie = ex & 0xFFFFu;
+                uint32_t o = (ex >> 16) + min(tie, need);
+                nsel = (tot >> 16) + min(tot & 0xFFFFu, need);
+#pragma unroll
+                for (int u = 0; u < kSelReg; ++u)
+                    if (u < cnt) {
+                        const bool eqk = key[u] == tau;
+                        if (key[u] > tau || (eqk && tie < need)) {
+                            if (o < topk) sel[o] = static_cast<int32_t>(pos[u]);
+                            ++o;
+                        }
+                        tie += eqk;
+                    }
+            } else if (m <= static_cast<uint32_t>(kSelCap)) {
                 // ---- the candidates fit in shared memory ----
                 // Entry j's sub-segment: every non-empty sub-segment writes its index at its
                 // first slot, then a running maximum fills the slots in between.  The loads
@@ -1478,7 +1734,7 @@ __global__ void __launch_bounds__(kThreads, 1) step_kernel(const StepParams p)
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kBarOffset);
-    __shared__ uint32_t scratch[64];
+    __shared__ __align__(16) uint32_t scratch[64];
     __shared__ uint32_t res[3];
     __shared__ int ok_s;
     __shared__ uint32_t epoch_s;
