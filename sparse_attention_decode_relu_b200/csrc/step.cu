@@ -46,7 +46,8 @@ constexpr int kBarSlots = 96;             // mbarriers (8 bytes each) after the 
 constexpr int kStepSmem = 1024 + kBarOffset + kBarSlots * 8;
 
 // mbarrier slots of each phase (disjoint, so no phase re-initialises another's)
-constexpr int kBarRawFull = 0, kBarShare = 16, kBarAccFull = 24, kBarSetup = 30;
+constexpr int kBarRawFull = 0, kBarAFull = 8, kBarAEmpty = 12, kBarAccFull = 16, kBarAccEmpty = 19, kBarRawEmpty = 22,
+              kBarSetup = 30;
 constexpr int kBarExtract = 32;           // [8 warps][4 stages]
 constexpr int kBarAttFull = 64, kBarAttEmpty = 80;
 
@@ -378,27 +379,26 @@ __device__ void radix_pass(ForEach for_each_key, uint32_t& lo, uint32_t& hi, uin
 
 // ==================================================================================
 // Phase 1: indexer scan on the fifth-generation tensor cores, a kernel of its own
-// (16 warps per SM: the per-tile work is a chain of latencies that four warps per
-// scheduler hide far better than two).  A tile of 128 keys is the M side of
-// tcgen05.mma kind::f16 (bf16 operands, fp32 accumulators in tensor memory), the
-// T x 16 indexer query heads the N side (16..128), the 64 dims K (four K = 16
-// steps).  The 16 warps are alike: warps w, w + 4, w + 8, w + 12 own the same 32
-// key rows (TMEM lanes 32 (w % 4) ..), and warp w, part p = w / 4, works on
-//   - (FP8 keys) the p-th quarter of every such row's 64 E4M3 codes (TMA tile
-//     with a 64-byte swizzle), widened exactly into bf16 straight into 8 columns
-//     of the tile's tensor-memory A buffer; bf16 keys arrive from TMA already as
-//     the shared-memory A operand (128-byte swizzle);
-//   - the epilogue of queries [p T / 4, (p + 1) T / 4): ReLU, head weights, a
-//     fixed-order sum over the 16 heads, the per-token scale; the fp32 score
-//     goes to global memory, and each thread keeps the largest key it has seen
-//     per query.
-// Every warp marks its share of a tile done on an mbarrier; tile j's MMAs (and
-// the TMA refill of the stage they free) are issued by warp j % 16, at the end
-// of its iteration two tiles earlier, so that the issue (a thread blocks while
-// the tensor core takes the instructions) rotates over the warps and its wait
-// for the other shares is long satisfied.  Otherwise warps wait only for data: a
-// TMA stage to land, an accumulator to be complete.  Tensor memory: three
-// accumulator buffers of 128 columns and four A buffers of 32 columns.
+// with 16 warps per SM in two roles, decoupled by tensor-memory buffers so that
+// each runs at its own pace.  A tile of 128 keys is the M side of tcgen05.mma
+// kind::f16 (bf16 operands, fp32 accumulators in tensor memory), the T x 16
+// indexer query heads the N side (16..128), the 64 dims K (four K = 16 steps).
+//   - Warps 0-3, one per TMEM lane quarter (32 key rows): (FP8 keys) widen each
+//     row's 64 E4M3 codes (TMA tile, 64-byte swizzle) exactly into bf16, straight
+//     into the tile's tensor-memory A buffer (four of them); bf16 keys arrive
+//     from TMA already as the shared-memory A operand (128-byte swizzle).  Tile
+//     j's MMAs, and the TMA refill of the stage it frees, are issued by warp j %
+//     4 once all four rows quarters are in and the accumulator buffer is free
+//     (the issuing thread blocks while the tensor core takes the instructions,
+//     so the duty rotates).
+//   - Warps 4-15, three per lane quarter: the epilogue of queries [e T / 3, (e +
+//     1) T / 3) for the e-th of them: load the accumulator columns, release the
+//     buffer, then ReLU, head weights, a fixed-order sum over the 16 heads, the
+//     per-token scale; the fp32 score goes to global memory, the largest key of
+//     each 32-position group (per query) to the group maxima, and each thread
+//     keeps the largest key it has seen per query.
+// Tensor memory: three accumulator buffers of 128 columns and four A buffers of
+// 32 columns.  Every wait is an mbarrier wait with a bound.
 //
 // First radix pass.  Each (thread, query) pair sees a fixed set of positions
 // (its key row of each of the block's tiles); the block histogram of top-12-bit
@@ -409,21 +409,26 @@ __device__ void radix_pass(ForEach for_each_key, uint32_t& lo, uint32_t& hi, uin
 // query, b* sits near the top 2048 / 18944 of the pair maxima, so for scores
 // without heavy ties the candidates number little more than topk.
 // ==================================================================================
-constexpr int kIdxThreads = 512;
-constexpr int kIdxWarps = kIdxThreads / 32;
-constexpr int kIdxParts = kIdxWarps / 4;     // warps per TMEM lane quarter
+constexpr int kConvWarps = 4;                // one per TMEM lane quarter
+constexpr int kEpiWarps = 8;                 // two per lane quarter
+constexpr int kEpiPerQuad = kEpiWarps / 4;
+constexpr int kIdxWarps = kConvWarps + kEpiWarps + 1;   // and the issuer
+constexpr int kIdxThreads = kIdxWarps * 32;
+constexpr int kIssuerWarp = kIdxWarps - 1;
+constexpr int kQStage = (kMaxT * kHI * 8 + kIdxThreads - 1) / kIdxThreads;   // query chunks staged per thread
 constexpr int kRawStagesF8 = 8, kRawStagesBf = 6;
 constexpr int kAccBufs = 3, kABufs = 4;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kACol = kAccBufs * 128;   // first column of the A buffers
 constexpr int kTileBytesBf16 = kKeyTile * kDI * 2;   // 16 KiB, one 128 x 64 bf16 operand tile
 constexpr int kIdxCounters = 16;             // shared words: issue marks
-static_assert(kIdxParts == 4 && kDI / kIdxParts == 16, "one 16-code chunk of a key row per warp");
+static_assert(kEpiPerQuad == 2 && (kMaxT + kEpiPerQuad - 1) / kEpiPerQuad <= 4, "at most four queries per epilogue warp");
 static_assert(kACol + kABufs * 32 <= kTmemCols, "tensor memory budget");
-static_assert(kRawStagesF8 * kKeyTile * kDI + kTileBytesBf16 + kMaxT * kHI * 4 + kHistWords * 2 + kIdxCounters * 4 <=
+static_assert(kRawStagesF8 <= kBarAFull - kBarRawFull && kRawStagesBf <= kBarSetup - kBarRawEmpty, "mbarrier slots");
+static_assert(kRawStagesF8 * kKeyTile * kDI + kTileBytesBf16 + 2 * kMaxT * kHI * 4 + kHistWords * 2 + kIdxCounters * 4 <=
                   kDataBytes,
               "FP8 indexer buffers fit the data region");
-static_assert(kRawStagesBf * kTileBytesBf16 + kTileBytesBf16 + kMaxT * kHI * 4 + kHistWords * 2 + kIdxCounters * 4 <=
+static_assert(kRawStagesBf * kTileBytesBf16 + kTileBytesBf16 + 2 * kMaxT * kHI * 4 + kHistWords * 2 + kIdxCounters * 4 <=
                   kDataBytes,
               "bf16 indexer buffers fit the data region");
 
@@ -441,22 +446,23 @@ struct IndexCtx {
     uint32_t* cnt;           // [0] loads issued; [1] MMA groups issued (for the drain after an abort)
     uint32_t* gmax;          // group maxima of the launch, or nullptr
     int64_t gmax_ld;
-    uint64_t* raw_full;
-    uint64_t* acc_full;
-    uint64_t* share;         // [kABufs or kAccBufs]: every warp's share of a tile done
+    uint64_t* raw_full;      // [S] TMA stage landed
+    uint64_t* raw_empty;     // [S] (bf16) the stage's MMAs are done
+    uint64_t* a_full;        // [4] all four lane quarters of an A buffer written
+    uint64_t* a_empty;       // [4] the A buffer's MMAs are done
+    uint64_t* acc_full;      // [3] accumulator complete
+    uint64_t* acc_empty;     // [3] every epilogue warp has loaded it
     const CUtensorMap* kmap;
     uint64_t policy;
     uint32_t tmem, idesc;
     uint64_t bdesc;
     int nloc;                // tiles of this block
-    int qa, nq;              // this warp's queries [qa, qa + nq)
 };
 
 template <bool FP8>
 struct IndexTile {
     static constexpr int S = FP8 ? kRawStagesF8 : kRawStagesBf;
     static constexpr int kRawBytes = kKeyTile * kDI * (FP8 ? 1 : 2);
-    static constexpr int kShareBufs = FP8 ? kABufs : kAccBufs;   // share barriers cycled by tile
     __device__ static int tile_of(int j) { return blockIdx.x + j * static_cast<int>(gridDim.x); }
 
     // TMA of local tile j into its ring stage (one thread).
@@ -467,7 +473,8 @@ struct IndexTile {
         tma_load_2d_hint(c.ring + stage * kRawBytes, c.kmap, 0, tile_of(j) * kKeyTile, &c.raw_full[stage], c.policy);
         red_max_shared(&c.cnt[0], static_cast<uint32_t>(j + 1));
     }
-    // MMAs of local tile j into accumulator buffer j % 3, committed to its barrier (one thread).
+    // MMAs of local tile j into accumulator buffer j % 3 (one thread), committed
+    // to the buffers they free and fill.
     __device__ static void mma(const IndexCtx& c, int j)
     {
         const uint32_t d = c.tmem + (j % kAccBufs) * 128;
@@ -475,82 +482,48 @@ struct IndexTile {
             const uint32_t a = c.tmem + kACol + (j % kABufs) * 32;
 #pragma unroll
             for (int k = 0; k < kDI / 16; ++k) tc_mma_bf16_tmem_a(d, a + k * 8, c.bdesc + 2 * k, c.idesc, k > 0 ? 1u : 0u);
+            tc_commit(&c.a_empty[j % kABufs]);
         } else {
             const uint64_t adesc = umma_desc_sw128(smem_u32(c.ring + (j % S) * kRawBytes));
 #pragma unroll
             for (int k = 0; k < kDI / 16; ++k) tc_mma_bf16(d, adesc + 2 * k, c.bdesc + 2 * k, c.idesc, k > 0 ? 1u : 0u);
+            tc_commit(&c.raw_empty[j % S]);
         }
         tc_commit(&c.acc_full[j % kAccBufs]);
         red_max_shared(&c.cnt[1], static_cast<uint32_t>(j + 1));
     }
-    // This warp's share of tile j is done (FP8: its A columns written; bf16: tile
-    // j's accumulator read).
-    __device__ static void done(const IndexCtx& c, int j, int lane)
-    {
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&c.share[j % kShareBufs]);
-    }
-    // Issue tile j's MMAs once every share is in (FP8: of tile j; bf16: of tile
-    // j - 3, whose accumulator buffer it reuses, and tile j's data has landed),
-    // and refill the stage freed (FP8: tile j's, with tile j + S; bf16: tile j -
-    // 3's, with tile j - 3 + S).  One thread; false if a wait ran out.
-    __device__ static bool issue(const IndexCtx& c, int j, uint32_t* err)
-    {
-        const int f = FP8 ? j : j - kAccBufs;   // the tile whose shares free what tile j needs
-        if (!mbar_wait(&c.share[f % kShareBufs], (f / kShareBufs) & 1, err)) return false;
-        if constexpr (!FP8) {
-            if (!mbar_wait(&c.raw_full[j % S], (j / S) & 1, err)) return false;
-        }
-        tc_fence_after();
-        mma(c, j);
-        if (f + S < c.nloc) load(c, f + S);
-        return true;
-    }
-    // FP8: this warp's quarter of its 32 key rows of tile j widened into the A
-    // buffer.  False if the wait for the data ran out.
-    __device__ static bool convert(const IndexCtx& c, int j, int row, int part, uint32_t lane_base, uint32_t* err)
-    {
-        const int stage = j % S;
-        if (__any_sync(0xffffffffu, !mbar_wait(&c.raw_full[stage], (j / S) & 1, err))) return false;
-        // 16-byte chunk q of the row is stored at chunk q ^ ((row >> 1) & 3)
-        const uint4 v = *reinterpret_cast<const uint4*>(c.ring + stage * kRawBytes + row * 64 +
-                                                        ((part ^ ((row >> 1) & 3)) << 4));
-        uint32_t r[8];
-        e4m3x4_to_bf16x4(v.x, r[0], r[1]);
-        e4m3x4_to_bf16x4(v.y, r[2], r[3]);
-        e4m3x4_to_bf16x4(v.z, r[4], r[5]);
-        e4m3x4_to_bf16x4(v.w, r[6], r[7]);
-        tmem_st8(c.tmem + lane_base + kACol + (j % kABufs) * 32 + part * 8, r);
-        tmem_st_wait();
-        return true;
-    }
 };
 
-// Math of one tile for this warp's queries (NQ of them, a compile-time count so
-// that the code is straight-line) from the accumulator registers.  w holds half
-// of each head weight: ReLU(x) w = (x + |x|) (w / 2) exactly (x + |x| is 2x or
-// +0, both exact; halving w is exact), so each head costs one add (with the
+// Epilogue math of one tile for NQ queries (a compile-time count: straight-line
+// code) from the accumulator registers r[u * 16 + j] (query u, head j).  w holds
+// half of each head weight: ReLU(x) w = (x + |x|) (w / 2) exactly (x + |x| is 2x
+// or +0, both exact; halving w is exact), so each head costs one add (with the
 // absolute value as an operand modifier) and half a packed FMA, all on the FMA
 // pipe, with the very rounding of fma(max(x, 0), w, acc).  FULL: every key of
 // the tile is in range and visible to the warp's queries (no per-key tests).
-template <int NQ, bool FULL>
-__device__ __forceinline__ void index_math(const StepParams& p, const uint32_t (&r)[32], const float4 (&w)[NQ][4],
-                                           int s, float scale, const int (&pos_q)[2], float* const (&out)[2],
-                                           float (&mx)[2], uint32_t (&key)[2])
+template <int U0, int N, bool FULL>
+__device__ __forceinline__ void index_math(const StepParams& p, const uint32_t (&r)[32], const float* w_half, int s,
+                                           float scale, const int (&pos_q)[4], float* const (&out)[4], float (&mx)[4],
+                                           uint32_t (&key)[4])
 {
+    float4 w[N][4];   // half of each head weight (shared memory)
 #pragma unroll
-    for (int u = 0; u < NQ; ++u) {
+    for (int i = 0; i < N; ++i)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) w[i][k] = reinterpret_cast<const float4*>(w_half + (U0 + i) * kHI)[k];
+#pragma unroll
+    for (int i = 0; i < N; ++i) {
+        const int u = U0 + i;
         // Four partial sums over heads {j, j+4, j+8, j+12}, j < 4, as two packed fp32
         // FMAs per four heads, combined in a fixed order.
-        const float* v = reinterpret_cast<const float*>(&r[u * 16]);
+        const float* v = reinterpret_cast<const float*>(&r[i * 16]);
         float2 p01 = make_float2(0.f, 0.f), p23 = make_float2(0.f, 0.f);
 #pragma unroll
         for (int g4 = 0; g4 < 4; ++g4) {
             const float* x = v + g4 * 4;
-            p01 = __ffma2_rn(make_float2(x[0] + fabsf(x[0]), x[1] + fabsf(x[1])), make_float2(w[u][g4].x, w[u][g4].y),
+            p01 = __ffma2_rn(make_float2(x[0] + fabsf(x[0]), x[1] + fabsf(x[1])), make_float2(w[i][g4].x, w[i][g4].y),
                              p01);
-            p23 = __ffma2_rn(make_float2(x[2] + fabsf(x[2]), x[3] + fabsf(x[3])), make_float2(w[u][g4].z, w[u][g4].w),
+            p23 = __ffma2_rn(make_float2(x[2] + fabsf(x[2]), x[3] + fabsf(x[3])), make_float2(w[i][g4].z, w[i][g4].w),
                              p23);
         }
         const float acc = ((p01.x + p01.y) + (p23.x + p23.y)) * scale;
@@ -578,7 +551,7 @@ __device__ void phase_index(const CUtensorMap& kmap, const StepParams& p, uint8_
     constexpr int S = Tile::S;
     constexpr int raw_bytes = Tile::kRawBytes;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int quad = warp & 3, part = warp >> 2;     // TMEM lane quarter; which quarter of the row / queries
+    const int quad = warp & 3;                        // TMEM lane quarter
     const int T = p.T;
     const int ntiles = (visible_max(p) + kKeyTile - 1) / kKeyTile;
 
@@ -586,27 +559,37 @@ __device__ void phase_index(const CUtensorMap& kmap, const StepParams& p, uint8_
     c.ring = smem;
     c.qsw = smem + S * raw_bytes;
     c.w_s = reinterpret_cast<const float*>(c.qsw + kTileBytesBf16);
-    c.hs = reinterpret_cast<uint32_t*>(c.qsw + kTileBytesBf16 + kMaxT * kHI * 4);
+    c.hs = reinterpret_cast<uint32_t*>(c.qsw + kTileBytesBf16 + 2 * kMaxT * kHI * 4);   // after the weights and halves
     c.cnt = c.hs + kHistWords / 2;
     c.gmax = p.gmax;
     c.gmax_ld = p.gmax_ld;
     c.raw_full = bars + kBarRawFull;
+    c.raw_empty = bars + kBarRawEmpty;
+    c.a_full = bars + kBarAFull;
+    c.a_empty = bars + kBarAEmpty;
     c.acc_full = bars + kBarAccFull;
-    c.share = bars + kBarShare;
+    c.acc_empty = bars + kBarAccEmpty;
     c.kmap = &kmap;
     c.policy = l2_evict_first_policy();   // keys are read once; the scores stay in L2
     c.nloc = ntiles > static_cast<int>(blockIdx.x) ? (ntiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
-    c.qa = part * T / kIdxParts;
-    c.nq = (part + 1) * T / kIdxParts - c.qa;        // 0, 1 or 2
     const bool hist = g_view.hist != nullptr;
     uint64_t* setup = bars + kBarSetup;
     float* w_s = const_cast<float*>(c.w_s);
 
     if (tid == 0) {
         prefetch_tmap(&kmap);
-        for (int s = 0; s < S; ++s) mbar_init(&c.raw_full[s], 1);
-        for (int b = 0; b < kAccBufs; ++b) mbar_init(&c.acc_full[b], 1);
-        for (int b = 0; b < Tile::kShareBufs; ++b) mbar_init(&c.share[b], kIdxWarps);
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&c.raw_full[s], 1);
+            if (!FP8) mbar_init(&c.raw_empty[s], 1);
+        }
+        for (int b = 0; b < kABufs; ++b) {
+            mbar_init(&c.a_full[b], kConvWarps);
+            mbar_init(&c.a_empty[b], 1);
+        }
+        for (int b = 0; b < kAccBufs; ++b) {
+            mbar_init(&c.acc_full[b], 1);
+            mbar_init(&c.acc_empty[b], kEpiWarps);
+        }
         mbar_init(setup, 1);
         fence_mbar_init();
         mbar_arrive_expect_tx(setup, T * kHI * 4);
@@ -617,14 +600,14 @@ __device__ void phase_index(const CUtensorMap& kmap, const StepParams& p, uint8_
     // The indexer queries as the B operand: row r = t*16 + j, 16-byte chunk k at
     // r*128 + (k ^ (r & 7))*16 (the 128B swizzle); rows >= T*16 are never read.
     {
-        uint4 v[kMaxT * kHI * 8 / kIdxThreads];   // every load in flight before the first store
+        uint4 v[kQStage];   // every load in flight before the first store
 #pragma unroll
-        for (int u = 0; u < kMaxT * kHI * 8 / kIdxThreads; ++u) {
+        for (int u = 0; u < kQStage; ++u) {
             const int i = tid + u * kIdxThreads;
             v[u] = i < T * kHI * 8 ? __ldg(reinterpret_cast<const uint4*>(p.q_idx) + i) : make_uint4(0u, 0u, 0u, 0u);
         }
 #pragma unroll
-        for (int u = 0; u < kMaxT * kHI * 8 / kIdxThreads; ++u) {
+        for (int u = 0; u < kQStage; ++u) {
             const int i = tid + u * kIdxThreads, r = i >> 3, k = i & 7;
             if (i < T * kHI * 8) *reinterpret_cast<uint4*>(c.qsw + r * 128 + ((k ^ (r & 7)) << 4)) = v[u];
         }
@@ -640,124 +623,175 @@ __device__ void phase_index(const CUtensorMap& kmap, const StepParams& p, uint8_
     c.bdesc = umma_desc_sw128(smem_u32(c.qsw));
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
     const int row = quad * 32 + lane;                // this thread's key row of every tile
-    bool aborted = false;
-    if (tid == 0) {
+    if (tid == 0)
         for (int j = 0; j < S && j < c.nloc; ++j) Tile::load(c, j);
-        if constexpr (!FP8) {   // the first accumulator buffers are free: their MMAs go out as the data lands
-            for (int j = 0; j < kAccBufs && j < c.nloc && !aborted; ++j) {
-                aborted = !mbar_wait(&c.raw_full[j], 0, p.err);
-                if (!aborted) Tile::mma(c, j);
-            }
-        }
-    }
-    aborted = __any_sync(0xffffffffu, aborted || !mbar_wait(setup, 0, p.err));   // warp-uniform from here on
-    int pos_q[2];                                    // positions of this warp's queries
-    float* out[2];                                   // their score rows
-    float mx[2] = {NAN, NAN};                        // largest score seen per query (NaN: none yet)
-    int pos_min = p.L;                               // tiles wholly below it and below L need no tests
-#pragma unroll
-    for (int u = 0; u < 2; ++u) {
-        pos_q[u] = u < c.nq ? query_pos_rt(p, c.qa + u) : -1;
-        out[u] = p.scores + (int64_t)min(c.qa + u, T - 1) * p.ld;
-        if (u < c.nq) pos_min = min(pos_min, pos_q[u] + 1);
-    }
+    bool aborted = __any_sync(0xffffffffu, !mbar_wait(setup, 0, p.err));   // warp-uniform from here on
+    // half of every head weight, next to the weights (see index_math)
+    float* w_half = w_s + kMaxT * kHI;
+    if (tid < T * kHI) w_half[tid] = 0.5f * w_s[tid];
+    __syncthreads();
 
-    auto run = [&](auto nq_tag) {
-        constexpr int NQ = decltype(nq_tag)::value;
-        float4 w[NQ > 0 ? NQ : 1][4];   // half of this warp's head weights, for every tile
-#pragma unroll
-        for (int u = 0; u < NQ; ++u)
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const float4 h = reinterpret_cast<const float4*>(c.w_s + (c.qa + u) * kHI)[k];
-                w[u][k] = make_float4(0.5f * h.x, 0.5f * h.y, 0.5f * h.z, 0.5f * h.w);
-            }
-        const bool scaled = p.scale != nullptr;
-        float scale_next = 1.0f;
-        if (NQ > 0 && scaled && c.nloc > 0) {
-            const int s = Tile::tile_of(0) * kKeyTile + row;
-            scale_next = s < p.L ? __ldg(p.scale + s) : 1.0f;
-        }
-        // Tile j's MMAs go out from warp j % 16 at the end of its iteration j - 2 (FP8:
-        // tiles 0 and 1 here; bf16: tiles 0..2 went out with the first loads).
-        auto issue_by_me = [&](int j) -> bool {
-            bool ok = true;
-            if (j < c.nloc && (FP8 || j >= kAccBufs) && warp == j % kIdxWarps && lane == 0) ok = Tile::issue(c, j, p.err);
-            return !__any_sync(0xffffffffu, !ok);
-        };
+    // per-thread key maxima of the epilogue warps' queries (NaN: none yet)
+    float mx[4] = {NAN, NAN, NAN, NAN};
+    const bool epi = warp >= kConvWarps && warp < kConvWarps + kEpiWarps;
+    const int e_idx = epi ? (warp - kConvWarps) / 4 : 0;
+    const int qa = e_idx * T / kEpiPerQuad;
+    const int nq = epi ? (e_idx + 1) * T / kEpiPerQuad - qa : 0;   // 0..4
+
+    if (warp < kConvWarps) {
+        // ---------------- converter / issuer warps ----------------
         if constexpr (FP8) {
-            for (int j = 0; j < 2 && j < c.nloc && !aborted; ++j) {
-                aborted = !Tile::convert(c, j, row, part, lane_base, p.err);
-                if (!aborted) {
-                    Tile::done(c, j, lane);
-                    aborted = !issue_by_me(j);
-                }
-            }
-        }
-        for (int e = 0; e < c.nloc && !aborted; ++e) {
-            const int s = Tile::tile_of(e) * kKeyTile + row;
-            const float scale = scale_next;
-            if (NQ > 0 && scaled && e + 1 < c.nloc) {   // next tile's scale, in flight during this tile
-                const int s2 = Tile::tile_of(e + 1) * kKeyTile + row;
-                scale_next = s2 < p.L ? __ldg(p.scale + s2) : 1.0f;
-            }
-            // tile e's accumulator: wait, start the loads, then (FP8) widen tile e + 2
-            // while they are in flight
-            const int cb = e % kAccBufs;
-            if (__any_sync(0xffffffffu, !mbar_wait(&c.acc_full[cb], (e / kAccBufs) & 1, p.err))) {
-                aborted = true;
-                break;
-            }
-            tc_fence_after();
-            uint32_t r[32];
-            if constexpr (NQ > 0) tmem_ld32_nowait(c.tmem + lane_base + cb * 128 + c.qa * kHI, r);
-            if (FP8 && e + 2 < c.nloc) {
-                if (!Tile::convert(c, e + 2, row, part, lane_base, p.err)) {
+            for (int j = 0; j < c.nloc && !aborted; ++j) {
+                const int ab = j % kABufs, stage = j % S;
+                bool ok = j < kABufs || mbar_wait(&c.a_empty[ab], ((j / kABufs) - 1) & 1, p.err);
+                ok = ok && mbar_wait(&c.raw_full[stage], (j / S) & 1, p.err);
+                if (__any_sync(0xffffffffu, !ok)) {
                     aborted = true;
                     break;
                 }
-                Tile::done(c, e + 2, lane);
-            }
-            if constexpr (NQ > 0) {
-                tmem_ld_wait();
+                // row `row`: 64 codes, 16-byte chunk q stored at chunk q ^ ((row >> 1) & 3)
+                const uint8_t* src = c.ring + stage * raw_bytes + row * 64;
+                uint4 v[4];
 #pragma unroll
-                for (int k = 0; k < 32; ++k) asm volatile("" : "+r"(r[k]));   // no use before the wait
-                uint32_t key[2];
-                if (Tile::tile_of(e) * kKeyTile + kKeyTile <= pos_min)
-                    index_math<NQ, true>(p, r, w, s, scale, pos_q, out, mx, key);
-                else
-                    index_math<NQ, false>(p, r, w, s, scale, pos_q, out, mx, key);
-                if (c.gmax != nullptr) {
-                    // the largest key of this warp's 32 positions per query (lane u stores
-                    // query u's): lets the extraction skip groups below its cut
-                    uint32_t mine = 0u;
+                for (int q = 0; q < 4; ++q) v[q] = *reinterpret_cast<const uint4*>(src + ((q ^ ((row >> 1) & 3)) << 4));
+                uint32_t r[32];
 #pragma unroll
-                    for (int u = 0; u < NQ; ++u) {
-                        const uint32_t m = __reduce_max_sync(0xffffffffu, key[u]);
-                        if (lane == u) mine = m;
-                    }
-                    if (lane < NQ)
-                        c.gmax[(int64_t)(c.qa + lane) * c.gmax_ld + Tile::tile_of(e) * (kKeyTile / 32) + quad] = mine;
+                for (int q = 0; q < 4; ++q) {
+                    e4m3x4_to_bf16x4(v[q].x, r[8 * q + 0], r[8 * q + 1]);
+                    e4m3x4_to_bf16x4(v[q].y, r[8 * q + 2], r[8 * q + 3]);
+                    e4m3x4_to_bf16x4(v[q].z, r[8 * q + 4], r[8 * q + 5]);
+                    e4m3x4_to_bf16x4(v[q].w, r[8 * q + 6], r[8 * q + 7]);
                 }
-            }
-            if constexpr (!FP8) Tile::done(c, e, lane);   // tile e's accumulator is read
-            if (!issue_by_me(e + 2)) {
-                aborted = true;
-                break;
+                tmem_st32(c.tmem + lane_base + kACol + ab * 32, r);
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&c.a_full[ab]);
             }
         }
-    };
-    if (c.nq == 2) {
-        run(std::integral_constant<int, 2>{});
-    } else if (c.nq == 1) {
-        run(std::integral_constant<int, 1>{});
+    } else if (warp == kIssuerWarp) {
+        // ---------------- the issuer: one thread issues every tile's MMAs ----------------
+        // once its A operand is in (FP8: all four lane quarters widened; bf16: the TMA
+        // tile landed) and its accumulator buffer is free, and refills the ring: FP8,
+        // tile j's stage (every converter has read it) with tile j + S; bf16, the stage
+        // two tiles behind once its MMAs are done.
+        bool ok = !aborted;
+        if (lane == 0 && ok) {
+            for (int j = 0; j < c.nloc && ok; ++j) {
+                if constexpr (FP8) ok = mbar_wait(&c.a_full[j % kABufs], (j / kABufs) & 1, p.err);
+                else ok = mbar_wait(&c.raw_full[j % S], (j / S) & 1, p.err);
+                ok = ok && (j < kAccBufs || mbar_wait(&c.acc_empty[j % kAccBufs], ((j / kAccBufs) - 1) & 1, p.err));
+                if (!ok) break;
+                tc_fence_after();
+                Tile::mma(c, j);
+                if constexpr (FP8) {
+                    if (j + S < c.nloc) Tile::load(c, j + S);
+                } else {
+                    const int f = j - 2;
+                    if (f >= 0 && f + S < c.nloc) {
+                        ok = mbar_wait(&c.raw_empty[f % S], (f / S) & 1, p.err);
+                        if (ok) Tile::load(c, f + S);
+                    }
+                }
+            }
+        }
+        aborted = __any_sync(0xffffffffu, !ok);
     } else {
-        run(std::integral_constant<int, 0>{});
+        // ---------------- epilogue warps ----------------
+        const float* wq = w_half + qa * kHI;         // this warp's queries' halved weights
+        int pos_q[4];                                // positions of this warp's queries
+        float* out[4];                               // their score rows
+        int pos_min = p.L;                           // tiles wholly below it and below L need no tests
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            pos_q[u] = u < nq ? query_pos_rt(p, qa + u) : -1;
+            out[u] = p.scores + (int64_t)min(qa + u, T - 1) * p.ld;
+            if (u < nq) pos_min = min(pos_min, pos_q[u] + 1);
+        }
+        auto run = [&](auto nq_tag) {
+            constexpr int NQ = decltype(nq_tag)::value;
+            const bool scaled = p.scale != nullptr;
+            float scale_next = 1.0f;
+            if (NQ > 0 && scaled && c.nloc > 0) {
+                const int s = Tile::tile_of(0) * kKeyTile + row;
+                scale_next = s < p.L ? __ldg(p.scale + s) : 1.0f;
+            }
+            for (int e = 0; e < c.nloc && !aborted; ++e) {
+                const int tile = Tile::tile_of(e);
+                const int s = tile * kKeyTile + row;
+                const float scale = scale_next;
+                if (NQ > 0 && scaled && e + 1 < c.nloc) {   // next tile's scale, in flight during this tile
+                    const int s2 = Tile::tile_of(e + 1) * kKeyTile + row;
+                    scale_next = s2 < p.L ? __ldg(p.scale + s2) : 1.0f;
+                }
+                const int cb = e % kAccBufs;
+                if (__any_sync(0xffffffffu, !mbar_wait(&c.acc_full[cb], (e / kAccBufs) & 1, p.err))) {
+                    aborted = true;
+                    break;
+                }
+                tc_fence_after();
+                // queries in groups of two: one 32-column load, then its math; the buffer is
+                // released after the last load, while the last group's math runs
+                const uint32_t tbase = c.tmem + lane_base + cb * 128 + qa * kHI;
+                const bool full = tile * kKeyTile + kKeyTile <= pos_min;
+                uint32_t key[4] = {0u, 0u, 0u, 0u};
+                auto group = [&](auto g_tag) {
+                    constexpr int G = decltype(g_tag)::value;             // queries [2G, 2G + n)
+                    constexpr int n = NQ - 2 * G >= 2 ? 2 : NQ - 2 * G;
+                    uint32_t r[32];
+                    if constexpr (n == 1) tmem_ld16_nowait(tbase + 32 * G, reinterpret_cast<uint32_t(&)[16]>(r[0]));
+                    else tmem_ld32_nowait(tbase + 32 * G, r);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int k = 0; k < n * 16; ++k) asm volatile("" : "+r"(r[k]));   // no use before the wait
+                    if (2 * G + n >= NQ) {   // the last load of this buffer
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&c.acc_empty[cb]);
+                    }
+                    if (full) index_math<2 * G, n, true>(p, r, wq, s, scale, pos_q, out, mx, key);
+                    else index_math<2 * G, n, false>(p, r, wq, s, scale, pos_q, out, mx, key);
+                };
+                if constexpr (NQ == 0) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&c.acc_empty[cb]);
+                } else {
+                    group(std::integral_constant<int, 0>{});
+                    if constexpr (NQ > 2) group(std::integral_constant<int, 1>{});
+                }
+                if constexpr (NQ > 0) {
+                    if (c.gmax != nullptr) {
+                        // the largest key of this warp's 32 positions per query (lane u stores
+                        // query u's): lets the extraction skip groups below its cut
+                        uint32_t mine = 0u;
+#pragma unroll
+                        for (int u = 0; u < NQ; ++u) {
+                            const uint32_t m = __reduce_max_sync(0xffffffffu, key[u]);
+                            if (lane == u) mine = m;
+                        }
+                        if (lane < NQ)
+                            c.gmax[(int64_t)(qa + lane) * c.gmax_ld + tile * (kKeyTile / 32) + quad] = mine;
+                    }
+                }
+            }
+        };
+        if (nq == 4) {
+            run(std::integral_constant<int, 4>{});
+        } else if (nq == 3) {
+            run(std::integral_constant<int, 3>{});
+        } else if (nq == 2) {
+            run(std::integral_constant<int, 2>{});
+        } else if (nq == 1) {
+            run(std::integral_constant<int, 1>{});
+        } else {
+            run(std::integral_constant<int, 0>{});
+        }
     }
     // A wait that ran out (error bit set) ends the loop for that warp; the others
     // run into bounded waits and stop too.  Copies and MMAs still in flight land
     // before the shared memory and tensor memory are reused: the last S loads and
-    // the last three MMA groups (every earlier one was waited for by an epilogue).
+    // the last three MMA groups.
     aborted = __syncthreads_or(aborted);
     if (aborted) {
         if (tid == 0) {
@@ -779,10 +813,10 @@ __device__ void phase_index(const CUtensorMap& kmap, const StepParams& p, uint8_
     if (hist) {
         // one count per (thread, query): its largest key's bin
 #pragma unroll
-        for (int u = 0; u < 2; ++u)
-            if (u < c.nq && !isnan(mx[u])) {
+        for (int u = 0; u < 4; ++u)
+            if (u < nq && !isnan(mx[u])) {
                 const uint32_t k = score_key(mx[u]);
-                atomicAdd(&c.hs[(c.qa + u) * (kHistBins / 2) + (k >> (kHistShift + 1))], 1u << (((k >> kHistShift) & 1u) << 4));
+                atomicAdd(&c.hs[(qa + u) * (kHistBins / 2) + (k >> (kHistShift + 1))], 1u << (((k >> kHistShift) & 1u) << 4));
             }
         __syncthreads();
         // the block's 16-bit counters (two per word) into the launch's histogram
