@@ -384,13 +384,12 @@ __device__ void radix_pass(ForEach for_each_key, uint32_t& lo, uint32_t& hi, uin
 // kind::f16 (bf16 operands, fp32 accumulators in tensor memory), the T x 16
 // indexer query heads the N side (16..128), the 64 dims K (four K = 16 steps).
 //   - Warps 0-3, one per TMEM lane quarter (32 key rows): (FP8 keys) widen each
-//     row's 64 E4M3 codes (TMA tile, 64-byte swizzle) exactly into bf16, straight
-//     into the tile's tensor-memory A buffer (four of them); bf16 keys arrive
-//     from TMA already as the shared-memory A operand (128-byte swizzle).  Tile
-//     j's MMAs, and the TMA refill of the stage it frees, are issued by warp j %
-//     4 once all four rows quarters are in and the accumulator buffer is free
-//     (the issuing thread blocks while the tensor core takes the instructions,
-//     so the duty rotates).
+//     row's 64 E4M3 codes (TMA tile, 64-byte swizzle) exactly into f16 (one
+//     conversion instruction per two codes), straight into the tile's
+//     tensor-memory A buffer (four of them); bf16 keys arrive from TMA already as
+//     the shared-memory A operand (128-byte swizzle).
+//   - Warp 16: one thread issues tile j's MMAs once its A operand is in and its
+//     accumulator buffer is free, and refills the TMA ring.
 //   - Warps 4-15, three per lane quarter: the epilogue of queries [e T / 3, (e +
 //     1) T / 3) for the e-th of them: load the accumulator columns, release the
 //     buffer, then ReLU, head weights, a fixed-order sum over the 16 heads, the
@@ -399,6 +398,16 @@ __device__ void radix_pass(ForEach for_each_key, uint32_t& lo, uint32_t& hi, uin
 //     keeps the largest key it has seen per query.
 // Tensor memory: three accumulator buffers of 128 columns and four A buffers of
 // 32 columns.  Every wait is an mbarrier wait with a bound.
+//
+// With FP8 keys the MMA runs on f16 operands: each query head row (t, j) is
+// scaled by a power of two 2^k so that its largest |q| lies in [2^14, 2^15), and
+// converted to f16, which is exact for every element down to 2^-32 of that
+// maximum (f16 holds bf16's 8 significant bits over that range); the head
+// weight is scaled by 2^-k.  Scaling by powers of two commutes with every
+// rounding of the fp32 accumulation and of the epilogue, so the scores are
+// bit-identical to the bf16 computation whenever the rows' elements are within
+// that range; an element below it contributes less than 2^-32 of the row's
+// largest term.
 //
 // First radix pass.  Each (thread, query) pair sees a fixed set of positions
 // (its key row of each of the block's tiles); the block histogram of top-12-bit
@@ -425,12 +434,22 @@ constexpr int kIdxCounters = 16;             // shared words: issue marks
 static_assert(kEpiPerQuad == 2 && (kMaxT + kEpiPerQuad - 1) / kEpiPerQuad <= 4, "at most four queries per epilogue warp");
 static_assert(kACol + kABufs * 32 <= kTmemCols, "tensor memory budget");
 static_assert(kRawStagesF8 <= kBarAFull - kBarRawFull && kRawStagesBf <= kBarSetup - kBarRawEmpty, "mbarrier slots");
-static_assert(kRawStagesF8 * kKeyTile * kDI + kTileBytesBf16 + 2 * kMaxT * kHI * 4 + kHistWords * 2 + kIdxCounters * 4 <=
+static_assert(kRawStagesF8 * kKeyTile * kDI + kTileBytesBf16 + 3 * kMaxT * kHI * 4 + kHistWords * 2 + kIdxCounters * 4 <=
                   kDataBytes,
               "FP8 indexer buffers fit the data region");
-static_assert(kRawStagesBf * kTileBytesBf16 + kTileBytesBf16 + 2 * kMaxT * kHI * 4 + kHistWords * 2 + kIdxCounters * 4 <=
+static_assert(kRawStagesBf * kTileBytesBf16 + kTileBytesBf16 + 3 * kMaxT * kHI * 4 + kHistWords * 2 + kIdxCounters * 4 <=
                   kDataBytes,
               "bf16 indexer buffers fit the data region");
+
+// Power-of-two exponent k for a query row whose largest |q| has the float bits
+// mbits: max * 2^k in [2^14, 2^15); 0 for an all-zero or non-finite row, at most
+// 100 (rows below 2^-86 lose low bits).
+__device__ __forceinline__ int f16_scale_exp(uint32_t mbits)
+{
+    const int e = static_cast<int>((mbits >> 23) & 0xFFu) - 127;
+    if (mbits == 0u || e == 128) return 0;
+    return min(14 - e, 100);
+}
 
 __device__ __forceinline__ void red_max_shared(uint32_t* a, uint32_t v)
 {
@@ -559,7 +578,7 @@ __device__ void phase_index(const CUtensorMap& kmap, const StepParams& p, uint8_
     c.ring = smem;
     c.qsw = smem + S * raw_bytes;
     c.w_s = reinterpret_cast<const float*>(c.qsw + kTileBytesBf16);
-    c.hs = reinterpret_cast<uint32_t*>(c.qsw + kTileBytesBf16 + 2 * kMaxT * kHI * 4);   // after the weights and halves
+    c.hs = reinterpret_cast<uint32_t*>(c.qsw + kTileBytesBf16 + 3 * kMaxT * kHI * 4);   // after weights, halves, exponents
     c.cnt = c.hs + kHistWords / 2;
     c.gmax = p.gmax;
     c.gmax_ld = p.gmax_ld;
@@ -599,6 +618,8 @@ __device__ void phase_index(const CUtensorMap& kmap, const StepParams& p, uint8_
     if (warp == 0) tmem_alloc(tmem_slot, kTmemCols);
     // The indexer queries as the B operand: row r = t*16 + j, 16-byte chunk k at
     // r*128 + (k ^ (r & 7))*16 (the 128B swizzle); rows >= T*16 are never read.
+    // FP8 keys: f16 queries, row r scaled by 2^rowk[r] (see above).
+    int* rowk = reinterpret_cast<int*>(w_s + 2 * kMaxT * kHI);
     {
         uint4 v[kQStage];   // every load in flight before the first store
 #pragma unroll
@@ -606,10 +627,45 @@ __device__ void phase_index(const CUtensorMap& kmap, const StepParams& p, uint8_
             const int i = tid + u * kIdxThreads;
             v[u] = i < T * kHI * 8 ? __ldg(reinterpret_cast<const uint4*>(p.q_idx) + i) : make_uint4(0u, 0u, 0u, 0u);
         }
+        if constexpr (FP8) {
+            if (tid < kMaxT * kHI) rowk[tid] = 0;   // first the bits of each row's max |q|
+            __syncthreads();
 #pragma unroll
-        for (int u = 0; u < kQStage; ++u) {
-            const int i = tid + u * kIdxThreads, r = i >> 3, k = i & 7;
-            if (i < T * kHI * 8) *reinterpret_cast<uint4*>(c.qsw + r * 128 + ((k ^ (r & 7)) << 4)) = v[u];
+            for (int u = 0; u < kQStage; ++u) {
+                const int i = tid + u * kIdxThreads;
+                if (i < T * kHI * 8) {
+                    const uint32_t x[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+                    uint32_t m = 0u;
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) m = max(m, max((x[q] << 16) & 0x7FFFFFFFu, x[q] & 0x7FFF0000u));
+                    atomicMax(reinterpret_cast<uint32_t*>(&rowk[i >> 3]), m);   // |q| bits order like |q|
+                }
+            }
+            __syncthreads();
+#pragma unroll
+            for (int u = 0; u < kQStage; ++u) {
+                const int i = tid + u * kIdxThreads, r = i >> 3, k = i & 7;
+                if (i < T * kHI * 8) {
+                    const float sc = __int_as_float((127 + f16_scale_exp(static_cast<uint32_t>(rowk[r]))) << 23);
+                    const uint32_t x[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+                    uint32_t y[4];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const __half2 h = __floats2half2_rn(__uint_as_float(x[q] << 16) * sc,
+                                                            __uint_as_float(x[q] & 0xFFFF0000u) * sc);
+                        y[q] = *reinterpret_cast<const uint32_t*>(&h);
+                    }
+                    *reinterpret_cast<uint4*>(c.qsw + r * 128 + ((k ^ (r & 7)) << 4)) = make_uint4(y[0], y[1], y[2], y[3]);
+                }
+            }
+            __syncthreads();
+            if (tid < kMaxT * kHI) rowk[tid] = f16_scale_exp(static_cast<uint32_t>(rowk[tid]));
+        } else {
+#pragma unroll
+            for (int u = 0; u < kQStage; ++u) {
+                const int i = tid + u * kIdxThreads, r = i >> 3, k = i & 7;
+                if (i < T * kHI * 8) *reinterpret_cast<uint4*>(c.qsw + r * 128 + ((k ^ (r & 7)) << 4)) = v[u];
+            }
         }
     }
     if (hist)
@@ -619,7 +675,7 @@ __device__ void phase_index(const CUtensorMap& kmap, const StepParams& p, uint8_
     __syncthreads();
     tc_fence_after();
     c.tmem = *tmem_slot;
-    c.idesc = umma_idesc_bf16(kKeyTile, T * kHI);
+    c.idesc = FP8 ? umma_idesc_f16(kKeyTile, T * kHI) : umma_idesc_bf16(kKeyTile, T * kHI);
     c.bdesc = umma_desc_sw128(smem_u32(c.qsw));
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
     const int row = quad * 32 + lane;                // this thread's key row of every tile
@@ -628,7 +684,7 @@ __device__ void phase_index(const CUtensorMap& kmap, const StepParams& p, uint8_
     bool aborted = __any_sync(0xffffffffu, !mbar_wait(setup, 0, p.err));   // warp-uniform from here on
     // half of every head weight, next to the weights (see index_math)
     float* w_half = w_s + kMaxT * kHI;
-    if (tid < T * kHI) w_half[tid] = 0.5f * w_s[tid];
+    if (tid < T * kHI) w_half[tid] = 0.5f * w_s[tid] * (FP8 ? __int_as_float((127 - rowk[tid]) << 23) : 1.0f);
     __syncthreads();
 
     // per-thread key maxima of the epilogue warps' queries (NaN: none yet)
@@ -657,10 +713,12 @@ __device__ void phase_index(const CUtensorMap& kmap, const StepParams& p, uint8_
                 uint32_t r[32];
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
-                    e4m3x4_to_bf16x4(v[q].x, r[8 * q + 0], r[8 * q + 1]);
-                    e4m3x4_to_bf16x4(v[q].y, r[8 * q + 2], r[8 * q + 3]);
-                    e4m3x4_to_bf16x4(v[q].z, r[8 * q + 4], r[8 * q + 5]);
-                    e4m3x4_to_bf16x4(v[q].w, r[8 * q + 6], r[8 * q + 7]);
+                    const uint32_t x[4] = {v[q].x, v[q].y, v[q].z, v[q].w};
+#pragma unroll
+                    for (int h = 0; h < 4; ++h) {
+                        r[8 * q + 2 * h] = e4m3x2_to_f16x2(x[h]);
+                        r[8 * q + 2 * h + 1] = e4m3x2_to_f16x2(x[h] >> 16);
+                    }
                 }
                 tmem_st32(c.tmem + lane_base + kACol + ab * 32, r);
                 tmem_st_wait();
