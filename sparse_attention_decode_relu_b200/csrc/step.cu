@@ -419,7 +419,7 @@ __device__ void radix_pass(ForEach for_each_key, uint32_t& lo, uint32_t& hi, uin
 // without heavy ties the candidates number little more than topk.
 // ==================================================================================
 constexpr int kConvWarps = 4;                // one per TMEM lane quarter
-constexpr int kEpiWarps = 8;                 // two per lane quarter
+constexpr int kEpiWarps = 12;                // three per lane quarter
 constexpr int kEpiPerQuad = kEpiWarps / 4;
 constexpr int kIdxWarps = kConvWarps + kEpiWarps + 1;   // and the issuer
 constexpr int kIdxThreads = kIdxWarps * 32;
@@ -431,7 +431,7 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kACol = kAccBufs * 128;   // first column of the A buffers
 constexpr int kTileBytesBf16 = kKeyTile * kDI * 2;   // 16 KiB, one 128 x 64 bf16 operand tile
 constexpr int kIdxCounters = 16;             // shared words: issue marks
-static_assert(kEpiPerQuad == 2 && (kMaxT + kEpiPerQuad - 1) / kEpiPerQuad <= 4, "at most four queries per epilogue warp");
+static_assert((kMaxT + kEpiPerQuad - 1) / kEpiPerQuad <= 4, "at most four queries per epilogue warp");
 static_assert(kACol + kABufs * 32 <= kTmemCols, "tensor memory budget");
 static_assert(kRawStagesF8 <= kBarAFull - kBarRawFull && kRawStagesBf <= kBarSetup - kBarRawEmpty, "mbarrier slots");
 static_assert(kRawStagesF8 * kKeyTile * kDI + kTileBytesBf16 + 3 * kMaxT * kHI * 4 + kHistWords * 2 + kIdxCounters * 4 <=
