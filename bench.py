@@ -52,12 +52,12 @@ def kernel_sources_sha256():
     return h.hexdigest()
 
 
-def profiled_traffic(workload):
-    """DRAM bytes per step-kernel launch from the committed ncu capture of this
+def profiled_traffic(kernel, workload):
+    """DRAM bytes per launch of `kernel` from the committed ncu capture of this
     workload, or None when there is none or the kernel sources changed since."""
     try:
         with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
-            rec = json.load(f)["step_kernel"]
+            rec = json.load(f)[kernel]
     except (OSError, KeyError, ValueError):
         return None
     if rec.get("source_sha256") != kernel_sources_sha256():
@@ -473,27 +473,47 @@ def main():
     # device->host copies of the outputs.  The caches stay resident.
     e2e = None
     if not args.no_e2e and args.op != "index":
-        h_in = {k: d[k].cpu().pin_memory() for k in (("q",) if args.op == "swa" else ("q", "q_idx", "w_idx"))}
-        dev_in = {k: torch.empty_like(d[k]) for k in h_in}
-        h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-        h_sel = torch.empty(sel.shape, dtype=sel.dtype).pin_memory()
-        h_pos = torch.tensor(w.pos, dtype=torch.int32).pin_memory()
-        e_pos = torch.empty_like(pos_dev)
-        h2d = sum(v.numel() * v.element_size() for v in h_in.values()) + (0 if args.op == "swa" else h_pos.numel() * 4)
-        d2h = h_out.numel() * h_out.element_size() + (0 if args.op == "swa" else h_sel.numel() * h_sel.element_size())
+        # The step's query-side inputs (and positions) are views of one device
+        # buffer filled by one copy from one pinned host buffer; the outputs are
+        # views of one device buffer read back by one copy.
+        names = ("q",) if args.op == "swa" else ("q", "q_idx", "w_idx")
+
+        def carve(buf, parts):
+            views, off = {}, 0
+            for k, (shape, dt) in parts.items():
+                n = int(np.prod(shape)) * torch.empty((), dtype=dt).element_size()
+                views[k] = buf[off:off + n].view(dt).view(shape)
+                off = (off + n + 255) // 256 * 256
+            return views
+
+        in_parts = {k: (tuple(d[k].shape), d[k].dtype) for k in names}
+        if args.op != "swa":
+            in_parts["pos"] = ((w.T,), torch.int32)
+        out_parts = {"out": (tuple(out.shape), out.dtype)}
+        if args.op != "swa":
+            out_parts["sel"] = (tuple(sel.shape), sel.dtype)
+        n_in = sum((int(np.prod(s_)) * torch.empty((), dtype=t_).element_size() + 255) // 256 * 256 for s_, t_ in in_parts.values())
+        n_out = sum((int(np.prod(s_)) * torch.empty((), dtype=t_).element_size() + 255) // 256 * 256 for s_, t_ in out_parts.values())
+        h_inbuf = torch.empty(n_in, dtype=torch.uint8).pin_memory()
+        d_inbuf = torch.empty(n_in, dtype=torch.uint8, device=dev)
+        h_outbuf = torch.empty(n_out, dtype=torch.uint8).pin_memory()
+        d_outbuf = torch.empty(n_out, dtype=torch.uint8, device=dev)
+        h_in, dev_in = carve(h_inbuf, in_parts), carve(d_inbuf, in_parts)
+        h_o, dev_o = carve(h_outbuf, out_parts), carve(d_outbuf, out_parts)
+        for k in names:
+            h_in[k].copy_(d[k].cpu())
+        if args.op != "swa":
+            h_in["pos"].copy_(torch.tensor(w.pos, dtype=torch.int32))
+        h2d, d2h = n_in, n_out
 
         def e2e_step():
-            for k in h_in:
-                dev_in[k].copy_(h_in[k], non_blocking=True)
+            d_inbuf.copy_(h_inbuf, non_blocking=True)
             if args.op == "swa":
-                dsa.dsa_swa_decode(dev_in["q"], d["kv"], w.pos, args.window, out, ws)
+                dsa.dsa_swa_decode(dev_in["q"], d["kv"], w.pos, args.window, dev_o["out"], ws)
             else:
-                e_pos.copy_(h_pos, non_blocking=True)
-                dsa.dsa_decode_devpos_ws(dev_in["q"], dev_in["q_idx"], dev_in["w_idx"], d["k_idx"], d["kv"], e_pos,
-                                         topk, out, sel, ws, k_scale=d["k_scale"])
-            h_out.copy_(out, non_blocking=True)
-            if args.op != "swa":
-                h_sel.copy_(sel, non_blocking=True)
+                dsa.dsa_decode_devpos_ws(dev_in["q"], dev_in["q_idx"], dev_in["w_idx"], d["k_idx"], d["kv"],
+                                         dev_in["pos"], topk, dev_o["out"], dev_o["sel"], ws, k_scale=d["k_scale"])
+            h_outbuf.copy_(d_outbuf, non_blocking=True)
 
         with torch.cuda.stream(stream):
             e2e_step()   # eager once (first-call set-up outside the capture)
@@ -518,28 +538,68 @@ def main():
             e_times.append(a.elapsed_time(b))
         dsa.dsa_device_status(stream)
         if args.op != "swa":   # the host copies hold the step's results
-            assert torch.equal(h_sel, sel.cpu()), "end-to-end selection differs from the device-timed step"
+            assert torch.equal(h_o["sel"], sel.cpu()), "end-to-end selection differs from the device-timed step"
         e_ms = reduce_max(statistics.mean(e_times), world)
         e2e = {"value": round(whole_job_gbs(ab["step"], e_ms, world), 3), "unit": "GB/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e_ms, 4),
-               "timing": "CUDA-graph replay of H2D copies + " +
+               "timing": "CUDA-graph replay of one H2D copy (inputs and positions) + " +
                          ("dsa_swa_decode" if args.op == "swa" else "dsa_decode_devpos_ws") +
-                         " + D2H copies, CUDA events per step, mean"}
+                         " + one D2H copy (outputs), CUDA events per step, mean"}
         del e_graph
 
-    # Roofline of the step kernel (the only kernel: every phase of the step runs in
-    # one cooperative launch), timed by the events around each graph replay.
+    # Roofline of the dominant kernel.  A step with the indexer launches two
+    # kernels: the indexer kernel, then the cooperative top-k/attention kernel.
+    # Their durations come from the library's stage events (one between the two
+    # launches) on eager calls of the same step, under the same cold-L2 protocol
+    # (the GPU spins while the host submits, so it never waits for the host);
+    # each kernel's algorithmic bytes are its share of the step's.
     peak, which = peaks()
-    achieved = ab["step"] / (ms * 1e-3) / 1e9
-    roof = {"kernel": "step_kernel", "bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+    bypassed = (args.op == "step" and not args.no_bypass and args.pos == "host"
+                and int(w.pos.max()) + 1 <= topk)   # no indexer phase then
+    kernels = {}
+    if args.op == "step" and not bypassed:
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+        with torch.cuda.stream(stream):
+            for e in evs:   # torch times only events it has seen recorded; the graph re-records them
+                e.record(stream)
+        stream.synchronize()
+        t_idx, t_coop = [], []
+        dsa.dsa_set_stage_events(evs)
+        for i in range(args.warmup + args.steps):
+            flush_l2()
+            stream.wait_stream(torch.cuda.current_stream())
+            with torch.cuda.stream(stream):
+                torch.cuda._sleep(SPIN_CYCLES)
+                step()
+            stream.synchronize()
+            if i >= args.warmup:
+                t_idx.append(evs[0].elapsed_time(evs[1]))
+                t_coop.append(evs[1].elapsed_time(evs[4]))
+        dsa.dsa_set_stage_events(None)
+        dsa.dsa_device_status(stream)
+        idx_in = w.T * (16 * 64 * 2 + 16 * 4)
+        kernels["index_kernel"] = {"us": reduce_max(statistics.mean(t_idx), world) * 1e3,
+                                   "bytes": ab["indexer"] + idx_in}
+        kernels["step_kernel"] = {"us": reduce_max(statistics.mean(t_coop), world) * 1e3,
+                                  "bytes": ab["step"] - ab["indexer"] - idx_in}
+    elif args.op == "index":
+        kernels["index_kernel"] = {"us": ms * 1e3, "bytes": ab["step"]}
+    else:
+        kernels["step_kernel"] = {"us": ms * 1e3, "bytes": ab["step"]}
+    dom = max(kernels, key=lambda k: kernels[k]["us"])
+    achieved = kernels[dom]["bytes"] / (kernels[dom]["us"] * 1e-6) / 1e9
+    key = w.name if args.op == "step" else f"{w.name}:{args.op}"
+    roof = {"kernel": dom, "bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
             "frac": round(achieved / peak, 4), "peak_source": which,
-            "traffic": profiled_traffic(w.name if args.op == "step" else f"{w.name}:{args.op}") if args.pos == "host" else None,
-            "algorithmic_bytes": ab["step"]}
+            "traffic": profiled_traffic(dom, key) if args.pos == "host" else None,
+            "algorithmic_bytes": kernels[dom]["bytes"], "duration_us": round(kernels[dom]["us"], 2),
+            "kernels": {k: {"us": round(v["us"], 2), "algorithmic_bytes": v["bytes"],
+                            "achieved_gbs": round(v["bytes"] / (v["us"] * 1e-6) / 1e9, 1)} for k, v in kernels.items()},
+            "timing": "stage events around each kernel of eager calls of the step, cold L2, mean"
+                      if args.op == "step" and not bypassed else "the step's own events"}
 
     # The indexer's tensor-core rate (tcgen05.mma), over its in-kernel phase time.
     tensor = None
-    bypassed = (args.op == "step" and not args.no_bypass and args.pos == "host"
-                and int(w.pos.max()) + 1 <= topk)   # no indexer phase then
     if args.op in ("step", "index") and not bypassed and phase_us.get("indexer", 0) > 0:
         tpk, tsrc = bf16_peak()
         tf = indexer_flops(w) / (phase_us["indexer"] * 1e-6) / 1e12

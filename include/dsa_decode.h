@@ -247,9 +247,11 @@ DSA_API uint64_t dsa_launch_count(void);
 
 /* Profiling hook for the calling host thread.  With n == 5, dsa_decode and
  * dsa_decode_ws record five cudaEvent_t on their stream: events[0] before the
- * first launch, events[1] after the indexer scan, events[2] after the top-k
- * selection, events[3] after the attention and events[4] at the end of the
- * call.  n == 0 disables; any other n is ignored. */
+ * first launch, events[1] between the indexer kernel and the cooperative
+ * top-k/attention kernel (when the indexer runs; the event then stands between
+ * them in the stream, so the second kernel's launch no longer overlaps the
+ * first's tail), events[2], events[3] and events[4] at the end of the call.
+ * n == 0 disables; any other n is ignored. */
 DSA_API void dsa_set_stage_events(void *const *events, int32_t n);
 
 /* Failure-detection test hook for the calling host thread (one launch only).

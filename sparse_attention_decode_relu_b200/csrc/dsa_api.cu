@@ -333,7 +333,8 @@ dsa_status_t launch(const CUtensorMap& map, StepParams& p, bool fp8, void* ws, c
         p.barrier_extra = 1;
         t_fail_barriers = 0;
     }
-    if ((e = launch_step(&map, p, fp8, stream)) != cudaSuccess) return cuda_fail(e, "step launch");
+    cudaEvent_t mid = t_stage_events_on ? static_cast<cudaEvent_t>(t_stage_events[1]) : nullptr;
+    if ((e = launch_step(&map, p, fp8, stream, mid)) != cudaSuccess) return cuda_fail(e, "step launch");
     g_launches += ((p.phases & kPhaseIndex) != 0) + ((p.phases & ~kPhaseIndex) != 0);   // indexer, cooperative kernel
     return DSA_OK;
 }
@@ -492,8 +493,8 @@ static dsa_status_t decode_ws(const dsa_tensor_t* q, const dsa_tensor_t* q_idx, 
     topk_params(p, workspace, l);
     attn_params(p, workspace, l, topk);
     stage_event(0, stream);
-    st = launch(map, p, sh.fp8, workspace, l, stream);
-    for (int i = 1; i < 5; ++i) stage_event(i, stream);
+    st = launch(map, p, sh.fp8, workspace, l, stream);   // events[1] between the indexer and the cooperative kernel
+    for (int i = 2; i < 5; ++i) stage_event(i, stream);
     return st;
 }
 

@@ -99,6 +99,10 @@ struct StepParams {
 
 int step_smem_bytes();
 int step_max_blocks(bool fp8);
-cudaError_t launch_step(const CUtensorMap* kmap, const StepParams& p, bool fp8, cudaStream_t s);
+// Launches the indexer kernel (when p.phases has kPhaseIndex) and then the
+// cooperative kernel for the remaining phases; mid_event (or nullptr) is recorded
+// on the stream between the two.
+cudaError_t launch_step(const CUtensorMap* kmap, const StepParams& p, bool fp8, cudaStream_t s,
+                        cudaEvent_t mid_event = nullptr);
 
 }  // namespace dsa

@@ -1895,7 +1895,7 @@ bool g_no_pdl[64] = {};
 
 int step_smem_bytes() { return kStepSmem; }
 
-cudaError_t launch_step(const CUtensorMap* kmap, const StepParams& p, bool fp8, cudaStream_t s)
+cudaError_t launch_step(const CUtensorMap* kmap, const StepParams& p, bool fp8, cudaStream_t s, cudaEvent_t mid_event)
 {
     int dev = 0;
     cudaGetDevice(&dev);
@@ -1912,6 +1912,7 @@ cudaError_t launch_step(const CUtensorMap* kmap, const StepParams& p, bool fp8, 
         kern<<<p.grid, kIdxThreads, kStepSmem, s>>>(*kmap, q);
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
+        if (mid_event != nullptr && (e = cudaEventRecord(mid_event, s)) != cudaSuccess) return e;
     }
     StepParams q = p;
     q.phases &= ~kPhaseIndex;

@@ -36,12 +36,13 @@ def test_window_bytes_by_hand():
 
 
 def test_traffic_only_for_the_profiled_sources(monkeypatch):
-    rec = bench.profiled_traffic("verify_block")
+    rec = bench.profiled_traffic("index_kernel", "verify_1m")
     if rec is not None:                                          # the committed capture matches these sources
-        assert rec > 30_000_000
-    assert bench.profiled_traffic("no_such_workload") is None
+        assert rec > 60_000_000                                  # at least the 1M keys' 64 MB
+    assert bench.profiled_traffic("index_kernel", "no_such_workload") is None
+    assert bench.profiled_traffic("no_such_kernel", "verify_1m") is None
     monkeypatch.setattr(bench, "kernel_sources_sha256", lambda: "0" * 64)
-    assert bench.profiled_traffic("verify_block") is None
+    assert bench.profiled_traffic("index_kernel", "verify_1m") is None
 
 
 def test_whole_job_rate_is_weak_scaling():
