@@ -116,7 +116,9 @@ typedef struct {
 #define DSA_WS_CTRL_BYTES 263168
 DSA_API size_t dsa_workspace_bytes(int32_t T, int64_t L, int32_t topk);
 
-/* The whole step: indexer scan, causal top-k, sparse attention.  Takes its
+/* The whole step: indexer scan, causal top-k, sparse attention -- two kernel
+ * launches on `stream` (the indexer, then the cooperative top-k/attention
+ * kernel as its programmatic dependent).  Takes its
  * workspace stream-ordered (cudaMallocAsync, a zeroing of its control words,
  * cudaFreeAsync, all on `stream`), so it
  * must not be captured into a CUDA graph on a device without memory-pool
@@ -264,8 +266,8 @@ DSA_API void dsa_set_stage_events(void *const *events, int32_t n);
  * words at zero, so the next call runs as usual.  Only waits between blocks are
  * affected; waits for a block's own copies in flight keep their normal bound.
  * NaiveAI research page, "NaiveRT > A DSA layer: from 29 kernels to one": the
- * single cooperative kernel depends on synchronisation between its CTAs, which
- * is what a bounded wait guards.  Returns DSA_ERR_INVALID_ARG for a limit
+ * cooperative top-k/attention kernel depends on synchronisation between its
+ * CTAs, which is what a bounded wait guards.  Returns DSA_ERR_INVALID_ARG for a limit
  * outside the range. */
 DSA_API dsa_status_t dsa_debug_fail_next_barriers(int64_t limit_cycles);
 
