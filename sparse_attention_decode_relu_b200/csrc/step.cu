@@ -76,6 +76,9 @@ __device__ bool wait_counter(const StepParams& p, const uint32_t* word, uint32_t
             atomicOr(p.err, ERR_WAIT_TIMEOUT);
             return false;
         }
+        // Hundreds of waiters poll words of one 128-byte line: a pause between polls
+        // keeps that L2 slice free for the data the others are moving.
+        __nanosleep(200);
     }
     return true;
 }
@@ -960,6 +963,19 @@ __device__ void phase_extract(const StepParams& p, uint8_t* smem, uint64_t* bars
     const int n = query_pos_rt(p, t) + 1;
     uint64_t* full = bars + kBarExtract + warp * kXStages;
     if (n > p.topk) {
+        const bool bound = p.hist_bound != 0;
+        const int R = p.chunk / kSegPerChunk;
+        const int s0 = c * p.chunk + warp * R, s1 = min(s0 + R, n);
+        // With group maxima: their first round is loaded now, in flight while the
+        // cut is found (they do not depend on it).
+        const bool use_gmax = p.gmax != nullptr && bound;
+        const uint32_t* gm = p.gmax + (int64_t)t * p.gmax_ld;
+        uint32_t m_first[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const int g = s0 + (k * 32 + lane) * 32;
+            m_first[k] = use_gmax && g < s1 ? __ldcg(gm + g / 32) : 0u;
+        }
         // threshold bin from the histogram (coalesced loads, all in flight)
         uint32_t* h = reinterpret_cast<uint32_t*>(smem + kXHistOff);
         {
@@ -980,7 +996,6 @@ __device__ void phase_extract(const StepParams& p, uint8_t* smem, uint64_t* bars
         // bin and above, those above it all selected.  Indexer histogram of per-thread
         // maxima (a lower bound): every key of bin >= b* is a candidate, to be
         // radix-selected from the top; with fewer than topk counts, every visible key.
-        const bool bound = p.hist_bound != 0;
         uint32_t cut = 0u, above = 0u, top = 0xFFFFFFFFu;
         if (res[2]) {
             cut = res[0] << kHistShift;
@@ -993,24 +1008,21 @@ __device__ void phase_extract(const StepParams& p, uint8_t* smem, uint64_t* bars
         }
         if (c == 0 && tid == 0) reinterpret_cast<uint4*>(p.cuts)[t] = make_uint4(cut, above, top, 0u);
 
-        const int R = p.chunk / kSegPerChunk;
-        const int s0 = c * p.chunk + warp * R, s1 = min(s0 + R, n);
         const int np = s1 > s0 ? (s1 - s0 + kXPiece - 1) / kXPiece : 0;
         const float* row = p.scores + (int64_t)t * p.ld;
         float* ring = reinterpret_cast<float*>(smem) + warp * kXStages * kXPiece;
         uint2* out = p.list + (int64_t)t * p.list_ld + s0;
         uint32_t count = 0;
-        if (p.gmax != nullptr && bound) {
+        if (use_gmax) {
             // Only the 32-position groups whose largest key reaches the cut are read:
             // eight rounds of 32 group maxima in flight per lane, then the hit groups'
             // scores four at a time, in position order.
-            const uint32_t* gm = p.gmax + (int64_t)t * p.gmax_ld;
             for (int base = s0; base < s1; base += 8 * 32 * 32) {
                 uint32_t m[8];
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {
                     const int g = base + (k * 32 + lane) * 32;
-                    m[k] = g < s1 ? __ldcg(gm + g / 32) : 0u;
+                    m[k] = base == s0 ? m_first[k] : (g < s1 ? __ldcg(gm + g / 32) : 0u);
                 }
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {
