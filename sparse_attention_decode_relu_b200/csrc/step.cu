@@ -1202,38 +1202,36 @@ __device__ void radix_pass_reg(const uint32_t (&k)[kSelReg], int cnt, uint32_t& 
     need -= res[1];
     lo = nlo;
     hi = nhi;
-    // A bin of at most 32 keys is resolved at once instead of by another pass: its
-    // keys go to a short list, and lane l of warp 0 ranks key l against the list;
-    // the key with (keys above it) < need <= (keys at or above it) is the exact one.
+    // A bin of at most 256 keys is resolved at once instead of by another pass: its
+    // keys go to a short list, and thread i ranks key i against the list (every
+    // thread reads the same entry at a time: broadcasts); the key with (keys above
+    // it) < need <= (keys at or above it) is the exact one.
     const uint32_t in_bin = h[res[0]];
     __syncthreads();
-    if (shift > 0 && in_bin <= 32u && res[2]) {
+    if (shift > 0 && in_bin <= static_cast<uint32_t>(kThreads) && res[2]) {
         uint32_t* list = h;   // the bins are no longer needed
-        if (tid == 0) res[1] = 0u;   // list length
+        if (tid == 0) {
+            res[1] = 0u;   // list length
+            res[2] = 0u;   // becomes the ties to take, once found
+        }
         __syncthreads();
 #pragma unroll
         for (int u = 0; u < kSelReg; ++u)
-            if (u < cnt && k[u] >= nlo && k[u] <= nhi) list[1 + atomicAdd(&res[1], 1u)] = k[u];
+            if (u < cnt && k[u] >= nlo && k[u] <= nhi) list[atomicAdd(&res[1], 1u)] = k[u];
         __syncthreads();
-        if (warp == 0) {
-            const uint32_t n = res[1];
-            const uint32_t mine = lane < static_cast<int>(n) ? list[1 + lane] : 0u;
-            uint32_t gt = 0, ge = 0;
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {   // every lane's key by shuffle, no serial loads
-                const uint32_t o = __shfl_sync(0xffffffffu, mine, j);
-                if (j < static_cast<int>(n)) {
-                    gt += o > mine;
-                    ge += o >= mine;
-                }
-            }
-            const bool hit = lane < static_cast<int>(n) && gt < need && need <= ge;
-            const uint32_t who = __ballot_sync(0xffffffffu, hit);
-            if (who != 0u && lane == __ffs(who) - 1) {
-                res[0] = mine;
-                res[2] = need - gt;   // ties of the exact key still to take
-            }
-            if (who == 0u && lane == 0) res[2] = 0u;
+        const uint32_t n = res[1];
+        const uint32_t mine = tid < static_cast<int>(n) ? list[tid] : 0u;
+        uint32_t gt = 0, ge = 0;
+#pragma unroll 4
+        for (uint32_t j = 0; j < n; ++j) {
+            const uint32_t o = list[j];
+            gt += o > mine;
+            ge += o >= mine;
+        }
+        // every holder of the exact key finds it; they agree on (key, need - gt)
+        if (tid < static_cast<int>(n) && gt < need && need <= ge) {
+            res[0] = mine;
+            res[2] = need - gt;
         }
         __syncthreads();
         if (res[2]) {
