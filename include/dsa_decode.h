@@ -109,9 +109,9 @@ typedef struct {
  * histograms that successive launches alternate between -- which must be zero
  * before the workspace's first use (one cudaMemsetAsync when it is created).  Every call leaves it ready for the next one (barrier and
  * per-query words back at zero, the histogram the next call uses cleared), so
- * later calls need no reset.  A launch that finds the grid-barrier words
- * (bytes 0..3 and 128..131) non-zero flags DSA_ERR_DEVICE (bit 8 of the error
- * word).  One workspace serves one call at a time: calls that may overlap on the
+ * later calls need no reset.  A launch that finds its barrier or per-query
+ * words non-zero flags DSA_ERR_DEVICE (error word bit 0x8) and skips the
+ * work that depends on them.  One workspace serves one call at a time: calls that may overlap on the
  * GPU need separate workspaces. */
 #define DSA_WS_CTRL_BYTES 263168
 DSA_API size_t dsa_workspace_bytes(int32_t T, int64_t L, int32_t topk);

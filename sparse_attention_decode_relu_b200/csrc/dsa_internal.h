@@ -38,7 +38,7 @@ constexpr int kTraceSlots = 32;             // phase-boundary stamps per block
 // clears histogram (e + 1) & 1 for the next one.  The whole region must be zero
 // before a workspace's first use.
 constexpr int kCtrlWordExit = 32, kCtrlWordEpoch = 64, kCtrlWordArrive = 96, kCtrlWordReady = 128,
-              kCtrlWordDone = 160;
+              kCtrlWordDone = 160, kCtrlWordBad = 192;
 constexpr int kCtrlBytes = 1024;
 constexpr int kHistWords = kMaxT * kHistBins;                 // one histogram buffer
 constexpr int kWsCtrlBytes = kCtrlBytes + 2 * kHistWords * 4;  // must be zero before first use

@@ -154,6 +154,7 @@ __device__ __forceinline__ void barrier_exit(const StepParams& p)
             if (ok) {
                 p.ctrl[0] = 0u;
                 p.ctrl[kCtrlWordExit] = 0u;
+                p.ctrl[kCtrlWordBad] = 0u;
                 for (int t = 0; t < kMaxT; ++t) {
                     p.ctrl[kCtrlWordArrive + t] = 0u;
                     p.ctrl[kCtrlWordReady + t] = 0u;
@@ -164,6 +165,23 @@ __device__ __forceinline__ void barrier_exit(const StepParams& p)
             }
         }
     }
+}
+
+// The control words are zero at launch but for the epoch (the previous launch on
+// the workspace left them so).  The indexer kernel checks them for the
+// cooperative kernel that follows it, before any of its blocks can write one
+// (they wait for the whole indexer grid first); if they are not, it flags the
+// workspace state and marks the words bad, and that kernel skips its phases.
+// The mark is written either way, so a stale one does not outlive the check.
+__device__ void check_ctrl_words(const StepParams& p)
+{
+    uint32_t any = *reinterpret_cast<volatile uint32_t*>(p.ctrl) | *reinterpret_cast<volatile uint32_t*>(p.ctrl + kCtrlWordExit);
+    for (int t = 0; t < kMaxT; ++t)
+        any |= *reinterpret_cast<volatile uint32_t*>(p.ctrl + kCtrlWordArrive + t) |
+               *reinterpret_cast<volatile uint32_t*>(p.ctrl + kCtrlWordReady + t) |
+               *reinterpret_cast<volatile uint32_t*>(p.ctrl + kCtrlWordDone + t);
+    if (any != 0u) atomicOr(p.err, ERR_WORKSPACE_STATE);
+    p.ctrl[kCtrlWordBad] = any != 0u ? 1u : 0u;
 }
 
 // Per-launch state every block reads at entry.
@@ -1215,18 +1233,36 @@ __device__ void radix_pass_reg(const uint32_t (&k)[kSelReg], int cnt, uint32_t& 
             res[2] = 0u;   // becomes the ties to take, once found
         }
         __syncthreads();
+        {   // one shared atomic per warp: a warp scan places each thread's keys
+            uint32_t c = 0;
 #pragma unroll
-        for (int u = 0; u < kSelReg; ++u)
-            if (u < cnt && k[u] >= nlo && k[u] <= nhi) list[atomicAdd(&res[1], 1u)] = k[u];
+            for (int u = 0; u < kSelReg; ++u) c += u < cnt && k[u] >= nlo && k[u] <= nhi;
+            const uint32_t incl = warp_incl_scan(c);
+            uint32_t base = 0;
+            if (lane == 31 && incl) base = atomicAdd(&res[1], incl);
+            uint32_t o = __shfl_sync(0xffffffffu, base, 31) + incl - c;
+#pragma unroll
+            for (int u = 0; u < kSelReg; ++u)
+                if (u < cnt && k[u] >= nlo && k[u] <= nhi) list[o++] = k[u];
+        }
         __syncthreads();
         const uint32_t n = res[1];
         const uint32_t mine = tid < static_cast<int>(n) ? list[tid] : 0u;
+        // four list entries per shared load (a broadcast); the entries past n are masked
         uint32_t gt = 0, ge = 0;
-#pragma unroll 4
-        for (uint32_t j = 0; j < n; ++j) {
-            const uint32_t o = list[j];
-            gt += o > mine;
-            ge += o >= mine;
+        if (warp * 32 < static_cast<int>(n)) {
+            const uint4* l4 = reinterpret_cast<const uint4*>(list);
+#pragma unroll 2
+            for (uint32_t j = 0; j < n; j += 4) {
+                const uint4 o = l4[j / 4];
+                const uint32_t e[4] = {o.x, o.y, o.z, o.w};
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    if (j + q < n) {
+                        gt += e[q] > mine;
+                        ge += e[q] >= mine;
+                    }
+            }
         }
         // every holder of the exact key finds it; they agree on (key, need - gt)
         if (tid < static_cast<int>(n) && gt < need && need <= ge) {
@@ -1301,7 +1337,8 @@ __device__ void phase_select(const StepParams& p, uint8_t* smem, uint32_t* res, 
                 // ---- few candidates: a run of up to 16 per thread, in registers ----
                 // The list into shared memory in list order, one thread per sub-segment (its
                 // loads, 16 entries at a time, all in flight); then thread i takes entries
-                // [i per, (i + 1) per).
+                // [i per, (i + 1) per).  (Loading each thread's run straight into registers
+                // is slower: every warp load then touches 32 scattered sectors.)
                 uint32_t* ckey = reinterpret_cast<uint32_t*>(smem + kSelEntOff);
                 uint32_t* cpos = ckey + kSelReg * kThreads;
                 for (int k = tid; k < nseg; k += kThreads) {
@@ -1777,18 +1814,24 @@ __device__ void phase_attend(const StepParams& p, uint8_t* smem, uint64_t* bars,
 // in flight at once; the max, the weights and the denominator come by warp
 // shuffles, the sink joins the denominator with no value row.
 // ==================================================================================
-__device__ void phase_merge(const StepParams& p)
+__device__ void phase_merge(const StepParams& p, int* ok_s)
 {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     constexpr int P = 2;                          // halves of the 128 dims per (t, h); two dims per lane
+    static_assert((kH * P) % kWarps == 0, "a block's items of one round belong to one query");
     const int items = p.T * kH * P;
     const int ns = p.nsplit;                      // <= kMaxSplitsQ
-    for (int i = blockIdx.x * kWarps + warp; i < items; i += gridDim.x * kWarps) {
-        const int t = i / (kH * P), h = (i / P) % kH, part = i % P;
-        int ok = 1;
-        if (lane == 0) ok = wait_counter(p, p.ctrl + kCtrlWordDone + t, static_cast<uint32_t>(ns)) ? 1 : 0;
-        ok = __shfl_sync(0xffffffffu, ok, 0);
-        if (!ok) continue;
+    for (int i0 = blockIdx.x * kWarps; i0 < items; i0 += gridDim.x * kWarps) {
+        // One thread waits for the query's splits, then the whole block goes on: the
+        // waiting stays out of the warps' loads.
+        const int t = i0 / (kH * P);
+        if (threadIdx.x == 0) *ok_s = wait_counter(p, p.ctrl + kCtrlWordDone + t, static_cast<uint32_t>(ns)) ? 1 : 0;
+        __syncthreads();
+        const bool ok = *ok_s != 0;
+        __syncthreads();   // every thread has read the flag before the next round writes it
+        const int i = i0 + warp;
+        if (!ok || i >= items) continue;
+        const int h = (i / P) % kH, part = i % P;
         const float2* ml = p.pml + (int64_t)t * ns * kH + h;
         const int d0 = part * (kD / P) + lane * 2;
         const float* po = p.po + ((int64_t)t * ns * kH + h) * kD + d0;
@@ -1863,6 +1906,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1) index_kernel(const __grid_cons
     // blocks take the SMs this grid leaves and wait for its completion
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     init_launch_view(p, p.hist_bound != 0);
+    if (p.hist_bound && p.ctrl != nullptr && blockIdx.x == 0 && threadIdx.x == 0) check_ctrl_words(p);
     __syncthreads();
     stamp(p, 0);
     if (p.trace != nullptr && threadIdx.x == 0) p.trace[(int64_t)blockIdx.x * kTraceSlots + 28] = clock64();
@@ -1899,7 +1943,8 @@ __global__ void __launch_bounds__(kThreads, 1) step_kernel(const StepParams p)
     // attention items done, 9 its merge items done, 30 end, 31 this kernel's
     // start; SM clock: 28 first kernel's start, 27 this kernel's start, 29 end.
     bool ok = true;
-    if (p.ctrl != nullptr) gb.enter();
+    const bool checked = p.hist_bound != 0;   // the indexer kernel checked the control words
+    if (p.ctrl != nullptr && !checked) gb.enter();
     // Launched as a programmatic dependent of the indexer kernel: everything above
     // touches nothing that grid writes; its scores and histogram are read below.
     asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -1915,7 +1960,16 @@ __global__ void __launch_bounds__(kThreads, 1) step_kernel(const StepParams p)
     if (p.phases & kPhaseHistScores) phase_hist_scores(p, smem);
     if (own_first) stamp(p, 1);
     if (p.phases & kPhaseTopk) {
-        ok = gb.sync(p, &ok_s);
+        if (!checked) {
+            ok = gb.sync(p, &ok_s);
+        } else if (p.ctrl != nullptr) {
+            // Nothing before the extraction depends on another block of this grid:
+            // the scores, histogram and group maxima are complete once the indexer
+            // kernel is, so no grid barrier; only its verdict on the control words.
+            if (threadIdx.x == 0) ok_s = *reinterpret_cast<volatile uint32_t*>(p.ctrl + kCtrlWordBad) == 0u;
+            __syncthreads();
+            ok = ok_s != 0;
+        }
         stamp(p, 2);
         if (ok) phase_extract(p, smem, bars, res, scratch);
         stamp(p, 3);
@@ -1929,7 +1983,7 @@ __global__ void __launch_bounds__(kThreads, 1) step_kernel(const StepParams p)
     if (p.phases & kPhaseAttend) {
         if (ok) phase_attend(p, smem, bars, (p.phases & kPhaseTopk) != 0, &ok_s);
         stamp(p, 7);
-        if (ok) phase_merge(p);
+        if (ok) phase_merge(p, &ok_s);
         __syncthreads();
         stamp(p, 9);
     }

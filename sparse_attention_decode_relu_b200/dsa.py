@@ -21,7 +21,7 @@ from . import build as _build
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_DEVICE = 0, 1, 2, 3, 4
 BF16, FP8_E4M3, F32, I32 = 0, 1, 2, 3
 WS_CTRL_BYTES = 263168   # DSA_WS_CTRL_BYTES: leading workspace bytes that must be zero before first use
-WS_WORDS_ZERO_AFTER_CALL = [0, 32] + list(range(96, 104)) + list(range(128, 136))   # int32 words a call leaves at 0
+WS_WORDS_ZERO_AFTER_CALL = [0, 32] + list(range(96, 104)) + list(range(128, 136)) + list(range(160, 168)) + [192]   # int32 words a call leaves at 0
 
 _lock = threading.Lock()
 _lib = None
