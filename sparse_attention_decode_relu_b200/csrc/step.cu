@@ -1033,8 +1033,10 @@ __device__ void phase_extract(const StepParams& p, uint8_t* smem, uint64_t* bars
         uint32_t count = 0;
         if (use_gmax) {
             // Only the 32-position groups whose largest key reaches the cut are read:
-            // eight rounds of 32 group maxima in flight per lane, then the hit groups'
-            // scores four at a time, in position order.
+            // eight rounds of 32 group maxima in flight per lane; the hit groups of all
+            // eight go to a short list in position order (in this warp's ring, idle
+            // here), then their scores are read eight groups at a time.
+            uint16_t* hl = reinterpret_cast<uint16_t*>(ring);   // group index within the round
             for (int base = s0; base < s1; base += 8 * 32 * 32) {
                 uint32_t m[8];
 #pragma unroll
@@ -1042,41 +1044,35 @@ __device__ void phase_extract(const StepParams& p, uint8_t* smem, uint64_t* bars
                     const int g = base + (k * 32 + lane) * 32;
                     m[k] = base == s0 ? m_first[k] : (g < s1 ? __ldcg(gm + g / 32) : 0u);
                 }
+                int nh = 0;
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {
-                    const int g0 = base + k * 32 * 32;
-                    uint32_t hit = __ballot_sync(0xffffffffu, g0 + lane * 32 < s1 && m[k] >= cut);
-                    while (hit) {
-                        int b[4];
-                        int nb = 0;
+                    const bool h = base + (k * 32 + lane) * 32 < s1 && m[k] >= cut;
+                    const uint32_t hm = __ballot_sync(0xffffffffu, h);
+                    if (h) hl[nh + __popc(hm & ((1u << lane) - 1u))] = static_cast<uint16_t>(k * 32 + lane);
+                    nh += __popc(hm);
+                }
+                __syncwarp();
+                for (int j = 0; j < nh; j += 8) {
+                    int sp[8];
+                    float f[8];
 #pragma unroll
-                        for (int u = 0; u < 4; ++u) {
-                            b[u] = 0;
-                            if (hit) {
-                                b[u] = __ffs(hit) - 1;
-                                hit &= hit - 1u;
-                                nb = u + 1;
-                            }
-                        }
-                        float f[4];
+                    for (int u = 0; u < 8; ++u) {
+                        sp[u] = j + u < nh ? base + static_cast<int>(hl[j + u]) * 32 + lane : s1;
+                        f[u] = sp[u] < s1 ? __ldcg(row + sp[u]) : -INFINITY;
+                    }
 #pragma unroll
-                        for (int u = 0; u < 4; ++u) {
-                            const int sp = g0 + b[u] * 32 + lane;
-                            f[u] = (u < nb && sp < s1) ? __ldcg(row + sp) : -INFINITY;
-                        }
-#pragma unroll
-                        for (int u = 0; u < 4; ++u) {
-                            if (u < nb) {
-                                const int sp = g0 + b[u] * 32 + lane;
-                                const uint32_t key = score_key(f[u]);
-                                const bool take = sp < s1 && key >= cut;
-                                const uint32_t tb = __ballot_sync(0xffffffffu, take);
-                                if (take) out[count + __popc(tb & ((1u << lane) - 1u))] = make_uint2(key, static_cast<uint32_t>(sp));
-                                count += __popc(tb);
-                            }
+                    for (int u = 0; u < 8; ++u) {
+                        if (j + u < nh) {
+                            const uint32_t key = score_key(f[u]);
+                            const bool take = sp[u] < s1 && key >= cut;
+                            const uint32_t tb = __ballot_sync(0xffffffffu, take);
+                            if (take) out[count + __popc(tb & ((1u << lane) - 1u))] = make_uint2(key, static_cast<uint32_t>(sp[u]));
+                            count += __popc(tb);
                         }
                     }
                 }
+                __syncwarp();   // the list is rewritten by the next round
             }
         } else {
             auto issue = [&](int j) {
