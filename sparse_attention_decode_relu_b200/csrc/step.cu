@@ -1292,6 +1292,8 @@ constexpr int kSelEntOff = kSelOffOff + kMaxSeg * 4;     // candidates (key, pos
 constexpr int kSelCap = (kDataBytes - kSelEntOff) / 10 / 256 * 256;   // with a 16-bit sub-segment index each
 constexpr int kSelSegOff = kSelEntOff + kSelCap * 8;     // [kSelCap] sub-segment of each candidate
 constexpr int kSelGOff = kSelEntOff + kMaxSeg * 4;       // (global path) second per-sub-segment array
+constexpr int kSelPieceOff = kSelEntOff + 2 * kSelReg * kThreads * 4;   // (register path) [kMaxSeg] first piece
+static_assert(kSelPieceOff + kMaxSeg * 4 <= kDataBytes, "piece numbers fit");
 static_assert(kSelCap >= 4096 && kSelSegOff + kSelCap * 2 <= kDataBytes && kSelGOff + kMaxSeg * 4 <= kDataBytes,
               "selection buffers fit");
 static_assert(kMaxSeg <= 65536, "sub-segment indices fit 16 bits");
@@ -1331,33 +1333,50 @@ __device__ void phase_select(const StepParams& p, uint8_t* smem, uint32_t* res, 
             uint32_t nsel = 0;
             if (m <= static_cast<uint32_t>(kSelReg * kThreads)) {
                 // ---- few candidates: a run of up to 16 per thread, in registers ----
-                // The list into shared memory in list order, one thread per sub-segment (its
-                // loads, 16 entries at a time, all in flight); then thread i takes entries
-                // [i per, (i + 1) per).  (Loading each thread's run straight into registers
-                // is slower: every warp load then touches 32 scattered sectors.)
+                // The list into shared memory in list order, in pieces of 16 entries: a scan
+                // of the sub-segments' piece counts numbers the pieces, thread i takes pieces
+                // i and i + 256 (a binary search finds each one's sub-segment), all loads in
+                // flight; then thread i takes entries [i per, (i + 1) per).  (Loading each
+                // thread's run straight into registers is slower: every warp load then
+                // touches 32 scattered sectors.)
                 uint32_t* ckey = reinterpret_cast<uint32_t*>(smem + kSelEntOff);
                 uint32_t* cpos = ckey + kSelReg * kThreads;
-                for (int k = tid; k < nseg; k += kThreads) {
-                    const uint32_t cnt = seg_cnt(k), o = off[k];
-                    const uint4* src = reinterpret_cast<const uint4*>(glist + seg_start(p, k));
-                    for (uint32_t j = 0; j < cnt; j += 16) {
-                        uint4 v[8];
+                uint32_t* cpre = reinterpret_cast<uint32_t*>(smem + kSelPieceOff);
+                for (int k = tid; k < nseg; k += kThreads) cpre[k] = (seg_cnt(k) + 15u) / 16u;
+                __syncthreads();
+                const uint32_t npiece = block_scan_array(cpre, nseg, scratch);   // cpre[k]: first piece of k
+                for (uint32_t q0 = tid; q0 < npiece; q0 += 2 * kThreads) {
+                    uint4 v[2][8];
+                    uint32_t jj[2], cc[2], oo[2];
+#pragma unroll
+                    for (int h2 = 0; h2 < 2; ++h2) {
+                        const uint32_t q = q0 + h2 * kThreads;
+                        int k = 0;   // the last sub-segment with cpre[k] <= q: a non-empty one
+                        for (int step = 1 << (31 - __clz(nseg)); step > 0; step >>= 1)
+                            if (k + step < nseg && cpre[k + step] <= q) k += step;
+                        const bool any = q < npiece;
+                        jj[h2] = any ? (q - cpre[k]) * 16u : 0u;
+                        cc[h2] = any ? seg_cnt(k) : 0u;
+                        oo[h2] = off[k];
+                        const uint4* src = reinterpret_cast<const uint4*>(glist + seg_start(p, k)) + jj[h2] / 2;
 #pragma unroll
                         for (int u = 0; u < 8; ++u)
-                            v[u] = j + 2 * u < cnt ? __ldcg(src + j / 2 + u) : make_uint4(0u, 0u, 0u, 0u);
+                            v[h2][u] = jj[h2] + 2 * u < cc[h2] ? __ldcg(src + u) : make_uint4(0u, 0u, 0u, 0u);
+                    }
+#pragma unroll
+                    for (int h2 = 0; h2 < 2; ++h2)
 #pragma unroll
                         for (int u = 0; u < 8; ++u) {
-                            const uint32_t e = j + 2 * u;
-                            if (e < cnt) {
-                                ckey[o + e] = v[u].x;
-                                cpos[o + e] = v[u].y;
+                            const uint32_t e = jj[h2] + 2 * u, o = oo[h2];
+                            if (e < cc[h2]) {
+                                ckey[o + e] = v[h2][u].x;
+                                cpos[o + e] = v[h2][u].y;
                             }
-                            if (e + 1 < cnt) {
-                                ckey[o + e + 1] = v[u].z;
-                                cpos[o + e + 1] = v[u].w;
+                            if (e + 1 < cc[h2]) {
+                                ckey[o + e + 1] = v[h2][u].z;
+                                cpos[o + e + 1] = v[h2][u].w;
                             }
                         }
-                    }
                 }
                 __syncthreads();
                 const uint32_t per = (m + kThreads - 1) / kThreads;
