@@ -40,15 +40,42 @@ METRIC = "µs per DSA decode/verify step and achieved HBM GB/s (% of B200 peak) 
 KEY_BYTES = {"bf16": 128, "fp8": 68}
 
 
+def source_code_only(src: str) -> str:
+    """C/C++ source without its comments, blank space collapsed; string and
+    character literals are kept as written."""
+    out, i, n = [], 0, len(src)
+    while i < n:
+        c = src[i]
+        if c in "\"'":
+            j = i + 1
+            while j < n and src[j] != c:
+                j += 2 if src[j] == "\\" else 1
+            out.append(src[i:j + 1])
+            i = j + 1
+        elif src.startswith("//", i):
+            j = src.find("\n", i)
+            i = n if j < 0 else j
+        elif src.startswith("/*", i):
+            j = src.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+            out.append(" ")
+        else:
+            out.append(c)
+            i += 1
+    return " ".join("".join(out).split())
+
+
 def kernel_sources_sha256():
-    """sha256 over the sorted file names and contents of the CUDA sources."""
+    """sha256 over the sorted file names and the code of the CUDA sources
+    (comments and blank space removed: a comment edit leaves a capture's record
+    valid, any change to the code does not)."""
     import hashlib
     d = os.path.join(ROOT, "sparse_attention_decode_relu_b200", "csrc")
     h = hashlib.sha256()
     for f in sorted(os.listdir(d)):
         h.update(f.encode())
-        with open(os.path.join(d, f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(d, f), encoding="utf-8") as fh:
+            h.update(source_code_only(fh.read()).encode())
     return h.hexdigest()
 
 

@@ -257,9 +257,9 @@ DSA_API uint64_t dsa_launch_count(void);
 DSA_API void dsa_set_stage_events(void *const *events, int32_t n);
 
 /* Failure-detection test hook for the calling host thread (one launch only).
- * The next step-kernel launch from this thread that uses grid barriers makes
- * each of them wait for one arrival more than its grid makes: a block that
- * never comes.  Every wait then runs into its bound after limit_cycles SM clocks
+ * The next cooperative-kernel launch from this thread makes each of its waits
+ * between blocks (the grid barrier where there is one, the per-query counters)
+ * wait for one arrival more than its grid makes: a block that never comes.  Every wait then runs into its bound after limit_cycles SM clocks
  * (1000 <= limit_cycles <= 2e9, the normal bound), sets the wait-timeout bit
  * (1) of the device error word and skips the work that depended on the
  * barrier; the launch still ends normally and leaves the workspace control
@@ -276,9 +276,9 @@ DSA_API dsa_status_t dsa_debug_fail_next_barriers(int64_t limit_cycles);
  * into ((uint64_t*)device_buffer)[b * 32 + k] at the phase boundaries of the
  * step: 0 start, 1 indexer scan done (both from the indexer kernel when it
  * runs), 31 start of the cooperative kernel, 2/3 candidate extraction (after
- * its grid barrier), 4/5 the per-query selection (blocks 0..T-1 only), 6 first
- * attention item starts (after its query's selection), 7 attention done, 8/9
- * merge, 30 end; slots 28, 27 and 29 hold the SM clock counter at the start of
+ * its grid barrier where there is one), 4/5 the per-query selection (blocks
+ * 0..T-1 only), 6 first attention item starts (after its query's selection), 7
+ * attention done, 9 merge done, 30 end; slots 28, 27 and 29 hold the SM clock counter at the start of
  * the first kernel, at the start of the cooperative kernel and at the end.  The
  * buffer must hold dsa_step_grid(...) * 32 entries.  NULL disables. */
 DSA_API void dsa_set_step_trace(void *device_buffer);

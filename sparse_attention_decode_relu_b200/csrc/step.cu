@@ -1,17 +1,19 @@
-// step.cu -- the DSA decode/verify step as one cooperative persistent kernel.
+// step.cu -- the DSA decode/verify step as two persistent kernels.
 //
 // NaiveAI research page (naive.ai/en/research), "NaiveRT > A DSA layer: from 29
 // kernels to one": a DSA layer runs as a single cooperative kernel across 148
-// CTAs in one grid.  Here one block per SM runs every phase of the step:
+// CTAs in one grid.  Here one block per SM runs the step in two launches:
 //
-//   1 index   : ReLU indexer scan over the key cache, warp-specialised on the
-//               fifth-generation tensor cores (TMA key tiles, FP8 keys widened
-//               into tensor memory, tcgen05.mma, an epilogue that writes fp32
-//               scores and counts every score's key in a per-query histogram of
-//               its top 12 bits -- the first radix pass of the top-k)
-//   -- grid barrier --
+//   1 index   : (index_kernel) ReLU indexer scan over the key cache,
+//               warp-specialised on the fifth-generation tensor cores (TMA key
+//               tiles, FP8 keys widened into tensor memory, tcgen05.mma, an
+//               epilogue that writes fp32 scores, per-32-position key maxima and
+//               a lower-bound histogram of the keys' top 12 bits -- the first
+//               radix pass of the top-k)
+//   -- step_kernel, a cooperative programmatic dependent of the first: its
+//      blocks wait for the whole indexer grid, no grid barrier of their own --
 //   2 extract : per (query, chunk): every score whose key reaches the query's
-//               threshold bin goes to a candidate sub-segment, in position order
+//               cut bin goes to a candidate sub-segment, in position order
 //   3 select  : per query (block t): the exact top-k among the candidates, ties
 //               to the lower position, written in ascending order; a release
 //               flag per query
@@ -24,7 +26,8 @@
 //   5 merge   : per (query, head), the splits merged in a fixed order, as soon
 //               as every split of the query is done
 //
-// Stage entry points run a sub-range of the phases.  Every reduction is either
+// Stage entry points run a sub-range of the phases (caller scores: the exact
+// histogram in step_kernel, then one grid barrier before the extraction).  Every reduction is either
 // integer or in a fixed order, so results are bitwise reproducible.
 #include <type_traits>
 

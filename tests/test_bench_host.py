@@ -45,5 +45,14 @@ def test_traffic_only_for_the_profiled_sources(monkeypatch):
     assert bench.profiled_traffic("index_kernel", "verify_1m") is None
 
 
+def test_code_hash_ignores_comments_only():
+    a = 'int x = 1; // one\nconst char* s = "a // b /* c */";\n/* block\n comment */ int y;'
+    b = 'int x = 1;\nconst char* s = "a // b /* c */"; int y;'
+    assert bench.source_code_only(a) == bench.source_code_only(b)
+    assert "a // b /* c */" in bench.source_code_only(a)            # literals stay as written
+    assert bench.source_code_only("int x = 1;") != bench.source_code_only("int x = 2;")
+    assert bench.source_code_only("char c = '/'; // x") == "char c = '/';"
+
+
 def test_whole_job_rate_is_weak_scaling():
     assert bench.whole_job_gbs(2e9, 1.0, 4) == 4 * bench.whole_job_gbs(2e9, 1.0, 1)

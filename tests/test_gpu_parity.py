@@ -361,7 +361,7 @@ def test_workspace_control_words_left_zero_and_checked():
 
 def test_barrier_wait_timeout_is_reported_and_recovers():
     """Failure detection of the single cooperative kernel: with the test hook,
-    every grid barrier of one launch waits for a block that never comes.  Each
+    every wait between blocks of one launch waits for a block that never comes.  Each
     bounded wait runs out (about 1 ms here), the launch reports the wait-timeout
     bit alone, leaves the workspace control words at zero, and the next call on
     the same workspace matches the oracle again."""
