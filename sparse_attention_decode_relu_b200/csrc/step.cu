@@ -403,7 +403,7 @@ __device__ void radix_pass(ForEach for_each_key, uint32_t& lo, uint32_t& hi, uin
 
 // ==================================================================================
 // Phase 1: indexer scan on the fifth-generation tensor cores, a kernel of its own
-// with 16 warps per SM in two roles, decoupled by tensor-memory buffers so that
+// with 17 warps per SM in three roles, decoupled by tensor-memory buffers so that
 // each runs at its own pace.  A tile of 128 keys is the M side of tcgen05.mma
 // kind::f16 (bf16 operands, fp32 accumulators in tensor memory), the T x 16
 // indexer query heads the N side (16..128), the 64 dims K (four K = 16 steps).
@@ -963,11 +963,14 @@ __device__ void phase_hist_scores(const StepParams& p, uint8_t* smem)
 
 // ==================================================================================
 // Phase 2: candidate extraction, one item per (query t, chunk c) and block.
-// The query's threshold bin b* (the bin of its topk-th largest key) comes from
-// the launch's histogram; every visible key in bin b* or above is a candidate.
-// Warp w of the block streams its own eighth of the chunk through a private
-// ring of 4 KiB bulk copies and appends its candidates, in position order, to
-// its sub-segment of the query's list (which starts at the sub-range's first
+// The query's cut bin comes from the launch's histogram: the threshold bin b*
+// (the bin of its topk-th largest key) for an exact histogram, a bin at or below
+// it for the indexer's lower-bound one; every visible key in the cut bin or
+// above is a candidate.  Warp w of the block takes its own eighth of the chunk:
+// with group maxima it reads only the scores of the 32-position groups whose
+// maximum reaches the cut, else it streams its scores through a private ring of
+// 4 KiB bulk copies; it appends its candidates, in position order, to its
+// sub-segment of the query's list (which starts at the sub-range's first
 // position, so it can never overflow).  No block-wide barrier in the loop.
 // ==================================================================================
 constexpr int kXStages = 4;
@@ -1281,9 +1284,9 @@ __device__ void radix_pass_reg(const uint32_t (&k)[kSelReg], int cnt, uint32_t& 
 
 // ==================================================================================
 // Phase 3: the selection of query t, by block t once every extraction item of
-// the query is done.  The candidates (every key in the threshold bin or above,
+// the query is done.  The candidates (every key in the cut bin or above,
 // position-ordered sub-segments) are gathered into shared memory in order; a
-// radix select over the threshold bin's low 20 bits finds tau, the topk-th
+// radix select from the top of their key range finds tau, the topk-th
 // largest key, and how many keys equal to tau are taken (the lowest positions,
 // i.e. the first ones in list order); an ordered compaction writes the
 // selected positions ascending.  More candidates than fit in shared memory
@@ -1911,7 +1914,7 @@ __device__ uint32_t init_launch_view(const StepParams& p, bool counts)
     return e;
 }
 
-// The indexer stage as a kernel of its own: one block per SM, 16 warps.  With a
+// The indexer stage as a kernel of its own: one block per SM, 17 warps.  With a
 // workspace it also counts the first radix pass into the launch's histogram.
 template <bool FP8>
 __global__ void __launch_bounds__(kIdxThreads, 1) index_kernel(const __grid_constant__ CUtensorMap kmap, const StepParams p)
